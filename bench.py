@@ -1,0 +1,695 @@
+#!/usr/bin/env python
+"""NSA / MoBA forward benchmark on B200 (one JSON line on rank 0).
+
+Default workload: NSA single-token decode, 32 sequences x 65536-token KV
+cache, 64 query heads / 4 KV heads, d = 128, bf16, top-16 blocks of 64,
+window 512 (metric: algorithmic KV GB/s). ``--workload`` selects the NSA
+prefill (TFLOP/s) or MoBA prefill (TFLOP/s) workloads instead.
+
+A step is one call of the hot path over one batch of inputs already resident
+in HBM. Timing: W warm-up steps, then exactly K steps between CUDA events on
+the launching stream, a barrier and a device synchronise on both sides, the
+max over ranks. Every step reads more than the 126 MB L2 (stated in config).
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the same
+workload instead (rank 0 only).
+
+Multi-GPU (torchrun): each rank runs its own batch (different seed); there is
+no collective on the data path (weak scaling); value = all ranks' work / the
+slowest rank's time.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from dynamic_block_sparse_nsa_b200 import inputs  # noqa: E402
+
+METRIC = "NSA decode KV GB/s & prefill TFLOP/s at 64k ctx; fraction of roofline"
+DEFAULT_WORKLOAD = "nsa_decode_bf16_b32_l65536"
+L2_BYTES = 126 * 2**20
+
+
+# --------------------------------------------------------------------------
+# peaks, clocks
+# --------------------------------------------------------------------------
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return dict(hbm=float(pk["hbm_gbs"]), bf16=float(pk["bf16_tflops"]),
+                    bf16_sus=float(pk["bf16_tflops_sustained"]), src="measured")
+    except (OSError, KeyError, ValueError):
+        return dict(hbm=6650.0, bf16=1590.0, bf16_sus=1400.0, src="fallback")
+
+
+_REASONS = {
+    0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+    0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+    0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+    0x100: "display_clock_setting",
+}
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    def __init__(self, device_index, period_s=0.005):
+        self.period = period_s
+        self.samples = []
+        self.max_mhz = None
+        self.err = None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # NVML missing: clocks reported as unavailable
+            self._nv = None
+            self.err = f"nvml unavailable: {e}"
+        self._t = None
+
+    def _reasons(self):
+        nv = self._nv
+        fn = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        return fn(self._h)
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                rs = self._reasons()
+                self.samples.append((mhz, rs))
+            except Exception as e:
+                self.err = str(e)
+                return
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [],
+                    "samples": 0, "note": self.err or "no samples"}
+        mhz = [s[0] for s in self.samples]
+        bits = 0
+        for _, r in self.samples:
+            bits |= int(r)
+        names = [n for b, n in _REASONS.items() if bits & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(mhz)}
+
+
+# --------------------------------------------------------------------------
+# algorithmic work (bytes for decode, flops for prefill)
+# --------------------------------------------------------------------------
+
+def n_cmp(T, l, s):
+    return 0 if T < l else (T - l) // s + 1
+
+
+def sel_tokens(sel, t, bs):
+    """Tokens of the selected blocks up to position t (sel: int array, -1 padded)."""
+    blk = sel[sel >= 0].astype(np.int64)
+    return int(np.sum(np.minimum(blk * bs + bs - 1, t) - blk * bs + 1))
+
+
+def decode_work(w, lens, sel_h):
+    """Algorithmic bytes of one decode step: every branch's reads counted once,
+    plus q/out/gate/selection traffic; and the union bytes (selected blocks and
+    window deduplicated)."""
+    d, Hkv, Hq, n, bs, win = w["d"], w["Hkv"], w["Hq"], w["top_n"], w["sel_block"], w["window"]
+    esz = 2 if w["dtype"] == "bf16" else 4
+    row = d * esz
+    total = union = 0
+    parts = dict(cmp=0, slc=0, win=0, io=0)
+    for b, L in enumerate(lens):
+        t = L - 1
+        nv = n_cmp(L, w["cmp_block"], w["cmp_stride"])
+        for g in range(Hkv):
+            ks = sel_tokens(sel_h[b, g], t, bs)
+            kw = min(win, L)
+            parts["cmp"] += 2 * nv * row
+            parts["slc"] += 2 * ks * row
+            parts["win"] += 2 * kw * row
+            toks = set()
+            for j in sel_h[b, g][sel_h[b, g] >= 0]:
+                toks.update(range(j * bs, min(j * bs + bs - 1, t) + 1))
+            toks.update(range(t - kw + 1, t + 1))
+            union += 2 * nv * row + 2 * len(toks) * row
+        io = 2 * Hq * d * esz + d * 3 * 4 + 4 + Hkv * n * 4
+        parts["io"] += io
+        union += io
+    total = sum(parts.values())
+    return total, union, parts
+
+
+def prefill_flops(w, sel_h):
+    """Algorithmic flops (4 d per query head and attended key, causal exact)."""
+    T, Hq, Hkv, d, bs, win = w["T"], w["Hq"], w["Hkv"], w["d"], w["sel_block"], w["window"]
+    G = Hq // Hkv
+    t = np.arange(T)
+    nvis = np.where(t + 1 >= w["cmp_block"], (t + 1 - w["cmp_block"]) // w["cmp_stride"] + 1, 0)
+    cmp_keys = int(nvis.sum()) * Hq
+    win_keys = int(np.minimum(win, t + 1).sum()) * Hq
+    sel = sel_h.reshape(-1, T, Hkv, sel_h.shape[-1]).astype(np.int64)
+    tt = np.broadcast_to(t[None, :, None, None], sel.shape)
+    ok = sel >= 0
+    cnt = np.where(ok, np.minimum(sel * bs + bs - 1, tt) - sel * bs + 1, 0)
+    slc_keys = int(cnt.sum()) * G
+    f = 4 * d
+    return dict(cmp=cmp_keys * f, slc=slc_keys * f, win=win_keys * f)
+
+
+def moba_flops(w, sel_h):
+    T, Hq, d, m = w["T"], w["Hq"], w["d"], w["block"]
+    t = np.arange(T)
+    sel = sel_h.reshape(-1, T, Hq, sel_h.shape[-1]).astype(np.int64)
+    tt = np.broadcast_to(t[None, :, None, None], sel.shape)
+    cnt = np.where(sel >= 0, np.minimum(sel * m + m - 1, tt) - sel * m + 1, 0)
+    attn = int(cnt.sum()) * 4 * d
+    gate = int((t // m).sum()) * Hq * 2 * d
+    return dict(attn=attn, gate=gate)
+
+
+# --------------------------------------------------------------------------
+# measured DRAM traffic (ncu) recorded under profiles/
+# --------------------------------------------------------------------------
+
+def kernel_traffic(name, workload):
+    """DRAM bytes per launch from profiles/dram_traffic.txt, if recorded for this
+    kernel and workload and the kernel's source has not changed since."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    for line in open(path):
+        f = line.split()
+        if len(f) != 5 or f[0].startswith("#"):
+            continue
+        kname, wl, src, sha, nbytes = f
+        if kname != name or wl != workload:
+            continue
+        sp = os.path.join(ROOT, "dynamic_block_sparse_nsa_b200", "csrc", src)
+        if not os.path.exists(sp):
+            return None
+        cur = hashlib.sha256(open(sp, "rb").read()).hexdigest()[:16]
+        return float(nbytes) if cur == sha else None
+    return None
+
+
+# --------------------------------------------------------------------------
+# distributed helpers
+# --------------------------------------------------------------------------
+
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def reduce_max(x, ws):
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(x, ws):
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------
+# the timed loops
+# --------------------------------------------------------------------------
+
+def timed(step, K, W, ws, device_index, trace=True):
+    from dynamic_block_sparse_nsa_b200 import nsa
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize()
+    barrier(ws)
+    torch.cuda.synchronize()
+    if trace:
+        nsa.trace_enable(True, capacity=K * 16 + 64)
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device_index) as clk:
+        e0.record(s)
+        for _ in range(K):
+            step()
+        e1.record(s)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    recs, launches = ([], 0)
+    if trace:
+        recs, launches = nsa.trace_records()
+        nsa.trace_enable(False)
+    barrier(ws)
+    return ms, recs, launches, clk.summary()
+
+
+def kernel_table(recs, K):
+    tab = {}
+    for name, ms in recs:
+        e = tab.setdefault(name, dict(launches=0, total_ms=0.0))
+        e["launches"] += 1
+        e["total_ms"] += ms
+    tot = sum(e["total_ms"] for e in tab.values()) or 1.0
+    for e in tab.values():
+        e["mean_us"] = 1000.0 * e["total_ms"] / max(1, e["launches"])
+        e["share"] = e["total_ms"] / tot
+    return tab
+
+
+def run_decode(w, K, W, ws, rank, local, e2e=True):
+    from dynamic_block_sparse_nsa_b200 import nsa
+    inp = inputs.make_decode(w, seed=w["seed"] + rank, device="cuda")
+    p = nsa.params(w["B"], w["T"], w["Hq"], w["Hkv"], w["d"], cmp_block=w["cmp_block"],
+                   cmp_stride=w["cmp_stride"], sel_block=w["sel_block"], top_n=w["top_n"],
+                   window=w["window"], dtype=inputs.DTYPES[w["dtype"]])
+    kc, vc = nsa.nsa_compress_kv(p, inp["k"], inp["v"], inp["w_cmp"])
+    ws_buf = nsa.workspace(p, nsa.OP_DECODE)
+    out = torch.empty(w["B"], w["Hq"], w["d"], dtype=inputs.DTYPES[w["dtype"]], device="cuda")
+    sel = torch.empty(w["B"], w["Hkv"], w["top_n"], dtype=torch.int32, device="cuda")
+    q, lens = inp["q"], inp["seq_lens"]
+
+    def step():
+        nsa.nsa_decode(p, q, inp["k"], inp["v"], lens, kc, vc, inp["w_gate"], out=out,
+                       sel_idx=sel, ws=ws_buf)
+
+    step()
+    nsa.nsa_check()
+    ms, recs, launches, clk = timed(step, K, W, ws, local)
+    nsa.nsa_check()
+    sel_h = sel.cpu().numpy()
+    lens_l = lens.cpu().tolist()
+    step_bytes, union_bytes, parts = decode_work(w, lens_l, sel_h)
+    res = dict(ms=ms, recs=recs, launches=launches, clk=clk, work=step_bytes,
+               union=union_bytes, parts=parts)
+    if e2e:
+        # through the public call with host buffers: H2D of the step's query and
+        # lengths, D2H of the output and selection; the KV caches are device-
+        # resident state (as in serving), not per-step inputs.
+        q_h = q.cpu().pin_memory()
+        lens_h = lens.cpu().pin_memory()
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        sel_h_p = torch.empty(sel.shape, dtype=sel.dtype).pin_memory()
+
+        def e2e_step():
+            q.copy_(q_h, non_blocking=True)
+            lens.copy_(lens_h, non_blocking=True)
+            step()
+            out_h.copy_(out, non_blocking=True)
+            sel_h_p.copy_(sel, non_blocking=True)
+
+        ems, _, _, _ = timed(e2e_step, K, max(3, W // 2), ws, local, trace=False)
+        res["e2e_ms"] = ems
+        res["h2d"] = q_h.numel() * q_h.element_size() + lens_h.numel() * 4
+        res["d2h"] = out_h.numel() * out_h.element_size() + sel_h_p.numel() * 4
+    return res
+
+
+def run_prefill(w, K, W, ws, rank, local, e2e=True):
+    from dynamic_block_sparse_nsa_b200 import nsa
+    inp = inputs.make_prefill(w, seed=w["seed"] + rank, device="cuda")
+    dt = inputs.DTYPES[w["dtype"]]
+    p = nsa.params(w["B"], w["T"], w["Hq"], w["Hkv"], w["d"], cmp_block=w["cmp_block"],
+                   cmp_stride=w["cmp_stride"], sel_block=w["sel_block"], top_n=w["top_n"],
+                   window=w["window"], dtype=dt)
+    Nc = nsa.num_cmp_blocks(w["T"], w["cmp_block"], w["cmp_stride"])
+    kc = torch.empty(w["B"], Nc, w["Hkv"], w["d"], dtype=dt, device="cuda")
+    vc = torch.empty_like(kc)
+    ws_buf = nsa.workspace(p, nsa.OP_PREFILL)
+    out = torch.empty_like(inp["q"])
+    sel = torch.empty(w["B"], w["T"], w["Hkv"], w["top_n"], dtype=torch.int32, device="cuda")
+
+    def step():
+        nsa.nsa_compress_kv(p, inp["k"], inp["v"], inp["w_cmp"], kc, vc)
+        nsa.nsa_prefill(p, inp["q"], inp["k"], inp["v"], kc, vc, inp["w_gate"], out=out,
+                        sel_idx=sel, ws=ws_buf)
+
+    step()
+    nsa.nsa_check()
+    ms, recs, launches, clk = timed(step, K, W, ws, local)
+    nsa.nsa_check()
+    fl = prefill_flops(w, sel.cpu().numpy())
+    res = dict(ms=ms, recs=recs, launches=launches, clk=clk, work=sum(fl.values()), parts=fl)
+    if e2e:
+        hq = inp["q"].cpu().pin_memory()
+        hk = inp["k"].cpu().pin_memory()
+        hv = inp["v"].cpu().pin_memory()
+        ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+        def e2e_step():
+            inp["q"].copy_(hq, non_blocking=True)
+            inp["k"].copy_(hk, non_blocking=True)
+            inp["v"].copy_(hv, non_blocking=True)
+            step()
+            ho.copy_(out, non_blocking=True)
+
+        ems, _, _, _ = timed(e2e_step, K, max(3, W // 2), ws, local, trace=False)
+        res["e2e_ms"] = ems
+        res["h2d"] = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+        res["d2h"] = ho.numel() * ho.element_size()
+    return res
+
+
+def run_moba(w, K, W, ws, rank, local, e2e=True):
+    from dynamic_block_sparse_nsa_b200 import nsa
+    inp = inputs.make_prefill(w, seed=w["seed"] + rank, device="cuda")
+    p = nsa.params(w["B"], w["T"], w["Hq"], w["Hkv"], w["d"], sel_block=w["block"],
+                   top_n=w["top_k"], dtype=inputs.DTYPES[w["dtype"]])
+    ws_buf = nsa.workspace(p, nsa.OP_MOBA_PREFILL)
+    out = torch.empty_like(inp["q"])
+    sel = torch.empty(w["B"], w["T"], w["Hq"], w["top_k"], dtype=torch.int32, device="cuda")
+
+    def step():
+        nsa.moba_prefill(p, inp["q"], inp["k"], inp["v"], out=out, sel_idx=sel, ws=ws_buf)
+
+    step()
+    nsa.nsa_check()
+    ms, recs, launches, clk = timed(step, K, W, ws, local)
+    nsa.nsa_check()
+    fl = moba_flops(w, sel.cpu().numpy())
+    res = dict(ms=ms, recs=recs, launches=launches, clk=clk, work=sum(fl.values()), parts=fl)
+    if e2e:
+        hq, hk, hv = (inp[x].cpu().pin_memory() for x in ("q", "k", "v"))
+        ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+
+        def e2e_step():
+            inp["q"].copy_(hq, non_blocking=True)
+            inp["k"].copy_(hk, non_blocking=True)
+            inp["v"].copy_(hv, non_blocking=True)
+            step()
+            ho.copy_(out, non_blocking=True)
+
+        ems, _, _, _ = timed(e2e_step, K, max(3, W // 2), ws, local, trace=False)
+        res["e2e_ms"] = ems
+        res["h2d"] = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
+        res["d2h"] = ho.numel() * ho.element_size()
+    return res
+
+
+# --------------------------------------------------------------------------
+# dominant kernel: algorithmic work per launch
+# --------------------------------------------------------------------------
+
+def kernel_work(kind, name, res, w):
+    """Algorithmic bytes (decode) or flops (prefill) of one launch of `name`,
+    and whether it is bandwidth ('hbm') or tensor ('tensor') bound."""
+    if kind == "decode":
+        p = res["parts"]
+        per = {
+            "nsa_rows_simt": p["cmp"] + p["slc"] + p["win"] + p["io"],
+            "dec_cmp_partial": p["cmp"],
+            "dec_sel_win": p["slc"] + p["win"],
+        }
+        return per.get(name), "hbm"
+    if kind == "prefill":
+        p = res["parts"]
+        per = {
+            "nsa_rows_simt": p["cmp"] + p["slc"] + p["win"],
+            "pf_cmp_attn": p["cmp"],
+            "pf_slc_attn": p["slc"],
+            "pf_win_attn": p["win"],
+        }
+        return per.get(name), "tensor"
+    p = res["parts"]
+    per = {"moba_rows_simt": p["attn"] + p["gate"], "moba_attn": p["attn"]}
+    return per.get(name), "tensor"
+
+
+# --------------------------------------------------------------------------
+# CPU oracle (baseline leg and reference arm)
+# --------------------------------------------------------------------------
+
+def oracle_sample(w, budget_s):
+    """Time the fp64 oracle on a bounded sample of the workload: returns
+    (work units of the sample in the metric's unit numerator, seconds, cores,
+    description)."""
+    import oracle
+    cores = os.cpu_count() or 1
+    kind = w["kind"]
+    if kind == "decode":
+        # unit: one query row (the G heads of a KV group) against one KV
+        # group's 65536-token cache and its compressed cache; `cores` units run
+        # in parallel per oracle call (OpenMP over rows).
+        one = dict(w, B=1)
+        inp = inputs.make_decode(one, seed=w["seed"] + 1000)
+        G = w["Hq"] // w["Hkv"]
+        op = dict(B=1, T=w["T"], Hq=G, Hkv=1, d=w["d"], cmp_block=w["cmp_block"],
+                  cmp_stride=w["cmp_stride"], sel_block=w["sel_block"], top_n=w["top_n"],
+                  window=w["window"], scale=0.0, gate_mode=0, store=w["dtype"], score_mode=0)
+        kg = np.ascontiguousarray(inp["k"][:, :, 0:1].double().numpy())
+        vg = np.ascontiguousarray(inp["v"][:, :, 0:1].double().numpy())
+        kc, vc = oracle.compress(op, kg, vg, inp["w_cmp"].double().numpy())
+        q = inp["q"][0, 0:G].double().numpy()
+        qrows = np.ascontiguousarray(np.broadcast_to(q, (cores, G, w["d"])))
+        wg = inp["w_gate"].double().numpy()
+        L = w["T"]
+        byt, secs, done = 0, 0.0, 0
+        while True:
+            t0 = time.perf_counter()
+            res = oracle.nsa_rows(op, [0] * cores, [L - 1] * cores, qrows, kg, vg, kc, vc, wg)
+            secs += time.perf_counter() - t0
+            for i in range(cores):
+                byt += decode_work(dict(w, Hkv=1, Hq=G), [L], res["sel"][i:i + 1])[0]
+            done += cores
+            if secs >= budget_s:
+                break
+        return byt, secs, cores, (f"{done} (query row, KV head) units of the 65536-token "
+                                  f"decode ({w['B'] * w['Hkv']} units make one step)")
+    if kind == "prefill":
+        inp = inputs.make_prefill(w, seed=w["seed"] + 1000)
+        op = dict(B=w["B"], T=w["T"], Hq=w["Hq"], Hkv=w["Hkv"], d=w["d"],
+                  cmp_block=w["cmp_block"], cmp_stride=w["cmp_stride"],
+                  sel_block=w["sel_block"], top_n=w["top_n"], window=w["window"], scale=0.0,
+                  gate_mode=0, store=w["dtype"], score_mode=0)
+        k64, v64 = inp["k"].double().numpy(), inp["v"].double().numpy()
+        kc, vc = oracle.compress(op, k64, v64, inp["w_cmp"].double().numpy())
+        q64 = inp["q"].double().numpy()
+        rng = np.random.default_rng(0)
+        fl, t_used, done = 0, 0.0, 0
+        while t_used < budget_s:
+            rows = np.sort(rng.integers(0, w["T"], cores))
+            t0 = time.perf_counter()
+            res = oracle.nsa_rows(op, [0] * len(rows), rows, q64[0, rows], k64, v64, kc, vc,
+                                  inp["w_gate"].double().numpy())
+            t_used += time.perf_counter() - t0
+            for i, t in enumerate(rows):
+                nv = n_cmp(t + 1, w["cmp_block"], w["cmp_stride"])
+                ks = sum(sel_tokens(res["sel"][i, g], t, w["sel_block"]) for g in range(w["Hkv"]))
+                fl += 4 * w["d"] * (nv * w["Hq"] + ks * (w["Hq"] // w["Hkv"])
+                                    + min(w["window"], t + 1) * w["Hq"])
+            done += len(rows)
+        return fl, t_used, cores, f"{done} uniformly sampled query rows (all heads)"
+    # moba
+    inp = inputs.make_prefill(dict(w, Hq=4, Hkv=4), seed=w["seed"] + 1000)
+    op = dict(B=1, T=w["T"], Hq=4, Hkv=4, d=w["d"], block=w["block"], top_k=w["top_k"],
+              scale=0.0)
+    k64, v64, q64 = (inp[x].double().numpy() for x in ("k", "v", "q"))
+    kbar = oracle.moba_block_means(op, k64)
+    rng = np.random.default_rng(0)
+    fl, t_used, done = 0, 0.0, 0
+    while t_used < budget_s:
+        rows = np.sort(rng.integers(0, w["T"], cores))
+        t0 = time.perf_counter()
+        res = oracle.moba_rows(op, [0] * len(rows), rows, q64[0, rows], k64, v64, kbar)
+        t_used += time.perf_counter() - t0
+        for i, t in enumerate(rows):
+            for h in range(4):
+                fl += 4 * w["d"] * sel_tokens(res["sel"][i, h], t, w["block"])
+                fl += 2 * w["d"] * (t // w["block"])
+        done += len(rows)
+    return fl, t_used, cores, f"{done} sampled query rows x 4 heads"
+
+
+def unit_of(kind):
+    return ("GB/s", 1e9) if kind == "decode" else ("TFLOP/s", 1e12)
+
+
+def run_reference(args, w):
+    """The oracle, as it stands, timed on the host cores: K steps of a bounded
+    sample each, sized so the whole run stays within a few minutes."""
+    kind = w["kind"]
+    unit, scale = unit_of(kind)
+    per_step = max(0.02, 150.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_sample(w, per_step)
+    work = secs = 0.0
+    cores, desc = 1, ""
+    for _ in range(args.steps):
+        wk, dt, cores, desc = oracle_sample(w, per_step)
+        work += wk
+        secs += dt
+    value = work / secs / scale
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": unit,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000.0 * secs / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, **config_of(w)},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
+                         "sample": f"each step: {desc}"},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w):
+    keys = [k for k in ("B", "T", "Hq", "Hkv", "d", "cmp_block", "cmp_stride", "sel_block",
+                        "top_n", "window", "block", "top_k", "dtype") if k in w]
+    c = {k: w[k] for k in keys}
+    return c
+
+
+# --------------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=None)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    args = ap.parse_args()
+    w = inputs.workload(args.workload)
+    kind = w["kind"]
+    if args.steps is None:
+        args.steps = {"decode": 2000, "prefill": 20, "moba": 10}[kind]
+    if args.warmup is None:
+        args.warmup = {"decode": 20, "prefill": 3, "moba": 3}[kind]
+    args.warmup = max(3, args.warmup)
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        if rank == 0:
+            run_reference(args, w)
+        return
+
+    ws, rank, local = dist_setup()
+    import dynamic_block_sparse_nsa_b200.nsa  # noqa: F401  (fails loudly if unbuilt)
+    runner = {"decode": run_decode, "prefill": run_prefill, "moba": run_moba}[kind]
+    res = runner(w, args.steps, args.warmup, ws, rank, local)
+
+    K = args.steps
+    ms_max = reduce_max(res["ms"], ws)
+    work_all = reduce_sum(res["work"] * K, ws)
+    unit, scale = unit_of(kind)
+    value = work_all / (ms_max / 1000.0) / scale
+    e2e = None
+    if "e2e_ms" in res:
+        e_ms = reduce_max(res["e2e_ms"], ws)
+        e2e = {"value": work_all / (e_ms / 1000.0) / scale, "unit": unit,
+               "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"],
+               "ms_per_step": e_ms / K}
+
+    tab = kernel_table(res["recs"], K)
+    peaks = load_peaks()
+    roof = None
+    if tab:
+        dom = max(tab, key=lambda n: tab[n]["total_ms"])
+        wk, bound = kernel_work(kind, dom, res, w)
+        mean_s = tab[dom]["total_ms"] / tab[dom]["launches"] / 1000.0
+        if wk is not None:
+            launches_per_step = tab[dom]["launches"] / K
+            per_launch = wk / launches_per_step
+            if bound == "hbm":
+                ach = per_launch / mean_s / 1e9
+                pk, u = peaks["hbm"], "GB/s"
+            else:
+                ach = per_launch / mean_s / 1e12
+                pk, u = peaks["bf16"], "TFLOP/s"
+            roof = {"kernel": dom, "bound": bound, "achieved": ach, "peak": pk, "unit": u,
+                    "frac": ach / pk, "peak_source": peaks["src"],
+                    "traffic": kernel_traffic(dom, args.workload),
+                    "algorithmic_per_launch": per_launch}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        wk, secs, cores, desc = oracle_sample(w, args.cpu_budget)
+        cpu = {"value": wk / secs / scale, "unit": unit, "cores": cores, "kind": "oracle",
+               "sample": desc, "seconds": secs}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": unit, "n_gpus": ws, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_max / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": w["dtype"], "data": "synthetic",
+            "config": {"workload": args.workload, **config_of(w),
+                       "l2": "inputs larger than L2 every step "
+                             f"({res['work'] / 1e6:.0f} MB read per step)" if kind == "decode"
+                       else "inputs larger than L2 every step"},
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": res["launches"],
+            "clocks": res["clk"],
+            "kernels": {n: {k: (round(v, 4) if isinstance(v, float) else v)
+                            for k, v in e.items()} for n, e in tab.items()},
+        }
+        if kind == "decode":
+            line["decode_bytes"] = {"per_step": res["work"], "union_per_step": res["union"],
+                                    **{k: v for k, v in res["parts"].items()}}
+            line["hbm_frac_nominal_8tbs"] = value / 8000.0
+        else:
+            line["flops_per_step"] = res["parts"]
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -49,15 +49,23 @@ def workload(name, **overrides):
 
 
 def _randn(gen, shape, scale, dtype):
-    x = torch.randn(*shape, generator=gen, dtype=torch.float32)
+    x = torch.randn(*shape, generator=gen, dtype=torch.float32, device=gen.device)
     if scale != 1.0:
         x.mul_(scale)
     return x.to(dtype)
 
 
-def make_prefill(w, seed=None):
-    """q [B,T,Hq,d], k/v [B,T,Hkv,d] in the run dtype; w_cmp [l], w_gate [d,3] fp32."""
-    gen = torch.Generator().manual_seed(w["seed"] if seed is None else seed)
+def _gen(seed, device):
+    return torch.Generator(device=device or "cpu").manual_seed(seed)
+
+
+def make_prefill(w, seed=None, device=None):
+    """q [B,T,Hq,d], k/v [B,T,Hkv,d] in the run dtype; w_cmp [l], w_gate [d,3] fp32.
+
+    device=None draws on the CPU generator (the recipe the tests use); a CUDA
+    device draws the same distributions from a CUDA generator (other numbers,
+    used by the benchmark to skip the host draw of multi-GB inputs)."""
+    gen = _gen(w["seed"] if seed is None else seed, device)
     dt = DTYPES[w["dtype"]]
     B, T, Hq, Hkv, d = w["B"], w["T"], w["Hq"], w["Hkv"], w["d"]
     sc = w.get("qkv_scale", 1.0)
@@ -67,30 +75,30 @@ def make_prefill(w, seed=None):
     out = dict(q=q, k=k, v=v)
     if "cmp_block" in w:
         l = w["cmp_block"]
-        out["w_cmp"] = torch.randn(l, generator=gen) * math.sqrt(1.0 / l)
-        out["w_gate"] = torch.randn(d, 3, generator=gen) * math.sqrt(1.0 / d)
+        out["w_cmp"] = torch.randn(l, generator=gen, device=gen.device) * math.sqrt(1.0 / l)
+        out["w_gate"] = torch.randn(d, 3, generator=gen, device=gen.device) * math.sqrt(1.0 / d)
     return out
 
 
-def make_decode(w, seed=None, seq_lens=None):
+def make_decode(w, seed=None, seq_lens=None, device=None):
     """q [B,Hq,d], k/v caches [B,T,Hkv,d], seq_lens [B] int32 (default: all T)."""
-    gen = torch.Generator().manual_seed(w["seed"] if seed is None else seed)
+    gen = _gen(w["seed"] if seed is None else seed, device)
     dt = DTYPES[w["dtype"]]
     B, T, Hq, Hkv, d = w["B"], w["T"], w["Hq"], w["Hkv"], w["d"]
     sc = w.get("qkv_scale", 1.0)
     q = _randn(gen, (B, Hq, d), sc, dt)
-    k = torch.empty(B, T, Hkv, d, dtype=dt)
-    v = torch.empty(B, T, Hkv, d, dtype=dt)
+    k = torch.empty(B, T, Hkv, d, dtype=dt, device=gen.device)
+    v = torch.empty(B, T, Hkv, d, dtype=dt, device=gen.device)
     for b in range(B):
         k[b] = _randn(gen, (T, Hkv, d), sc, dt)
     for b in range(B):
         v[b] = _randn(gen, (T, Hkv, d), sc, dt)
     l = w["cmp_block"]
-    w_cmp = torch.randn(l, generator=gen) * math.sqrt(1.0 / l)
-    w_gate = torch.randn(d, 3, generator=gen) * math.sqrt(1.0 / d)
+    w_cmp = torch.randn(l, generator=gen, device=gen.device) * math.sqrt(1.0 / l)
+    w_gate = torch.randn(d, 3, generator=gen, device=gen.device) * math.sqrt(1.0 / d)
     if seq_lens is None:
         seq_lens = [T] * B
-    lens = torch.tensor(seq_lens, dtype=torch.int32)
+    lens = torch.tensor(seq_lens, dtype=torch.int32, device=gen.device)
     return dict(q=q, k=k, v=v, w_cmp=w_cmp, w_gate=w_gate, seq_lens=lens)
 
 

@@ -1,0 +1,187 @@
+/*
+ * nsa.h -- C ABI of the B200 (sm_100a) Native Sparse Attention / MoBA
+ * forward library (libnsa_b200.so).
+ *
+ * Operations (the sources print no equations; each operation is the plain
+ * reading of their prose with the constants of the workload statement):
+ *   - nsa_compress_kv: token compression, "Zhang Xiaojun EP94 notes" §五 branch
+ *     one; lchairun.cn NSA article, compression paragraph.
+ *   - nsa_prefill / nsa_decode: the three-branch NSA forward, EP94 notes §五
+ *     (compressed, selected and sliding-window branches, gating) and §六 (GQA
+ *     group-shared selection); lchairun.cn NSA article, selection, window and
+ *     gate paragraphs (decode is bound by KV bytes moved).
+ *   - moba_prefill: MoBA, EP94 notes §九/§十/§十六 (mean-pooled block keys,
+ *     parameter-free per-head top-k, block 512, top-3); LateTalk ep.103 (the
+ *     query's own block is always attended).
+ *
+ * Conventions for every call:
+ *   - Tensors are plain device pointers, contiguous, row-major, in the layout
+ *     given per argument ("bshd": [batch, tokens, heads, head_dim]). The caller
+ *     allocates and owns all of them; the library never allocates or frees
+ *     device memory and never synchronises, except nsa_check.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream). All work is enqueued asynchronously on it.
+ *   - Arguments are validated on the host before anything is launched; on an
+ *     error nothing is written and a status other than NSA_OK is returned,
+ *     with a message in nsa_last_error_detail().
+ *   - Launch failures return NSA_ERR_CUDA. Faults found on the device (a
+ *     bounded wait that gave up, a sequence length out of range) set a
+ *     per-device error word that nsa_check reports.
+ *   - Thread safety: calls on different streams may run concurrently; the
+ *     error-detail string is thread-local.
+ */
+#ifndef NSA_B200_H_
+#define NSA_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define NSA_API __attribute__((visibility("default")))
+#else
+#define NSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  NSA_OK = 0,
+  NSA_ERR_INVALID_ARGUMENT = 1, /* bad pointer, shape, size or mode          */
+  NSA_ERR_UNSUPPORTED = 2,      /* valid but not implemented (e.g. head dim) */
+  NSA_ERR_WORKSPACE_TOO_SMALL = 3,
+  NSA_ERR_CUDA = 4,             /* a CUDA runtime call or launch failed      */
+  NSA_ERR_DEVICE_TIMEOUT = 5    /* a bounded device-side wait gave up        */
+} nsa_status;
+
+typedef enum { NSA_DTYPE_F32 = 0, NSA_DTYPE_BF16 = 1 } nsa_dtype;
+
+/* Operation ids for nsa_workspace_size. */
+typedef enum {
+  NSA_OP_COMPRESS = 0,
+  NSA_OP_PREFILL = 1,
+  NSA_OP_DECODE = 2,
+  NSA_OP_MOBA_PREFILL = 3
+} nsa_op;
+
+/* Problem description shared by all calls.
+ *   B, T       batch and tokens (prefill: every sequence has T tokens; decode:
+ *              T is the KV-cache capacity, the live length comes from seq_lens;
+ *              MoBA: tokens per sequence).
+ *   Hq, Hkv    query heads and KV heads; Hq % Hkv == 0; query head h reads KV
+ *              head h / (Hq / Hkv) (consecutive heads form a GQA group).
+ *   d          head dimension: 64 or 128.
+ *   cmp_block, cmp_stride   compression length l and stride s (l >= s >= 1).
+ *   sel_block  selection block size (NSA: 64); MoBA block size m (512).
+ *   top_n      NSA: blocks kept per (token, KV head), block 0 included;
+ *              MoBA: blocks kept per (token, head), the own block included.
+ *   window     sliding-window length w (>= 1).
+ *   softmax_scale  0 selects 1/sqrt(d).
+ *   gate_mode  0: g = sigmoid(q . Wg) per branch (Wg [d,3], order cmp, slc,
+ *              win, raw unscaled q); 1: g = fixed_gates for every query.
+ *   dtype      element type of q, k, v, compressed k/v and out.
+ * MoBA uses B, T, Hq, Hkv, d, sel_block, top_n, softmax_scale and dtype. */
+typedef struct {
+  int B, T, Hq, Hkv, d;
+  int cmp_block, cmp_stride;
+  int sel_block, top_n, window;
+  float softmax_scale;
+  int gate_mode;
+  float fixed_gates[3];
+  nsa_dtype dtype;
+} nsa_params;
+
+/* Bytes of caller-provided device workspace `op` needs for `p` (0 is
+ * possible). The workspace must be 256-byte aligned. */
+NSA_API nsa_status nsa_workspace_size(const nsa_params* p, int op, size_t* bytes);
+
+/* Number of compressed blocks for T tokens: floor((T - l) / s) + 1, or 0 when
+ * T < l. Compressed block i covers tokens [i*s, i*s + l - 1]. */
+NSA_API int nsa_num_cmp_blocks(int T, int cmp_block, int cmp_stride);
+
+/* Token compression (EP94 notes §五 branch one).
+ *   k, v       [B, T, Hkv, d] dtype.
+ *   w_cmp      [cmp_block] fp32 weights shared by keys and values.
+ *   k_cmp, v_cmp  [B, Nc, Hkv, d] dtype outputs, Nc = nsa_num_cmp_blocks(T):
+ *              k_cmp[b,i,g,:] = sum_j w_cmp[j] * k[b, i*s + j, g, :]
+ *              (accumulated in fp64, rounded once to dtype, nearest-even). */
+NSA_API nsa_status nsa_compress_kv(const nsa_params* p, const void* k, const void* v,
+                           const float* w_cmp, void* k_cmp, void* v_cmp, void* stream);
+
+/* NSA causal prefill (EP94 notes §五, §六).
+ *   q          [B, T, Hq, d]; k, v [B, T, Hkv, d]; k_cmp, v_cmp [B, Nc, Hkv, d]
+ *              (from nsa_compress_kv).
+ *   w_gate     [d, 3] fp32 (ignored when gate_mode == 1; may then be NULL).
+ *   out        [B, T, Hq, d] dtype.
+ *   sel_idx    [B, T, Hkv, top_n] int32 or NULL: the selected blocks of each
+ *              (token, KV head), ascending, block 0 first, -1 padded when
+ *              fewer than top_n blocks exist.
+ *   workspace  device scratch of nsa_workspace_size(NSA_OP_PREFILL) bytes. */
+NSA_API nsa_status nsa_prefill(const nsa_params* p, const void* q, const void* k, const void* v,
+                       const void* k_cmp, const void* v_cmp, const float* w_gate, void* out,
+                       int32_t* sel_idx, void* workspace, size_t ws_bytes, void* stream);
+
+/* NSA single-token decode over a KV cache (EP94 notes §六; lchairun.cn NSA
+ * article: decode moves the group's one shared KV subset).
+ *   q          [B, Hq, d]: the query of the token at position seq_lens[b]-1.
+ *   k_cache, v_cache  [B, T, Hkv, d] (T = capacity); positions < seq_lens[b]
+ *              are live and include the current token.
+ *   seq_lens   [B] int32 device array, 1 <= seq_lens[b] <= T (violations set
+ *              the device error word and zero that sequence's output).
+ *   k_cmp, v_cmp  [B, Nc(T), Hkv, d]; entries of blocks ending before
+ *              seq_lens[b] are read.
+ *   w_gate, out [B, Hq, d], sel_idx [B, Hkv, top_n], workspace: as prefill. */
+NSA_API nsa_status nsa_decode(const nsa_params* p, const void* q, const void* k_cache,
+                      const void* v_cache, const int32_t* seq_lens, const void* k_cmp,
+                      const void* v_cmp, const float* w_gate, void* out, int32_t* sel_idx,
+                      void* workspace, size_t ws_bytes, void* stream);
+
+/* MoBA causal prefill (EP94 notes §九/§十).
+ *   q [B, T, Hq, d]; k, v [B, T, Hkv, d]; out [B, T, Hq, d].
+ *   Block m = sel_block; each (token t, head h) keeps its own block t/m and the
+ *   top_n - 1 earlier blocks by q . mean(K_block) (ties to the lower index),
+ *   then one causal softmax over the kept tokens.
+ *   sel_idx    [B, T, Hq, top_n] int32 or NULL (ascending, -1 padded). */
+NSA_API nsa_status moba_prefill(const nsa_params* p, const void* q, const void* k, const void* v,
+                        void* out, int32_t* sel_idx, void* workspace, size_t ws_bytes,
+                        void* stream);
+
+/* Synchronise `stream`, then read and clear this device's error word:
+ * NSA_ERR_DEVICE_TIMEOUT if a bounded wait gave up, NSA_ERR_INVALID_ARGUMENT
+ * if a kernel met an out-of-range sequence length, else NSA_OK (or
+ * NSA_ERR_CUDA if the synchronisation itself failed). */
+NSA_API nsa_status nsa_check(void* stream);
+
+/* Test hook for the failure path: launches one kernel that waits for *flag
+ * (device int) to become nonzero for at most max_iters polls, then sets the
+ * error word and returns. Nothing sets the flag in the test, so nsa_check must
+ * report NSA_ERR_DEVICE_TIMEOUT while the context stays usable. */
+NSA_API nsa_status nsa_debug_bounded_wait(const int32_t* flag, int max_iters, void* stream);
+
+/* Kernel trace (timing aid). While enabled, every kernel this library
+ * launches is bracketed by two CUDA events recorded on its stream; records
+ * accumulate until the next nsa_trace_enable call. Enabling clears the
+ * record; at most `capacity` launches are kept (later ones are counted but
+ * not timed). Events are created at enable time, so the traced region itself
+ * creates none. Not for concurrent use from several host threads. */
+NSA_API nsa_status nsa_trace_enable(int on, int capacity);
+
+/* Number of launches since the trace was enabled (including untimed ones). */
+NSA_API int nsa_trace_count(void);
+
+/* Name and device duration (ms) of traced launch i (synchronises on its stop
+ * event). Returns NSA_ERR_INVALID_ARGUMENT for i out of range. */
+NSA_API nsa_status nsa_trace_get(int i, const char** name, float* ms);
+
+/* Static description of a status code. */
+NSA_API const char* nsa_status_string(nsa_status s);
+
+/* Detail of the last error returned on this host thread ("" if none). */
+NSA_API const char* nsa_last_error_detail(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NSA_B200_H_ */

@@ -1,0 +1,73 @@
+"""Parity rules shared by the GPU tests.
+
+Selection: the GPU's block set must equal the oracle's wherever the oracle's
+last kept and first dropped non-forced candidates differ by more than 1e-5
+relative. Elsewhere the GPU set must still be a valid top set of the oracle's
+scores within that tolerance; those rows are then re-run through the oracle
+with the GPU's selection forced, and outputs are compared on every row.
+
+Outputs: fp32 max |err| <= 1e-4; bf16 max |err| <= 2e-2 and mean |err| <= 2e-3.
+"""
+import numpy as np
+
+SEL_REL = 1e-5
+TOL = {"f32": dict(max=1e-4, mean=1e-4), "bf16": dict(max=2e-2, mean=2e-3)}
+
+
+def _ranked(scores, lo, hi):
+    """Candidate indices lo..hi-1 sorted by (score desc, index asc)."""
+    idx = np.arange(lo, hi)
+    return idx[np.lexsort((idx, -scores[lo:hi]))]
+
+
+def check_selection(gpu_sel, ora_sel, ora_scores, ncand, n_keep, forced_first=True,
+                    forced_block=None):
+    """Compare one row's selection. Returns True if the sets are equal, False if
+    they differ but the difference is allowed (a near tie); raises otherwise.
+
+    ncand: candidate blocks are 0..ncand-1 (NSA) -- for MoBA pass the number of
+    earlier blocks and forced_block = own block.
+    """
+    g = sorted(int(x) for x in gpu_sel if x >= 0)
+    o = sorted(int(x) for x in ora_sel if x >= 0)
+    if g == o:
+        return True
+    lo = 1 if forced_first else 0
+    want = n_keep - 1  # non-forced picks
+    if forced_first and ncand <= n_keep:
+        raise AssertionError(f"selection differs with no choice to make: gpu {g} oracle {o}")
+    ranked = _ranked(ora_scores, lo, ncand)
+    if len(ranked) <= want:
+        raise AssertionError(f"selection differs with no choice to make: gpu {g} oracle {o}")
+    s_last = ora_scores[ranked[want - 1]]
+    s_next = ora_scores[ranked[want]]
+    gap = abs(s_last - s_next)
+    if gap > SEL_REL * abs(s_last):
+        raise AssertionError(
+            f"selection differs beyond the tie tolerance: gpu {g} oracle {o} "
+            f"(gap {gap:.3e}, last kept {s_last:.9e})")
+    forced = 0 if forced_first else forced_block
+    free = [j for j in g if j != forced]
+    if forced is not None:
+        assert forced in g, f"forced block {forced} missing from gpu selection {g}"
+    assert len(free) == want, f"gpu kept {len(free)} blocks, expected {want}"
+    tol = SEL_REL * abs(s_last)
+    for j in free:
+        assert ora_scores[j] >= s_last - tol, f"gpu kept block {j} well below the cut"
+    dropped = [j for j in ranked if j not in free]
+    for j in dropped:
+        assert ora_scores[j] <= s_last + tol, f"gpu dropped block {j} well above the cut"
+    return False
+
+
+def check_output(gpu, ref, dtype, what="out"):
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert gpu.shape == ref.shape, (gpu.shape, ref.shape)
+    assert np.all(np.isfinite(gpu)), f"{what}: non-finite GPU values"
+    err = np.abs(gpu - ref)
+    mx, mean = float(err.max(initial=0.0)), float(err.mean()) if err.size else 0.0
+    tol = TOL[dtype]
+    assert mx <= tol["max"], f"{what}: max |err| {mx:.3e} > {tol['max']}"
+    assert mean <= tol["mean"], f"{what}: mean |err| {mean:.3e} > {tol['mean']}"
+    return mx, mean

@@ -1,0 +1,88 @@
+"""Host-only checks of the C ABI (no GPU needed, no kernel launched).
+
+* the library loads and exports every function include/nsa.h declares;
+* argument validation happens on the host before any CUDA call.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+from tests.conftest import ROOT
+
+nsa = pytest.importorskip("dynamic_block_sparse_nsa_b200.nsa")
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "nsa.h")).read()
+    return sorted(set(re.findall(r"NSA_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_functions() == sorted(nsa.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(nsa.LIB_PATH)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings():
+    for code, name in nsa.STATUS.items():
+        assert nsa.LIB.nsa_status_string(code).decode() == name
+
+
+def test_num_cmp_blocks():
+    assert nsa.num_cmp_blocks(65536, 32, 16) == 4095
+    assert nsa.num_cmp_blocks(8192, 32, 16) == 511
+    assert nsa.num_cmp_blocks(31, 32, 16) == 0
+
+
+def _status(fn, *args):
+    return fn(*args)
+
+
+def test_workspace_size_validation():
+    n = ctypes.c_size_t(7)
+    assert nsa.LIB.nsa_workspace_size(None, 0, ctypes.byref(n)) == 1
+    p = nsa.params(1, 1024, 4, 1, 64)
+    assert nsa.LIB.nsa_workspace_size(ctypes.byref(p), 99, ctypes.byref(n)) == 1
+    bad = nsa.params(1, 1024, 4, 1, 96)
+    assert nsa.LIB.nsa_workspace_size(ctypes.byref(bad), nsa.OP_PREFILL, ctypes.byref(n)) == 2
+    assert b"head dim" in nsa.LIB.nsa_last_error_detail()
+    bad = nsa.params(1, 1024, 6, 4, 64)
+    assert nsa.LIB.nsa_workspace_size(ctypes.byref(bad), nsa.OP_PREFILL, ctypes.byref(n)) == 1
+    bad = nsa.params(1, 1024, 4, 1, 64, cmp_block=8, cmp_stride=16)
+    assert nsa.LIB.nsa_workspace_size(ctypes.byref(bad), nsa.OP_PREFILL, ctypes.byref(n)) == 1
+    moba = nsa.params(2, 131072, 32, 32, 128, sel_block=512, top_n=3)
+    assert nsa.workspace_size(moba, nsa.OP_MOBA_PREFILL) == 2 * 256 * 32 * 128 * 4
+
+
+def test_calls_reject_null_pointers_before_launching():
+    p = nsa.params(1, 1024, 4, 1, 64)
+    L = nsa.LIB
+    assert L.nsa_compress_kv(ctypes.byref(p), None, None, None, None, None, None) == 1
+    assert L.nsa_prefill(ctypes.byref(p), None, None, None, None, None, None, None, None, None,
+                         0, None) == 1
+    assert L.nsa_decode(ctypes.byref(p), None, None, None, None, None, None, None, None, None,
+                        None, 0, None) == 1
+    assert L.moba_prefill(ctypes.byref(p), None, None, None, None, None, None, 0, None) == 1
+    assert L.nsa_debug_bounded_wait(None, 10, None) == 1
+    # gate weights are required for learned gates only
+    fake = ctypes.c_void_p(256)
+    assert L.nsa_prefill(ctypes.byref(p), fake, fake, fake, fake, fake, None, fake, None, None,
+                         0, None) == 1
+    assert b"w_gate" in L.nsa_last_error_detail()
+
+
+def test_moba_rejects_small_workspace_before_launching():
+    p = nsa.params(1, 4096, 4, 4, 128, sel_block=512, top_n=3)
+    fake = ctypes.c_void_p(256)
+    need = nsa.workspace_size(p, nsa.OP_MOBA_PREFILL)
+    st = nsa.LIB.moba_prefill(ctypes.byref(p), fake, fake, fake, fake, None, fake, need - 1, None)
+    assert st == 3
+    st = nsa.LIB.moba_prefill(ctypes.byref(p), fake, fake, fake, fake, None, ctypes.c_void_p(264),
+                              need, None)
+    assert st == 1  # misaligned workspace
