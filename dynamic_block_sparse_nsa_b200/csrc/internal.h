@@ -2,6 +2,7 @@
 // Every launcher enqueues on `stream` and returns the launch status.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cstddef>
 #include <cstdint>
@@ -51,6 +52,38 @@ struct MobaArgs {
   nsa_dtype dtype;
 };
 
+// Arguments of the bf16 / d=128 / 16-heads-per-group decode kernels.
+struct DecFastArgs {
+  const void* q;
+  const int32_t* seq_lens;
+  const float* w_gate;
+  void* out;
+  int32_t* sel_out;
+  unsigned* err;
+  int B, T, Hq, Hkv, Nc, l, s, bs, n, w;
+  int nbt;        // selection blocks one 64-key compressed tile can overlap (bound)
+  int tiles_max;  // 64-key compressed tiles per sequence at capacity T
+  int items_max;  // 128-key items of the selected + window branches per unit
+  int grid1;      // CTAs of the compressed-branch kernel
+  float scale_log2;
+  int gate_mode;
+  float fixed_gates[3];
+  float* part1;   // compressed-branch partials, slot = cta + unit
+  float* trec;    // per-tile block-score records
+  float* oacc;    // g0 * o_cmp per unit
+  float* gates;   // per unit [16][3]
+  int* sel;       // per unit [n]
+  float* part3;   // selected / window partials per (unit, item)
+  unsigned* cnt3; // finished items per unit
+};
+
+bool decode_fast_eligible(const nsa_params& p);
+size_t decode_fast_ws_bytes(const nsa_params& p);
+cudaError_t launch_decode_fast(const nsa_params& p, const void* q, const void* k, const void* v,
+                               const int32_t* seq_lens, const void* kc, const void* vc,
+                               const float* w_gate, void* out, int32_t* sel_out, void* ws,
+                               unsigned* err, cudaStream_t stream);
+
 // Kernel trace: bracket a launch with events when tracing is on.
 void trace_begin(const char* name, cudaStream_t stream);
 void trace_end(cudaStream_t stream);
@@ -60,6 +93,11 @@ struct TraceScope {
   TraceScope(const char* name, cudaStream_t st) : s(st) { trace_begin(name, st); }
   ~TraceScope() { trace_end(s); }
 };
+
+// 3-D TMA map over a contiguous bf16 array [dim2][dim1][dim0] with a box of
+// (box0, box1, box2) elements; false if the driver rejects it.
+bool make_tmap_bf16_3d(CUtensorMap* m, const void* base, uint64_t dim0, uint64_t dim1,
+                       uint64_t dim2, uint32_t box0, uint32_t box1, uint32_t box2, bool swizzle128);
 
 cudaError_t launch_compress(const nsa_params& p, const void* k, const void* v, const float* w,
                             void* kc, void* vc, cudaStream_t stream);

@@ -150,11 +150,16 @@ nsa_status nsa_workspace_size(const nsa_params* p, int op, size_t* bytes) {
   *bytes = 0;
   switch (op) {
     case NSA_OP_COMPRESS:
-    case NSA_OP_PREFILL:
-    case NSA_OP_DECODE: {
+    case NSA_OP_PREFILL: {
       nsa_status s = check_nsa(p);
       if (s != NSA_OK) return s;
       *bytes = 0;
+      return NSA_OK;
+    }
+    case NSA_OP_DECODE: {
+      nsa_status s = check_nsa(p);
+      if (s != NSA_OK) return s;
+      *bytes = decode_fast_ws_bytes(*p);
       return NSA_OK;
     }
     case NSA_OP_MOBA_PREFILL: {
@@ -174,6 +179,7 @@ nsa_status nsa_compress_kv(const nsa_params* p, const void* k, const void* v, co
   g_detail.clear();
   nsa_status s = check_nsa(p);
   if (s != NSA_OK) return s;
+  if (nsa_num_cmp_blocks(p->T, p->cmp_block, p->cmp_stride) == 0) return NSA_OK;  // nothing to write
   if (!k || !v || !w_cmp || !k_cmp || !v_cmp)
     return fail(NSA_ERR_INVALID_ARGUMENT, "k, v, w_cmp, k_cmp, v_cmp must be non-NULL");
   cudaError_t e = launch_compress(*p, k, v, w_cmp, k_cmp, v_cmp, (cudaStream_t)stream);
@@ -219,10 +225,15 @@ nsa_status nsa_decode(const nsa_params* p, const void* q, const void* k_cache, c
                 "q, k_cache, v_cache, seq_lens, k_cmp, v_cmp, out must be non-NULL");
   if (p->gate_mode == 0 && !w_gate)
     return fail(NSA_ERR_INVALID_ARGUMENT, "w_gate must be non-NULL when gate_mode == 0");
-  (void)workspace;
-  (void)ws_bytes;
   unsigned* err = err_word(&s);
   if (!err) return s;
+  if (decode_fast_eligible(*p)) {
+    s = check_workspace(workspace, ws_bytes, decode_fast_ws_bytes(*p));
+    if (s != NSA_OK) return s;
+    cudaError_t e = launch_decode_fast(*p, q, k_cache, v_cache, seq_lens, k_cmp, v_cmp, w_gate,
+                                       out, sel_idx, workspace, err, (cudaStream_t)stream);
+    return e == cudaSuccess ? NSA_OK : cuda_fail(e, "decode launch");
+  }
   NsaRowArgs a = row_args(p);
   a.q = q; a.k = k_cache; a.v = v_cache; a.kc = k_cmp; a.vc = v_cmp;
   a.w_gate = w_gate; a.out = out; a.sel_idx = sel_idx; a.seq_lens = seq_lens; a.err = err;

@@ -183,8 +183,8 @@ __device__ inline void add_branch(const Ctx& c, int which, bool normalise) {
 
 // Top selection over scores[lo, ncand): keeps `forced` (>= 0) plus the best
 // `want` others by (score desc, index asc); writes sel[0..) ascending and
-// returns the count. Taken entries of scores are overwritten with -1 (valid
-// scores are >= 0 for NSA; MoBA scores are shifted by the caller).
+// returns the count. Taken entries of scores are overwritten with -inf and
+// -inf entries are never picked.
 __device__ inline int select_top(const Ctx& c, int lo, int ncand, int forced, int want) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int ns = 0;

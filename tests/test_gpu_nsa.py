@@ -76,3 +76,29 @@ def test_decode_f32_ragged():
 def test_decode_bf16_full_size_sampled_sequences():
     w = inputs.workload("nsa_decode_bf16_b32_l65536")
     gc.run_nsa_decode(w, None, check_b=[0, 13, 31])
+
+
+def test_decode_bf16_many_units_ragged():
+    # many (sequence, KV head) units per CTA and units split across CTAs
+    w = inputs.workload("nsa_decode_bf16_b32_l65536", B=16, T=20000)
+    lens = inputs.ragged_lens(16, 20000, seed=5, lo=1)
+    gc.run_nsa_decode(w, lens, check_b=[0, 3, 7, 11, 15])
+
+
+def test_decode_bf16_group_of_8_generic_path():
+    w = inputs.workload("nsa_decode_bf16_b32_l65536", B=3, T=4000, Hq=32, Hkv=4)
+    gc.run_nsa_decode(w, [4000, 1234, 64])
+
+
+def test_decode_repeat_is_deterministic(cuda_ok):
+    from dynamic_block_sparse_nsa_b200 import nsa
+    w = inputs.workload("nsa_decode_bf16_b32_l65536", B=4, T=9000)
+    inp = inputs.make_decode(w, seq_lens=[9000, 5000, 777, 8999])
+    p = gc.nsa_params_for(w)
+    dev = {k_: v_.cuda() for k_, v_ in inp.items()}
+    kc, vc = nsa.nsa_compress_kv(p, dev["k"], dev["v"], dev["w_cmp"])
+    outs = [nsa.nsa_decode(p, dev["q"], dev["k"], dev["v"], dev["seq_lens"], kc, vc,
+                           dev["w_gate"]) for _ in range(3)]
+    nsa.nsa_check()
+    for o, s in outs[1:]:
+        assert torch.equal(o, outs[0][0]) and torch.equal(s, outs[0][1])
