@@ -577,7 +577,8 @@ def run_reference(args, w):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 * secs / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, **config_of(w)},
+        "config": {"workload": args.workload, **config_of(w),
+                   **({"overrides": args.set} if args.set else {})},
         "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle",
                          "sample": f"each step: {desc}"},
         "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -603,9 +604,17 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(inputs.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--set", action="append", default=[], metavar="KEY=VALUE",
+                    help="override a workload field (smaller cases for profiling)")
     args = ap.parse_args()
     w = inputs.workload(args.workload)
+    for kv in args.set:
+        key, val = kv.split("=", 1)
+        w[key] = type(w[key])(val) if key in w else int(val)
     kind = w["kind"]
+    if args.set and args.impl == "ours":
+        args.no_cpu_baseline = True
     if args.steps is None:
         args.steps = {"decode": 2000, "prefill": 20, "moba": 10}[kind]
     if args.warmup is None:
@@ -621,7 +630,7 @@ def main():
     ws, rank, local = dist_setup()
     import dynamic_block_sparse_nsa_b200.nsa  # noqa: F401  (fails loudly if unbuilt)
     runner = {"decode": run_decode, "prefill": run_prefill, "moba": run_moba}[kind]
-    res = runner(w, args.steps, args.warmup, ws, rank, local)
+    res = runner(w, args.steps, args.warmup, ws, rank, local, e2e=not args.no_e2e)
 
     K = args.steps
     ms_max = reduce_max(res["ms"], ws)
@@ -668,6 +677,7 @@ def main():
             "warmup": args.warmup, "ms_per_step": ms_max / K, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": w["dtype"], "data": "synthetic",
             "config": {"workload": args.workload, **config_of(w),
+                       **({"overrides": args.set} if args.set else {}),
                        "l2": "inputs larger than L2 every step "
                              f"({res['work'] / 1e6:.0f} MB read per step)" if kind == "decode"
                        else "inputs larger than L2 every step"},

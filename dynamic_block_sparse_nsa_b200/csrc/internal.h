@@ -53,6 +53,7 @@ struct MobaArgs {
 };
 
 // Arguments of the bf16 / d=128 / 16-heads-per-group decode kernels.
+constexpr int kDecMaxNbt = 48;
 struct DecFastArgs {
   const void* q;
   const int32_t* seq_lens;
@@ -63,18 +64,18 @@ struct DecFastArgs {
   int B, T, Hq, Hkv, Nc, l, s, bs, n, w;
   int nbt;        // selection blocks one 64-key compressed tile can overlap (bound)
   int tiles_max;  // 64-key compressed tiles per sequence at capacity T
-  int items_max;  // 128-key items of the selected + window branches per unit
-  int grid1;      // CTAs of the compressed-branch kernel
+  int grid1;      // CTAs of the compressed-branch stream kernel
+  int grid3;      // CTAs of the selected/window stream kernel
   float scale_log2;
   int gate_mode;
   float fixed_gates[3];
+  int8_t klo[kDecMaxNbt], khi[kDecMaxNbt];  // per block of a tile: its key range
   float* part1;   // compressed-branch partials, slot = cta + unit
   float* trec;    // per-tile block-score records
   float* oacc;    // g0 * o_cmp per unit
   float* gates;   // per unit [16][3]
   int* sel;       // per unit [n]
-  float* part3;   // selected / window partials per (unit, item)
-  unsigned* cnt3; // finished items per unit
+  float* part3;   // selected / window partials, slot = cta + 2 * unit + branch
 };
 
 bool decode_fast_eligible(const nsa_params& p);
