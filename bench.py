@@ -271,30 +271,68 @@ def reduce_sum(x, ws):
 # the timed loops
 # --------------------------------------------------------------------------
 
-def timed(step, K, W, ws, device_index, trace=True):
+def _run_steps(step, K, graph, trace_only=None, trace_all=False, sampler=None):
+    """Run K steps (optionally as one CUDA graph) between CUDA events on the
+    launching stream; returns (ms, trace records, launches, clock summary)."""
     from dynamic_block_sparse_nsa_b200 import nsa
+    tracing = trace_all or trace_only is not None
+    g = None
+    if graph:
+        if tracing:
+            nsa.trace_enable(True, capacity=K * 8 + 64, only=trace_only)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(K):
+                step()
+        g.replay()  # untimed: uploads the graph
+        torch.cuda.synchronize()
+    s = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if tracing and not graph:
+        nsa.trace_enable(True, capacity=K * 8 + 64, only=trace_only)
+    clk = ClockSampler(sampler) if sampler is not None else None
+    if clk:
+        clk.__enter__()
+    e0.record(s)
+    if graph:
+        g.replay()
+    else:
+        for _ in range(K):
+            step()
+    e1.record(s)
+    torch.cuda.synchronize()
+    if clk:
+        clk.__exit__()
+    ms = e0.elapsed_time(e1)
+    recs, launches = [], 0
+    if tracing:
+        recs, launches = nsa.trace_records()
+        nsa.trace_enable(False)  # (graph: launches counted at capture = one replay)
+    del g
+    return ms, recs, launches, (clk.summary() if clk else None)
+
+
+def timed(step, K, W, ws, device_index, graph=False):
+    """W warm-up steps; a short traced pass names the dominant kernel; then two
+    timed regions of exactly K steps, each between a barrier and a device
+    synchronise: (A) uninstrumented -- the step time and clocks; (B) events
+    around every launch of the dominant kernel only -- its mean duration.
+    Event-record nodes between kernels delay the next launch, hence (A)."""
     for _ in range(W):
         step()
     torch.cuda.synchronize()
+    _, recs0, _, _ = _run_steps(step, min(K, 50), graph, trace_all=True)
+    table0 = kernel_table(recs0, min(K, 50))
+    dom = max(table0, key=lambda n: table0[n]["total_ms"]) if table0 else None
     barrier(ws)
     torch.cuda.synchronize()
-    if trace:
-        nsa.trace_enable(True, capacity=K * 16 + 64)
-    s = torch.cuda.current_stream()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with ClockSampler(device_index) as clk:
-        e0.record(s)
-        for _ in range(K):
-            step()
-        e1.record(s)
-        torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1)
-    recs, launches = ([], 0)
-    if trace:
-        recs, launches = nsa.trace_records()
-        nsa.trace_enable(False)
+    ms, _, _, clk = _run_steps(step, K, graph, sampler=device_index)
     barrier(ws)
-    return ms, recs, launches, clk.summary()
+    torch.cuda.synchronize()
+    msb, recs, launches, _ = _run_steps(step, K, graph, trace_only=dom or "")
+    barrier(ws)
+    return dict(ms=ms, ms_traced=msb, recs=recs, launches=launches, clk=clk, table0=table0,
+                dom=dom)
 
 
 def kernel_table(recs, K):
@@ -310,7 +348,7 @@ def kernel_table(recs, K):
     return tab
 
 
-def run_decode(w, K, W, ws, rank, local, e2e=True):
+def run_decode(w, K, W, ws, rank, local, e2e=True, use_graph=True):
     from dynamic_block_sparse_nsa_b200 import nsa
     inp = inputs.make_decode(w, seed=w["seed"] + rank, device="cuda")
     p = nsa.params(w["B"], w["T"], w["Hq"], w["Hkv"], w["d"], cmp_block=w["cmp_block"],
@@ -328,13 +366,12 @@ def run_decode(w, K, W, ws, rank, local, e2e=True):
 
     step()
     nsa.nsa_check()
-    ms, recs, launches, clk = timed(step, K, W, ws, local)
+    res = timed(step, K, W, ws, local, graph=use_graph)
     nsa.nsa_check()
     sel_h = sel.cpu().numpy()
     lens_l = lens.cpu().tolist()
     step_bytes, union_bytes, parts = decode_work(w, lens_l, sel_h)
-    res = dict(ms=ms, recs=recs, launches=launches, clk=clk, work=step_bytes,
-               union=union_bytes, parts=parts)
+    res.update(work=step_bytes, union=union_bytes, parts=parts)
     if e2e:
         # through the public call with host buffers: H2D of the step's query and
         # lengths, D2H of the output and selection; the KV caches are device-
@@ -351,8 +388,12 @@ def run_decode(w, K, W, ws, rank, local, e2e=True):
             out_h.copy_(out, non_blocking=True)
             sel_h_p.copy_(sel, non_blocking=True)
 
-        ems, _, _, _ = timed(e2e_step, K, max(3, W // 2), ws, local, trace=False)
-        res["e2e_ms"] = ems
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(ws)
+        res["e2e_ms"] = _run_steps(e2e_step, K, False)[0]
+        barrier(ws)
         res["h2d"] = q_h.numel() * q_h.element_size() + lens_h.numel() * 4
         res["d2h"] = out_h.numel() * out_h.element_size() + sel_h_p.numel() * 4
     return res
@@ -379,10 +420,10 @@ def run_prefill(w, K, W, ws, rank, local, e2e=True):
 
     step()
     nsa.nsa_check()
-    ms, recs, launches, clk = timed(step, K, W, ws, local)
+    res = timed(step, K, W, ws, local)
     nsa.nsa_check()
     fl = prefill_flops(w, sel.cpu().numpy())
-    res = dict(ms=ms, recs=recs, launches=launches, clk=clk, work=sum(fl.values()), parts=fl)
+    res.update(work=sum(fl.values()), parts=fl)
     if e2e:
         hq = inp["q"].cpu().pin_memory()
         hk = inp["k"].cpu().pin_memory()
@@ -396,8 +437,12 @@ def run_prefill(w, K, W, ws, rank, local, e2e=True):
             step()
             ho.copy_(out, non_blocking=True)
 
-        ems, _, _, _ = timed(e2e_step, K, max(3, W // 2), ws, local, trace=False)
-        res["e2e_ms"] = ems
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(ws)
+        res["e2e_ms"] = _run_steps(e2e_step, K, False)[0]
+        barrier(ws)
         res["h2d"] = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
         res["d2h"] = ho.numel() * ho.element_size()
     return res
@@ -417,10 +462,10 @@ def run_moba(w, K, W, ws, rank, local, e2e=True):
 
     step()
     nsa.nsa_check()
-    ms, recs, launches, clk = timed(step, K, W, ws, local)
+    res = timed(step, K, W, ws, local)
     nsa.nsa_check()
     fl = moba_flops(w, sel.cpu().numpy())
-    res = dict(ms=ms, recs=recs, launches=launches, clk=clk, work=sum(fl.values()), parts=fl)
+    res.update(work=sum(fl.values()), parts=fl)
     if e2e:
         hq, hk, hv = (inp[x].cpu().pin_memory() for x in ("q", "k", "v"))
         ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
@@ -432,8 +477,12 @@ def run_moba(w, K, W, ws, rank, local, e2e=True):
             step()
             ho.copy_(out, non_blocking=True)
 
-        ems, _, _, _ = timed(e2e_step, K, max(3, W // 2), ws, local, trace=False)
-        res["e2e_ms"] = ems
+        for _ in range(3):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(ws)
+        res["e2e_ms"] = _run_steps(e2e_step, K, False)[0]
+        barrier(ws)
         res["h2d"] = sum(t.numel() * t.element_size() for t in (hq, hk, hv))
         res["d2h"] = ho.numel() * ho.element_size()
     return res
@@ -605,6 +654,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time decode steps as separate launches instead of one CUDA graph")
     ap.add_argument("--set", action="append", default=[], metavar="KEY=VALUE",
                     help="override a workload field (smaller cases for profiling)")
     args = ap.parse_args()
@@ -630,7 +681,8 @@ def main():
     ws, rank, local = dist_setup()
     import dynamic_block_sparse_nsa_b200.nsa  # noqa: F401  (fails loudly if unbuilt)
     runner = {"decode": run_decode, "prefill": run_prefill, "moba": run_moba}[kind]
-    res = runner(w, args.steps, args.warmup, ws, rank, local, e2e=not args.no_e2e)
+    kw = {"use_graph": not args.no_graph} if kind == "decode" else {}
+    res = runner(w, args.steps, args.warmup, ws, rank, local, e2e=not args.no_e2e, **kw)
 
     K = args.steps
     ms_max = reduce_max(res["ms"], ws)
@@ -647,13 +699,13 @@ def main():
     tab = kernel_table(res["recs"], K)
     peaks = load_peaks()
     roof = None
-    if tab:
-        dom = max(tab, key=lambda n: tab[n]["total_ms"])
+    dom = res["dom"]
+    if dom and dom in tab:
         wk, bound = kernel_work(kind, dom, res, w)
         mean_s = tab[dom]["total_ms"] / tab[dom]["launches"] / 1000.0
+        mean_s = reduce_max(mean_s, ws)
         if wk is not None:
-            launches_per_step = tab[dom]["launches"] / K
-            per_launch = wk / launches_per_step
+            per_launch = wk / (tab[dom]["launches"] / K)
             if bound == "hbm":
                 ach = per_launch / mean_s / 1e9
                 pk, u = peaks["hbm"], "GB/s"
@@ -663,7 +715,10 @@ def main():
             roof = {"kernel": dom, "bound": bound, "achieved": ach, "peak": pk, "unit": u,
                     "frac": ach / pk, "peak_source": peaks["src"],
                     "traffic": kernel_traffic(dom, args.workload),
-                    "algorithmic_per_launch": per_launch}
+                    "algorithmic_per_launch": per_launch,
+                    "mean_launch_us": mean_s * 1e6,
+                    "timing": "events around each launch of this kernel over a second "
+                              "timed region of the same K steps"}
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -685,9 +740,11 @@ def main():
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": res["launches"],
+            "timing": "cuda_graph" if (kind == "decode" and not args.no_graph) else "stream",
             "clocks": res["clk"],
-            "kernels": {n: {k: (round(v, 4) if isinstance(v, float) else v)
-                            for k, v in e.items()} for n, e in tab.items()},
+            "kernels_event_bracketed": {
+                n: {k: (round(v, 4) if isinstance(v, float) else v) for k, v in e.items()}
+                for n, e in res["table0"].items()},
         }
         if kind == "decode":
             line["decode_bytes"] = {"per_step": res["work"], "union_per_step": res["union"],

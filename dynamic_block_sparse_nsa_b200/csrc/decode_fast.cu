@@ -17,14 +17,15 @@
 //  dec_sel_win      stream kernel over the selected blocks, then the window.
 //  dec_combine      one CTA per unit: out = g0 o_cmp + g1 o_slc + g2 o_win.
 //
-// Stream kernel: persistent, one CTA per SM, 1 TMA producer warp + 4 consumer
-// warps. The global sequence of 64-key tiles (sequence-major, then KV head,
-// then tile) is split evenly over the CTAs. K and V halves of each tile go
-// through a ring of 16 KB slots (128B-swizzled TMA boxes, L2 evict-first),
-// each slot released as soon as it has been read. Consumer warps take tiles
-// round-robin and keep online-softmax partials (m, l, O); at every segment
-// boundary (unit, or unit and branch) the four warps merge their partials and
-// write one per (CTA, segment), slot = cta + segment.
+// Stream kernel: persistent, one CTA per SM, 1 TMA producer warp + 3 pairs of
+// consumer warps (7 warps: at most two per SM sub-partition, whose register
+// file then holds up to 255 registers a thread). The global sequence of 64-key
+// tiles (sequence-major, then KV head, then tile) is split evenly over the
+// SMs x 3 pair streams; each pair has a private ring of four 16 KB slots (K or
+// V of a tile, 128B-swizzled TMA boxes, L2 evict-first) so no stream waits on
+// another's slot. The two warps of a pair take 32 keys each of every tile and
+// keep online-softmax partials (m, l, O), written once per segment they touch
+// (segment = unit, or unit and branch).
 // Softmax runs in the log2 domain: z2 = (q . k) * scale * log2(e).
 #include <algorithm>
 #include <climits>
@@ -39,13 +40,9 @@ namespace {
 constexpr int G = 16;                       // query heads per KV head
 constexpr int D = 128;                      // head dim
 constexpr int TK = 64;                      // keys per tile
-constexpr int NCW = 4;                      // consumer warps
-constexpr int SLOTS = 12;                   // ring of half-tiles (K or V)
 constexpr int HALF_BYTES = TK * 64 * 2;     // 64 rows x 64 dims of bf16 (one TMA box)
 constexpr int SLOT_BYTES = 2 * HALF_BYTES;  // 64 keys x 128 dims
 constexpr int PART = 2 * G + G * D;         // m[16], l[16], o[16][128]
-constexpr int MERGE_FLOATS = NCW * PART;
-constexpr int SCR_PITCH = TK + 2;  // even: float2 stores stay aligned
 constexpr uint64_t kWaitNs = 2000000000ull;
 
 enum { MODE_CMP = 0, MODE_SW = 1 };
@@ -72,50 +69,74 @@ __device__ __forceinline__ int unit_tiles(int L, const DecFastArgs& a) {
 }
 
 // ---------------------------------------------------------------------------
-// consumer math (one warp: 16 heads x 64 keys)
+// consumer math (one warp: 16 heads x 32 keys of a 64-key tile)
 // ---------------------------------------------------------------------------
 
-__device__ __forceinline__ void load_q_frags(uint32_t (&qa)[8][4], const __nv_bfloat16* q,
-                                             int lane) {
-  const uint32_t* qw = reinterpret_cast<const uint32_t*>(q);
-  const int r0 = lane >> 2, c = (lane & 3) * 2;
-#pragma unroll
-  for (int ks = 0; ks < 8; ++ks) {
-    qa[ks][0] = __ldg(qw + (r0 * D + ks * 16 + c) / 2);
-    qa[ks][1] = __ldg(qw + ((r0 + 8) * D + ks * 16 + c) / 2);
-    qa[ks][2] = __ldg(qw + (r0 * D + ks * 16 + 8 + c) / 2);
-    qa[ks][3] = __ldg(qw + ((r0 + 8) * D + ks * 16 + 8 + c) / 2);
-  }
-}
+constexpr int WK = 32;  // keys per consumer warp per tile (two warps share a tile)
 
-// S[16 x 64] = Q K^T over a swizzled 64-key tile.
-__device__ __forceinline__ void qk_tile(float (&s)[8][4], const uint32_t (&qa)[8][4],
-                                        uint32_t kbase, int lane) {
+// S[16 x 8*NT] = Q K^T with the query block in shared memory (row r's 16-byte
+// chunk c stored at chunk c ^ (r & 7)); even and odd k-steps accumulate in
+// separate registers so consecutive tensor-core ops do not wait on each other.
+template <int NT>
+__device__ __forceinline__ void qk_tile_q(float (&s)[NT][4], uint32_t qbase, uint32_t kbase,
+                                          int key0, int lane) {
+  float t[NT][4];
 #pragma unroll
-  for (int nt = 0; nt < 8; ++nt) s[nt][0] = s[nt][1] = s[nt][2] = s[nt][3] = 0.f;
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) s[nt][i] = t[nt][i] = 0.f;
   const int mi = lane >> 3, r = lane & 7;
 #pragma unroll
   for (int ks = 0; ks < 8; ++ks) {
+    uint32_t qa[4];
+    {
+      const int row = (mi & 1) * 8 + r;
+      const int chunk = 2 * ks + (mi >> 1);
+      ptx::ldsm_x4(qbase + row * 256 + ((chunk ^ (row & 7)) << 4), qa[0], qa[1], qa[2], qa[3]);
+    }
 #pragma unroll
-    for (int np = 0; np < 4; ++np) {
-      const int key = (2 * np + (mi >> 1)) * 8 + r;
+    for (int np = 0; np < NT / 2; ++np) {
+      const int key = key0 + (2 * np + (mi >> 1)) * 8 + r;
       const int chunk = 2 * ks + (mi & 1);
       const uint32_t addr =
           kbase + (chunk >> 3) * HALF_BYTES + key * 128 + (((chunk & 7) ^ (key & 7)) << 4);
       uint32_t b0, b1, b2, b3;
       ptx::ldsm_x4(addr, b0, b1, b2, b3);
-      ptx::mma_16816(s[2 * np], qa[ks], b0, b1);
-      ptx::mma_16816(s[2 * np + 1], qa[ks], b2, b3);
+      if (ks & 1) {
+        ptx::mma_16816(t[2 * np], qa, b0, b1);
+        ptx::mma_16816(t[2 * np + 1], qa, b2, b3);
+      } else {
+        ptx::mma_16816(s[2 * np], qa, b0, b1);
+        ptx::mma_16816(s[2 * np + 1], qa, b2, b3);
+      }
     }
+  }
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) s[nt][i] += t[nt][i];
+}
+
+// The 16 x 128 query block of a unit into shared memory (swizzled as above);
+// the two warps of a pair copy 8 rows each.
+__device__ __forceinline__ void stage_q_half(unsigned char* qs, const __nv_bfloat16* q, int hw,
+                                             int lane) {
+  const uint4* src = reinterpret_cast<const uint4*>(q);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int x = hw * 128 + i * 32 + lane;  // 16-byte chunk: row x / 16, chunk x % 16
+    const int r = x >> 4, c = x & 15;
+    *reinterpret_cast<uint4*>(qs + r * 256 + ((c ^ (r & 7)) << 4)) = __ldg(src + x);
   }
 }
 
-// O[16 x 128] += P[16 x 64] V over a swizzled 64-key tile.
-__device__ __forceinline__ void pv_tile(float (&o)[16][4], const float (&p)[8][4], uint32_t vbase,
-                                        int lane) {
+// O[16 x 128] += P[16 x 16*KS] V for keys [key0, key0 + 16*KS) of a swizzled tile.
+template <int KS>
+__device__ __forceinline__ void pv_tile(float (&o)[16][4], const float (&p)[2 * KS][4],
+                                        uint32_t vbase, int key0, int lane) {
   const int mi = lane >> 3, r = lane & 7;
 #pragma unroll
-  for (int kk = 0; kk < 4; ++kk) {
+  for (int kk = 0; kk < KS; ++kk) {
     uint32_t a[4];
     a[0] = ptx::pack_bf16(p[2 * kk][0], p[2 * kk][1]);
     a[1] = ptx::pack_bf16(p[2 * kk][2], p[2 * kk][3]);
@@ -123,7 +144,7 @@ __device__ __forceinline__ void pv_tile(float (&o)[16][4], const float (&p)[8][4
     a[3] = ptx::pack_bf16(p[2 * kk + 1][2], p[2 * kk + 1][3]);
 #pragma unroll
     for (int dp = 0; dp < 8; ++dp) {
-      const int key = kk * 16 + (mi & 1) * 8 + r;
+      const int key = key0 + kk * 16 + (mi & 1) * 8 + r;
       const int chunk = 2 * dp + (mi >> 1);
       const uint32_t addr =
           vbase + (chunk >> 3) * HALF_BYTES + key * 128 + (((chunk & 7) ^ (key & 7)) << 4);
@@ -145,16 +166,17 @@ __device__ __forceinline__ float quad_sum(float x) {
   return x + __shfl_xor_sync(0xffffffffu, x, 2);
 }
 
-// Online-softmax step over one 64-key tile: mask keys >= nvalid, scale to the
-// log2 domain, update running max/sum of rows r0 = lane/4 and r1 = r0 + 8,
-// rescale O, and turn s into p = exp2(z - m_new).
-__device__ __forceinline__ void softmax_step(float (&s)[8][4], float (&o)[16][4], float& m0,
+// Online-softmax step over NT n-tiles (8 keys each): mask keys >= nvalid,
+// scale to the log2 domain, update running max/sum of rows r0 = lane/4 and
+// r1 = r0 + 8, rescale O, and turn s into p = exp2(z - m_new).
+template <int NT>
+__device__ __forceinline__ void softmax_step(float (&s)[NT][4], float (&o)[16][4], float& m0,
                                              float& m1, float& l0, float& l1, int nvalid,
                                              float scale_log2, int lane) {
   const int c = (lane & 3) * 2;
   float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-  for (int nt = 0; nt < 8; ++nt)
+  for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       const bool ok = nt * 8 + c + e < nvalid;
@@ -170,7 +192,7 @@ __device__ __forceinline__ void softmax_step(float (&s)[8][4], float (&o)[16][4]
   const float c1 = mn1 == -INFINITY ? 1.f : exp2f(m1 - mn1);
   float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
-  for (int nt = 0; nt < 8; ++nt)
+  for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       s[nt][e] = mn0 == -INFINITY ? 0.f : exp2f(s[nt][e] - mn0);
@@ -193,17 +215,219 @@ __device__ __forceinline__ void softmax_step(float (&s)[8][4], float (&o)[16][4]
   }
 }
 
-__device__ __forceinline__ void write_warp_partial(float* mrg, int w, int lane, float m0, float m1,
-                                                   float l0, float l1, const float (&o)[16][4]) {
-  float* pw = mrg + w * PART;
+// As softmax_step, but the running max only moves when some row's tile max
+// exceeds it by more than 8 (log2 units): below that, p = exp2(z - m) <= 256
+// stays well inside fp32 and bf16, the normalisation by l stays exact, and the
+// common case skips rescaling the accumulators.
+template <int NT>
+__device__ __forceinline__ void softmax_step_lazy(float (&s)[NT][4], float (&o)[16][4], float& m0,
+                                                  float& m1, float& l0, float& l1, int nvalid,
+                                                  float scale_log2, int lane) {
+  const int c = (lane & 3) * 2;
+  float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const bool ok = nt * 8 + c + e < nvalid;
+      s[nt][e] = ok ? s[nt][e] * scale_log2 : -INFINITY;
+      s[nt][2 + e] = ok ? s[nt][2 + e] * scale_log2 : -INFINITY;
+      mx0 = fmaxf(mx0, s[nt][e]);
+      mx1 = fmaxf(mx1, s[nt][2 + e]);
+    }
+  mx0 = quad_max(mx0);
+  mx1 = quad_max(mx1);
+  const bool grow = mx0 > m0 + 8.f || mx1 > m1 + 8.f;
+  if (__any_sync(0xffffffffu, grow)) {
+    const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+    const float c0 = exp2f(m0 - mn0), c1 = exp2f(m1 - mn1);  // 0 when m was -inf
+    l0 *= c0;
+    l1 *= c1;
+#pragma unroll
+    for (int dt = 0; dt < 16; ++dt) {
+      o[dt][0] *= c0;
+      o[dt][1] *= c0;
+      o[dt][2] *= c1;
+      o[dt][3] *= c1;
+    }
+    m0 = mn0;
+    m1 = mn1;
+  }
+  float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      s[nt][e] = exp2f(s[nt][e] - m0);
+      s[nt][2 + e] = exp2f(s[nt][2 + e] - m1);
+      sum0 += s[nt][e];
+      sum1 += s[nt][2 + e];
+    }
+  l0 += quad_sum(sum0);
+  l1 += quad_sum(sum1);
+}
+
+// ---------------------------------------------------------------------------
+// global tile order and its even split over the pair streams
+// ---------------------------------------------------------------------------
+
+struct StreamPlan {
+  int len;  // 64-key tiles of this stream
+  int b, g, tile, ntiles;
+};
+
+// Walk of the global tile order (sequence-major, then KV head, then tile),
+// caching the current sequence's length and selected-block count. `lens`
+// points at the sequence lengths (a shared-memory copy when it fits).
+template <int MODE>
+struct Walker {
+  int b, g, tile, ntiles, L, ns;
+  __device__ void init(const DecFastArgs& a, const int* lens, const StreamPlan& p) {
+    b = p.b;
+    g = p.g;
+    tile = p.tile;
+    ntiles = p.ntiles;
+    L = lens[b];
+    ns = n_selected(L, a);
+  }
+  __device__ void advance(const DecFastArgs& a, const int* lens) {
+    if (++tile < ntiles) return;
+    tile = 0;
+    if (++g < a.Hkv) return;
+    g = 0;
+    do {
+      ++b;
+      L = b < a.B ? lens[b] : 1;
+      ntiles = b < a.B ? unit_tiles<MODE>(L, a) : 1;
+    } while (ntiles == 0);
+    ns = n_selected(L, a);
+  }
+  __device__ int segment(const DecFastArgs& a) const {
+    const int u = b * a.Hkv + g;
+    return MODE == MODE_CMP ? u : 2 * u + (tile >= ns ? 1 : 0);
+  }
+};
+
+constexpr int LENS_CAP = 1024;  // sequence lengths kept in shared memory
+
+// Plans of the NS streams of this CTA (computed by one warp). Stream
+// v = cta * NS + i owns global tiles [total*v/V, total*(v+1)/V). `pre` is
+// scratch for the per-sequence prefix of tile counts (cap entries); `lens_s`
+// receives a copy of the lengths when B <= LENS_CAP.
+template <int MODE, int NS>
+__device__ void make_plans(const DecFastArgs& a, StreamPlan* plans, int* lens_s, long long* pre,
+                           int cap, int lane) {
+  const bool cached = a.B <= LENS_CAP;
+  const bool use_pre = a.B + 1 <= cap;
+  long long carry = 0;
+  if (use_pre && lane == 0) pre[0] = 0;
+  for (int base = 0; base < a.B; base += 32) {
+    const int b = base + lane;
+    const int L = b < a.B ? __ldg(a.seq_lens + b) : 0;
+    if (cached && b < a.B) lens_s[b] = L;
+    long long x = b < a.B ? (long long)unit_tiles<MODE>(L, a) * a.Hkv : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {  // inclusive warp scan
+      const long long y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (use_pre && b < a.B) pre[b + 1] = carry + x;
+    carry += __shfl_sync(0xffffffffu, x, 31);
+  }
+  __syncwarp();
+  const long long total = carry;
+  const long long V = (long long)gridDim.x * NS;
+  if (lane < NS) {
+    const long long v = (long long)blockIdx.x * NS + lane;
+    const long long t0 = total * v / V, t1 = total * (v + 1) / V;
+    StreamPlan p{};
+    p.len = (int)(t1 - t0);
+    p.ntiles = 1;
+    if (t1 > t0) {
+      int b;
+      long long acc;
+      if (use_pre) {  // first b with pre[b + 1] > t0
+        int lo = 0, hi = a.B - 1;
+        while (lo < hi) {
+          const int mid = (lo + hi) >> 1;
+          if (pre[mid + 1] > t0) hi = mid;
+          else lo = mid + 1;
+        }
+        b = lo;
+        acc = pre[b];
+      } else {
+        acc = 0;
+        for (b = 0; b < a.B; ++b) {
+          const long long span = (long long)unit_tiles<MODE>(__ldg(a.seq_lens + b), a) * a.Hkv;
+          if (t0 < acc + span) break;
+          acc += span;
+        }
+      }
+      const int nt = unit_tiles<MODE>(__ldg(a.seq_lens + b), a);
+      const long long off = t0 - acc;
+      p.b = b;
+      p.g = (int)(off / nt);
+      p.tile = (int)(off % nt);
+      p.ntiles = nt;
+    }
+    plans[lane] = p;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// the stream kernel
+// ---------------------------------------------------------------------------
+
+constexpr int NPAIR = 4;              // consumer warp pairs = tile streams per CTA
+constexpr int PSLOTS = 3;             // ring slots per pair: K and V of a tile + one ahead
+constexpr int SLOTS = NPAIR * PSLOTS;
+constexpr int NCW = 2 * NPAIR;        // consumer warps; + 1 producer = 9 warps
+constexpr int RPITCH = WK + 2;        // record scratch pitch (floats)
+constexpr int QBYTES = G * D * 2;     // query block of a pair
+
+template <int MODE>
+struct StreamCfg {
+  static constexpr size_t SMEM = 1024 + (size_t)SLOTS * SLOT_BYTES + NPAIR * QBYTES +
+                                 2 * SLOTS * 8 + SLOTS * 4 + NPAIR * sizeof(StreamPlan) +
+                                 NPAIR * 6 * 4 + 64 + LENS_CAP * 4;
+};
+
+struct TileSrc {
+  int row;     // TMA row (outer coordinate)
+  int nvalid;  // valid keys in the 64-key tile
+};
+
+template <int MODE>
+__device__ __forceinline__ TileSrc tile_source(const DecFastArgs& a, const Walker<MODE>& wk) {
+  TileSrc ts;
+  if (MODE == MODE_CMP) {
+    ts.row = wk.b * a.Nc + wk.tile * TK;
+    ts.nvalid = min(TK, n_visible(wk.L, a.l, a.s, a.Nc) - wk.tile * TK);
+  } else {
+    const int t = wk.L - 1;
+    int start;
+    if (wk.tile < wk.ns) {
+      start = __ldg(a.sel + (long)(wk.b * a.Hkv + wk.g) * a.n + wk.tile) * a.bs;
+    } else {
+      start = t - min(a.w, wk.L) + 1 + (wk.tile - wk.ns) * TK;
+    }
+    ts.row = wk.b * a.T + start;
+    ts.nvalid = min(TK, t - start + 1);
+  }
+  return ts;
+}
+
+// Write one warp's (m, l, unnormalised O) partial straight to global.
+__device__ __forceinline__ void store_partial(float* dst, int lane, float m0, float m1, float l0,
+                                              float l1, const float (&o)[16][4]) {
   const int r0 = lane >> 2, c = (lane & 3) * 2;
   if ((lane & 3) == 0) {
-    pw[r0] = m0;
-    pw[r0 + 8] = m1;
-    pw[G + r0] = l0;
-    pw[G + r0 + 8] = l1;
+    dst[r0] = m0;
+    dst[r0 + 8] = m1;
+    dst[G + r0] = l0;
+    dst[G + r0 + 8] = l1;
   }
-  float* po = pw + 2 * G;
+  float* po = dst + 2 * G;
 #pragma unroll
   for (int dt = 0; dt < 16; ++dt) {
     *reinterpret_cast<float2*>(po + r0 * D + dt * 8 + c) = make_float2(o[dt][0], o[dt][1]);
@@ -211,171 +435,41 @@ __device__ __forceinline__ void write_warp_partial(float* mrg, int w, int lane, 
   }
 }
 
-// 128 consumer threads combine the NCW warp partials into dst.
-__device__ __forceinline__ void merge_warps_to(float* dst, const float* mrg, int tid) {
-  const int h = tid >> 3, e0 = (tid & 7) * 16;
-  float M = -INFINITY;
-#pragma unroll
-  for (int w = 0; w < NCW; ++w) M = fmaxf(M, mrg[w * PART + h]);
-  float f[NCW], L = 0.f;
-#pragma unroll
-  for (int w = 0; w < NCW; ++w) {
-    const float mw = mrg[w * PART + h];
-    f[w] = (M == -INFINITY || mw == -INFINITY) ? 0.f : exp2f(mw - M);
-    L += f[w] * mrg[w * PART + G + h];
-  }
-  if ((tid & 7) == 0) {
-    dst[h] = M;
-    dst[G + h] = L;
-  }
-#pragma unroll
-  for (int e = e0; e < e0 + 16; e += 4) {
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int w = 0; w < NCW; ++w) {
-      const float4 v = *reinterpret_cast<const float4*>(mrg + w * PART + 2 * G + h * D + e);
-      acc.x += f[w] * v.x;
-      acc.y += f[w] * v.y;
-      acc.z += f[w] * v.z;
-      acc.w += f[w] * v.w;
-    }
-    *reinterpret_cast<float4*>(dst + 2 * G + h * D + e) = acc;
-  }
-}
-
-// ---------------------------------------------------------------------------
-// global tile order and its even split over CTAs
-// ---------------------------------------------------------------------------
-
-struct Plan {
-  long long t0, t1;
-  int b, g, tile, ntiles;
-};
-
+// One CTA per SM: warps 0..5 are three pairs of consumers, warp 6 the TMA
+// producer. Pair p streams its own range of 64-key tiles through its own ring
+// of four 16 KB slots (K and V of the current and the next tile); warp h of
+// the pair handles keys [32h, 32h + 32) of every tile, with its own online
+// softmax state, and writes its partial to slot 2 * (stream + segment) + h.
+// Every consumer takes part in every phase of its pair's slots, so the mbarrier
+// phase parity is always unambiguous. The producer polls the three rings
+// without blocking on any one of them.
 template <int MODE>
-struct Walker {
-  int b, g, tile, ntiles;
-  __device__ void advance(const DecFastArgs& a) {
-    if (++tile < ntiles) return;
-    tile = 0;
-    if (++g < a.Hkv) return;
-    g = 0;
-    do {
-      ++b;
-      ntiles = b < a.B ? unit_tiles<MODE>(a.seq_lens[b], a) : 1;
-    } while (ntiles == 0);
-  }
-};
-
-template <int MODE>
-__device__ long long total_tiles_warp(const DecFastArgs& a, int lane) {
-  long long total = 0;
-  for (int base = 0; base < a.B; base += 32) {
-    const int b = base + lane;
-    long long tb = b < a.B ? (long long)unit_tiles<MODE>(a.seq_lens[b], a) * a.Hkv : 0;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) tb += __shfl_xor_sync(0xffffffffu, tb, o);
-    total += tb;
-  }
-  return total;
-}
-
-template <int MODE>
-__device__ void make_plan(const DecFastArgs& a, Plan* plan, int lane) {
-  const long long total = total_tiles_warp<MODE>(a, lane);
-  const long long c = blockIdx.x, grid = gridDim.x;
-  const long long t0 = total * c / grid, t1 = total * (c + 1) / grid;
-  if (lane == 0) {
-    plan->t0 = t0;
-    plan->t1 = t1;
-    plan->b = plan->g = plan->tile = 0;
-    plan->ntiles = 1;
-    if (t1 > t0) {
-      long long acc = 0;
-      for (int b = 0; b < a.B; ++b) {
-        const int nt = unit_tiles<MODE>(a.seq_lens[b], a);
-        const long long span = (long long)nt * a.Hkv;
-        if (t0 < acc + span) {
-          const long long off = t0 - acc;
-          plan->b = b;
-          plan->g = (int)(off / nt);
-          plan->tile = (int)(off % nt);
-          plan->ntiles = nt;
-          break;
-        }
-        acc += span;
-      }
-    }
-  }
-}
-
-// CTA (of `grid`) whose share of `total` tiles holds global tile `tile`.
-__device__ __forceinline__ int owner_cta(long long tile, long long total, long long grid) {
-  long long cc = tile * grid / total;
-  while (cc > 0 && total * cc / grid > tile) --cc;
-  while (cc + 1 < grid && total * (cc + 1) / grid <= tile) ++cc;
-  return (int)cc;
-}
-
-// ---------------------------------------------------------------------------
-// the stream kernel
-// ---------------------------------------------------------------------------
-
-template <int MODE>
-struct TileSrc {
-  int row;      // TMA row (outer coordinate)
-  int nvalid;   // valid keys in the tile
-};
-
-template <int MODE>
-__device__ __forceinline__ TileSrc<MODE> tile_source(const DecFastArgs& a, int b, int g, int tile) {
-  TileSrc<MODE> ts;
-  const int L = a.seq_lens[b];
-  if (MODE == MODE_CMP) {
-    ts.row = b * a.Nc + tile * TK;
-    ts.nvalid = min(TK, n_visible(L, a.l, a.s, a.Nc) - tile * TK);
-  } else {
-    const int t = L - 1, ns = n_selected(L, a);
-    int start;
-    if (tile < ns) {
-      start = a.sel[(long)(b * a.Hkv + g) * a.n + tile] * a.bs;
-    } else {
-      start = t - min(a.w, L) + 1 + (tile - ns) * TK;
-    }
-    ts.row = b * a.T + start;
-    ts.nvalid = min(TK, t - start + 1);
-  }
-  return ts;
-}
-
-template <int MODE>
-__device__ __forceinline__ int segment_of(const DecFastArgs& a, int b, int g, int tile) {
-  const int u = b * a.Hkv + g;
-  if (MODE == MODE_CMP) return u;
-  return 2 * u + (tile >= n_selected(a.seq_lens[b], a) ? 1 : 0);
-}
-
-template <int MODE>
-__global__ void __launch_bounds__(160, 1)
+__global__ void __launch_bounds__((NCW + 1) * 32, 1)
     dec_stream_kernel(const __grid_constant__ DecFastArgs a, const __grid_constant__ CUtensorMap tk,
                       const __grid_constant__ CUtensorMap tv) {
+  using C = StreamCfg<MODE>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   unsigned char* slots = smem;
-  float* mrg = reinterpret_cast<float*>(smem + SLOTS * SLOT_BYTES);
-  uint64_t* full = reinterpret_cast<uint64_t*>(mrg + MERGE_FLOATS);
+  unsigned char* qsm = slots + SLOTS * SLOT_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(qsm + NPAIR * QBYTES);
   uint64_t* empty = full + SLOTS;
-  Plan* plan = reinterpret_cast<Plan*>(empty + SLOTS);
-  int* abort_flag = reinterpret_cast<int*>(plan + 1);
+  int* info = reinterpret_cast<int*>(empty + SLOTS);
+  StreamPlan* plans = reinterpret_cast<StreamPlan*>(info + SLOTS);
+  Walker<MODE>* pwk = reinterpret_cast<Walker<MODE>*>(plans + NPAIR);
+  int* abort_flag = reinterpret_cast<int*>(pwk + NPAIR);
+  int* lens_s = abort_flag + 1;  // [LENS_CAP]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp == NCW) {
-    make_plan<MODE>(a, plan, lane);
+    // the slot ring is idle until the pipeline starts: use it as plan scratch
+    make_plans<MODE, NPAIR>(a, plans, lens_s, reinterpret_cast<long long*>(slots),
+                            SLOTS * SLOT_BYTES / 8, lane);
     if (lane == 0) {
       for (int i = 0; i < SLOTS; ++i) {
         ptx::mbar_init(&full[i], 1);
-        ptx::mbar_init(&empty[i], 1);
+        ptx::mbar_init(&empty[i], 2);
       }
       *abort_flag = 0;
       ptx::fence_mbar_init();
@@ -384,166 +478,304 @@ __global__ void __launch_bounds__(160, 1)
     }
   }
   __syncthreads();
-  const long long ntl = plan->t1 - plan->t0;
-  if (ntl <= 0) return;
+  const int* lens_p = a.B <= LENS_CAP ? lens_s : a.seq_lens;
   float* part = MODE == MODE_CMP ? a.part1 : a.part3;
 
   if (warp == NCW) {
-    // ---------------- producer: half-tile i = 2k (K) or 2k+1 (V) ----------------
-    if (lane == 0) {
-      const uint64_t pol = ptx::policy_evict_first();
-      Walker<MODE> wk{plan->b, plan->g, plan->tile, plan->ntiles};
-      long long i = 0;
-      TileSrc<MODE> ts{};
-      for (; i < 2 * ntl; ++i) {
-        const int sl = (int)(i % SLOTS);
-        const long long use = i / SLOTS;
-        if (use > 0 && !ptx::mbar_wait(&empty[sl], (uint32_t)((use - 1) & 1), kWaitNs)) {
-          atomicOr(a.err, kErrTimeout);
-          atomicExch(abort_flag, 1);
+    // ---------------- producer ----------------
+    if (lane != 0) return;
+    const uint64_t pol = ptx::policy_evict_first();
+    int h[NPAIR], hend[NPAIR];
+    TileSrc ts[NPAIR];
+    long long remaining = 0;
+#pragma unroll
+    for (int p = 0; p < NPAIR; ++p) {
+      h[p] = 0;
+      hend[p] = 2 * plans[p].len;
+      remaining += hend[p];
+      if (hend[p] > 0) {
+        pwk[p].init(a, lens_p, plans[p]);
+        ts[p] = tile_source<MODE>(a, pwk[p]);
+      }
+    }
+    uint64_t t_last = ptx::globaltimer();
+    while (remaining > 0) {
+      bool progressed = false;
+#pragma unroll
+      for (int p = 0; p < NPAIR; ++p) {
+        if (h[p] >= hend[p]) continue;
+        const int sl = p * PSLOTS + h[p] % PSLOTS;
+        const int use = h[p] / PSLOTS;
+        if (use > 0 && !ptx::mbar_try_wait(&empty[sl], (uint32_t)((use - 1) & 1))) continue;
+        const bool isv = h[p] & 1;
+        if (!isv) {
+          // first / last stream of each segment, for the merging kernels
+          const Walker<MODE>& wk = pwk[p];
+          const int u = wk.b * a.Hkv + wk.g;
+          const int v = blockIdx.x * NPAIR + p;
+          if (MODE == MODE_CMP) {
+            if (wk.tile == 0) a.rng1[2 * u] = v;
+            if (wk.tile == wk.ntiles - 1) a.rng1[2 * u + 1] = v;
+          } else {
+            if (wk.tile == 0) a.rng3[4 * u] = v;
+            if (wk.tile == wk.ns - 1) a.rng3[4 * u + 1] = v;
+            if (wk.tile == wk.ns) a.rng3[4 * u + 2] = v;
+            if (wk.tile == wk.ntiles - 1) a.rng3[4 * u + 3] = v;
+          }
         }
-        if (*(volatile int*)abort_flag) break;
-        const bool isv = i & 1;
-        if (!isv) ts = tile_source<MODE>(a, wk.b, wk.g, wk.tile);
+        info[sl] = ts[p].nvalid;
         unsigned char* dst = slots + sl * SLOT_BYTES;
         const CUtensorMap* m = isv ? &tv : &tk;
         ptx::mbar_arrive_expect_tx(&full[sl], SLOT_BYTES);
-        ptx::tma_load_3d(dst, m, &full[sl], 0, wk.g, ts.row, pol);
-        ptx::tma_load_3d(dst + HALF_BYTES, m, &full[sl], 64, wk.g, ts.row, pol);
-        if (isv) wk.advance(a);
+        ptx::tma_load_3d(dst, m, &full[sl], 0, pwk[p].g, ts[p].row, pol);
+        ptx::tma_load_3d(dst + HALF_BYTES, m, &full[sl], 64, pwk[p].g, ts[p].row, pol);
+        if (isv) {
+          pwk[p].advance(a, lens_p);
+          if (h[p] + 1 < hend[p]) ts[p] = tile_source<MODE>(a, pwk[p]);  // next tile, early
+        }
+        ++h[p];
+        --remaining;
+        progressed = true;
       }
-      // every issued load must have landed before the CTA exits
-      const long long issued = i;
-      for (int sl = 0; sl < SLOTS && sl < issued; ++sl) {
-        const long long last_use = (issued - 1 - sl) / SLOTS;
-        if (!ptx::mbar_wait(&full[sl], (uint32_t)(last_use & 1), kWaitNs))
-          atomicOr(a.err, kErrTimeout);
+      if (progressed) {
+        t_last = ptx::globaltimer();
+      } else if (ptx::globaltimer() - t_last > kWaitNs || *(volatile int*)abort_flag) {
+        atomicOr(a.err, kErrTimeout);
+        atomicExch(abort_flag, 1);
+        break;
       }
     }
+    // every issued load must have landed before the CTA exits
+#pragma unroll
+    for (int p = 0; p < NPAIR; ++p)
+      for (int k = 0; k < PSLOTS && k < h[p]; ++k) {
+        const int last = h[p] - 1 - ((h[p] - 1 - k) % PSLOTS);  // last half-tile in slot k
+        if (!ptx::mbar_wait(&full[p * PSLOTS + last % PSLOTS],
+                            (uint32_t)((last / PSLOTS) & 1), kWaitNs))
+          atomicOr(a.err, kErrTimeout);
+      }
     return;
   }
 
   // ---------------- consumers ----------------
-  const int tid = threadIdx.x;
-  float* scr = mrg + warp * (G * SCR_PITCH);
-  Walker<MODE> wk{plan->b, plan->g, plan->tile, plan->ntiles};
-  int cur_seg = segment_of<MODE>(a, wk.b, wk.g, wk.tile);
+  const int pair = warp >> 1, hw = warp & 1;
+  const int my_len = plans[pair].len;
+  if (my_len <= 0) return;
+  unsigned char* qs = qsm + pair * QBYTES;
+  const uint32_t qbase = ptx::smem_u32(qs);
+  const long long vstream = (long long)blockIdx.x * NPAIR + pair;
+  Walker<MODE> wk;
+  wk.init(a, lens_p, plans[pair]);
+  int cur_seg = wk.segment(a);
   int cur_b = wk.b, cur_g = wk.g;
-  uint32_t qa[8][4];
-  const __nv_bfloat16* qbase = reinterpret_cast<const __nv_bfloat16*>(a.q);
-  load_q_frags(qa, qbase + ((long)cur_b * a.Hq + cur_g * G) * D, lane);
+  const __nv_bfloat16* qg = reinterpret_cast<const __nv_bfloat16*>(a.q);
+  stage_q_half(qs, qg + ((long)cur_b * a.Hq + cur_g * G) * D, hw, lane);
+  ptx::named_bar_sync(1 + pair, 64);
   float o[16][4];
 #pragma unroll
   for (int dt = 0; dt < 16; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
   float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
   const int r0 = lane >> 2, c = (lane & 3) * 2;
-
-  auto flush = [&](int seg) {
-    ptx::named_bar_sync(1, NCW * 32);
-    write_warp_partial(mrg, warp, lane, m0, m1, l0, l1, o);
-    ptx::named_bar_sync(1, NCW * 32);
-    merge_warps_to(part + (long)(blockIdx.x + seg) * PART, mrg, tid);
-    ptx::named_bar_sync(1, NCW * 32);
-#pragma unroll
-    for (int dt = 0; dt < 16; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
-    m0 = m1 = -INFINITY;
-    l0 = l1 = 0.f;
-  };
-
-  for (long long k = 0; k < ntl; ++k) {
-    const int seg = segment_of<MODE>(a, wk.b, wk.g, wk.tile);
+  for (int r = 0; r < my_len; ++r) {
+    const int seg = wk.segment(a);
     if (seg != cur_seg) {
-      flush(cur_seg);
+      store_partial(part + (2 * (vstream + cur_seg) + hw) * PART, lane, m0, m1, l0, l1, o);
+#pragma unroll
+      for (int dt = 0; dt < 16; ++dt) o[dt][0] = o[dt][1] = o[dt][2] = o[dt][3] = 0.f;
+      m0 = m1 = -INFINITY;
+      l0 = l1 = 0.f;
       cur_seg = seg;
       if (wk.b != cur_b || wk.g != cur_g) {
         cur_b = wk.b;
         cur_g = wk.g;
-        load_q_frags(qa, qbase + ((long)cur_b * a.Hq + cur_g * G) * D, lane);
+        ptx::named_bar_sync(1 + pair, 64);  // both warps are done with the old block
+        stage_q_half(qs, qg + ((long)cur_b * a.Hq + cur_g * G) * D, hw, lane);
+        ptx::named_bar_sync(1 + pair, 64);
       }
     }
-    if ((int)(k % NCW) == warp) {
-      const int slk = (int)((2 * k) % SLOTS), slv = (int)((2 * k + 1) % SLOTS);
-      const uint32_t pk = (uint32_t)(((2 * k) / SLOTS) & 1);
-      const uint32_t pv = (uint32_t)(((2 * k + 1) / SLOTS) & 1);
-      const TileSrc<MODE> ts = tile_source<MODE>(a, wk.b, wk.g, wk.tile);
-      bool ok = !*(volatile int*)abort_flag;
-      if (ok && !ptx::mbar_wait(&full[slk], pk, kWaitNs)) {
-        if (lane == 0) {
-          atomicOr(a.err, kErrTimeout);
-          atomicExch(abort_flag, 1);
-        }
-        ok = false;
+    const int hk = 2 * r, hv = 2 * r + 1;
+    const int slk = pair * PSLOTS + hk % PSLOTS, slv = pair * PSLOTS + hv % PSLOTS;
+    bool ok = !*(volatile int*)abort_flag;
+    if (ok && !ptx::mbar_wait(&full[slk], (uint32_t)((hk / PSLOTS) & 1), kWaitNs)) {
+      if (lane == 0) {
+        atomicOr(a.err, kErrTimeout);
+        atomicExch(abort_flag, 1);
       }
-      float s[8][4];
-      if (ok) qk_tile(s, qa, ptx::smem_u32(slots + slk * SLOT_BYTES), lane);
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&empty[slk]);
-      if (ok) {
-        softmax_step(s, o, m0, m1, l0, l1, ts.nvalid, a.scale_log2, lane);
-        if (MODE == MODE_CMP) {
-          // tile record: running max per head, and exp-sums per overlapped block
+      ok = false;
+    }
+    const int nvalid = ok ? min(WK, info[slk] - WK * hw) : 0;
+    float s[4][4];
+    if (nvalid > 0) qk_tile_q<4>(s, qbase, ptx::smem_u32(slots + slk * SLOT_BYTES), WK * hw, lane);
+    if (nvalid > 0) {
+      softmax_step_lazy<4>(s, o, m0, m1, l0, l1, nvalid, a.scale_log2, lane);
+      if (MODE == MODE_CMP) {
+        // record of this 32-key sub-tile: running max per head, and per
+        // overlapped selection block the exp-sum of its keys. Scratch: this
+        // warp's own 32 key rows of the K slot (first TMA box), already read.
+        __syncwarp();
+        float* scr = reinterpret_cast<float*>(slots + slk * SLOT_BYTES + hw * (WK * 128));
 #pragma unroll
-          for (int nt = 0; nt < 8; ++nt) {
-            *reinterpret_cast<float2*>(scr + r0 * SCR_PITCH + nt * 8 + c) =
-                make_float2(s[nt][0], s[nt][1]);
-            *reinterpret_cast<float2*>(scr + (r0 + 8) * SCR_PITCH + nt * 8 + c) =
-                make_float2(s[nt][2], s[nt][3]);
-          }
-          __syncwarp();
-          const int u = wk.b * a.Hkv + wk.g;
-          float* rec = a.trec + ((long)u * a.tiles_max + wk.tile) * (G * (1 + a.nbt));
-          if ((lane & 3) == 0) {
-            rec[r0] = m0;
-            rec[r0 + 8] = m1;
-          }
-          for (int x = lane; x < G * a.nbt; x += 32) {
-            const int jl = x >> 4, h = x & 15;
-            const int lo = a.klo[jl], hi = min((int)a.khi[jl], ts.nvalid - 1);
-            float acc = 0.f;
-            for (int kk = lo; kk <= hi; ++kk) acc += scr[h * SCR_PITCH + kk];
-            rec[G + x] = acc;  // [1 + jl][h]
-          }
-          __syncwarp();
+        for (int nt = 0; nt < 4; ++nt) {
+          *reinterpret_cast<float2*>(scr + r0 * RPITCH + nt * 8 + c) =
+              make_float2(s[nt][0], s[nt][1]);
+          *reinterpret_cast<float2*>(scr + (r0 + 8) * RPITCH + nt * 8 + c) =
+              make_float2(s[nt][2], s[nt][3]);
         }
-      }
-      if (ok && !ptx::mbar_wait(&full[slv], pv, kWaitNs)) {
-        if (lane == 0) {
-          atomicOr(a.err, kErrTimeout);
-          atomicExch(abort_flag, 1);
+        __syncwarp();
+        const int u = wk.b * a.Hkv + wk.g;
+        float* rec = a.trec + ((long)u * a.tiles_max + 2 * wk.tile + hw) * (G * (1 + a.nbt));
+        if ((lane & 3) == 0) {
+          rec[r0] = m0;
+          rec[r0 + 8] = m1;
         }
-        ok = false;
+        for (int x = lane; x < G * a.nbt; x += 32) {
+          const int jl = x >> 4, hh = x & 15;
+          const int lo = a.klo[jl], hi = min((int)a.khi[jl], nvalid - 1);
+          float acc = 0.f;
+          for (int kk = lo; kk <= hi; ++kk) acc += scr[hh * RPITCH + kk];
+          rec[G + x] = acc;  // [1 + jl][h]
+        }
+        ptx::fence_proxy_async();  // scratch writes before the slot's next TMA fill
       }
-      if (ok) pv_tile(o, s, ptx::smem_u32(slots + slv * SLOT_BYTES), lane);
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&empty[slv]);
     }
-    wk.advance(a);
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(&empty[slk]);
+    if (ok && !ptx::mbar_wait(&full[slv], (uint32_t)((hv / PSLOTS) & 1), kWaitNs)) {
+      if (lane == 0) {
+        atomicOr(a.err, kErrTimeout);
+        atomicExch(abort_flag, 1);
+      }
+      ok = false;
+    }
+    if (ok && nvalid > 0) pv_tile<2>(o, s, ptx::smem_u32(slots + slv * SLOT_BYTES), WK * hw, lane);
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(&empty[slv]);
+    wk.advance(a, lens_p);
   }
-  flush(cur_seg);
+  store_partial(part + (2 * (vstream + cur_seg) + hw) * PART, lane, m0, m1, l0, l1, o);
+}
+
+// ---------------------------------------------------------------------------
+// merging stream partials (dec_select, dec_combine)
+// ---------------------------------------------------------------------------
+
+constexpr int MP = 64;  // partials staged per chunk
+
+// Online merge of the softmax partials in slots [first, first + np): per head
+// M = max m_p and L = sum_p exp2(m_p - M) l_p (left in sM / sL), and
+//   acc[h][e0 .. e0+7] += scale_h / L_h * sum_p exp2(m_p - M_h) o_p[h][e].
+// Partials are staged MP at a time with a running max and sum, so any count
+// works; one chunk costs two load-dependent steps. Threads (h, 8 dims): the
+// first 256 threads of the block accumulate; all NT take part in staging.
+template <int NT>
+__device__ void merge_online(const float* part, long long first, int np, const float* scale,
+                             float* pm, float* pl, float* sM, float* sL, float* sR, int h, int e0,
+                             float (&acc)[8]) {
+  const int tid = threadIdx.x;
+  float run[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  if (tid < 16) {
+    sM[tid] = -INFINITY;
+    sL[tid] = 0.f;
+  }
+  for (int p0 = 0; p0 < np; p0 += MP) {
+    const int pc = min(MP, np - p0);
+    __syncthreads();
+    for (int x = tid; x < pc * 16; x += NT) {
+      const float* src = part + (first + p0 + (x >> 4)) * PART;
+      pm[x] = __ldcg(src + (x & 15));
+      pl[x] = __ldcg(src + G + (x & 15));
+    }
+    __syncthreads();
+    if (tid < 16) {
+      float Mc = -INFINITY;
+      for (int pp = 0; pp < pc; ++pp) Mc = fmaxf(Mc, pm[pp * 16 + tid]);
+      const float Mo = sM[tid], Mn = fmaxf(Mo, Mc);
+      const float r = Mo == -INFINITY ? 0.f : exp2f(Mo - Mn);
+      float Lc = 0.f;
+      for (int pp = 0; pp < pc; ++pp) {
+        const float mm = pm[pp * 16 + tid];
+        if (mm != -INFINITY) Lc += exp2f(mm - Mn) * pl[pp * 16 + tid];
+      }
+      sL[tid] = sL[tid] * r + Lc;
+      sM[tid] = Mn;
+      sR[tid] = r;
+    }
+    __syncthreads();
+    for (int x = tid; x < pc * 16; x += NT) {
+      const float mm = pm[x];
+      pm[x] = mm == -INFINITY ? 0.f : exp2f(mm - sM[x & 15]);
+    }
+    __syncthreads();
+    if (tid < 256) {
+      const float r = sR[h];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) run[e] *= r;
+#pragma unroll 4
+      for (int pp = 0; pp < pc; ++pp) {
+        const float f = pm[pp * 16 + h];
+        const float4* src =
+            reinterpret_cast<const float4*>(part + (first + p0 + pp) * PART + 2 * G + h * D + e0);
+        const float4 v0 = __ldcg(src), v1 = __ldcg(src + 1);
+        run[0] += f * v0.x;
+        run[1] += f * v0.y;
+        run[2] += f * v0.z;
+        run[3] += f * v0.w;
+        run[4] += f * v1.x;
+        run[5] += f * v1.y;
+        run[6] += f * v1.z;
+        run[7] += f * v1.w;
+      }
+    }
+  }
+  __syncthreads();
+  if (tid < 256) {
+    const float sc = sL[h] > 0.f ? scale[h] / sL[h] : 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] += sc * run[e];
+  }
 }
 
 // ---------------------------------------------------------------------------
 // dec_select
 // ---------------------------------------------------------------------------
 
-constexpr int SEL_THREADS = 256;
+constexpr int SEL_THREADS = 512;
+constexpr int SEL_WARPS = SEL_THREADS / 32;
+constexpr int MAXSEL = 64;       // top_n bound of the fast path
+constexpr int MAXCAND = 4096;    // selection blocks bound of the fast path (T <= 262144)
+
+// Sort key of a candidate block: higher score first, then the lower index.
+// Scores are >= 0, so their IEEE bits order like the values; the low word is
+// the inverted index. Keys are unique, so the top set is exact.
+__device__ __forceinline__ unsigned long long sel_key(float score, int j) {
+  return ((unsigned long long)__float_as_uint(score) << 32) | (0xffffffffu - (unsigned)j);
+}
 
 __global__ void __launch_bounds__(SEL_THREADS) dec_select_kernel(const __grid_constant__ DecFastArgs a) {
-  extern __shared__ __align__(16) float sm[];
+  // dynamic: records [tiles_max][16 (1 + nbt)] | keys [npow] u64 | fac [tiles_max][16]
+  //          | tsum [tiles_max][16]
+  extern __shared__ __align__(128) unsigned char dyn_raw[];
+  __shared__ float mS[G], lS[G], sR[G], lse2[G], gate[3 * G], scl[G];
+  __shared__ __align__(16) float pm[MP * G], pl[MP * G];
+  __shared__ float wg_s[D * 3];
+  __shared__ float q_s[G * D];
+  __shared__ int sel[MAXSEL];
+  __shared__ unsigned hist[256];
+  __shared__ int cut_bin, cut_above, nsel_s;
+  __shared__ __align__(8) uint64_t rec_bar;
+
   const int u = blockIdx.x, b = u / a.Hkv, g = u - b * a.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int nblk = (a.T + a.bs - 1) / a.bs;
-  long long* red_ll = reinterpret_cast<long long*>(sm);  // [16]
-  float* lse2 = sm + 32;                  // [16]
-  float* gate = lse2 + G;                 // [16][3]
-  float* fac = gate + 3 * G;              // [tiles_max][16]
-  float* scores = fac + a.tiles_max * G;  // [nblk]
-  float* red_s = scores + nblk;           // [8]
-  int* red_j = reinterpret_cast<int*>(red_s + 8);
-  int* sel = red_j + 8;                   // [n]
-  __shared__ int c_first, c_last;
+  int npow = 1;
+  while (npow < nblk) npow <<= 1;
+  const int rec_floats = G * (1 + a.nbt);
+  float* recs = reinterpret_cast<float*>(dyn_raw);
+  unsigned long long* keys = reinterpret_cast<unsigned long long*>(recs + (size_t)a.tiles_max * rec_floats);
+  float* fac = reinterpret_cast<float*>(keys + npow);
+  float* tsum = fac + (size_t)a.tiles_max * G;
 
-  const int L = a.seq_lens[b];
+  const int L = __ldg(a.seq_lens + b);
   float* oacc = a.oacc + (long)u * G * D;
   if (!len_ok(L, a)) {
     for (int x = tid; x < G * D; x += SEL_THREADS)
@@ -557,20 +789,36 @@ __global__ void __launch_bounds__(SEL_THREADS) dec_select_kernel(const __grid_co
   const int t = L - 1;
   const int nvis = n_visible(L, a.l, a.s, a.Nc);
   const int ncand = t / a.bs + 1;
-  const int tiles_u = (nvis + TK - 1) / TK;
+  const int rtiles_u = (nvis + WK - 1) / WK;  // 32-key record sub-tiles
+
+  // The unit's score records, in one bulk copy that lands while the partials merge.
+  if (tid == 0) {
+    ptx::mbar_init(&rec_bar, 1);
+    ptx::fence_mbar_init();
+    if (rtiles_u > 0) {
+      const uint32_t bytes = (uint32_t)rtiles_u * rec_floats * 4;
+      ptx::mbar_arrive_expect_tx(&rec_bar, bytes);
+      ptx::bulk_load(recs, a.trec + (long)u * a.tiles_max * rec_floats, bytes, &rec_bar);
+    }
+  }
   const __nv_bfloat16* qg =
       reinterpret_cast<const __nv_bfloat16*>(a.q) + ((long)b * a.Hq + g * G) * D;
+  for (int x = tid; x < G * D; x += SEL_THREADS) q_s[x] = __bfloat162float(qg[x]);
+  if (a.gate_mode == 0)
+    for (int x = tid; x < D * 3; x += SEL_THREADS) wg_s[x] = __ldg(a.w_gate + x);
+  const int2 rg = *reinterpret_cast<const int2*>(a.rng1 + 2 * u);
+  __syncthreads();
 
-  // gates (EP94 notes §五 gating): one warp per (head, branch) dot product
-  for (int x = warp; x < 3 * G; x += SEL_THREADS / 32) {
+  // gates (EP94 notes §五 gating), from the raw query: a warp per dot product
+  for (int x = warp; x < 3 * G; x += SEL_WARPS) {
     const int h = x / 3, br = x - h * 3;
     float gv;
     if (a.gate_mode == 1) {
       gv = a.fixed_gates[br];
     } else {
       float dot = 0.f;
-      for (int e = lane; e < D; e += 32)
-        dot = fmaf(__bfloat162float(qg[h * D + e]), __ldg(a.w_gate + e * 3 + br), dot);
+#pragma unroll
+      for (int e = lane; e < D; e += 32) dot = fmaf(q_s[h * D + e], wg_s[e * 3 + br], dot);
       dot = warp_sum(dot);
       gv = 1.f / (1.f + expf(-dot));
     }
@@ -579,152 +827,139 @@ __global__ void __launch_bounds__(SEL_THREADS) dec_select_kernel(const __grid_co
       a.gates[(long)u * 3 * G + x] = gv;
     }
   }
-  for (int j = tid; j < ncand; j += SEL_THREADS) scores[j] = 0.f;
+  __syncthreads();
 
   if (nvis > 0) {
-    long long before = 0, total = 0;
-    for (int bb = tid; bb < a.B; bb += SEL_THREADS) {
-      const long long nt = (long long)unit_tiles<MODE_CMP>(a.seq_lens[bb], a) * a.Hkv;
-      total += nt;
-      if (bb < b) before += nt;
+    if (tid < 16) scl[tid] = gate[tid * 3];
+    const int h = (tid & 255) >> 4, e0 = (tid & 15) * 8;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    merge_online<SEL_THREADS>(a.part1, 2 * ((long long)rg.x + u), 2 * (rg.y - rg.x + 1), scl, pm,
+                              pl, mS, lS, sR, h, e0, acc);
+    if (tid < 16) lse2[tid] = mS[tid] + log2f(lS[tid]);
+    if (tid < 256) {
+      float4* dst = reinterpret_cast<float4*>(oacc + h * D + e0);
+      dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
     }
-    for (int o = 16; o > 0; o >>= 1) {
-      total += __shfl_xor_sync(0xffffffffu, total, o);
-      before += __shfl_xor_sync(0xffffffffu, before, o);
-    }
-    if (lane == 0) {
-      red_ll[2 * warp] = total;
-      red_ll[2 * warp + 1] = before;
+    // records landed? then factors exp2(m_ref - lse) per (sub-tile, head)
+    if (!ptx::mbar_wait(&rec_bar, 0, kWaitNs) && tid == 0) atomicOr(a.err, kErrTimeout);
+    __syncthreads();
+    for (int x = tid; x < rtiles_u * G; x += SEL_THREADS) {
+      const int tau = x >> 4, h = x & 15;
+      fac[x] = exp2f(recs[tau * rec_floats + h] - lse2[h]);
     }
     __syncthreads();
-    if (tid == 0) {
-      long long T0 = 0, P0 = 0;
-      for (int w = 0; w < SEL_THREADS / 32; ++w) {
-        T0 += red_ll[2 * w];
-        P0 += red_ll[2 * w + 1];
-      }
-      const long long Pu = P0 + (long long)g * tiles_u;
-      c_first = owner_cta(Pu, T0, a.grid1);
-      c_last = owner_cta(Pu + tiles_u - 1, T0, a.grid1);
-    }
-    __syncthreads();
-    if (tid < G) {
-      float M = -INFINITY;
-      for (int cc = c_first; cc <= c_last; ++cc)
-        M = fmaxf(M, a.part1[(long)(cc + u) * PART + tid]);
-      float Ls = 0.f;
-      for (int cc = c_first; cc <= c_last; ++cc) {
-        const float* pp = a.part1 + (long)(cc + u) * PART;
-        Ls += exp2f(pp[tid] - M) * pp[G + tid];
-      }
-      lse2[tid] = M + log2f(Ls);
-    }
-    __syncthreads();
-    for (int x = tid; x < G * D; x += SEL_THREADS) {
-      const int h = x / D;
-      float acc = 0.f;
-      for (int cc = c_first; cc <= c_last; ++cc) {
-        const float* pp = a.part1 + (long)(cc + u) * PART;
-        acc += exp2f(pp[h] - lse2[h]) * pp[2 * G + x];
-      }
-      oacc[x] = gate[h * 3] * acc;
-    }
-    const float* rec = a.trec + (long)u * a.tiles_max * (G * (1 + a.nbt));
-    for (int x = tid; x < tiles_u * G; x += SEL_THREADS) {
-      const int tau = x / G, h = x - tau * G;
-      fac[x] = exp2f(rec[(long)tau * G * (1 + a.nbt) + h] - lse2[h]);
-    }
-    __syncthreads();
-    // block j gets its record entries from tile j / R and, for its first
-    // compressed key, possibly the tile before (R = blocks per tile start)
-    const int R = (TK * a.s) / a.bs;
-    for (int j = tid; j < ncand; j += SEL_THREADS) {
-      float acc = 0.f;
-      const int tau_hi = min(j / R, tiles_u - 1);
-      const int tau_lo = max(0, (j - a.nbt + R) / R);
-      for (int tau = tau_lo; tau <= tau_hi; ++tau) {
-        const int jl = j - tau * R;
-        if (jl < 0 || jl >= a.nbt) continue;
-        const float4* rt = reinterpret_cast<const float4*>(
-            rec + (long)tau * G * (1 + a.nbt) + G * (1 + jl));
-        const float* f = fac + tau * G;
+    // per (sub-tile, block slot): the head-weighted sum of the record, as a
+    // 16-wide dot product of two contiguous shared-memory rows
+    for (int x = tid; x < rtiles_u * 16; x += SEL_THREADS) {
+      const int tau = x >> 4, jl = x & 15;
+      float v = 0.f;
+      if (jl < a.nbt) {
+        const float4* rt = reinterpret_cast<const float4*>(recs + tau * rec_floats + G * (1 + jl));
+        const float4* f = reinterpret_cast<const float4*>(fac + tau * G);
+        float v0 = 0.f, v1 = 0.f;
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          const float4 v = __ldg(rt + q4);
-          acc += f[4 * q4] * v.x;
-          acc += f[4 * q4 + 1] * v.y;
-          acc += f[4 * q4 + 2] * v.z;
-          acc += f[4 * q4 + 3] * v.w;
+        for (int q4 = 0; q4 < 4; q4 += 2) {
+          const float4 r0 = rt[q4], f0 = f[q4], r1 = rt[q4 + 1], f1 = f[q4 + 1];
+          v0 += r0.x * f0.x + r0.y * f0.y + r0.z * f0.z + r0.w * f0.w;
+          v1 += r1.x * f1.x + r1.y * f1.y + r1.z * f1.z + r1.w * f1.w;
         }
+        v = v0 + v1;
       }
-      scores[j] = acc;
+      tsum[x] = v;
+    }
+    __syncthreads();
+    // block j collects the slots of the sub-tiles whose block ranges include it
+    const int rsh = a.r_shift;  // blocks between sub-tile starts = 1 << rsh
+    for (int j = tid; j < ncand; j += SEL_THREADS) {
+      float v = 0.f;
+      const int tau_hi = min(j >> rsh, rtiles_u - 1);
+      const int tau_lo = max(0, (j - a.nbt + (1 << rsh)) >> rsh);
+      for (int tau = tau_lo; tau <= tau_hi; ++tau) {
+        const int jl = j - (tau << rsh);
+        if (jl >= 0 && jl < a.nbt) v += tsum[tau * 16 + jl];
+      }
+      keys[j] = sel_key(v, j);
     }
   } else {
     for (int x = tid; x < G * D; x += SEL_THREADS) oacc[x] = 0.f;
+    for (int j = tid; j < ncand; j += SEL_THREADS) keys[j] = sel_key(0.f, j);
   }
+  if (tid == 0) nsel_s = 0;
   __syncthreads();
 
-  // top-n: block 0 kept, the best n-1 others (ties to the lower index)
+  // top-n: block 0 kept, the best n-1 others (ties to the lower index). The
+  // (n-1)-th largest key among blocks 1..ncand-1 is found by radix selection
+  // on 8-bit digits (keys are unique); every key at or above it is kept.
   int ns;
   if (ncand <= a.n) {
     for (int j = tid; j < ncand; j += SEL_THREADS) sel[j] = j;
     ns = ncand;
-  } else {
+  } else if (a.n == 1) {
     if (tid == 0) sel[0] = 0;
-    for (int r = 1; r < a.n; ++r) {
-      float bs = -INFINITY;
-      int bj = INT_MAX;
+    ns = 1;
+  } else {
+    int need = a.n - 1;
+    unsigned long long prefix = 0ull, mask = 0ull;
+    for (int shift = 56; shift >= 0; shift -= 8) {
+      if (tid < 256) hist[tid] = 0u;
+      __syncthreads();
       for (int j = 1 + tid; j < ncand; j += SEL_THREADS) {
-        const float sj = scores[j];
-        if (sj != -INFINITY && sel_better(sj, j, bs, bj)) {
-          bs = sj;
-          bj = j;
-        }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float os = __shfl_xor_sync(0xffffffffu, bs, o);
-        const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
-        if (sel_better(os, oj, bs, bj)) {
-          bs = os;
-          bj = oj;
-        }
-      }
-      if (lane == 0) {
-        red_s[warp] = bs;
-        red_j[warp] = bj;
+        const unsigned long long k = keys[j];
+        if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
       }
       __syncthreads();
       if (warp == 0) {
-        float s0 = lane < SEL_THREADS / 32 ? red_s[lane] : -INFINITY;
-        int j0 = lane < SEL_THREADS / 32 ? red_j[lane] : INT_MAX;
+        // lane l holds bins 255-8l .. 248-8l (descending)
+        unsigned c[8], tot = 0;
 #pragma unroll
-        for (int o = 4; o > 0; o >>= 1) {
-          const float os = __shfl_xor_sync(0xffffffffu, s0, o);
-          const int oj = __shfl_xor_sync(0xffffffffu, j0, o);
-          if (sel_better(os, oj, s0, j0)) {
-            s0 = os;
-            j0 = oj;
-          }
+        for (int i = 0; i < 8; ++i) {
+          c[i] = hist[255 - 8 * lane - i];
+          tot += c[i];
         }
-        if (lane == 0) {
-          sel[r] = j0;
-          scores[j0] = -INFINITY;
+        unsigned incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const unsigned y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        const unsigned excl = incl - tot;
+        const bool here = excl < (unsigned)need && (unsigned)need <= incl;
+        if (here) {
+          unsigned cum = excl;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            if (cum + c[i] >= (unsigned)need) {
+              cut_bin = 255 - 8 * lane - i;
+              cut_above = (int)cum;
+              break;
+            }
+            cum += c[i];
+          }
         }
       }
       __syncthreads();
+      const int d = cut_bin;
+      need -= cut_above;
+      prefix |= (unsigned long long)d << shift;
+      mask |= 255ull << shift;
+      if ((int)hist[d] == need) break;  // all of bin d is kept
+      __syncthreads();
     }
-    if (tid == 0) {
-      for (int x = 1; x < a.n; ++x) {
-        const int v = sel[x];
-        int p = x - 1;
-        while (p >= 0 && sel[p] > v) {
-          sel[p + 1] = sel[p];
-          --p;
-        }
-        sel[p + 1] = v;
-      }
+    // keys >= prefix are exactly the n-1 kept blocks
+    for (int j = 1 + tid; j < ncand; j += SEL_THREADS)
+      if (keys[j] >= prefix) sel[1 + atomicAdd(&nsel_s, 1)] = j;
+    if (tid == 0) sel[0] = 0;
+    __syncthreads();
+    // ascending order: each entry's rank among the n kept
+    if (tid < a.n) {
+      const int v = sel[tid];
+      int rank = 0;
+      for (int k = 0; k < a.n; ++k) rank += sel[k] < v;
+      hist[rank] = (unsigned)v;  // hist is free: reuse as the sorted list
     }
+    __syncthreads();
+    if (tid < a.n) sel[tid] = (int)hist[tid];
     ns = a.n;
   }
   __syncthreads();
@@ -739,75 +974,35 @@ __global__ void __launch_bounds__(SEL_THREADS) dec_select_kernel(const __grid_co
 // dec_combine
 // ---------------------------------------------------------------------------
 
-__global__ void __launch_bounds__(128) dec_combine_kernel(const __grid_constant__ DecFastArgs a) {
+constexpr int CMB_THREADS = 256;
+
+__global__ void __launch_bounds__(CMB_THREADS) dec_combine_kernel(const __grid_constant__ DecFastArgs a) {
   const int u = blockIdx.x, b = u / a.Hkv, g = u - b * a.Hkv;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  __shared__ long long red[8];
-  __shared__ int crange[4];
-  const int L = a.seq_lens[b];
+  const int tid = threadIdx.x;
+  __shared__ float mS[G], lS[G], sR[G], scl[2][G];
+  __shared__ __align__(16) float pm[MP * G], pl[MP * G];
+  const int L = __ldg(a.seq_lens + b);
   if (!len_ok(L, a)) return;  // output zeroed by dec_select
-  const int ns = n_selected(L, a);
-  const int nw = (min(a.w, L) + TK - 1) / TK;
-  long long total = 0, before = 0;
-  for (int bb = tid; bb < a.B; bb += 128) {
-    const long long nt = (long long)unit_tiles<MODE_SW>(a.seq_lens[bb], a) * a.Hkv;
-    total += nt;
-    if (bb < b) before += nt;
+  const int4 rg = *reinterpret_cast<const int4*>(a.rng3 + (long)u * 4);  // written by dec_sel_win
+  const int h = tid >> 4, e0 = (tid & 15) * 8;
+  float acc[8];
+  {
+    const float4* oc = reinterpret_cast<const float4*>(a.oacc + (long)u * G * D + h * D + e0);
+    const float4 v0 = oc[0], v1 = oc[1];
+    acc[0] = v0.x; acc[1] = v0.y; acc[2] = v0.z; acc[3] = v0.w;
+    acc[4] = v1.x; acc[5] = v1.y; acc[6] = v1.z; acc[7] = v1.w;
   }
-  for (int o = 16; o > 0; o >>= 1) {
-    total += __shfl_xor_sync(0xffffffffu, total, o);
-    before += __shfl_xor_sync(0xffffffffu, before, o);
-  }
-  if (lane == 0) {
-    red[2 * warp] = total;
-    red[2 * warp + 1] = before;
-  }
-  __syncthreads();
-  if (tid == 0) {
-    long long T0 = 0, P0 = 0;
-    for (int w = 0; w < 4; ++w) {
-      T0 += red[2 * w];
-      P0 += red[2 * w + 1];
-    }
-    const long long Pu = P0 + (long long)g * (ns + nw);
-    crange[0] = owner_cta(Pu, T0, a.grid3);
-    crange[1] = owner_cta(Pu + ns - 1, T0, a.grid3);
-    crange[2] = owner_cta(Pu + ns, T0, a.grid3);
-    crange[3] = owner_cta(Pu + ns + nw - 1, T0, a.grid3);
-  }
-  __syncthreads();
-  const int h = tid >> 3, e0 = (tid & 7) * 16;
-  float res[16];
-  const float* oc = a.oacc + (long)u * G * D + h * D + e0;
-#pragma unroll
-  for (int e = 0; e < 16; ++e) res[e] = oc[e];
-#pragma unroll
-  for (int br = 0; br < 2; ++br) {
-    const int seg = 2 * u + br;
-    const int c0 = crange[2 * br], c1 = crange[2 * br + 1];
-    float M = -INFINITY;
-    for (int cc = c0; cc <= c1; ++cc) M = fmaxf(M, a.part3[(long)(cc + seg) * PART + h]);
-    float Ls = 0.f;
-    float acc[16];
-#pragma unroll
-    for (int e = 0; e < 16; ++e) acc[e] = 0.f;
-    for (int cc = c0; cc <= c1; ++cc) {
-      const float* pp = a.part3 + (long)(cc + seg) * PART;
-      const float mm = pp[h];
-      const float f = mm == -INFINITY ? 0.f : exp2f(mm - M);
-      Ls += f * pp[G + h];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) acc[e] += f * pp[2 * G + h * D + e0 + e];
-    }
-    const float gs = a.gates[(long)u * 3 * G + h * 3 + 1 + br] / Ls;
-#pragma unroll
-    for (int e = 0; e < 16; ++e) res[e] += gs * acc[e];
-  }
+  if (tid < 2 * G) scl[tid >> 4][tid & 15] = a.gates[(long)u * 3 * G + (tid & 15) * 3 + 1 + (tid >> 4)];
+  // selected branch (segment 2u), then window branch (segment 2u + 1)
+  merge_online<CMB_THREADS>(a.part3, 2 * ((long long)rg.x + 2 * u), 2 * (rg.y - rg.x + 1), scl[0],
+                            pm, pl, mS, lS, sR, h, e0, acc);
+  merge_online<CMB_THREADS>(a.part3, 2 * ((long long)rg.z + 2 * u + 1), 2 * (rg.w - rg.z + 1),
+                            scl[1], pm, pl, mS, lS, sR, h, e0, acc);
   __nv_bfloat16* orow =
       reinterpret_cast<__nv_bfloat16*>(a.out) + ((long)b * a.Hq + g * G + h) * D + e0;
 #pragma unroll
-  for (int e = 0; e < 16; e += 2)
-    *reinterpret_cast<__nv_bfloat162*>(orow + e) = __floats2bfloat162_rn(res[e], res[e + 1]);
+  for (int e = 0; e < 8; e += 2)
+    *reinterpret_cast<__nv_bfloat162*>(orow + e) = __floats2bfloat162_rn(acc[e], acc[e + 1]);
 }
 
 // ---------------------------------------------------------------------------
@@ -816,20 +1011,33 @@ __global__ void __launch_bounds__(128) dec_combine_kernel(const __grid_constant_
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// True the first time kernel `id` is launched on the current device.
+bool first_use(int id) {
+  static bool seen[2][64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return true;
+  const bool f = !seen[id][dev];
+  seen[id][dev] = true;
+  return f;
+}
+
 struct WsLayout {
-  size_t part1, trec, oacc, gates, sel, part3, total;
+  size_t part1, trec, oacc, gates, sel, part3, rng1, rng3, total;
 };
 
 WsLayout ws_layout(const DecFastArgs& a) {
   WsLayout w{};
   const size_t units = (size_t)a.B * a.Hkv;
   size_t off = 0;
-  w.part1 = off; off = align256(off + (size_t)(a.grid1 + units) * PART * 4);
+  w.part1 = off; off = align256(off + 2 * (size_t)(a.grid1 + units) * PART * 4);
   w.trec = off; off = align256(off + units * a.tiles_max * G * (1 + a.nbt) * 4);
   w.oacc = off; off = align256(off + units * G * D * 4);
   w.gates = off; off = align256(off + units * 3 * G * 4);
   w.sel = off; off = align256(off + units * a.n * 4);
-  w.part3 = off; off = align256(off + (size_t)(a.grid3 + 2 * units) * PART * 4);
+  w.part3 = off; off = align256(off + 2 * (size_t)(a.grid3 + 2 * units) * PART * 4);
+  w.rng1 = off; off = align256(off + units * 2 * 4);
+  w.rng3 = off; off = align256(off + units * 4 * 4);
   w.total = off;
   return w;
 }
@@ -846,21 +1054,21 @@ DecFastArgs base_args(const nsa_params& p) {
   a.n = p.top_n;
   a.w = p.window;
   a.Nc = nsa_num_cmp_blocks(p.T, p.cmp_block, p.cmp_stride);
-  a.nbt = (63 * a.s + a.l - 1) / a.bs + 2;
-  a.tiles_max = (a.Nc + TK - 1) / TK;
+  a.nbt = ((WK - 1) * a.s + a.l - 1) / a.bs + 2;
+  a.r_shift = 0;
+  while ((1 << a.r_shift) < (WK * a.s) / a.bs) ++a.r_shift;
+  a.tiles_max = (a.Nc + WK - 1) / WK;  // 32-key record sub-tiles
   for (int jl = 0; jl < a.nbt && jl < kDecMaxNbt; ++jl) {
-    // keys of a 64-key tile (relative index) overlapping its jl-th block
+    // keys of a 32-key sub-tile (relative index) overlapping its jl-th block
     const int num = jl * a.bs - a.l + 1;
     const int lo = num <= 0 ? 0 : (num + a.s - 1) / a.s;
-    const int hi = std::min(TK - 1, (jl * a.bs + a.bs - 1) / a.s);
+    const int hi = std::min(WK - 1, (jl * a.bs + a.bs - 1) / a.s);
     a.klo[jl] = (int8_t)std::min(lo, 127);
     a.khi[jl] = (int8_t)hi;
   }
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  a.grid1 = sms;
-  a.grid3 = sms;
+  const int sms = device_sm_count();
+  a.grid1 = sms * NPAIR;  // tile streams: one per consumer pair
+  a.grid3 = sms * NPAIR;
   const float scale = p.softmax_scale != 0.f ? p.softmax_scale : 1.f / sqrtf((float)p.d);
   a.scale_log2 = scale * 1.4426950408889634f;
   a.gate_mode = p.gate_mode;
@@ -868,19 +1076,20 @@ DecFastArgs base_args(const nsa_params& p) {
   return a;
 }
 
-constexpr size_t kStreamSmem =
-    1024 + SLOTS * SLOT_BYTES + MERGE_FLOATS * 4 + 2 * SLOTS * 8 + sizeof(Plan) + 16;
 
 }  // namespace
 
 bool decode_fast_eligible(const nsa_params& p) {
   if (!(p.dtype == NSA_DTYPE_BF16 && p.d == D && p.Hq == G * p.Hkv && p.sel_block == TK &&
-        p.top_n <= 256 && p.T >= 1))
+        p.top_n <= MAXSEL && p.T >= 1 && (p.T + p.sel_block - 1) / p.sel_block <= MAXCAND))
     return false;
-  // 64-key compressed tiles must start on selection-block boundaries
-  if ((TK * p.cmp_stride) % p.sel_block != 0) return false;
-  const int nbt = (63 * p.cmp_stride + p.cmp_block - 1) / p.sel_block + 2;
-  return nbt <= kDecMaxNbt;
+  // 32-key compressed sub-tiles must start on selection-block boundaries, a
+  // power-of-two number of blocks apart
+  if ((WK * p.cmp_stride) % p.sel_block != 0) return false;
+  const int R = (WK * p.cmp_stride) / p.sel_block;
+  if ((R & (R - 1)) != 0) return false;
+  const int nbt = ((WK - 1) * p.cmp_stride + p.cmp_block - 1) / p.sel_block + 2;
+  return nbt <= 16 && nbt <= kDecMaxNbt;
 }
 
 size_t decode_fast_ws_bytes(const nsa_params& p) {
@@ -907,6 +1116,8 @@ cudaError_t launch_decode_fast(const nsa_params& p, const void* q, const void* k
   a.gates = reinterpret_cast<float*>(w + L.gates);
   a.sel = reinterpret_cast<int*>(w + L.sel);
   a.part3 = reinterpret_cast<float*>(w + L.part3);
+  a.rng1 = reinterpret_cast<int*>(w + L.rng1);
+  a.rng3 = reinterpret_cast<int*>(w + L.rng3);
 
   CUtensorMap tkc, tvc, tk, tv;
   const uint64_t rows = (uint64_t)p.B * p.T;
@@ -923,30 +1134,37 @@ cudaError_t launch_decode_fast(const nsa_params& p, const void* q, const void* k
   cudaError_t e;
   if (a.Nc > 0) {
     TraceScope trace("dec_cmp_partial", stream);
-    cudaFuncSetAttribute(dec_stream_kernel<MODE_CMP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)kStreamSmem);
-    dec_stream_kernel<MODE_CMP><<<a.grid1, 160, kStreamSmem, stream>>>(a, tkc, tvc);
+    constexpr size_t smem = StreamCfg<MODE_CMP>::SMEM;
+    if (first_use(0))
+      cudaFuncSetAttribute(dec_stream_kernel<MODE_CMP>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    dec_stream_kernel<MODE_CMP><<<a.grid1 / NPAIR, (NCW + 1) * 32, smem, stream>>>(a, tkc, tvc);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   {
     const int nblk = (p.T + p.sel_block - 1) / p.sel_block;
-    const size_t smem = (size_t)(32 + G + 3 * G + a.tiles_max * G + nblk + 8) * 4 + 8 * 4 +
-                        (size_t)a.n * 4 + 16;
+    int npow = 1;
+    while (npow < nblk) npow <<= 1;
+    const size_t smem = (size_t)a.tiles_max * G * (1 + a.nbt) * 4 + (size_t)npow * 8 +
+                        2 * (size_t)a.tiles_max * G * 4 + 16;
     TraceScope trace("dec_select", stream);
-    cudaFuncSetAttribute(dec_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (smem > 48 * 1024)
+      cudaFuncSetAttribute(dec_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     dec_select_kernel<<<p.B * p.Hkv, SEL_THREADS, smem, stream>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   {
     TraceScope trace("dec_sel_win", stream);
-    cudaFuncSetAttribute(dec_stream_kernel<MODE_SW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)kStreamSmem);
-    dec_stream_kernel<MODE_SW><<<a.grid3, 160, kStreamSmem, stream>>>(a, tk, tv);
+    constexpr size_t smem = StreamCfg<MODE_SW>::SMEM;
+    if (first_use(1))
+      cudaFuncSetAttribute(dec_stream_kernel<MODE_SW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
+    dec_stream_kernel<MODE_SW><<<a.grid3 / NPAIR, (NCW + 1) * 32, smem, stream>>>(a, tk, tv);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   {
     TraceScope trace("dec_combine", stream);
-    dec_combine_kernel<<<p.B * p.Hkv, 128, 0, stream>>>(a);
+    dec_combine_kernel<<<p.B * p.Hkv, CMB_THREADS, 0, stream>>>(a);
     return cudaGetLastError();
   }
 }

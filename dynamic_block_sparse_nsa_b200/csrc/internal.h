@@ -62,20 +62,23 @@ struct DecFastArgs {
   int32_t* sel_out;
   unsigned* err;
   int B, T, Hq, Hkv, Nc, l, s, bs, n, w;
-  int nbt;        // selection blocks one 64-key compressed tile can overlap (bound)
+  int nbt;        // selection blocks one 32-key compressed sub-tile can overlap (bound)
+  int r_shift;    // log2 of the selection blocks between sub-tile starts
   int tiles_max;  // 64-key compressed tiles per sequence at capacity T
-  int grid1;      // CTAs of the compressed-branch stream kernel
-  int grid3;      // CTAs of the selected/window stream kernel
+  int grid1;      // tile streams (CTAs x consumer pairs) of the compressed-branch kernel
+  int grid3;      // tile streams of the selected/window kernel
   float scale_log2;
   int gate_mode;
   float fixed_gates[3];
   int8_t klo[kDecMaxNbt], khi[kDecMaxNbt];  // per block of a tile: its key range
-  float* part1;   // compressed-branch partials, slot = cta + unit
+  float* part1;   // compressed-branch partials, slot = 2 * (stream + unit) + half
   float* trec;    // per-tile block-score records
   float* oacc;    // g0 * o_cmp per unit
   float* gates;   // per unit [16][3]
   int* sel;       // per unit [n]
-  float* part3;   // selected / window partials, slot = cta + 2 * unit + branch
+  float* part3;   // selected / window partials, slot = 2 * (stream + 2 * unit + branch) + half
+  int* rng1;      // per unit: first/last stream of its compressed tiles
+  int* rng3;      // per unit: first/last stream of its selected and window tiles
 };
 
 bool decode_fast_eligible(const nsa_params& p);
@@ -94,6 +97,9 @@ struct TraceScope {
   TraceScope(const char* name, cudaStream_t st) : s(st) { trace_begin(name, st); }
   ~TraceScope() { trace_end(s); }
 };
+
+// Multiprocessor count of the current device (cached per device).
+int device_sm_count();
 
 // 3-D TMA map over a contiguous bf16 array [dim2][dim1][dim0] with a box of
 // (box0, box1, box2) elements; false if the driver rejects it.

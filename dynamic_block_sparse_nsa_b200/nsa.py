@@ -29,7 +29,8 @@ _TORCH_DTYPE = {DTYPE_F32: torch.float32, DTYPE_BF16: torch.bfloat16}
 EXPORTS = (
     "nsa_workspace_size", "nsa_num_cmp_blocks", "nsa_compress_kv", "nsa_prefill", "nsa_decode",
     "moba_prefill", "nsa_check", "nsa_debug_bounded_wait", "nsa_status_string",
-    "nsa_last_error_detail", "nsa_trace_enable", "nsa_trace_count", "nsa_trace_get",
+    "nsa_last_error_detail", "nsa_trace_enable", "nsa_trace_set_filter", "nsa_trace_count",
+    "nsa_trace_timed", "nsa_trace_get",
 )
 
 
@@ -73,6 +74,8 @@ def _load():
         "nsa_last_error_detail": [],
         "nsa_trace_enable": [ctypes.c_int, ctypes.c_int],
         "nsa_trace_count": [],
+        "nsa_trace_timed": [],
+        "nsa_trace_set_filter": [ctypes.c_char_p],
         "nsa_trace_get": [ctypes.c_int, ctypes.POINTER(ctypes.c_char_p),
                           ctypes.POINTER(ctypes.c_float)],
     }
@@ -230,7 +233,9 @@ def status_of_check(stream=None):
     return LIB.nsa_check(_stream(stream))
 
 
-def trace_enable(on=True, capacity=4096):
+def trace_enable(on=True, capacity=4096, only=None):
+    """Bracket launches with CUDA events; `only`: a kernel-name prefix to time."""
+    _raise(LIB.nsa_trace_set_filter(only.encode() if only else None))
     _raise(LIB.nsa_trace_enable(1 if on else 0, capacity))
 
 
@@ -238,7 +243,7 @@ def trace_records():
     """[(kernel name, device ms)] of the launches traced since trace_enable."""
     out = []
     n = LIB.nsa_trace_count()
-    for i in range(n):
+    for i in range(LIB.nsa_trace_timed()):
         name, ms = ctypes.c_char_p(), ctypes.c_float()
         if LIB.nsa_trace_get(i, ctypes.byref(name), ctypes.byref(ms)) != NSA_OK:
             break

@@ -167,11 +167,20 @@ NSA_API nsa_status nsa_debug_bounded_wait(const int32_t* flag, int max_iters, vo
  * creates none. Not for concurrent use from several host threads. */
 NSA_API nsa_status nsa_trace_enable(int on, int capacity);
 
+/* Restrict event brackets to kernels whose name starts with `prefix` (NULL or
+ * "" = every kernel). Every launch is still counted. Events between kernels
+ * delay the next launch slightly, so timing only the kernel of interest keeps
+ * the rest of the timeline undisturbed. */
+NSA_API nsa_status nsa_trace_set_filter(const char* prefix);
+
 /* Number of launches since the trace was enabled (including untimed ones). */
 NSA_API int nsa_trace_count(void);
 
-/* Name and device duration (ms) of traced launch i (synchronises on its stop
- * event). Returns NSA_ERR_INVALID_ARGUMENT for i out of range. */
+/* Number of launches bracketed with events (see nsa_trace_set_filter). */
+NSA_API int nsa_trace_timed(void);
+
+/* Name and device duration (ms) of timed launch i (0 <= i < nsa_trace_timed();
+ * synchronises on its stop event). NSA_ERR_INVALID_ARGUMENT when out of range. */
 NSA_API nsa_status nsa_trace_get(int i, const char** name, float* ms);
 
 /* Static description of a status code. */
