@@ -311,7 +311,8 @@ struct Walker {
 constexpr int LENS_CAP = 1024;  // sequence lengths kept in shared memory
 
 // Plans of the NS streams of this CTA (computed by one warp). Stream
-// v = cta * NS + i owns global tiles [total*v/V, total*(v+1)/V). `pre` is
+// v = cta * NS + i owns global tiles [total*v/V, total*(v+1)/V), where
+// V = min(all streams, total) (streams v >= V are idle). `pre` is
 // scratch for the per-sequence prefix of tile counts (cap entries); `lens_s`
 // receives a copy of the lengths when B <= LENS_CAP.
 template <int MODE, int NS>
@@ -336,10 +337,12 @@ __device__ void make_plans(const DecFastArgs& a, StreamPlan* plans, int* lens_s,
   }
   __syncwarp();
   const long long total = carry;
-  const long long V = (long long)gridDim.x * NS;
+  // At most one stream per tile: then every stream owns at least one tile, so
+  // the streams between a segment's first and last owner all wrote partials.
+  const long long V = min((long long)gridDim.x * NS, total);
   if (lane < NS) {
     const long long v = (long long)blockIdx.x * NS + lane;
-    const long long t0 = total * v / V, t1 = total * (v + 1) / V;
+    const long long t0 = v < V ? total * v / V : 0, t1 = v < V ? total * (v + 1) / V : 0;
     StreamPlan p{};
     p.len = (int)(t1 - t0);
     p.ntiles = 1;
@@ -743,6 +746,17 @@ constexpr int SEL_THREADS = 512;
 constexpr int SEL_WARPS = SEL_THREADS / 32;
 constexpr int MAXSEL = 64;       // top_n bound of the fast path
 constexpr int MAXCAND = 4096;    // selection blocks bound of the fast path (T <= 262144)
+constexpr size_t kSelDynSmemMax = 192 * 1024;  // dec_select dynamic shared memory (+ ~18 KB static)
+
+// Dynamic shared memory of dec_select: the unit's score records, the sort keys,
+// and two per-(sub-tile, head) arrays.
+__host__ __device__ inline size_t sel_dyn_smem(int T, int sel_block, int tiles_max, int nbt) {
+  const int nblk = (T + sel_block - 1) / sel_block;
+  int npow = 1;
+  while (npow < nblk) npow <<= 1;
+  return (size_t)tiles_max * 16 * (1 + nbt) * 4 + (size_t)npow * 8 + 2 * (size_t)tiles_max * 16 * 4 +
+         16;
+}
 
 // Sort key of a candidate block: higher score first, then the lower index.
 // Scores are >= 0, so their IEEE bits order like the values; the low word is
@@ -1013,7 +1027,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // True the first time kernel `id` is launched on the current device.
 bool first_use(int id) {
-  static bool seen[2][64] = {};
+  static bool seen[3][64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return true;
@@ -1089,7 +1103,10 @@ bool decode_fast_eligible(const nsa_params& p) {
   const int R = (WK * p.cmp_stride) / p.sel_block;
   if ((R & (R - 1)) != 0) return false;
   const int nbt = ((WK - 1) * p.cmp_stride + p.cmp_block - 1) / p.sel_block + 2;
-  return nbt <= 16 && nbt <= kDecMaxNbt;
+  if (nbt > 16 || nbt > kDecMaxNbt) return false;
+  // dec_select keeps a whole unit's score records in shared memory
+  const int Nc = nsa_num_cmp_blocks(p.T, p.cmp_block, p.cmp_stride);
+  return sel_dyn_smem(p.T, p.sel_block, (Nc + WK - 1) / WK, nbt) <= kSelDynSmemMax;
 }
 
 size_t decode_fast_ws_bytes(const nsa_params& p) {
@@ -1142,14 +1159,11 @@ cudaError_t launch_decode_fast(const nsa_params& p, const void* q, const void* k
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   {
-    const int nblk = (p.T + p.sel_block - 1) / p.sel_block;
-    int npow = 1;
-    while (npow < nblk) npow <<= 1;
-    const size_t smem = (size_t)a.tiles_max * G * (1 + a.nbt) * 4 + (size_t)npow * 8 +
-                        2 * (size_t)a.tiles_max * G * 4 + 16;
+    const size_t smem = sel_dyn_smem(p.T, p.sel_block, a.tiles_max, a.nbt);
     TraceScope trace("dec_select", stream);
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(dec_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (first_use(2))
+      cudaFuncSetAttribute(dec_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kSelDynSmemMax);
     dec_select_kernel<<<p.B * p.Hkv, SEL_THREADS, smem, stream>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }

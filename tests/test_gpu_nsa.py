@@ -102,3 +102,24 @@ def test_decode_repeat_is_deterministic(cuda_ok):
     nsa.nsa_check()
     for o, s in outs[1:]:
         assert torch.equal(o, outs[0][0]) and torch.equal(s, outs[0][1])
+
+
+def test_decode_independent_of_stale_workspace(cuda_ok):
+    # Workspace contents left by an earlier call (another shape) must not leak
+    # into a later one: fill the workspace with garbage and compare.
+    from dynamic_block_sparse_nsa_b200 import nsa
+    w = inputs.workload("nsa_decode_bf16_b32_l65536", B=6, T=12000)
+    inp = inputs.make_decode(w, seed=11, seq_lens=[12000, 9000, 4097, 777, 64, 11999])
+    p = gc.nsa_params_for(w)
+    dev = {k_: v_.cuda() for k_, v_ in inp.items()}
+    kc, vc = nsa.nsa_compress_kv(p, dev["k"], dev["v"], dev["w_cmp"])
+    outs = []
+    for fill in (0, 0x7f, 0x3c):
+        ws = nsa.workspace(p, nsa.OP_DECODE)
+        ws.fill_(fill)
+        outs.append(nsa.nsa_decode(p, dev["q"], dev["k"], dev["v"], dev["seq_lens"], kc, vc,
+                                   dev["w_gate"], ws=ws))
+    nsa.nsa_check()
+    for o, s in outs[1:]:
+        assert torch.equal(o, outs[0][0]) and torch.equal(s, outs[0][1])
+    gc.run_nsa_decode(w, [12000, 9000, 4097, 777, 64, 11999], seed=11)
