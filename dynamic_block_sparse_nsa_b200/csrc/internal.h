@@ -98,6 +98,9 @@ struct TraceScope {
   ~TraceScope() { trace_end(s); }
 };
 
+// Record `msg` as this host thread's error detail (nsa_last_error_detail).
+void set_last_error(nsa_status s, const char* msg);
+
 // Multiprocessor count of the current device (cached per device).
 int device_sm_count();
 

@@ -133,6 +133,9 @@ nsa_status check_workspace(void* ws, size_t have, size_t need) {
 }
 
 }  // namespace
+
+void set_last_error(nsa_status, const char* msg) { g_detail = msg ? msg : ""; }
+
 }  // namespace nsa
 
 using namespace nsa;

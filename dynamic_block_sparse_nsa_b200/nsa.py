@@ -28,7 +28,7 @@ _TORCH_DTYPE = {DTYPE_F32: torch.float32, DTYPE_BF16: torch.bfloat16}
 # Every symbol include/nsa.h declares.
 EXPORTS = (
     "nsa_workspace_size", "nsa_num_cmp_blocks", "nsa_compress_kv", "nsa_prefill", "nsa_decode",
-    "moba_prefill", "nsa_check", "nsa_debug_bounded_wait", "nsa_status_string",
+    "moba_prefill", "nsa_decode_noalloc", "nsa_check", "nsa_debug_bounded_wait", "nsa_status_string",
     "nsa_last_error_detail", "nsa_trace_enable", "nsa_trace_set_filter", "nsa_trace_count",
     "nsa_trace_timed", "nsa_trace_get",
 )
@@ -68,6 +68,7 @@ def _load():
         "nsa_prefill": [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
         "nsa_decode": [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
         "moba_prefill": [P, vp, vp, vp, vp, vp, vp, sz, vp],
+        "nsa_decode_noalloc": [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
         "nsa_check": [vp],
         "nsa_debug_bounded_wait": [vp, ctypes.c_int, vp],
         "nsa_status_string": [ctypes.c_int],
@@ -204,6 +205,30 @@ def nsa_decode(p, q, k_cache, v_cache, seq_lens, k_cmp, v_cmp, w_gate=None, out=
     _raise(LIB.nsa_decode(ctypes.byref(p), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens),
                           _ptr(k_cmp), _ptr(v_cmp), _ptr(w_gate), _ptr(out), _ptr(sel_idx),
                           _ptr(ws), nbytes, _stream(stream)))
+    return out, sel_idx
+
+
+def nsa_decode_noalloc(p, q, k_cache, v_cache, seq_lens, k_cmp, v_cmp, w_gate=None, out=None,
+                       sel_idx=None, stream=None, want_sel=True):
+    """nsa_decode with the library's static scratch instead of a workspace, for
+    callers that cannot allocate device memory (include/nsa.h gives the limits;
+    calls must not overlap on the GPU). The C call allocates nothing; this
+    wrapper allocates `out` / `sel_idx` only when they are not given."""
+    dt = p.torch_dtype
+    for t, nm in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"), (k_cmp, "k_cmp"),
+                  (v_cmp, "v_cmp")):
+        _dev(t, nm, dt)
+    _dev(seq_lens, "seq_lens", torch.int32)
+    _dev(w_gate, "w_gate", torch.float32)
+    if out is None:
+        out = torch.empty(p.B, p.Hq, p.d, dtype=dt, device=q.device)
+    if sel_idx is None and want_sel:
+        sel_idx = torch.empty(p.B, p.Hkv, p.top_n, dtype=torch.int32, device=q.device)
+    _dev(out, "out", dt)
+    _dev(sel_idx, "sel_idx", torch.int32)
+    _raise(LIB.nsa_decode_noalloc(ctypes.byref(p), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                  _ptr(seq_lens), _ptr(k_cmp), _ptr(v_cmp), _ptr(w_gate),
+                                  _ptr(out), _ptr(sel_idx), _stream(stream)))
     return out, sel_idx
 
 

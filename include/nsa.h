@@ -137,6 +137,31 @@ NSA_API nsa_status nsa_decode(const nsa_params* p, const void* q, const void* k_
                       const void* v_cmp, const float* w_gate, void* out, int32_t* sel_idx,
                       void* workspace, size_t ws_bytes, void* stream);
 
+/* nsa_decode without a workspace argument, for callers that cannot allocate
+ * device memory: code that runs while a stream capture is in progress
+ * (cudaMalloc is not permitted during a global-mode capture), real-time or
+ * callback threads that must not block in an allocator, and hosts whose device
+ * memory is owned by another runtime's pool. Nothing here states whether the
+ * call itself can be captured into a graph.
+ * The sources describe no such call; it has no counterpart in the method.
+ *   Same arguments and results as nsa_decode, minus workspace / ws_bytes. The
+ *   scratch is a static 64 MiB device array in this library, held on every GPU
+ *   that loads it until the process exits. Shapes whose decode scratch
+ *   (nsa_workspace_size(NSA_OP_DECODE)) exceeds 64 MiB are rejected with
+ *   NSA_ERR_UNSUPPORTED before anything runs (32 sequences of 65536 tokens
+ *   with 4 KV heads need about 39 MB).
+ *   The first call on each device looks the scratch's address up (once, with
+ *   that device current); make that first call before any stream capture.
+ *   All calls share the one scratch: calls that overlap on the GPU (different
+ *   streams, no ordering) race and corrupt each other's results. Nothing in
+ *   it must start at zero: every call writes each scratch byte it reads.
+ *   No device memory is allocated or freed, by this call or any library
+ *   routine it uses. */
+NSA_API nsa_status nsa_decode_noalloc(const nsa_params* p, const void* q, const void* k_cache,
+                                      const void* v_cache, const int32_t* seq_lens,
+                                      const void* k_cmp, const void* v_cmp, const float* w_gate,
+                                      void* out, int32_t* sel_idx, void* stream);
+
 /* MoBA causal prefill (EP94 notes §九/§十).
  *   q [B, T, Hq, d]; k, v [B, T, Hkv, d]; out [B, T, Hq, d].
  *   Block m = sel_block; each (token t, head h) keeps its own block t/m and the
