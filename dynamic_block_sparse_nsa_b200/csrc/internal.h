@@ -88,6 +88,14 @@ cudaError_t launch_decode_fast(const nsa_params& p, const void* q, const void* k
                                const float* w_gate, void* out, int32_t* sel_out, void* ws,
                                unsigned* err, cudaStream_t stream);
 
+// Tensor-core prefill: bf16, d = 128, 16 query heads per KV head, l = 32,
+// s = 16, selection block 64, top_n <= 16.
+bool prefill_tc_eligible(const nsa_params& p);
+size_t prefill_tc_ws_bytes(const nsa_params& p);
+cudaError_t launch_prefill_tc(const nsa_params& p, const void* q, const void* k, const void* v,
+                              const void* kc, const void* vc, const float* w_gate, void* out,
+                              int32_t* sel_out, void* ws, unsigned* err, cudaStream_t stream);
+
 // Kernel trace: bracket a launch with events when tracing is on.
 void trace_begin(const char* name, cudaStream_t stream);
 void trace_end(cudaStream_t stream);

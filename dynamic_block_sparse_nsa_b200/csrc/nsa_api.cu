@@ -152,11 +152,16 @@ nsa_status nsa_workspace_size(const nsa_params* p, int op, size_t* bytes) {
   if (!bytes) return fail(NSA_ERR_INVALID_ARGUMENT, "bytes is NULL");
   *bytes = 0;
   switch (op) {
-    case NSA_OP_COMPRESS:
-    case NSA_OP_PREFILL: {
+    case NSA_OP_COMPRESS: {
       nsa_status s = check_nsa(p);
       if (s != NSA_OK) return s;
       *bytes = 0;
+      return NSA_OK;
+    }
+    case NSA_OP_PREFILL: {
+      nsa_status s = check_nsa(p);
+      if (s != NSA_OK) return s;
+      *bytes = prefill_tc_eligible(*p) ? prefill_tc_ws_bytes(*p) : 0;
       return NSA_OK;
     }
     case NSA_OP_DECODE: {
@@ -200,10 +205,15 @@ nsa_status nsa_prefill(const nsa_params* p, const void* q, const void* k, const 
     return fail(NSA_ERR_INVALID_ARGUMENT, "q, k, v, k_cmp, v_cmp, out must be non-NULL");
   if (p->gate_mode == 0 && !w_gate)
     return fail(NSA_ERR_INVALID_ARGUMENT, "w_gate must be non-NULL when gate_mode == 0");
-  (void)workspace;
-  (void)ws_bytes;
   unsigned* err = err_word(&s);
   if (!err) return s;
+  if (prefill_tc_eligible(*p)) {
+    s = check_workspace(workspace, ws_bytes, prefill_tc_ws_bytes(*p));
+    if (s != NSA_OK) return s;
+    cudaError_t e = launch_prefill_tc(*p, q, k, v, k_cmp, v_cmp, w_gate, out, sel_idx, workspace,
+                                      err, (cudaStream_t)stream);
+    return e == cudaSuccess ? NSA_OK : cuda_fail(e, "prefill launch");
+  }
   NsaRowArgs a = row_args(p);
   a.q = q; a.k = k; a.v = v; a.kc = k_cmp; a.vc = v_cmp;
   a.w_gate = w_gate; a.out = out; a.sel_idx = sel_idx; a.err = err; a.decode = 0;

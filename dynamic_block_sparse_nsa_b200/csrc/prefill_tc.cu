@@ -1,0 +1,956 @@
+// NSA causal prefill on the sm_100a tensor cores (tcgen05 MMAs with TMEM
+// accumulators, operands staged by TMA), for bf16 inputs, head dimension 128
+// and 16 query heads per KV head, with compression block 32 at stride 16 and
+// selection block 64 (EP94 notes section five; lchairun NSA article, the three
+// branches and the gate).
+//
+// Two kernels:
+//  pf_main  one CTA per (sequence, KV head, 8 consecutive tokens): the 128 rows
+//           (token, head of the group) share every K / V tile (GQA group
+//           sharing, EP94 notes section six).
+//           1. compressed attention over the visible compressed blocks (online
+//              softmax, P kept in TMEM as the A operand of the PV MMA);
+//           2. sliding-window attention over [t - w + 1, t];
+//           3. the block scores: S^T = K~ Q^T is recomputed with the final
+//              log-sum-exp of step 1, so each thread holds one compressed key
+//              and sums its probabilities over the 16 heads of the group in
+//              registers; a selection block j collects compressed blocks
+//              4j-1 .. 4j+3;
+//           4. top-n per token with block 0 forced (ties to the lower index);
+//           5. g_cmp * o_cmp + g_win * o_win (fp32) and g_slc to the workspace.
+//  pf_slc   persistent; one unit per (sequence, token, KV head): the selected
+//           blocks, two per 128-key tile, give S^T = K_sel Q^T (M = 128 keys,
+//           N = 16 heads); an exact softmax over all selected keys per head;
+//           O^T = V_sel^T P^T; out = acc + g_slc * o_slc in bf16.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <algorithm>
+#include <cstdint>
+
+#include "internal.h"
+#include "ptx.cuh"
+#include "tcgen05.cuh"
+
+namespace nsa {
+namespace {
+
+constexpr int G = 16;             // query heads per KV head
+constexpr int D = 128;            // head dimension
+constexpr int TQ = 8;             // tokens per pf_main tile (TQ * G = 128 rows)
+constexpr int KT = 128;           // keys per tile
+constexpr int CL = 32, CS = 16;   // compression block and stride
+constexpr int SB = 64;            // selection block
+constexpr uint32_t ATOM = 16384;  // one d-half of a 128-row bf16 tile
+constexpr uint32_t TILE = 32768;  // a 128 x 128 bf16 tile
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr int kMaxSel = 16;       // top_n bound: 8 tiles of two blocks in pf_slc
+constexpr int kMainStagesMax = 4;
+constexpr int kMainThreads = 192; // TMA, MMA, 4 softmax warps
+constexpr int kSlcThreads = 256;  // K TMA, V TMA, MMA, TMEM owner, 4 softmax warps
+constexpr int kSlcKStages = 3, kSlcVStages = 2;
+constexpr uint32_t kQ16 = 4096;   // 16 rows x 128 d bf16
+
+struct PfArgs {
+  const float* w_gate;
+  float* acc;    // [B, T, Hq, d]: g_cmp * o_cmp + g_win * o_win
+  float* gslc;   // [B, T, Hq]
+  int32_t* sel;  // [B, T, Hkv, n]
+  __nv_bfloat16* out;
+  unsigned* err;
+  int B, T, Hq, Hkv, Nc, n, w, nblk, stages;
+  float c;       // softmax scale * log2(e)
+  int gate_mode;
+  float fixed_gates[3];
+};
+
+__device__ __forceinline__ unsigned char* align1024(unsigned char* p) {
+  return (unsigned char*)(((uintptr_t)p + 1023) & ~(uintptr_t)1023);
+}
+
+// Bounded wait that records a timeout and switches the CTA to abort mode
+// (every later wait returns at once, loops run out with their fixed bounds).
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                              unsigned* err) {
+  if (*abort) return false;
+  if (ptx::mbar_wait(bar, parity, kWaitNs)) return true;
+  *abort = 1;
+  atomicOr(err, kErrTimeout);
+  return false;
+}
+
+// K-major SW128 operand of a 128-row (or 16-row) tile, MMA step ks of 8.
+__device__ __forceinline__ uint64_t kmaj(uint32_t base, int ks, uint32_t half_bytes) {
+  return tc::sdesc(base + (ks >> 2) * half_bytes + (ks & 3) * 32, 16, 1024, tc::kSw128);
+}
+
+// MN-major SW128 operand of a [128 keys][128 d] tile (d contiguous), step ks.
+__device__ __forceinline__ uint64_t mnmaj(uint32_t base, int ks) {
+  return tc::sdesc(base + ks * 2048, ATOM, 1024, tc::kSw128);
+}
+
+__device__ __forceinline__ float sigmoidf(float x) { return 1.f / (1.f + __expf(-x)); }
+
+// The three gates of query row `row` of a K-major SW128 Q tile (two d-halves
+// of `half_bytes` each): sigmoid(q . Wg[:, k]) or the fixed gates.
+__device__ __forceinline__ void row_gates(const PfArgs& a, const unsigned char* q, int row,
+                                          uint32_t half_bytes, float (&gt)[3]) {
+  if (a.gate_mode != 0) {
+    gt[0] = a.fixed_gates[0];
+    gt[1] = a.fixed_gates[1];
+    gt[2] = a.fixed_gates[2];
+    return;
+  }
+  float z0 = 0.f, z1 = 0.f, z2 = 0.f;
+#pragma unroll
+  for (int ch = 0; ch < 16; ++ch) {
+    const int hf = ch >> 3, c8 = ch & 7;
+    const uint4 v = *reinterpret_cast<const uint4*>(q + hf * half_bytes + row * 128 +
+                                                    ((c8 ^ (row & 7)) << 4));
+    const __nv_bfloat162* e = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 f = __bfloat1622float2(e[k]);
+      const int dd = ch * 8 + 2 * k;
+      z0 += f.x * __ldg(a.w_gate + dd * 3 + 0) + f.y * __ldg(a.w_gate + dd * 3 + 3);
+      z1 += f.x * __ldg(a.w_gate + dd * 3 + 1) + f.y * __ldg(a.w_gate + dd * 3 + 4);
+      z2 += f.x * __ldg(a.w_gate + dd * 3 + 2) + f.y * __ldg(a.w_gate + dd * 3 + 5);
+    }
+  }
+  gt[0] = sigmoidf(z0);
+  gt[1] = sigmoidf(z1);
+  gt[2] = sigmoidf(z2);
+}
+
+// ============================================================================
+// pf_main
+// ============================================================================
+
+struct MainBars {
+  uint64_t full[kMainStagesMax], empty[kMainStagesMax];
+  uint64_t q_full, s_full[2], p_full[2], o_done[2], fin;
+  uint32_t tmem;
+  int abort;
+};
+
+// TMEM columns of pf_main.
+constexpr uint32_t kO1 = 0, kO2 = 128, kS0 = 256;  // S buffers at 256 and 384
+
+__global__ void __launch_bounds__(kMainThreads, 1)
+    pf_main_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tkc,
+                   const __grid_constant__ CUtensorMap tvc, const __grid_constant__ CUtensorMap tk,
+                   const __grid_constant__ CUtensorMap tv, const PfArgs a) {
+  extern __shared__ unsigned char smraw[];
+  unsigned char* base = align1024(smraw);
+  unsigned char* sQ = base;
+  unsigned char* ring = base + TILE;
+  float* sc = reinterpret_cast<float*>(ring + a.stages * TILE);  // [TQ][nblk]
+  float* slse = sc + TQ * a.nblk;                                  // [128]
+  MainBars* bars = reinterpret_cast<MainBars*>(slse + 128);
+  volatile int* abort = &bars->abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = a.stages;
+  const int ntq = (a.T + TQ - 1) / TQ;
+  const int BH = a.B * a.Hkv;
+  const int bg = blockIdx.x % BH;
+  const int r = ntq - 1 - (int)(blockIdx.x / BH);  // longest tiles first
+  const int b = bg / a.Hkv, g = bg % a.Hkv;
+  const int t0 = r * TQ;
+  const int tlast = min(t0 + TQ - 1, a.T - 1);
+  const int nvis = tlast >= CL - 1 ? min(a.Nc, (tlast - (CL - 1)) / CS + 1) : 0;
+  const int J1 = (nvis + KT - 1) / KT;
+  const int ks0 = max(0, t0 - a.w + 1);
+  const int J2 = (tlast - ks0 + KT) / KT;
+  const int A = J1 + J2;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      ptx::mbar_init(&bars->full[i], 1);
+      ptx::mbar_init(&bars->empty[i], 1);
+    }
+    ptx::mbar_init(&bars->q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&bars->s_full[i], 1);
+      ptx::mbar_init(&bars->p_full[i], 128);
+      ptx::mbar_init(&bars->o_done[i], 1);
+    }
+    ptx::mbar_init(&bars->fin, 1);
+    bars->abort = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 1) {
+    tc::tmem_alloc(&bars->tmem, 512);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = bars->tmem;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tq);
+      ptx::prefetch_tmap(&tkc);
+      ptx::prefetch_tmap(&tvc);
+      ptx::prefetch_tmap(&tk);
+      ptx::prefetch_tmap(&tv);
+      const uint64_t keep = ptx::policy_evict_last(), once = ptx::policy_evict_first();
+      const int qrow = b * a.T + t0;
+      ptx::mbar_arrive_expect_tx(&bars->q_full, TILE);
+      ptx::tma_load_3d(sQ, &tq, &bars->q_full, 0, g * G, qrow, once);
+      ptx::tma_load_3d(sQ + ATOM, &tq, &bars->q_full, 64, g * G, qrow, once);
+      int c = 0;
+      bool ok = true;
+      auto load = [&](const CUtensorMap* m, int z) {
+        if (!ok) return;
+        const int st = c % S;
+        if (c >= S && !wait_or_abort(&bars->empty[st], (uint32_t)(((c / S) - 1) & 1), abort,
+                                     a.err)) {
+          ok = false;
+          return;
+        }
+        unsigned char* dst = ring + st * TILE;
+        ptx::mbar_arrive_expect_tx(&bars->full[st], TILE);
+        ptx::tma_load_3d(dst, m, &bars->full[st], 0, g, z, keep);
+        ptx::tma_load_3d(dst + ATOM, m, &bars->full[st], 64, g, z, keep);
+        ++c;
+      };
+      auto k_of = [&](int i) {
+        if (i < J1) load(&tkc, b * a.Nc + i * KT);
+        else load(&tk, b * a.T + ks0 + (i - J1) * KT);
+      };
+      auto v_of = [&](int i) {
+        if (i < J1) load(&tvc, b * a.Nc + i * KT);
+        else load(&tv, b * a.T + ks0 + (i - J1) * KT);
+      };
+      for (int i = 0; i < A; ++i) {
+        k_of(i);
+        if (i >= 1) v_of(i - 1);
+      }
+      if (A >= 1) v_of(A - 1);
+      for (int i = 0; i < J1; ++i) load(&tkc, b * a.Nc + i * KT);
+      // every issued load must land before the CTA exits
+      for (int k = max(0, c - S); k < c; ++k)
+        if (!ptx::mbar_wait(&bars->full[k % S], (uint32_t)((k / S) & 1), kWaitNs))
+          atomicOr(a.err, kErrTimeout);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t iss = tc::idesc_bf16(128, 128, false, false);
+      const uint32_t its = tc::idesc_bf16(128, 128, false, true);
+      const uint32_t q0 = ptx::smem_u32(sQ), r0 = ptx::smem_u32(ring);
+      bool ok = wait_or_abort(&bars->q_full, 0, abort, a.err);
+      tc::fence_after_sync();
+      int c = 0;
+      auto take = [&]() -> int {
+        const int st = c % S;
+        if (ok) ok = wait_or_abort(&bars->full[st], (uint32_t)((c / S) & 1), abort, a.err);
+        tc::fence_after_sync();
+        return st;
+      };
+      for (int i = 0; ok && i <= A; ++i) {
+        if (i < A) {
+          const int bs = i & 1;
+          if (i >= 2) ok = ok && wait_or_abort(&bars->p_full[bs], (uint32_t)(((i - 2) >> 1) & 1),
+                                               abort, a.err);
+          const int st = take();
+          if (!ok) break;
+          const uint32_t kb = r0 + st * TILE;
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            tc::mma_ss(tmem + kS0 + bs * 128, kmaj(q0, ks, ATOM), kmaj(kb, ks, ATOM), iss, ks > 0);
+          tc::commit(&bars->empty[st]);
+          tc::commit(&bars->s_full[bs]);
+          ++c;
+        }
+        if (i >= 1) {
+          const int pj = i - 1, pb = pj & 1;
+          ok = ok && wait_or_abort(&bars->p_full[pb], (uint32_t)((pj >> 1) & 1), abort, a.err);
+          tc::fence_after_sync();
+          const int st = take();
+          if (!ok) break;
+          const uint32_t vb = r0 + st * TILE;
+          const uint32_t od = tmem + (pj < J1 ? kO1 : kO2);
+          const bool first = (pj == 0 || pj == J1);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            tc::mma_ts(od, tmem + kS0 + pb * 128 + ks * 8, mnmaj(vb, ks), its, (!first || ks > 0));
+          tc::commit(&bars->empty[st]);
+          tc::commit(&bars->o_done[pj & 1]);
+          ++c;
+        }
+      }
+      for (int jj = 0; ok && jj < J1; ++jj) {
+        const int j = A + jj, bs = j & 1;
+        if (j >= 2) ok = wait_or_abort(&bars->p_full[bs], (uint32_t)(((j - 2) >> 1) & 1), abort,
+                                       a.err);
+        const int st = take();
+        if (!ok) break;
+        const uint32_t kb = r0 + st * TILE;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          tc::mma_ss(tmem + kS0 + bs * 128, kmaj(kb, ks, ATOM), kmaj(q0, ks, ATOM), iss, ks > 0);
+        tc::commit(&bars->empty[st]);
+        tc::commit(&bars->s_full[bs]);
+        ++c;
+      }
+      tc::commit(&bars->fin);
+      if (!ptx::mbar_wait(&bars->fin, 0, kWaitNs)) atomicOr(a.err, kErrTimeout);
+    }
+  } else {
+    // ---------------- softmax / scores / selection / epilogue ----------------
+    const int qd = warp & 3;
+    const int row = qd * 32 + lane;  // TMEM lane: query row in steps 1-2, key in step 3
+    const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
+    const int tt = row >> 4, h = row & 15;
+    const int t = min(t0 + tt, a.T - 1);
+    const bool row_ok = t0 + tt < a.T;
+    const int nv_t = t >= CL - 1 ? min(a.Nc, (t - (CL - 1)) / CS + 1) : 0;
+    const int wlo = max(0, t - a.w + 1);
+    for (int i = row; i < TQ * a.nblk; i += 128) sc[i] = 0.f;
+
+    float m1 = -INFINITY, l1 = 0.f, m2 = -INFINITY, l2 = 0.f;
+    for (int j = 0; j < A; ++j) {
+      const int bs = j & 1;
+      wait_or_abort(&bars->s_full[bs], (uint32_t)((j >> 1) & 1), abort, a.err);
+      tc::fence_after_sync();
+      const bool cmp = j < J1;
+      const int kb = cmp ? j * KT : ks0 + (j - J1) * KT;
+      const int lo = cmp ? 0 : wlo, hi = cmp ? nv_t - 1 : t;
+      float s[128];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t u[32];
+        tc::ld32(tl + kS0 + bs * 128 + q4 * 32, u);
+        tc::ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) s[q4 * 32 + e] = __uint_as_float(u[e]);
+      }
+      float mt = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < 128; ++e) {
+        const int key = kb + e;
+        s[e] = (key >= lo && key <= hi) ? s[e] * a.c : -INFINITY;
+        mt = fmaxf(mt, s[e]);
+      }
+      float& m = cmp ? m1 : m2;
+      float& l = cmp ? l1 : l2;
+      const float mn = fmaxf(m, mt);
+      if (mn != -INFINITY && (m == -INFINITY || mn > m + 8.f)) {
+        if (m != -INFINITY) {
+          // rescale this row of O once the previous PV MMA has finished
+          const float f = exp2f(m - mn);
+          l *= f;
+          wait_or_abort(&bars->o_done[(j - 1) & 1], (uint32_t)(((j - 1) >> 1) & 1), abort, a.err);
+          tc::fence_after_sync();
+          const uint32_t oc = tl + (cmp ? kO1 : kO2);
+#pragma unroll
+          for (int q4 = 0; q4 < 8; ++q4) {
+            uint32_t u[16];
+            tc::ld16(oc + q4 * 16, u);
+            tc::ld_wait();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * f);
+            tc::st16(oc + q4 * 16, u);
+          }
+          tc::st_wait();
+        }
+        m = mn;
+      }
+      const float mref = m;
+      float ls = 0.f;
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t u[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = exp2f(s[q4 * 32 + 2 * e] - mref);
+          const float p1 = exp2f(s[q4 * 32 + 2 * e + 1] - mref);
+          ls += p0 + p1;
+          u[e] = ptx::pack_bf16(p0, p1);
+        }
+        tc::st16(tl + kS0 + bs * 128 + q4 * 16, u);
+      }
+      l += ls;
+      tc::st_wait();
+      tc::fence_before_sync();
+      ptx::mbar_arrive(&bars->p_full[bs]);
+    }
+
+    // log-sum-exp (log2 domain) of the compressed branch for step 3
+    slse[row] = l1 > 0.f ? m1 + __log2f(l1) : INFINITY;
+    ptx::named_bar_sync(1, 128);
+
+    // step 3: block scores, thread = compressed key `row` of each tile
+    for (int jj = 0; jj < J1; ++jj) {
+      const int j = A + jj, bs = j & 1;
+      wait_or_abort(&bars->s_full[bs], (uint32_t)((j >> 1) & 1), abort, a.err);
+      tc::fence_after_sync();
+      float s[128];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t u[32];
+        tc::ld32(tl + kS0 + bs * 128 + q4 * 32, u);
+        tc::ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) s[q4 * 32 + e] = __uint_as_float(u[e]);
+      }
+      tc::fence_before_sync();
+      ptx::mbar_arrive(&bars->p_full[bs]);
+      const int kk = jj * KT + row;
+      float pt[TQ];
+#pragma unroll
+      for (int x = 0; x < TQ; ++x) {
+        const int tok = t0 + x;
+        float acc = 0.f;
+        if (tok < a.T && kk < a.Nc && kk * CS + CL - 1 <= tok) {
+#pragma unroll
+          for (int hh = 0; hh < G; ++hh) acc += exp2f(s[x * G + hh] * a.c - slse[x * G + hh]);
+        }
+        pt[x] = acc;
+      }
+      const int blk = kk >> 2;  // compressed block kk overlaps selection blocks kk/4 and, when
+                                // kk % 4 == 3, kk/4 + 1
+#pragma unroll
+      for (int x = 0; x < TQ; ++x) {
+        float g4 = pt[x];
+        g4 += __shfl_xor_sync(0xffffffffu, g4, 1);
+        g4 += __shfl_xor_sync(0xffffffffu, g4, 2);
+        if ((lane & 3) == 0 && g4 != 0.f && blk < a.nblk) atomicAdd(&sc[x * a.nblk + blk], g4);
+        if ((lane & 3) == 3 && pt[x] != 0.f && blk + 1 < a.nblk)
+          atomicAdd(&sc[x * a.nblk + blk + 1], pt[x]);
+      }
+    }
+    ptx::named_bar_sync(1, 128);
+
+    // step 4: top-n per token, one warp per two tokens
+    for (int x = 2 * qd; x < 2 * qd + 2; ++x) {
+      const int tok = t0 + x;
+      if (tok >= a.T) continue;
+      const int ncand = tok / SB + 1;
+      int32_t* dst = a.sel + ((size_t)(b * a.T + tok) * a.Hkv + g) * a.n;
+      if (ncand <= a.n) {
+        for (int i = lane; i < a.n; i += 32) dst[i] = i < ncand ? i : -1;
+        continue;
+      }
+      float* scx = sc + x * a.nblk;
+      int mine = lane == 0 ? 0 : 0x7fffffff;
+      for (int k = 0; k < a.n - 1; ++k) {
+        float best = -1.f;
+        int bi = 0x7fffffff;
+        for (int jb = 1 + lane; jb < ncand; jb += 32) {
+          const float v = scx[jb];
+          if (v > best) {
+            best = v;
+            bi = jb;
+          }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, best, off);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+          if (ov > best || (ov == best && oi < bi)) {
+            best = ov;
+            bi = oi;
+          }
+        }
+        if (lane == k + 1) mine = bi;
+        __syncwarp();
+        if (lane == 0) scx[bi] = -2.f;
+        __syncwarp();
+      }
+      // ascending order: rank of each lane's block among the n chosen
+      int rank = 0;
+      for (int o = 0; o < 32; ++o) {
+        const int v = __shfl_sync(0xffffffffu, mine, o);
+        rank += (v < mine) ? 1 : 0;
+      }
+      if (lane < a.n) dst[rank] = mine;
+    }
+
+    // step 5: gated compressed + window outputs, and g_slc
+    if (A >= 1)
+      wait_or_abort(&bars->o_done[(A - 1) & 1], (uint32_t)(((A - 1) >> 1) & 1), abort, a.err);
+    tc::fence_after_sync();
+    float gt[3];
+    row_gates(a, sQ, row, ATOM, gt);
+    const float i1 = l1 > 0.f ? gt[0] / l1 : 0.f;
+    const float i2 = l2 > 0.f ? gt[2] / l2 : 0.f;
+    float* dst = a.acc + ((size_t)(b * a.T + t) * a.Hq + g * G + h) * D;
+#pragma unroll
+    for (int q4 = 0; q4 < 8; ++q4) {
+      uint32_t u1[16], u2[16];
+      tc::ld16(tl + kO1 + q4 * 16, u1);
+      tc::ld16(tl + kO2 + q4 * 16, u2);
+      tc::ld_wait();
+      if (row_ok) {
+#pragma unroll
+        for (int e = 0; e < 16; e += 4) {
+          float4 o;
+          o.x = (i1 != 0.f ? __uint_as_float(u1[e]) * i1 : 0.f) + __uint_as_float(u2[e]) * i2;
+          o.y = (i1 != 0.f ? __uint_as_float(u1[e + 1]) * i1 : 0.f) + __uint_as_float(u2[e + 1]) * i2;
+          o.z = (i1 != 0.f ? __uint_as_float(u1[e + 2]) * i1 : 0.f) + __uint_as_float(u2[e + 2]) * i2;
+          o.w = (i1 != 0.f ? __uint_as_float(u1[e + 3]) * i1 : 0.f) + __uint_as_float(u2[e + 3]) * i2;
+          *reinterpret_cast<float4*>(dst + q4 * 16 + e) = o;
+        }
+      }
+    }
+    if (row_ok) a.gslc[(size_t)(b * a.T + t) * a.Hq + g * G + h] = gt[1];
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == 1) tc::tmem_dealloc(tmem, 512);
+}
+
+// ============================================================================
+// pf_slc
+// ============================================================================
+
+struct SlcBars {
+  uint64_t kfull[kSlcKStages], kempty[kSlcKStages];
+  uint64_t vfull[kSlcVStages], vempty[kSlcVStages];
+  uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2], o_free[2], fin;
+  uint32_t tmem;
+  int abort;
+  float red[2][4][G];
+};
+
+// TMEM columns of pf_slc: S^T of unit parity p at 128 p (8 tiles x 16 heads),
+// O^T at 256 + 16 p.
+constexpr uint32_t kSlcO = 256;
+
+// Number of valid (non-negative) entries of a sorted selection row.
+__device__ __forceinline__ int count_sel(const int32_t* s, int n) {
+  int c = 0;
+  for (int i = 0; i < n; ++i) c += s[i] >= 0 ? 1 : 0;
+  return c;
+}
+
+__global__ void __launch_bounds__(kSlcThreads, 1)
+    pf_slc_kernel(const __grid_constant__ CUtensorMap tq16, const __grid_constant__ CUtensorMap tk64,
+                  const __grid_constant__ CUtensorMap tv64, const PfArgs a) {
+  extern __shared__ unsigned char smraw[];
+  unsigned char* base = align1024(smraw);
+  unsigned char* kring = base;                               // 3 x 32 KB
+  unsigned char* vring = kring + kSlcKStages * TILE;         // 2 x 32 KB
+  unsigned char* sP = vring + kSlcVStages * TILE;            // 32 KB: [1024 keys][16] SW32
+  unsigned char* sQ = sP + 32768;                            // 2 x 4 KB
+  SlcBars* bars = reinterpret_cast<SlcBars*>(sQ + 2 * kQ16);
+  volatile int* abort = &bars->abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const long long BT = (long long)a.B * a.T;
+  const long long U = BT * a.Hkv;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kSlcKStages; ++i) {
+      ptx::mbar_init(&bars->kfull[i], 1);
+      ptx::mbar_init(&bars->kempty[i], 1);
+    }
+    for (int i = 0; i < kSlcVStages; ++i) {
+      ptx::mbar_init(&bars->vfull[i], 1);
+      ptx::mbar_init(&bars->vempty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&bars->q_full[i], 1);
+      ptx::mbar_init(&bars->q_empty[i], 1);
+      ptx::mbar_init(&bars->s_full[i], 1);
+      ptx::mbar_init(&bars->p_full[i], 128);
+      ptx::mbar_init(&bars->o_full[i], 1);
+      ptx::mbar_init(&bars->o_free[i], 128);
+    }
+    ptx::mbar_init(&bars->fin, 1);
+    bars->abort = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 3) {
+    tc::tmem_alloc(&bars->tmem, 512);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = bars->tmem;
+
+  // unit u -> (g, b, t): group-major so that concurrent CTAs share one group's K/V in L2
+  auto unit_of = [&](long long u, int& b, int& t, int& g) {
+    g = (int)(u / BT);
+    const long long bt = u % BT;
+    b = (int)(bt / a.T);
+    t = (int)(bt % a.T);
+  };
+
+  if (warp == 0 || warp == 1) {
+    // ---------------- TMA producers: warp 0 K (and Q), warp 1 V ----------------
+    if (lane == 0) {
+      const bool isk = warp == 0;
+      const CUtensorMap* m = isk ? &tk64 : &tv64;
+      ptx::prefetch_tmap(m);
+      if (isk) ptx::prefetch_tmap(&tq16);
+      const uint64_t keep = ptx::policy_evict_last(), once = ptx::policy_evict_first();
+      const int NS = isk ? kSlcKStages : kSlcVStages;
+      uint64_t* full = isk ? bars->kfull : bars->vfull;
+      uint64_t* empty = isk ? bars->kempty : bars->vempty;
+      unsigned char* ringp = isk ? kring : vring;
+      int c = 0, k = 0;
+      bool ok = true;
+      for (long long u = blockIdx.x; ok && u < U; u += gridDim.x, ++k) {
+        int b, t, g;
+        unit_of(u, b, t, g);
+        const int32_t* sl = a.sel + ((size_t)(b * a.T + t) * a.Hkv + g) * a.n;
+        const int nsel = count_sel(sl, a.n);
+        if (isk) {
+          const int qs = k & 1;
+          if (k >= 2 && !wait_or_abort(&bars->q_empty[qs], (uint32_t)(((k >> 1) - 1) & 1), abort,
+                                       a.err)) {
+            ok = false;
+            break;
+          }
+          unsigned char* qd = sQ + qs * kQ16;
+          ptx::mbar_arrive_expect_tx(&bars->q_full[qs], kQ16);
+          ptx::tma_load_3d(qd, &tq16, &bars->q_full[qs], 0, g * G, b * a.T + t, once);
+          ptx::tma_load_3d(qd + kQ16 / 2, &tq16, &bars->q_full[qs], 64, g * G, b * a.T + t, once);
+        }
+        for (int i = 0; i < (nsel + 1) / 2; ++i) {
+          const int st = c % NS;
+          if (c >= NS && !wait_or_abort(&empty[st], (uint32_t)(((c / NS) - 1) & 1), abort, a.err)) {
+            ok = false;
+            break;
+          }
+          unsigned char* dst = ringp + st * TILE;
+          ptx::mbar_arrive_expect_tx(&full[st], TILE);
+#pragma unroll
+          for (int hb = 0; hb < 2; ++hb) {
+            // a missing second block reads past the tensor: zero fill
+            const int z = (2 * i + hb < nsel) ? b * a.T + SB * __ldg(sl + 2 * i + hb) : (int)BT;
+            ptx::tma_load_3d(dst + hb * (ATOM / 2), m, &full[st], 0, g, z, keep);
+            ptx::tma_load_3d(dst + ATOM + hb * (ATOM / 2), m, &full[st], 64, g, z, keep);
+          }
+          ++c;
+        }
+      }
+      for (int kq = max(0, c - NS); kq < c; ++kq)
+        if (!ptx::mbar_wait(&full[kq % NS], (uint32_t)((kq / NS) & 1), kWaitNs))
+          atomicOr(a.err, kErrTimeout);
+      if (isk)
+        for (int kq = max(0, k - 2); kq < k; ++kq)
+          if (!ptx::mbar_wait(&bars->q_full[kq & 1], (uint32_t)((kq >> 1) & 1), kWaitNs))
+            atomicOr(a.err, kErrTimeout);
+    }
+  } else if (warp == 2) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t is16 = tc::idesc_bf16(128, 16, false, false);
+      const uint32_t ipv = tc::idesc_bf16(128, 16, true, true);
+      const uint32_t kr = ptx::smem_u32(kring), vr = ptx::smem_u32(vring);
+      const uint32_t pb0 = ptx::smem_u32(sP), qb = ptx::smem_u32(sQ);
+      int ck = 0, cv = 0, k = 0, prev_tiles = 0;
+      bool ok = true;
+      auto pv = [&](int kk, int ntile) {
+        const int pp = kk & 1;
+        ok = ok && wait_or_abort(&bars->p_full[pp], (uint32_t)((kk >> 1) & 1), abort, a.err);
+        if (kk >= 2)
+          ok = ok && wait_or_abort(&bars->o_free[pp], (uint32_t)(((kk >> 1) - 1) & 1), abort, a.err);
+        tc::fence_after_sync();
+        for (int i = 0; ok && i < ntile; ++i) {
+          const int st = cv % kSlcVStages;
+          ok = wait_or_abort(&bars->vfull[st], (uint32_t)((cv / kSlcVStages) & 1), abort, a.err);
+          tc::fence_after_sync();
+          if (!ok) break;
+          const uint32_t vb = vr + st * TILE;
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            tc::mma_ss(tmem + kSlcO + pp * 16, mnmaj(vb, ks),
+                       tc::sdesc(pb0 + i * 4096 + ks * 512, 16, 256, tc::kSw32), ipv,
+                       (i > 0 || ks > 0));
+          tc::commit(&bars->vempty[st]);
+          ++cv;
+        }
+        tc::commit(&bars->o_full[pp]);
+      };
+      for (long long u = blockIdx.x; ok && u < U; u += gridDim.x, ++k) {
+        int b, t, g;
+        unit_of(u, b, t, g);
+        const int32_t* sl = a.sel + ((size_t)(b * a.T + t) * a.Hkv + g) * a.n;
+        const int ntile = (count_sel(sl, a.n) + 1) / 2;
+        const int pk = k & 1;
+        ok = wait_or_abort(&bars->q_full[pk], (uint32_t)((k >> 1) & 1), abort, a.err);
+        tc::fence_after_sync();
+        const uint32_t qd = qb + pk * kQ16;
+        for (int i = 0; ok && i < ntile; ++i) {
+          const int st = ck % kSlcKStages;
+          ok = wait_or_abort(&bars->kfull[st], (uint32_t)((ck / kSlcKStages) & 1), abort, a.err);
+          tc::fence_after_sync();
+          if (!ok) break;
+          const uint32_t kb = kr + st * TILE;
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks)
+            tc::mma_ss(tmem + pk * 128 + i * 16, kmaj(kb, ks, ATOM), kmaj(qd, ks, kQ16 / 2), is16,
+                       ks > 0);
+          tc::commit(&bars->kempty[st]);
+          ++ck;
+        }
+        tc::commit(&bars->q_empty[pk]);
+        tc::commit(&bars->s_full[pk]);
+        if (k >= 1 && ok) pv(k - 1, prev_tiles);
+        prev_tiles = ntile;
+      }
+      if (k >= 1 && ok) pv(k - 1, prev_tiles);
+      tc::commit(&bars->fin);
+      if (!ptx::mbar_wait(&bars->fin, 0, kWaitNs)) atomicOr(a.err, kErrTimeout);
+    }
+  } else if (warp >= 4) {
+    // ---------------- softmax and epilogue ----------------
+    const int qd = warp & 3;
+    const int r = qd * 32 + lane;  // TMEM lane: key row of a tile, then d in the epilogue
+    const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
+    int k = 0;
+    int pb = 0, pt = 0, pg = 0;
+    float pl[G];
+    auto epilogue = [&](int kk) {
+      const int pp = kk & 1;
+      uint32_t u[16];
+      tc::ld16(tl + kSlcO + pp * 16, u);
+      tc::ld_wait();
+      const size_t rowbase = (size_t)(pb * a.T + pt) * a.Hq + pg * G;
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) {
+        const size_t o = (rowbase + hh) * D + r;
+        const float gs = __ldg(a.gslc + rowbase + hh);
+        const float v = a.acc[o] + gs * __uint_as_float(u[hh]) / pl[hh];
+        a.out[o] = __float2bfloat16_rn(v);
+      }
+      tc::fence_before_sync();
+      ptx::mbar_arrive(&bars->o_free[pp]);
+    };
+    for (long long u = blockIdx.x; u < U; u += gridDim.x, ++k) {
+      int b, t, g;
+      unit_of(u, b, t, g);
+      const int32_t* sl = a.sel + ((size_t)(b * a.T + t) * a.Hkv + g) * a.n;
+      const int nsel = count_sel(sl, a.n);
+      const int ntile = (nsel + 1) / 2;
+      const int pk = k & 1;
+      wait_or_abort(&bars->s_full[pk], (uint32_t)((k >> 1) & 1), abort, a.err);
+      tc::fence_after_sync();
+      float s[8][G];
+      float mh[G];
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) mh[hh] = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (i < ntile) {
+          uint32_t uu[16];
+          tc::ld16(tl + pk * 128 + i * 16, uu);
+          tc::ld_wait();
+          const int bi = 2 * i + (r >> 6);
+          const bool valid = bi < nsel && SB * __ldg(sl + bi) + (r & 63) <= t;
+#pragma unroll
+          for (int hh = 0; hh < G; ++hh) {
+            s[i][hh] = valid ? __uint_as_float(uu[hh]) * a.c : -INFINITY;
+            mh[hh] = fmaxf(mh[hh], s[i][hh]);
+          }
+        }
+      }
+      // per-head maximum over all selected keys: warp, then the four warps
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+          mh[hh] = fmaxf(mh[hh], __shfl_xor_sync(0xffffffffu, mh[hh], off));
+      }
+      if (lane == 0)
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) bars->red[0][qd][hh] = mh[hh];
+      ptx::named_bar_sync(1, 128);
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh)
+        mh[hh] = fmaxf(fmaxf(bars->red[0][0][hh], bars->red[0][1][hh]),
+                       fmaxf(bars->red[0][2][hh], bars->red[0][3][hh]));
+      float lh[G];
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) lh[hh] = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (i < ntile) {
+#pragma unroll
+          for (int hh = 0; hh < G; ++hh) {
+            s[i][hh] = exp2f(s[i][hh] - mh[hh]);  // 0 for masked keys; mh is finite (block 0)
+            lh[hh] += s[i][hh];
+          }
+        }
+      }
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1)
+          lh[hh] += __shfl_xor_sync(0xffffffffu, lh[hh], off);
+      }
+      if (lane == 0)
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) bars->red[1][qd][hh] = lh[hh];
+      // P of the previous unit must have been read by its PV MMA
+      if (k >= 1)
+        wait_or_abort(&bars->o_full[(k - 1) & 1], (uint32_t)(((k - 1) >> 1) & 1), abort, a.err);
+      tc::fence_after_sync();
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (i < ntile) {
+          const int R = i * KT + r;
+          unsigned char* rowp = sP + (R >> 3) * 256 + (R & 7) * 32;
+          uint4 lo, hi;
+          lo.x = ptx::pack_bf16(s[i][0], s[i][1]);
+          lo.y = ptx::pack_bf16(s[i][2], s[i][3]);
+          lo.z = ptx::pack_bf16(s[i][4], s[i][5]);
+          lo.w = ptx::pack_bf16(s[i][6], s[i][7]);
+          hi.x = ptx::pack_bf16(s[i][8], s[i][9]);
+          hi.y = ptx::pack_bf16(s[i][10], s[i][11]);
+          hi.z = ptx::pack_bf16(s[i][12], s[i][13]);
+          hi.w = ptx::pack_bf16(s[i][14], s[i][15]);
+          const bool sw = (R & 7) >= 4;  // 32-byte swizzle: rows 4..7 swap halves
+          *reinterpret_cast<uint4*>(rowp + (sw ? 16 : 0)) = lo;
+          *reinterpret_cast<uint4*>(rowp + (sw ? 0 : 16)) = hi;
+        }
+      }
+      ptx::fence_proxy_async();
+      tc::fence_before_sync();
+      ptx::mbar_arrive(&bars->p_full[pk]);
+      if (k >= 1) epilogue(k - 1);
+      ptx::named_bar_sync(1, 128);  // red[1] complete; red[0] free for the next unit
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh)
+        pl[hh] = bars->red[1][0][hh] + bars->red[1][1][hh] + bars->red[1][2][hh] +
+                 bars->red[1][3][hh];
+      pb = b;
+      pt = t;
+      pg = g;
+    }
+    if (k >= 1) {
+      wait_or_abort(&bars->o_full[(k - 1) & 1], (uint32_t)(((k - 1) >> 1) & 1), abort, a.err);
+      tc::fence_after_sync();
+      epilogue(k - 1);
+    }
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == 3) tc::tmem_dealloc(tmem, 512);
+}
+
+size_t main_smem(int stages, int nblk) {
+  return 1024 + TILE + (size_t)stages * TILE + (size_t)TQ * nblk * 4 + 128 * 4 + sizeof(MainBars);
+}
+
+size_t slc_smem() {
+  return 1024 + (kSlcKStages + kSlcVStages) * (size_t)TILE + 32768 + 2 * kQ16 + sizeof(SlcBars);
+}
+
+int main_stages(int nblk) {
+  for (int s = kMainStagesMax; s >= 2; --s)
+    if (main_smem(s, nblk) <= 227 * 1024) return s;
+  return 0;
+}
+
+bool first_use(int id) {
+  static bool seen[2][64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return true;
+  const bool f = !seen[id][dev];
+  seen[id][dev] = true;
+  return f;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
+bool prefill_tc_eligible(const nsa_params& p) {
+  if (p.dtype != NSA_DTYPE_BF16 || p.d != D || p.Hkv < 1 || p.Hq != G * p.Hkv) return false;
+  if (p.cmp_block != CL || p.cmp_stride != CS || p.sel_block != SB) return false;
+  if (p.top_n < 1 || p.top_n > kMaxSel || p.window < 1) return false;
+  if ((long long)p.B * p.T >= (1ll << 30)) return false;
+  const int nblk = (p.T + SB - 1) / SB;
+  return main_stages(nblk) >= 2;
+}
+
+size_t prefill_tc_ws_bytes(const nsa_params& p) {
+  const size_t rows = (size_t)p.B * p.T * p.Hq;
+  return align256(rows * D * 4) + align256(rows * 4) +
+         align256((size_t)p.B * p.T * p.Hkv * p.top_n * 4);
+}
+
+cudaError_t launch_prefill_tc(const nsa_params& p, const void* q, const void* k, const void* v,
+                              const void* kc, const void* vc, const float* w_gate, void* out,
+                              int32_t* sel_out, void* ws, unsigned* err, cudaStream_t stream) {
+  PfArgs a{};
+  const size_t rows = (size_t)p.B * p.T * p.Hq;
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  a.acc = reinterpret_cast<float*>(w);
+  w += align256(rows * D * 4);
+  a.gslc = reinterpret_cast<float*>(w);
+  w += align256(rows * 4);
+  a.sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(w);
+  a.w_gate = w_gate;
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.err = err;
+  a.B = p.B;
+  a.T = p.T;
+  a.Hq = p.Hq;
+  a.Hkv = p.Hkv;
+  a.Nc = nsa_num_cmp_blocks(p.T, p.cmp_block, p.cmp_stride);
+  a.n = p.top_n;
+  a.w = p.window;
+  a.nblk = (p.T + SB - 1) / SB;
+  a.stages = main_stages(a.nblk);
+  const float scale = p.softmax_scale > 0.f ? p.softmax_scale : 1.f / sqrtf((float)p.d);
+  a.c = scale * 1.4426950408889634f;
+  a.gate_mode = p.gate_mode;
+  for (int i = 0; i < 3; ++i) a.fixed_gates[i] = p.fixed_gates[i];
+
+  const uint64_t BT = (uint64_t)p.B * p.T;
+  CUtensorMap tq, tq16, tk, tv, tk64, tv64, tkc, tvc;
+  bool ok = make_tmap_bf16_3d(&tq, q, D, p.Hq, BT, 64, G, TQ, true) &&
+            make_tmap_bf16_3d(&tq16, q, D, p.Hq, BT, 64, G, 1, true) &&
+            make_tmap_bf16_3d(&tk, k, D, p.Hkv, BT, 64, 1, KT, true) &&
+            make_tmap_bf16_3d(&tv, v, D, p.Hkv, BT, 64, 1, KT, true) &&
+            make_tmap_bf16_3d(&tk64, k, D, p.Hkv, BT, 64, 1, SB, true) &&
+            make_tmap_bf16_3d(&tv64, v, D, p.Hkv, BT, 64, 1, SB, true);
+  if (a.Nc > 0) {
+    ok = ok && make_tmap_bf16_3d(&tkc, kc, D, p.Hkv, (uint64_t)p.B * a.Nc, 64, 1, KT, true) &&
+         make_tmap_bf16_3d(&tvc, vc, D, p.Hkv, (uint64_t)p.B * a.Nc, 64, 1, KT, true);
+  } else {
+    tkc = tk;  // never read: no compressed block is visible anywhere
+    tvc = tv;
+  }
+  if (!ok) return cudaErrorInvalidValue;
+
+  cudaError_t e;
+  const size_t sm1 = main_smem(a.stages, a.nblk);
+  if (first_use(0))
+    cudaFuncSetAttribute(pf_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  {
+    TraceScope trace("pf_cmp_win", stream);
+    const long long grid = (long long)p.B * p.Hkv * ((p.T + TQ - 1) / TQ);
+    pf_main_kernel<<<(unsigned)grid, kMainThreads, sm1, stream>>>(tq, tkc, tvc, tk, tv, a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  const size_t sm2 = slc_smem();
+  if (first_use(1))
+    cudaFuncSetAttribute(pf_slc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
+  {
+    TraceScope trace("pf_slc_attn", stream);
+    const long long U = (long long)p.B * p.T * p.Hkv;
+    const int grid = (int)std::min<long long>(U, device_sm_count());
+    pf_slc_kernel<<<grid, kSlcThreads, sm2, stream>>>(tq16, tk64, tv64, a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace nsa

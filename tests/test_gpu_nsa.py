@@ -55,6 +55,36 @@ def test_prefill_bf16_small_all_rows(over):
     gc.run_nsa_prefill(w, rows=gc.sample_rows(w["T"], 400))
 
 
+# Tensor-core prefill path (bf16, d = 128, 16 query heads per KV head): edges of
+# its 8-token row tiles, 128-key tiles and the selection.
+@pytest.mark.parametrize("over", [
+    dict(T=1003),                                  # ragged last row tile and key tiles
+    dict(B=2, T=517, window=100),                  # two sequences
+    dict(T=20),                                    # no compressed block visible
+    dict(T=300, window=1, top_n=2),                # window of one token
+    dict(T=700, window=3000, top_n=16),            # window longer than the sequence
+    dict(T=640, top_n=16),                         # every block selected up to t = 639
+    dict(T=1500, gate_mode=1, fixed_gates=(0.2, 0.5, 0.3), top_n=5),
+    dict(T=1200, Hq=32, Hkv=2, top_n=7, window=200),
+])
+def test_prefill_bf16_tensor_core_edges(over):
+    w = inputs.workload("nsa_prefill_bf16_t8192", **dict(dict(Hq=16, Hkv=1), **over))
+    gc.run_nsa_prefill(w, seed=7)
+
+
+def test_prefill_bf16_runs_the_tensor_core_kernels():
+    from dynamic_block_sparse_nsa_b200 import nsa
+    w = inputs.workload("nsa_prefill_bf16_t8192", T=600, Hq=16, Hkv=1)
+    nsa.trace_enable(True, 64)
+    try:
+        gc.run_nsa_prefill(w, rows=gc.sample_rows(w["T"], 50))
+        recs, _ = nsa.trace_records()
+        names = {nm for nm, _ in recs}
+    finally:
+        nsa.trace_enable(False)
+    assert {"pf_cmp_win", "pf_slc_attn"} <= names, names
+
+
 def test_prefill_bf16_t65536_sampled_rows():
     w = inputs.workload("nsa_prefill_bf16_t65536")
     gc.run_nsa_prefill(w, rows=gc.sample_rows(w["T"], 40))
