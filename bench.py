@@ -507,9 +507,8 @@ def kernel_work(kind, name, res, w):
         p = res["parts"]
         per = {
             "nsa_rows_simt": p["cmp"] + p["slc"] + p["win"],
-            "pf_cmp_attn": p["cmp"],
+            "pf_cmp_win": p["cmp"] + p["win"],
             "pf_slc_attn": p["slc"],
-            "pf_win_attn": p["win"],
         }
         return per.get(name), "tensor"
     p = res["parts"]
@@ -752,6 +751,17 @@ def main():
             line["hbm_frac_nominal_8tbs"] = value / 8000.0
         else:
             line["flops_per_step"] = res["parts"]
+            # every traced kernel against the bf16 peak (first timed region's events)
+            per = {}
+            for n, e in res["table0"].items():
+                wk, _ = kernel_work(kind, n, res, w)
+                if wk is None or not e["launches"]:
+                    continue
+                per_launch = wk / (e["launches"] / min(K, 50))
+                ach = per_launch / (e["total_ms"] / e["launches"] / 1000.0) / 1e12
+                per[n] = {"tflops": ach, "frac": ach / peaks["bf16"],
+                          "mean_launch_us": 1000.0 * e["total_ms"] / e["launches"]}
+            line["kernel_tflops"] = per
         print(json.dumps(line), flush=True)
     if ws > 1:
         import torch.distributed as dist

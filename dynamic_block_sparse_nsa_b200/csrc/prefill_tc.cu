@@ -50,6 +50,7 @@ constexpr int kMainThreads = 192; // TMA, MMA, 4 softmax warps
 constexpr int kSlcThreads = 256;  // K TMA, V TMA, MMA, TMEM owner, 4 softmax warps
 constexpr int kSlcKStages = 3, kSlcVStages = 2;
 constexpr uint32_t kQ16 = 4096;   // 16 rows x 128 d bf16
+constexpr uint32_t kNegInf = 0xff800000u;  // bits of -inf
 
 struct PfArgs {
   const float* w_gate;
@@ -93,8 +94,9 @@ __device__ __forceinline__ float sigmoidf(float x) { return 1.f / (1.f + __expf(
 
 // The three gates of query row `row` of a K-major SW128 Q tile (two d-halves
 // of `half_bytes` each): sigmoid(q . Wg[:, k]) or the fixed gates.
-__device__ __forceinline__ void row_gates(const PfArgs& a, const unsigned char* q, int row,
-                                          uint32_t half_bytes, float (&gt)[3]) {
+__device__ __forceinline__ void row_gates(const PfArgs& a, const unsigned char* q,
+                                          const float* wg, int row, uint32_t half_bytes,
+                                          float (&gt)[3]) {
   if (a.gate_mode != 0) {
     gt[0] = a.fixed_gates[0];
     gt[1] = a.fixed_gates[1];
@@ -102,19 +104,28 @@ __device__ __forceinline__ void row_gates(const PfArgs& a, const unsigned char* 
     return;
   }
   float z0 = 0.f, z1 = 0.f, z2 = 0.f;
-#pragma unroll
-  for (int ch = 0; ch < 16; ++ch) {
+#pragma unroll 1
+  for (int ch = 0; ch < 16; ++ch) {  // runs once per row: kept compact
     const int hf = ch >> 3, c8 = ch & 7;
     const uint4 v = *reinterpret_cast<const uint4*>(q + hf * half_bytes + row * 128 +
                                                     ((c8 ^ (row & 7)) << 4));
     const __nv_bfloat162* e = reinterpret_cast<const __nv_bfloat162*>(&v);
+    // Wg rows ch*8 .. ch*8+7: 24 floats, six 16-byte loads
+    float w[24];
+#pragma unroll
+    for (int i = 0; i < 6; ++i) {
+      const float4 w4 = reinterpret_cast<const float4*>(wg + ch * 24)[i];
+      w[4 * i] = w4.x;
+      w[4 * i + 1] = w4.y;
+      w[4 * i + 2] = w4.z;
+      w[4 * i + 3] = w4.w;
+    }
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
       const float2 f = __bfloat1622float2(e[k]);
-      const int dd = ch * 8 + 2 * k;
-      z0 += f.x * __ldg(a.w_gate + dd * 3 + 0) + f.y * __ldg(a.w_gate + dd * 3 + 3);
-      z1 += f.x * __ldg(a.w_gate + dd * 3 + 1) + f.y * __ldg(a.w_gate + dd * 3 + 4);
-      z2 += f.x * __ldg(a.w_gate + dd * 3 + 2) + f.y * __ldg(a.w_gate + dd * 3 + 5);
+      z0 += f.x * w[6 * k + 0] + f.y * w[6 * k + 3];
+      z1 += f.x * w[6 * k + 1] + f.y * w[6 * k + 4];
+      z2 += f.x * w[6 * k + 2] + f.y * w[6 * k + 5];
     }
   }
   gt[0] = sigmoidf(z0);
@@ -146,7 +157,10 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   unsigned char* ring = base + TILE;
   float* sc = reinterpret_cast<float*>(ring + a.stages * TILE);  // [TQ][nblk]
   float* slse = sc + TQ * a.nblk;                                  // [128]
-  MainBars* bars = reinterpret_cast<MainBars*>(slse + 128);
+  float* spk = slse + 128;                                          // [TQ][128]
+  float* scarry = spk + TQ * KT;                                    // [TQ] (+ pad)
+  float* swg = scarry + 16;                                         // [D][3]
+  MainBars* bars = reinterpret_cast<MainBars*>(swg + D * 3);
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -189,25 +203,32 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   const uint32_t tmem = bars->tmem;
 
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
-    if (lane == 0) {
-      ptx::prefetch_tmap(&tq);
-      ptx::prefetch_tmap(&tkc);
-      ptx::prefetch_tmap(&tvc);
-      ptx::prefetch_tmap(&tk);
-      ptx::prefetch_tmap(&tv);
+    // ---------------- TMA producers: lane L < S issues loads c = L (mod S) ----------------
+    // (one issuing thread keeps only a few bulk copies moving; S threads in
+    // parallel reach the SM's ingest rate)
+    if (lane < S) {
+      if (lane == 0) {
+        ptx::prefetch_tmap(&tq);
+        ptx::prefetch_tmap(&tkc);
+        ptx::prefetch_tmap(&tvc);
+        ptx::prefetch_tmap(&tk);
+        ptx::prefetch_tmap(&tv);
+      }
       const uint64_t keep = ptx::policy_evict_last(), once = ptx::policy_evict_first();
-      const int qrow = b * a.T + t0;
-      ptx::mbar_arrive_expect_tx(&bars->q_full, TILE);
-      ptx::tma_load_3d(sQ, &tq, &bars->q_full, 0, g * G, qrow, once);
-      ptx::tma_load_3d(sQ + ATOM, &tq, &bars->q_full, 64, g * G, qrow, once);
-      int c = 0;
+      if (lane == 0) {
+        const int qrow = b * a.T + t0;
+        ptx::mbar_arrive_expect_tx(&bars->q_full, TILE);
+        ptx::tma_load_3d(sQ, &tq, &bars->q_full, 0, g * G, qrow, once);
+        ptx::tma_load_3d(sQ + ATOM, &tq, &bars->q_full, 64, g * G, qrow, once);
+      }
+      int c = 0, mine = 0;
       bool ok = true;
       auto load = [&](const CUtensorMap* m, int z) {
-        if (!ok) return;
-        const int st = c % S;
-        if (c >= S && !wait_or_abort(&bars->empty[st], (uint32_t)(((c / S) - 1) & 1), abort,
-                                     a.err)) {
+        const int cc = c++;
+        if (!ok || cc % S != lane) return;
+        const int st = lane;
+        if (cc >= S && !wait_or_abort(&bars->empty[st], (uint32_t)(((cc / S) - 1) & 1), abort,
+                                      a.err)) {
           ok = false;
           return;
         }
@@ -215,7 +236,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         ptx::mbar_arrive_expect_tx(&bars->full[st], TILE);
         ptx::tma_load_3d(dst, m, &bars->full[st], 0, g, z, keep);
         ptx::tma_load_3d(dst + ATOM, m, &bars->full[st], 64, g, z, keep);
-        ++c;
+        ++mine;
       };
       auto k_of = [&](int i) {
         if (i < J1) load(&tkc, b * a.Nc + i * KT);
@@ -231,10 +252,13 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       }
       if (A >= 1) v_of(A - 1);
       for (int i = 0; i < J1; ++i) load(&tkc, b * a.Nc + i * KT);
-      // every issued load must land before the CTA exits
-      for (int k = max(0, c - S); k < c; ++k)
-        if (!ptx::mbar_wait(&bars->full[k % S], (uint32_t)((k / S) & 1), kWaitNs))
+      // this lane's last load must land before the CTA exits (earlier ones on
+      // the same stage completed before their stage was reused)
+      if (mine > 0) {
+        const int last = lane + (mine - 1) * S;
+        if (!ptx::mbar_wait(&bars->full[lane], (uint32_t)((last / S) & 1), kWaitNs))
           atomicOr(a.err, kErrTimeout);
+      }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
@@ -311,6 +335,9 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     const int nv_t = t >= CL - 1 ? min(a.Nc, (t - (CL - 1)) / CS + 1) : 0;
     const int wlo = max(0, t - a.w + 1);
     for (int i = row; i < TQ * a.nblk; i += 128) sc[i] = 0.f;
+    if (row < TQ) scarry[row] = 0.f;
+    if (a.gate_mode == 0)
+      for (int i = row; i < D * 3; i += 128) swg[i] = __ldg(a.w_gate + i);
 
     float m1 = -INFINITY, l1 = 0.f, m2 = -INFINITY, l2 = 0.f;
     for (int j = 0; j < A; ++j) {
@@ -320,22 +347,24 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       const bool cmp = j < J1;
       const int kb = cmp ? j * KT : ks0 + (j - J1) * KT;
       const int lo = cmp ? 0 : wlo, hi = cmp ? nv_t - 1 : t;
-      float s[128];
+      uint32_t u[128];
+      tc::ld128_sync(tl + kS0 + bs * 128, u);
+      if (kb < lo || kb + KT - 1 > hi) {  // the tile straddles this row's key range
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        uint32_t u[32];
-        tc::ld32(tl + kS0 + bs * 128 + q4 * 32, u);
-        tc::ld_wait();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) s[q4 * 32 + e] = __uint_as_float(u[e]);
+        for (int e = 0; e < 128; ++e) {
+          const int key = kb + e;
+          if (key < lo || key > hi) u[e] = kNegInf;
+        }
       }
-      float mt = -INFINITY;
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-      for (int e = 0; e < 128; ++e) {
-        const int key = kb + e;
-        s[e] = (key >= lo && key <= hi) ? s[e] * a.c : -INFINITY;
-        mt = fmaxf(mt, s[e]);
+      for (int e = 0; e < 128; e += 4) {
+        mx0 = fmaxf(mx0, __uint_as_float(u[e]));
+        mx1 = fmaxf(mx1, __uint_as_float(u[e + 1]));
+        mx2 = fmaxf(mx2, __uint_as_float(u[e + 2]));
+        mx3 = fmaxf(mx3, __uint_as_float(u[e + 3]));
       }
+      const float mt = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * a.c;
       float& m = cmp ? m1 : m2;
       float& l = cmp ? l1 : l2;
       const float mn = fmaxf(m, mt);
@@ -350,8 +379,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
 #pragma unroll
           for (int q4 = 0; q4 < 8; ++q4) {
             uint32_t u[16];
-            tc::ld16(oc + q4 * 16, u);
-            tc::ld_wait();
+            tc::ld16_sync(oc + q4 * 16, u);
 #pragma unroll
             for (int e = 0; e < 16; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * f);
             tc::st16(oc + q4 * 16, u);
@@ -360,28 +388,31 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         }
         m = mn;
       }
-      const float mref = m;
-      float ls = 0.f;
+      // p = 2^(s c - m); masked keys (-inf) give 0; a row without any valid key
+      // so far keeps m = -inf and gets p = 0 through a zero offset
+      const float nm = m == -INFINITY ? 0.f : -m;
+      float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
-        uint32_t u[16];
+        uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = exp2f(s[q4 * 32 + 2 * e] - mref);
-          const float p1 = exp2f(s[q4 * 32 + 2 * e + 1] - mref);
-          ls += p0 + p1;
-          u[e] = ptx::pack_bf16(p0, p1);
+          const float p0 = ptx::ex2(fmaf(__uint_as_float(u[q4 * 32 + 2 * e]), a.c, nm));
+          const float p1 = ptx::ex2(fmaf(__uint_as_float(u[q4 * 32 + 2 * e + 1]), a.c, nm));
+          ls0 += p0;
+          ls1 += p1;
+          pk[e] = ptx::pack_bf16(p0, p1);
         }
-        tc::st16(tl + kS0 + bs * 128 + q4 * 16, u);
+        tc::st16(tl + kS0 + bs * 128 + q4 * 16, pk);
       }
-      l += ls;
+      l += ls0 + ls1;
       tc::st_wait();
       tc::fence_before_sync();
       ptx::mbar_arrive(&bars->p_full[bs]);
     }
 
     // log-sum-exp (log2 domain) of the compressed branch for step 3
-    slse[row] = l1 > 0.f ? m1 + __log2f(l1) : INFINITY;
+    slse[row] = l1 > 0.f ? -(m1 + __log2f(l1)) : -INFINITY;  // negated, for fma
     ptx::named_bar_sync(1, 128);
 
     // step 3: block scores, thread = compressed key `row` of each tile
@@ -389,15 +420,8 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       const int j = A + jj, bs = j & 1;
       wait_or_abort(&bars->s_full[bs], (uint32_t)((j >> 1) & 1), abort, a.err);
       tc::fence_after_sync();
-      float s[128];
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        uint32_t u[32];
-        tc::ld32(tl + kS0 + bs * 128 + q4 * 32, u);
-        tc::ld_wait();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) s[q4 * 32 + e] = __uint_as_float(u[e]);
-      }
+      uint32_t u[128];
+      tc::ld128_sync(tl + kS0 + bs * 128, u);
       tc::fence_before_sync();
       ptx::mbar_arrive(&bars->p_full[bs]);
       const int kk = jj * KT + row;
@@ -405,70 +429,110 @@ __global__ void __launch_bounds__(kMainThreads, 1)
 #pragma unroll
       for (int x = 0; x < TQ; ++x) {
         const int tok = t0 + x;
-        float acc = 0.f;
+        float acc0 = 0.f, acc1 = 0.f;
         if (tok < a.T && kk < a.Nc && kk * CS + CL - 1 <= tok) {
+          const float4* nl = reinterpret_cast<const float4*>(slse + x * G);
 #pragma unroll
-          for (int hh = 0; hh < G; ++hh) acc += exp2f(s[x * G + hh] * a.c - slse[x * G + hh]);
+          for (int q = 0; q < 4; ++q) {
+            const float4 l4 = nl[q];
+            acc0 += ptx::ex2(fmaf(__uint_as_float(u[x * G + 4 * q]), a.c, l4.x));
+            acc1 += ptx::ex2(fmaf(__uint_as_float(u[x * G + 4 * q + 1]), a.c, l4.y));
+            acc0 += ptx::ex2(fmaf(__uint_as_float(u[x * G + 4 * q + 2]), a.c, l4.z));
+            acc1 += ptx::ex2(fmaf(__uint_as_float(u[x * G + 4 * q + 3]), a.c, l4.w));
+          }
         }
-        pt[x] = acc;
+        pt[x] = acc0 + acc1;
       }
-      const int blk = kk >> 2;  // compressed block kk overlaps selection blocks kk/4 and, when
-                                // kk % 4 == 3, kk/4 + 1
+      // selection block q of this tile collects compressed keys 4q-1 .. 4q+3
+      // (key 4q-1 of block 0 comes from the previous tile)
 #pragma unroll
-      for (int x = 0; x < TQ; ++x) {
-        float g4 = pt[x];
-        g4 += __shfl_xor_sync(0xffffffffu, g4, 1);
-        g4 += __shfl_xor_sync(0xffffffffu, g4, 2);
-        if ((lane & 3) == 0 && g4 != 0.f && blk < a.nblk) atomicAdd(&sc[x * a.nblk + blk], g4);
-        if ((lane & 3) == 3 && pt[x] != 0.f && blk + 1 < a.nblk)
-          atomicAdd(&sc[x * a.nblk + blk + 1], pt[x]);
+      for (int x = 0; x < TQ; ++x) spk[x * KT + row] = pt[x];
+      ptx::named_bar_sync(1, 128);
+      {
+        const int x = row >> 4, q0 = (row & 15) * 2;
+        const float* px = spk + x * KT;
+        float nc = 0.f;
+        if ((row & 15) == 15) nc = px[KT - 1];
+#pragma unroll
+        for (int qq = 0; qq < 2; ++qq) {
+          const int q = q0 + qq;
+          const int jb = jj * (KT / 4) + q;
+          const float prev = q > 0 ? px[4 * q - 1] : scarry[x];
+          const float v = prev + px[4 * q] + px[4 * q + 1] + px[4 * q + 2] + px[4 * q + 3];
+          if (jb < a.nblk) sc[x * a.nblk + jb] = v;
+        }
+        ptx::named_bar_sync(1, 128);
+        if ((row & 15) == 15) {
+          scarry[x] = nc;
+          // the block after the last tile holds only the carried key
+          if (jj == J1 - 1 && J1 * (KT / 4) < a.nblk) sc[x * a.nblk + J1 * (KT / 4)] = nc;
+        }
       }
     }
     ptx::named_bar_sync(1, 128);
 
-    // step 4: top-n per token, one warp per two tokens
-    for (int x = 2 * qd; x < 2 * qd + 2; ++x) {
-      const int tok = t0 + x;
-      if (tok >= a.T) continue;
-      const int ncand = tok / SB + 1;
-      int32_t* dst = a.sel + ((size_t)(b * a.T + tok) * a.Hkv + g) * a.n;
-      if (ncand <= a.n) {
-        for (int i = lane; i < a.n; i += 32) dst[i] = i < ncand ? i : -1;
-        continue;
+    // step 4: top-n per token, one warp per two tokens (processed together).
+    // A candidate's key is (score bits + 1, ~index): unique, ordered by score
+    // and then by the lower index; a taken block gets key 0.
+    {
+      int tokx[2], ncand[2], mine[2];
+      uint32_t bh[2], bl[2];
+      int32_t* dst[2];
+#pragma unroll
+      for (int z = 0; z < 2; ++z) {
+        const int x = 2 * qd + z, tok = t0 + x;
+        tokx[z] = x;
+        ncand[z] = tok < a.T ? tok / SB + 1 : 0;
+        dst[z] = a.sel + ((size_t)(b * a.T + min(tok, a.T - 1)) * a.Hkv + g) * a.n;
+        mine[z] = lane == 0 ? 0 : 0x7fffffff;
+        bh[z] = 0;
+        bl[z] = 0;
+        if (tok < a.T && ncand[z] <= a.n) {
+          for (int i = lane; i < a.n; i += 32) dst[z][i] = i < ncand[z] ? i : -1;
+          ncand[z] = 0;  // done
+        }
       }
-      float* scx = sc + x * a.nblk;
-      int mine = lane == 0 ? 0 : 0x7fffffff;
-      for (int k = 0; k < a.n - 1; ++k) {
-        float best = -1.f;
-        int bi = 0x7fffffff;
-        for (int jb = 1 + lane; jb < ncand; jb += 32) {
+      auto rescan = [&](int z) {
+        const float* scx = sc + tokx[z] * a.nblk;
+        uint32_t h = 0, l = 0;
+        for (int jb = 1 + lane; jb < ncand[z]; jb += 32) {
           const float v = scx[jb];
-          if (v > best) {
-            best = v;
-            bi = jb;
+          const uint32_t kh = v < 0.f ? 0u : __float_as_uint(v) + 1u;
+          const uint32_t kl = ~(uint32_t)jb;
+          if (kh > h || (kh == h && kl > l)) {
+            h = kh;
+            l = kl;
           }
+        }
+        bh[z] = h;
+        bl[z] = l;
+      };
+      rescan(0);
+      rescan(1);
+      for (int k = 0; k < a.n - 1; ++k) {
+        int pick[2];
+#pragma unroll
+        for (int z = 0; z < 2; ++z) {
+          const uint32_t mh = __reduce_max_sync(0xffffffffu, bh[z]);
+          const uint32_t ml = __reduce_max_sync(0xffffffffu, bh[z] == mh ? bl[z] : 0u);
+          pick[z] = (int)~ml;
+          if (lane == k + 1) mine[z] = pick[z];
         }
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-          const float ov = __shfl_xor_sync(0xffffffffu, best, off);
-          const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-          if (ov > best || (ov == best && oi < bi)) {
-            best = ov;
-            bi = oi;
+        for (int z = 0; z < 2; ++z) {
+          if (ncand[z] > 0 && ((pick[z] - 1) & 31) == lane) {
+            sc[tokx[z] * a.nblk + pick[z]] = -1.f;
+            rescan(z);
           }
         }
-        if (lane == k + 1) mine = bi;
-        __syncwarp();
-        if (lane == 0) scx[bi] = -2.f;
-        __syncwarp();
       }
-      // ascending order: rank of each lane's block among the n chosen
-      int rank = 0;
-      for (int o = 0; o < 32; ++o) {
-        const int v = __shfl_sync(0xffffffffu, mine, o);
-        rank += (v < mine) ? 1 : 0;
+#pragma unroll
+      for (int z = 0; z < 2; ++z) {
+        if (ncand[z] == 0) continue;  // warp-uniform
+        int rank = 0;
+        for (int o = 0; o < 32; ++o) rank += (__shfl_sync(0xffffffffu, mine[z], o) < mine[z]) ? 1 : 0;
+        if (lane < a.n) dst[z][rank] = mine[z];
       }
-      if (lane < a.n) dst[rank] = mine;
     }
 
     // step 5: gated compressed + window outputs, and g_slc
@@ -476,16 +540,16 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       wait_or_abort(&bars->o_done[(A - 1) & 1], (uint32_t)(((A - 1) >> 1) & 1), abort, a.err);
     tc::fence_after_sync();
     float gt[3];
-    row_gates(a, sQ, row, ATOM, gt);
+    row_gates(a, sQ, swg, row, ATOM, gt);
     const float i1 = l1 > 0.f ? gt[0] / l1 : 0.f;
     const float i2 = l2 > 0.f ? gt[2] / l2 : 0.f;
     float* dst = a.acc + ((size_t)(b * a.T + t) * a.Hq + g * G + h) * D;
-#pragma unroll
-    for (int q4 = 0; q4 < 8; ++q4) {
+    // (O1 is never written when no compressed block is visible: i1 = 0 skips it)
+#pragma unroll 1
+    for (int c16 = 0; c16 < 8; ++c16) {  // runs once per row: kept compact
       uint32_t u1[16], u2[16];
-      tc::ld16(tl + kO1 + q4 * 16, u1);
-      tc::ld16(tl + kO2 + q4 * 16, u2);
-      tc::ld_wait();
+      tc::ld16_sync(tl + kO1 + c16 * 16, u1);
+      tc::ld16_sync(tl + kO2 + c16 * 16, u2);
       if (row_ok) {
 #pragma unroll
         for (int e = 0; e < 16; e += 4) {
@@ -494,7 +558,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
           o.y = (i1 != 0.f ? __uint_as_float(u1[e + 1]) * i1 : 0.f) + __uint_as_float(u2[e + 1]) * i2;
           o.z = (i1 != 0.f ? __uint_as_float(u1[e + 2]) * i1 : 0.f) + __uint_as_float(u2[e + 2]) * i2;
           o.w = (i1 != 0.f ? __uint_as_float(u1[e + 3]) * i1 : 0.f) + __uint_as_float(u2[e + 3]) * i2;
-          *reinterpret_cast<float4*>(dst + q4 * 16 + e) = o;
+          *reinterpret_cast<float4*>(dst + c16 * 16 + e) = o;
         }
       }
     }
@@ -515,14 +579,45 @@ struct SlcBars {
   uint64_t kfull[kSlcKStages], kempty[kSlcKStages];
   uint64_t vfull[kSlcVStages], vempty[kSlcVStages];
   uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2], o_free[2], fin;
+  uint64_t a_full[2], a_empty[2];
   uint32_t tmem;
   int abort;
-  float red[2][4][G];
+  alignas(16) float red[2][4][G];
 };
+
+constexpr uint32_t kAccBytes = G * D * 4;  // one unit's acc rows
+constexpr uint32_t kAccSlot = kAccBytes + 256;  // + its 16 gates
 
 // TMEM columns of pf_slc: S^T of unit parity p at 128 p (8 tiles x 16 heads),
 // O^T at 256 + 16 p.
 constexpr uint32_t kSlcO = 256;
+
+// Reduces v[16] (one value per head) over the 32 lanes of a warp with 16
+// shuffles: each step exchanges the half of the values the partner keeps, so
+// lane L ends with the reduction of head L / 2.
+template <bool MAX>
+__device__ __forceinline__ float xreduce16(const float (&v)[G], int lane) {
+  auto op = [](float x, float y) { return MAX ? fmaxf(x, y) : x + y; };
+  float w8[8], w4[4], w2[2];
+  const bool b4 = lane & 16, b3 = lane & 8, b2 = lane & 4, b1 = lane & 2;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const float send = b4 ? v[j] : v[j + 8];
+    w8[j] = op(b4 ? v[j + 8] : v[j], __shfl_xor_sync(0xffffffffu, send, 16));
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float send = b3 ? w8[j] : w8[j + 4];
+    w4[j] = op(b3 ? w8[j + 4] : w8[j], __shfl_xor_sync(0xffffffffu, send, 8));
+  }
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const float send = b2 ? w4[j] : w4[j + 2];
+    w2[j] = op(b2 ? w4[j + 2] : w4[j], __shfl_xor_sync(0xffffffffu, send, 4));
+  }
+  const float w1 = op(b1 ? w2[1] : w2[0], __shfl_xor_sync(0xffffffffu, b1 ? w2[0] : w2[1], 2));
+  return op(w1, __shfl_xor_sync(0xffffffffu, w1, 1));
+}
 
 // Number of valid (non-negative) entries of a sorted selection row.
 __device__ __forceinline__ int count_sel(const int32_t* s, int n) {
@@ -540,7 +635,8 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
   unsigned char* vring = kring + kSlcKStages * TILE;         // 2 x 32 KB
   unsigned char* sP = vring + kSlcVStages * TILE;            // 32 KB: [1024 keys][16] SW32
   unsigned char* sQ = sP + 32768;                            // 2 x 4 KB
-  SlcBars* bars = reinterpret_cast<SlcBars*>(sQ + 2 * kQ16);
+  unsigned char* sA = sQ + 2 * kQ16;                         // 2 x (acc 8 KB + gates)
+  SlcBars* bars = reinterpret_cast<SlcBars*>(sA + 2 * kAccSlot);
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -549,11 +645,11 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kSlcKStages; ++i) {
-      ptx::mbar_init(&bars->kfull[i], 1);
+      ptx::mbar_init(&bars->kfull[i], 4);  // one arrival per issuing lane
       ptx::mbar_init(&bars->kempty[i], 1);
     }
     for (int i = 0; i < kSlcVStages; ++i) {
-      ptx::mbar_init(&bars->vfull[i], 1);
+      ptx::mbar_init(&bars->vfull[i], 4);
       ptx::mbar_init(&bars->vempty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
@@ -563,6 +659,8 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
       ptx::mbar_init(&bars->p_full[i], 128);
       ptx::mbar_init(&bars->o_full[i], 1);
       ptx::mbar_init(&bars->o_free[i], 128);
+      ptx::mbar_init(&bars->a_full[i], 1);
+      ptx::mbar_init(&bars->a_empty[i], 128);
     }
     ptx::mbar_init(&bars->fin, 1);
     bars->abort = 0;
@@ -587,16 +685,22 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
 
   if (warp == 0 || warp == 1) {
     // ---------------- TMA producers: warp 0 K (and Q), warp 1 V ----------------
-    if (lane == 0) {
+    // Lane L < 4 issues box L of every tile (selected block L / 2, d-half L % 2):
+    // four issuing threads keep enough bulk copies moving to reach the SM's
+    // ingest rate. A tile's full barrier takes one arrival per lane.
+    if (lane < 4) {
       const bool isk = warp == 0;
       const CUtensorMap* m = isk ? &tk64 : &tv64;
-      ptx::prefetch_tmap(m);
-      if (isk) ptx::prefetch_tmap(&tq16);
+      if (lane == 0) {
+        ptx::prefetch_tmap(m);
+        if (isk) ptx::prefetch_tmap(&tq16);
+      }
       const uint64_t keep = ptx::policy_evict_last(), once = ptx::policy_evict_first();
       const int NS = isk ? kSlcKStages : kSlcVStages;
       uint64_t* full = isk ? bars->kfull : bars->vfull;
       uint64_t* empty = isk ? bars->kempty : bars->vempty;
       unsigned char* ringp = isk ? kring : vring;
+      const int hb = lane >> 1, dh = lane & 1;
       int c = 0, k = 0;
       bool ok = true;
       for (long long u = blockIdx.x; ok && u < U; u += gridDim.x, ++k) {
@@ -604,7 +708,7 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
         unit_of(u, b, t, g);
         const int32_t* sl = a.sel + ((size_t)(b * a.T + t) * a.Hkv + g) * a.n;
         const int nsel = count_sel(sl, a.n);
-        if (isk) {
+        if (isk && lane == 0) {
           const int qs = k & 1;
           if (k >= 2 && !wait_or_abort(&bars->q_empty[qs], (uint32_t)(((k >> 1) - 1) & 1), abort,
                                        a.err)) {
@@ -615,6 +719,17 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
           ptx::mbar_arrive_expect_tx(&bars->q_full[qs], kQ16);
           ptx::tma_load_3d(qd, &tq16, &bars->q_full[qs], 0, g * G, b * a.T + t, once);
           ptx::tma_load_3d(qd + kQ16 / 2, &tq16, &bars->q_full[qs], 64, g * G, b * a.T + t, once);
+          // the unit's acc rows and g_slc, for the epilogue
+          if (k >= 2 && !wait_or_abort(&bars->a_empty[qs], (uint32_t)(((k >> 1) - 1) & 1), abort,
+                                       a.err)) {
+            ok = false;
+            break;
+          }
+          const size_t row0 = (size_t)(b * a.T + t) * a.Hq + g * G;
+          unsigned char* ad = sA + qs * kAccSlot;
+          ptx::mbar_arrive_expect_tx(&bars->a_full[qs], kAccBytes + G * 4);
+          ptx::bulk_load(ad, a.acc + row0 * D, kAccBytes, &bars->a_full[qs]);
+          ptx::bulk_load(ad + kAccBytes, a.gslc + row0, G * 4, &bars->a_full[qs]);
         }
         for (int i = 0; i < (nsel + 1) / 2; ++i) {
           const int st = c % NS;
@@ -622,25 +737,24 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
             ok = false;
             break;
           }
-          unsigned char* dst = ringp + st * TILE;
-          ptx::mbar_arrive_expect_tx(&full[st], TILE);
-#pragma unroll
-          for (int hb = 0; hb < 2; ++hb) {
-            // a missing second block reads past the tensor: zero fill
-            const int z = (2 * i + hb < nsel) ? b * a.T + SB * __ldg(sl + 2 * i + hb) : (int)BT;
-            ptx::tma_load_3d(dst + hb * (ATOM / 2), m, &full[st], 0, g, z, keep);
-            ptx::tma_load_3d(dst + ATOM + hb * (ATOM / 2), m, &full[st], 64, g, z, keep);
-          }
+          unsigned char* dst = ringp + st * TILE + dh * ATOM + hb * (ATOM / 2);
+          // a missing second block reads past the tensor: zero fill
+          const int z = (2 * i + hb < nsel) ? b * a.T + SB * __ldg(sl + 2 * i + hb) : (int)BT;
+          ptx::mbar_arrive_expect_tx(&full[st], ATOM / 2);
+          ptx::tma_load_3d(dst, m, &full[st], dh * 64, g, z, keep);
           ++c;
         }
       }
       for (int kq = max(0, c - NS); kq < c; ++kq)
         if (!ptx::mbar_wait(&full[kq % NS], (uint32_t)((kq / NS) & 1), kWaitNs))
           atomicOr(a.err, kErrTimeout);
-      if (isk)
-        for (int kq = max(0, k - 2); kq < k; ++kq)
+      if (isk && lane == 0)
+        for (int kq = max(0, k - 2); kq < k; ++kq) {
           if (!ptx::mbar_wait(&bars->q_full[kq & 1], (uint32_t)((kq >> 1) & 1), kWaitNs))
             atomicOr(a.err, kErrTimeout);
+          if (!ptx::mbar_wait(&bars->a_full[kq & 1], (uint32_t)((kq >> 1) & 1), kWaitNs))
+            atomicOr(a.err, kErrTimeout);
+        }
     }
   } else if (warp == 2) {
     // ---------------- MMA issuer ----------------
@@ -708,6 +822,7 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
     // ---------------- softmax and epilogue ----------------
     const int qd = warp & 3;
     const int r = qd * 32 + lane;  // TMEM lane: key row of a tile, then d in the epilogue
+    const int half = r >> 6, kr = r & (SB - 1);
     const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
     int k = 0;
     int pb = 0, pt = 0, pg = 0;
@@ -715,102 +830,97 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
     auto epilogue = [&](int kk) {
       const int pp = kk & 1;
       uint32_t u[16];
-      tc::ld16(tl + kSlcO + pp * 16, u);
-      tc::ld_wait();
-      const size_t rowbase = (size_t)(pb * a.T + pt) * a.Hq + pg * G;
+      tc::ld16_sync(tl + kSlcO + pp * 16, u);
+      wait_or_abort(&bars->a_full[pp], (uint32_t)((kk >> 1) & 1), abort, a.err);
+      const float* accs = reinterpret_cast<const float*>(sA + pp * kAccSlot);
+      __nv_bfloat16* o = a.out + ((size_t)(pb * a.T + pt) * a.Hq + pg * G) * D + r;
 #pragma unroll
-      for (int hh = 0; hh < G; ++hh) {
-        const size_t o = (rowbase + hh) * D + r;
-        const float gs = __ldg(a.gslc + rowbase + hh);
-        const float v = a.acc[o] + gs * __uint_as_float(u[hh]) / pl[hh];
-        a.out[o] = __float2bfloat16_rn(v);
-      }
+      for (int hh = 0; hh < G; ++hh)
+        o[hh * D] = __float2bfloat16_rn(
+            fmaf(accs[G * D + hh] / pl[hh], __uint_as_float(u[hh]), accs[hh * D + r]));
       tc::fence_before_sync();
       ptx::mbar_arrive(&bars->o_free[pp]);
+      ptx::mbar_arrive(&bars->a_empty[pp]);
     };
     for (long long u = blockIdx.x; u < U; u += gridDim.x, ++k) {
       int b, t, g;
       unit_of(u, b, t, g);
       const int32_t* sl = a.sel + ((size_t)(b * a.T + t) * a.Hkv + g) * a.n;
-      const int nsel = count_sel(sl, a.n);
-      const int ntile = (nsel + 1) / 2;
+      int selv[kMaxSel];
+#pragma unroll
+      for (int i = 0; i < kMaxSel; ++i) selv[i] = i < a.n ? __ldg(sl + i) : -1;
+      int nsel = 0;
+#pragma unroll
+      for (int i = 0; i < kMaxSel; ++i) nsel += selv[i] >= 0 ? 1 : 0;
       const int pk = k & 1;
       wait_or_abort(&bars->s_full[pk], (uint32_t)((k >> 1) & 1), abort, a.err);
       tc::fence_after_sync();
-      float s[8][G];
+      // uu: S^T of this key lane (8 tiles x 16 heads), masked in place, then
+      // the probabilities
+      uint32_t uu[128];
+      tc::ld128_sync(tl + pk * 128, uu);
       float mh[G];
 #pragma unroll
       for (int hh = 0; hh < G; ++hh) mh[hh] = -INFINITY;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        if (i < ntile) {
-          uint32_t uu[16];
-          tc::ld16(tl + pk * 128 + i * 16, uu);
-          tc::ld_wait();
-          const int bi = 2 * i + (r >> 6);
-          const bool valid = bi < nsel && SB * __ldg(sl + bi) + (r & 63) <= t;
+        const int blk = half ? selv[2 * i + 1] : selv[2 * i];
+        if (!(2 * i + half < nsel && blk * SB + kr <= t)) {
 #pragma unroll
-          for (int hh = 0; hh < G; ++hh) {
-            s[i][hh] = valid ? __uint_as_float(uu[hh]) * a.c : -INFINITY;
-            mh[hh] = fmaxf(mh[hh], s[i][hh]);
-          }
+          for (int hh = 0; hh < G; ++hh) uu[i * G + hh] = kNegInf;
         }
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) mh[hh] = fmaxf(mh[hh], __uint_as_float(uu[i * G + hh]));
       }
-      // per-head maximum over all selected keys: warp, then the four warps
-#pragma unroll
-      for (int hh = 0; hh < G; ++hh) {
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
-          mh[hh] = fmaxf(mh[hh], __shfl_xor_sync(0xffffffffu, mh[hh], off));
-      }
-      if (lane == 0)
-#pragma unroll
-        for (int hh = 0; hh < G; ++hh) bars->red[0][qd][hh] = mh[hh];
+      // per-head maximum over the 128 keys of the four warps, then over warps
+      const float mw = xreduce16<true>(mh, lane);
+      if ((lane & 1) == 0) bars->red[0][qd][lane >> 1] = mw;
       ptx::named_bar_sync(1, 128);
+      float nmc[G];  // -max * c; finite, since key 0 of block 0 is always valid
 #pragma unroll
-      for (int hh = 0; hh < G; ++hh)
-        mh[hh] = fmaxf(fmaxf(bars->red[0][0][hh], bars->red[0][1][hh]),
-                       fmaxf(bars->red[0][2][hh], bars->red[0][3][hh]));
+      for (int q = 0; q < 4; ++q) {
+        const float4 r0 = reinterpret_cast<const float4*>(bars->red[0][0])[q];
+        const float4 r1 = reinterpret_cast<const float4*>(bars->red[0][1])[q];
+        const float4 r2 = reinterpret_cast<const float4*>(bars->red[0][2])[q];
+        const float4 r3 = reinterpret_cast<const float4*>(bars->red[0][3])[q];
+        nmc[4 * q] = -fmaxf(fmaxf(r0.x, r1.x), fmaxf(r2.x, r3.x)) * a.c;
+        nmc[4 * q + 1] = -fmaxf(fmaxf(r0.y, r1.y), fmaxf(r2.y, r3.y)) * a.c;
+        nmc[4 * q + 2] = -fmaxf(fmaxf(r0.z, r1.z), fmaxf(r2.z, r3.z)) * a.c;
+        nmc[4 * q + 3] = -fmaxf(fmaxf(r0.w, r1.w), fmaxf(r2.w, r3.w)) * a.c;
+      }
       float lh[G];
 #pragma unroll
       for (int hh = 0; hh < G; ++hh) lh[hh] = 0.f;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        if (i < ntile) {
 #pragma unroll
-          for (int hh = 0; hh < G; ++hh) {
-            s[i][hh] = exp2f(s[i][hh] - mh[hh]);  // 0 for masked keys; mh is finite (block 0)
-            lh[hh] += s[i][hh];
-          }
+        for (int hh = 0; hh < G; ++hh) {
+          const float x = ptx::ex2(fmaf(__uint_as_float(uu[i * G + hh]), a.c, nmc[hh]));
+          uu[i * G + hh] = __float_as_uint(x);
+          lh[hh] += x;
         }
       }
-#pragma unroll
-      for (int hh = 0; hh < G; ++hh) {
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1)
-          lh[hh] += __shfl_xor_sync(0xffffffffu, lh[hh], off);
-      }
-      if (lane == 0)
-#pragma unroll
-        for (int hh = 0; hh < G; ++hh) bars->red[1][qd][hh] = lh[hh];
+      const float lw = xreduce16<false>(lh, lane);
+      if ((lane & 1) == 0) bars->red[1][qd][lane >> 1] = lw;
       // P of the previous unit must have been read by its PV MMA
       if (k >= 1)
         wait_or_abort(&bars->o_full[(k - 1) & 1], (uint32_t)(((k - 1) >> 1) & 1), abort, a.err);
       tc::fence_after_sync();
+      const int ntile = (nsel + 1) / 2;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         if (i < ntile) {
           const int R = i * KT + r;
           unsigned char* rowp = sP + (R >> 3) * 256 + (R & 7) * 32;
           uint4 lo, hi;
-          lo.x = ptx::pack_bf16(s[i][0], s[i][1]);
-          lo.y = ptx::pack_bf16(s[i][2], s[i][3]);
-          lo.z = ptx::pack_bf16(s[i][4], s[i][5]);
-          lo.w = ptx::pack_bf16(s[i][6], s[i][7]);
-          hi.x = ptx::pack_bf16(s[i][8], s[i][9]);
-          hi.y = ptx::pack_bf16(s[i][10], s[i][11]);
-          hi.z = ptx::pack_bf16(s[i][12], s[i][13]);
-          hi.w = ptx::pack_bf16(s[i][14], s[i][15]);
+          lo.x = ptx::pack_bf16(__uint_as_float(uu[i * G + 0]), __uint_as_float(uu[i * G + 1]));
+          lo.y = ptx::pack_bf16(__uint_as_float(uu[i * G + 2]), __uint_as_float(uu[i * G + 3]));
+          lo.z = ptx::pack_bf16(__uint_as_float(uu[i * G + 4]), __uint_as_float(uu[i * G + 5]));
+          lo.w = ptx::pack_bf16(__uint_as_float(uu[i * G + 6]), __uint_as_float(uu[i * G + 7]));
+          hi.x = ptx::pack_bf16(__uint_as_float(uu[i * G + 8]), __uint_as_float(uu[i * G + 9]));
+          hi.y = ptx::pack_bf16(__uint_as_float(uu[i * G + 10]), __uint_as_float(uu[i * G + 11]));
+          hi.z = ptx::pack_bf16(__uint_as_float(uu[i * G + 12]), __uint_as_float(uu[i * G + 13]));
+          hi.w = ptx::pack_bf16(__uint_as_float(uu[i * G + 14]), __uint_as_float(uu[i * G + 15]));
           const bool sw = (R & 7) >= 4;  // 32-byte swizzle: rows 4..7 swap halves
           *reinterpret_cast<uint4*>(rowp + (sw ? 16 : 0)) = lo;
           *reinterpret_cast<uint4*>(rowp + (sw ? 0 : 16)) = hi;
@@ -822,9 +932,16 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
       if (k >= 1) epilogue(k - 1);
       ptx::named_bar_sync(1, 128);  // red[1] complete; red[0] free for the next unit
 #pragma unroll
-      for (int hh = 0; hh < G; ++hh)
-        pl[hh] = bars->red[1][0][hh] + bars->red[1][1][hh] + bars->red[1][2][hh] +
-                 bars->red[1][3][hh];
+      for (int q = 0; q < 4; ++q) {
+        const float4 r0 = reinterpret_cast<const float4*>(bars->red[1][0])[q];
+        const float4 r1 = reinterpret_cast<const float4*>(bars->red[1][1])[q];
+        const float4 r2 = reinterpret_cast<const float4*>(bars->red[1][2])[q];
+        const float4 r3 = reinterpret_cast<const float4*>(bars->red[1][3])[q];
+        pl[4 * q] = (r0.x + r1.x) + (r2.x + r3.x);
+        pl[4 * q + 1] = (r0.y + r1.y) + (r2.y + r3.y);
+        pl[4 * q + 2] = (r0.z + r1.z) + (r2.z + r3.z);
+        pl[4 * q + 3] = (r0.w + r1.w) + (r2.w + r3.w);
+      }
       pb = b;
       pt = t;
       pg = g;
@@ -843,11 +960,13 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
 }
 
 size_t main_smem(int stages, int nblk) {
-  return 1024 + TILE + (size_t)stages * TILE + (size_t)TQ * nblk * 4 + 128 * 4 + sizeof(MainBars);
+  return 1024 + TILE + (size_t)stages * TILE + (size_t)TQ * nblk * 4 + 128 * 4 +
+         (size_t)TQ * KT * 4 + 16 * 4 + D * 3 * 4 + sizeof(MainBars);
 }
 
 size_t slc_smem() {
-  return 1024 + (kSlcKStages + kSlcVStages) * (size_t)TILE + 32768 + 2 * kQ16 + sizeof(SlcBars);
+  return 1024 + (kSlcKStages + kSlcVStages) * (size_t)TILE + 32768 + 2 * kQ16 + 2 * kAccSlot +
+         sizeof(SlcBars);
 }
 
 int main_stages(int nblk) {
