@@ -643,6 +643,31 @@ def config_of(w):
 
 # --------------------------------------------------------------------------
 
+def prefill_summary(ws, rank, local, peaks, K=5, W=3):
+    """The 65536-token bf16 prefill (the metric's prefill half), timed like the
+    main line: whole-step TFLOP/s and every kernel against the bf16 peak."""
+    name = "nsa_prefill_bf16_t65536"
+    w = inputs.workload(name)
+    res = run_prefill(w, K, W, ws, rank, local, e2e=False)
+    ms_max = reduce_max(res["ms"], ws)
+    work_all = reduce_sum(res["work"] * K, ws)
+    per = {}
+    for n, e in res["table0"].items():
+        wk, _ = kernel_work("prefill", n, res, w)
+        if wk is None or not e["launches"]:
+            continue
+        per_launch = wk / (e["launches"] / min(K, 50))
+        ach = per_launch / (e["total_ms"] / e["launches"] / 1000.0) / 1e12
+        per[n] = {"tflops": ach, "frac": ach / peaks["bf16"], "peak": peaks["bf16"],
+                  "mean_launch_us": 1000.0 * e["total_ms"] / e["launches"]}
+    return {"workload": name, "value": work_all / (ms_max / 1000.0) / 1e12, "unit": "TFLOP/s",
+            "ms_per_step": ms_max / K, "steps": K, "warmup": W,
+            "flops_per_step": res["parts"], "kernel_tflops": per,
+            "peak_source": peaks["src"], "clocks": res["clk"],
+            "note": "algorithmic flops (4 d per query head and attended key); "
+                    "a step is nsa_compress_kv + nsa_prefill on device-resident inputs"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -653,6 +678,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="skip the 65536-token prefill measured beside the default decode line")
     ap.add_argument("--no-graph", action="store_true",
                     help="time decode steps as separate launches instead of one CUDA graph")
     ap.add_argument("--set", action="append", default=[], metavar="KEY=VALUE",
@@ -719,6 +746,10 @@ def main():
                     "timing": "events around each launch of this kernel over a second "
                               "timed region of the same K steps"}
 
+    pf = None
+    if kind == "decode" and not args.set and not args.no_prefill and args.workload == DEFAULT_WORKLOAD:
+        pf = prefill_summary(ws, rank, local, peaks)
+
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         wk, secs, cores, desc = oracle_sample(w, args.cpu_budget)
@@ -762,6 +793,8 @@ def main():
                 per[n] = {"tflops": ach, "frac": ach / peaks["bf16"],
                           "mean_launch_us": 1000.0 * e["total_ms"] / e["launches"]}
             line["kernel_tflops"] = per
+        if pf is not None:
+            line["prefill_64k"] = pf
         print(json.dumps(line), flush=True)
     if ws > 1:
         import torch.distributed as dist
