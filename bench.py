@@ -643,6 +643,37 @@ def config_of(w):
 
 # --------------------------------------------------------------------------
 
+def run_dense(w, K, W, rank):
+    """Dense causal attention of the prefill's shape, in this build: nsa_prefill
+    with gates fixed to (0, 0, 1) and a window covering the sequence (the
+    closed form in which NSA is dense attention; the zero-gated branches are
+    skipped). Returns (ms per step, algorithmic flops per step)."""
+    from dynamic_block_sparse_nsa_b200 import nsa
+    inp = inputs.make_prefill(w, seed=w["seed"] + rank, device="cuda")
+    dt = inputs.DTYPES[w["dtype"]]
+    p = nsa.params(w["B"], w["T"], w["Hq"], w["Hkv"], w["d"], cmp_block=w["cmp_block"],
+                   cmp_stride=w["cmp_stride"], sel_block=w["sel_block"], top_n=w["top_n"],
+                   window=w["T"], dtype=dt, gate_mode=1, fixed_gates=(0.0, 0.0, 1.0))
+    Nc = nsa.num_cmp_blocks(w["T"], w["cmp_block"], w["cmp_stride"])
+    kc = torch.zeros(w["B"], Nc, w["Hkv"], w["d"], dtype=dt, device="cuda")
+    vc = torch.zeros_like(kc)
+    ws_buf = nsa.workspace(p, nsa.OP_PREFILL)
+    out = torch.empty_like(inp["q"])
+
+    def step():
+        nsa.nsa_prefill(p, inp["q"], inp["k"], inp["v"], kc, vc, None, out=out, ws=ws_buf,
+                        want_sel=False)
+
+    for _ in range(W):
+        step()
+    nsa.nsa_check()
+    ms = _run_steps(step, K, False)[0] / K
+    nsa.nsa_check()
+    T = w["T"]
+    flops = w["B"] * (T * (T + 1) // 2) * w["Hq"] * 4 * w["d"]
+    return ms, flops
+
+
 def prefill_summary(ws, rank, local, peaks, K=5, W=3):
     """The 65536-token bf16 prefill (the metric's prefill half), timed like the
     main line: whole-step TFLOP/s and every kernel against the bf16 peak."""
@@ -660,8 +691,15 @@ def prefill_summary(ws, rank, local, peaks, K=5, W=3):
         ach = per_launch / (e["total_ms"] / e["launches"] / 1000.0) / 1e12
         per[n] = {"tflops": ach, "frac": ach / peaks["bf16"], "peak": peaks["bf16"],
                   "mean_launch_us": 1000.0 * e["total_ms"] / e["launches"]}
+    dms, dfl = run_dense(w, 2, 1, rank)
+    dms = reduce_max(dms, ws)
+    dense = {"ms_per_step": dms, "tflops": dfl / (dms / 1000.0) / 1e12, "flops_per_step": dfl,
+             "frac": dfl / (dms / 1000.0) / 1e12 / peaks["bf16"],
+             "nsa_speedup": dms / (ms_max / K),
+             "how": "nsa_prefill with gates fixed to (0, 0, 1) and window = T (dense causal "
+                    "attention, same shape), 2 timed steps after 1 warm-up"}
     return {"workload": name, "value": work_all / (ms_max / 1000.0) / 1e12, "unit": "TFLOP/s",
-            "ms_per_step": ms_max / K, "steps": K, "warmup": W,
+            "ms_per_step": ms_max / K, "steps": K, "warmup": W, "dense_causal": dense,
             "flops_per_step": res["parts"], "kernel_tflops": per,
             "peak_source": peaks["src"], "clocks": res["clk"],
             "note": "algorithmic flops (4 d per query head and attended key); "

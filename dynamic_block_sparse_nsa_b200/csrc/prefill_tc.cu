@@ -63,6 +63,11 @@ struct PfArgs {
   float c;       // softmax scale * log2(e)
   int gate_mode;
   float fixed_gates[3];
+  // Branches a fixed zero gate removes (the output is unchanged without them):
+  int run_cmp;     // compressed attention (pass 1), needed for its output or the selection
+  int need_sel;    // block scores and top-n (pass 3, step 4)
+  int run_win;     // window attention (pass 2)
+  int direct_out;  // no selected branch: pf_main writes the bf16 output itself
 };
 
 __device__ __forceinline__ unsigned char* align1024(unsigned char* p) {
@@ -173,9 +178,10 @@ __global__ void __launch_bounds__(kMainThreads, 1)
   const int t0 = r * TQ;
   const int tlast = min(t0 + TQ - 1, a.T - 1);
   const int nvis = tlast >= CL - 1 ? min(a.Nc, (tlast - (CL - 1)) / CS + 1) : 0;
-  const int J1 = (nvis + KT - 1) / KT;
+  const int J1 = a.run_cmp ? (nvis + KT - 1) / KT : 0;  // compressed tiles (passes 1 and 3)
   const int ks0 = max(0, t0 - a.w + 1);
-  const int J2 = (tlast - ks0 + KT) / KT;
+  const int J2 = a.run_win ? (tlast - ks0 + KT) / KT : 0;  // window tiles
+  const int J3 = a.need_sel ? J1 : 0;                       // score tiles
   const int A = J1 + J2;
 
   if (threadIdx.x == 0) {
@@ -251,7 +257,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         if (i >= 1) v_of(i - 1);
       }
       if (A >= 1) v_of(A - 1);
-      for (int i = 0; i < J1; ++i) load(&tkc, b * a.Nc + i * KT);
+      for (int i = 0; i < J3; ++i) load(&tkc, b * a.Nc + i * KT);
       // this lane's last load must land before the CTA exits (earlier ones on
       // the same stage completed before their stage was reused)
       if (mine > 0) {
@@ -307,7 +313,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
           ++c;
         }
       }
-      for (int jj = 0; ok && jj < J1; ++jj) {
+      for (int jj = 0; ok && jj < J3; ++jj) {
         const int j = A + jj, bs = j & 1;
         if (j >= 2) ok = wait_or_abort(&bars->p_full[bs], (uint32_t)(((j - 2) >> 1) & 1), abort,
                                        a.err);
@@ -416,7 +422,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     ptx::named_bar_sync(1, 128);
 
     // step 3: block scores, thread = compressed key `row` of each tile
-    for (int jj = 0; jj < J1; ++jj) {
+    for (int jj = 0; jj < J3; ++jj) {
       const int j = A + jj, bs = j & 1;
       wait_or_abort(&bars->s_full[bs], (uint32_t)((j >> 1) & 1), abort, a.err);
       tc::fence_after_sync();
@@ -474,7 +480,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     // step 4: top-n per token, one warp per two tokens (processed together).
     // A candidate's key is (score bits + 1, ~index): unique, ordered by score
     // and then by the lower index; a taken block gets key 0.
-    {
+    if (a.need_sel) {
       int tokx[2], ncand[2], mine[2];
       uint32_t bh[2], bl[2];
       int32_t* dst[2];
@@ -543,26 +549,36 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     row_gates(a, sQ, swg, row, ATOM, gt);
     const float i1 = l1 > 0.f ? gt[0] / l1 : 0.f;
     const float i2 = l2 > 0.f ? gt[2] / l2 : 0.f;
-    float* dst = a.acc + ((size_t)(b * a.T + t) * a.Hq + g * G + h) * D;
-    // (O1 is never written when no compressed block is visible: i1 = 0 skips it)
+    const size_t orow = ((size_t)(b * a.T + t) * a.Hq + g * G + h) * D;
+    // An accumulator a branch never wrote (no visible key, or the branch
+    // skipped) has l = 0, so i = 0 keeps its unwritten columns out.
 #pragma unroll 1
     for (int c16 = 0; c16 < 8; ++c16) {  // runs once per row: kept compact
       uint32_t u1[16], u2[16];
       tc::ld16_sync(tl + kO1 + c16 * 16, u1);
       tc::ld16_sync(tl + kO2 + c16 * 16, u2);
-      if (row_ok) {
+      float o[16];
 #pragma unroll
-        for (int e = 0; e < 16; e += 4) {
-          float4 o;
-          o.x = (i1 != 0.f ? __uint_as_float(u1[e]) * i1 : 0.f) + __uint_as_float(u2[e]) * i2;
-          o.y = (i1 != 0.f ? __uint_as_float(u1[e + 1]) * i1 : 0.f) + __uint_as_float(u2[e + 1]) * i2;
-          o.z = (i1 != 0.f ? __uint_as_float(u1[e + 2]) * i1 : 0.f) + __uint_as_float(u2[e + 2]) * i2;
-          o.w = (i1 != 0.f ? __uint_as_float(u1[e + 3]) * i1 : 0.f) + __uint_as_float(u2[e + 3]) * i2;
-          *reinterpret_cast<float4*>(dst + c16 * 16 + e) = o;
+      for (int e = 0; e < 16; ++e)
+        o[e] = (i1 != 0.f ? __uint_as_float(u1[e]) * i1 : 0.f) +
+               (i2 != 0.f ? __uint_as_float(u2[e]) * i2 : 0.f);
+      if (row_ok) {
+        if (a.direct_out) {
+          uint4 pk[2];
+          uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) pw[e] = ptx::pack_bf16(o[2 * e], o[2 * e + 1]);
+          uint4* dst = reinterpret_cast<uint4*>(a.out + orow + c16 * 16);
+          dst[0] = pk[0];
+          dst[1] = pk[1];
+        } else {
+          float4* dst = reinterpret_cast<float4*>(a.acc + orow + c16 * 16);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dst[e] = make_float4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
         }
       }
     }
-    if (row_ok) a.gslc[(size_t)(b * a.T + t) * a.Hq + g * G + h] = gt[1];
+    if (row_ok && !a.direct_out) a.gslc[(size_t)(b * a.T + t) * a.Hq + g * G + h] = gt[1];
   }
 
   tc::fence_before_sync();
@@ -1031,6 +1047,12 @@ cudaError_t launch_prefill_tc(const nsa_params& p, const void* q, const void* k,
   a.c = scale * 1.4426950408889634f;
   a.gate_mode = p.gate_mode;
   for (int i = 0; i < 3; ++i) a.fixed_gates[i] = p.fixed_gates[i];
+  const bool fixed = p.gate_mode == 1;
+  const bool slc_branch = !(fixed && p.fixed_gates[1] == 0.f);
+  a.need_sel = slc_branch || sel_out != nullptr;
+  a.run_cmp = !(fixed && p.fixed_gates[0] == 0.f) || a.need_sel;
+  a.run_win = !(fixed && p.fixed_gates[2] == 0.f);
+  a.direct_out = !slc_branch;
 
   const uint64_t BT = (uint64_t)p.B * p.T;
   CUtensorMap tq, tq16, tk, tv, tk64, tv64, tkc, tvc;
@@ -1059,6 +1081,7 @@ cudaError_t launch_prefill_tc(const nsa_params& p, const void* q, const void* k,
     pf_main_kernel<<<(unsigned)grid, kMainThreads, sm1, stream>>>(tq, tkc, tvc, tk, tv, a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
+  if (a.direct_out) return cudaSuccess;
   const size_t sm2 = slc_smem();
   if (first_use(1))
     cudaFuncSetAttribute(pf_slc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);

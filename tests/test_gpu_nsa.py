@@ -153,3 +153,31 @@ def test_decode_independent_of_stale_workspace(cuda_ok):
     for o, s in outs[1:]:
         assert torch.equal(o, outs[0][0]) and torch.equal(s, outs[0][1])
     gc.run_nsa_decode(w, [12000, 9000, 4097, 777, 64, 11999], seed=11)
+
+
+@pytest.mark.parametrize("want_sel", [False, True])
+def test_prefill_bf16_dense_closed_form(want_sel):
+    # Gates fixed to (0, 0, 1) and a window covering the sequence reduce NSA to
+    # dense causal attention; the tensor-core path then skips the zero-gated
+    # branches (and the selection, unless sel_idx is requested).
+    from dynamic_block_sparse_nsa_b200 import nsa
+    from tests import dense_ref, parity
+    T = 700
+    w = inputs.workload("nsa_prefill_bf16_t8192", T=T, Hq=16, Hkv=1, window=4096, gate_mode=1,
+                        fixed_gates=(0.0, 0.0, 1.0))
+    inp = inputs.make_prefill(w, 5)
+    p = gc.nsa_params_for(w)
+    dev = {k_: v_.cuda() for k_, v_ in inp.items()}
+    kc, vc = nsa.nsa_compress_kv(p, dev["k"], dev["v"], dev["w_cmp"])
+    out, sel = nsa.nsa_prefill(p, dev["q"], dev["k"], dev["v"], kc, vc, None, want_sel=want_sel)
+    nsa.nsa_check()
+    q, k, v = gc.f64(inp["q"])[0], gc.f64(inp["k"])[0], gc.f64(inp["v"])[0]
+    ref = np.stack([dense_ref.masked_attention(q[:, h], k[:, 0], v[:, 0], dense_ref.causal_mask(T),
+                                               1.0 / np.sqrt(128))[0] for h in range(16)], axis=1)
+    parity.check_output(gc.f64(out)[0], ref, "bf16")
+    if want_sel:
+        s = sel.cpu().numpy()[0, :, 0]
+        assert (s[:, 0] == 0).all()
+        for t in range(T):
+            row = s[t][s[t] >= 0]
+            assert len(row) == min(w["top_n"], t // 64 + 1) and (np.diff(row) > 0).all()
