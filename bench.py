@@ -194,8 +194,9 @@ def moba_flops(w, sel_h):
     tt = np.broadcast_to(t[None, :, None, None], sel.shape)
     cnt = np.where(sel >= 0, np.minimum(sel * m + m - 1, tt) - sel * m + 1, 0)
     attn = int(cnt.sum()) * 4 * d
+    own = int((t - (t // m) * m + 1).sum()) * Hq * sel.shape[0] * 4 * d
     gate = int((t // m).sum()) * Hq * 2 * d
-    return dict(attn=attn, gate=gate)
+    return dict(attn=attn, gate=gate, attn_own=own, attn_past=attn - own)
 
 
 # --------------------------------------------------------------------------
@@ -465,7 +466,7 @@ def run_moba(w, K, W, ws, rank, local, e2e=True):
     res = timed(step, K, W, ws, local)
     nsa.nsa_check()
     fl = moba_flops(w, sel.cpu().numpy())
-    res.update(work=sum(fl.values()), parts=fl)
+    res.update(work=fl["attn"] + fl["gate"], parts=fl)
     if e2e:
         hq, hk, hv = (inp[x].cpu().pin_memory() for x in ("q", "k", "v"))
         ho = torch.empty(out.shape, dtype=out.dtype).pin_memory()
@@ -512,7 +513,8 @@ def kernel_work(kind, name, res, w):
         }
         return per.get(name), "tensor"
     p = res["parts"]
-    per = {"moba_rows_simt": p["attn"] + p["gate"], "moba_attn": p["attn"]}
+    per = {"moba_rows_simt": p["attn"] + p["gate"], "moba_own": p["attn_own"],
+           "moba_blk": p["attn_past"]}
     return per.get(name), "tensor"
 
 
@@ -819,7 +821,7 @@ def main():
                                     **{k: v for k, v in res["parts"].items()}}
             line["hbm_frac_nominal_8tbs"] = value / 8000.0
         else:
-            line["flops_per_step"] = res["parts"]
+            line["flops_per_step"] = {k: v for k, v in res["parts"].items()}
             # every traced kernel against the bf16 peak (first timed region's events)
             per = {}
             for n, e in res["table0"].items():

@@ -126,6 +126,15 @@ cudaError_t launch_nsa_rows_simt(const NsaRowArgs& a, cudaStream_t stream);
 
 size_t moba_simt_smem(const MobaArgs& a);
 cudaError_t launch_moba_simt(const MobaArgs& a, cudaStream_t stream);
+cudaError_t launch_moba_block_mean(const MobaArgs& a, cudaStream_t stream);
+
+// Tensor-core MoBA: bf16, d = 128, block a multiple of 128 (<= 2048),
+// top_k <= 8. Its workspace starts with the block means (kbar_bytes).
+bool moba_tc_eligible(const nsa_params& p);
+size_t moba_tc_ws_bytes(const nsa_params& p, size_t kbar_bytes);
+cudaError_t launch_moba_tc(const nsa_params& p, const void* q, const void* k, const void* v,
+                           void* out, int32_t* sel_out, void* ws, size_t kbar_bytes,
+                           unsigned* err, cudaStream_t stream);
 
 cudaError_t launch_bounded_wait(const int32_t* flag, int max_iters, unsigned* err,
                                 cudaStream_t stream);

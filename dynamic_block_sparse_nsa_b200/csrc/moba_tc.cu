@@ -1,0 +1,860 @@
+// MoBA causal prefill on the sm_100a tensor cores, block-centric (EP94 notes
+// sections nine and ten: mean-pooled block keys, parameter-free top-k gating,
+// the query's own block always attended; LateTalk ep.103). bf16, d = 128,
+// block m a multiple of 128 (m <= 2048), top_k <= 8.
+//
+// A query row (token t, head h) attends to its own block c = t / m over
+// [c m, t] and to top_k - 1 earlier blocks chosen by q . mean(K_block). With
+// independent per-row choices no two rows share much, so the work is grouped
+// by key block instead of by query (the gather / re-index view of the pages):
+//   moba_gate  scores and picks per row on CUDA cores in fp32 (block means
+//              staged in shared memory), the selection row, and per-(head,
+//              block) pick counts;
+//   moba_scan  offsets of each (sequence, head, block) bucket and of its
+//              128-row tiles;
+//   moba_fill  the rows of every bucket (token, slot);
+//   moba_blk   per bucket tile: 128 gathered query rows against the block's m
+//              keys (tcgen05, TMEM accumulators), written as a normalised
+//              partial output and its log-sum-exp;
+//   moba_own   per 128 consecutive tokens of one head: causal attention over
+//              the own block, merged with the row's partials into the output.
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include <algorithm>
+#include <cstdint>
+
+#include "internal.h"
+#include "ptx.cuh"
+#include "tcgen05.cuh"
+
+namespace nsa {
+namespace {
+
+constexpr int D = 128;
+constexpr int KT = 128;           // keys per tile, rows per query tile
+constexpr uint32_t ATOM = 16384;  // one d-half of a 128-row bf16 tile
+constexpr uint32_t TILE = 32768;
+constexpr uint64_t kWaitNs = 2000000000ull;
+constexpr int kMaxTopk = 8;
+constexpr int kStages = 4;
+constexpr int kThreads = 192;     // TMA lanes, MMA thread, 4 softmax warps
+constexpr uint32_t kNegInf = 0xff800000u;
+constexpr int kGateChunk = 64;    // block means staged per round in moba_gate
+
+struct MobaTcArgs {
+  const __nv_bfloat16* q;
+  const float* kbar;      // [B, nfull, Hkv, d]
+  __nv_bfloat16* out;
+  int32_t* sel;           // [B, T, Hq, topk]
+  int32_t* cnt;           // [NB] picks per bucket (b, h, j)
+  int32_t* off;           // [NB] first row of each bucket in `list`
+  int32_t* toff;          // [NB + 1] first tile of each bucket
+  int32_t* cur;           // [NB] fill cursors
+  int32_t* list;          // rows: t * 8 + slot
+  float* po;              // [B, T, Hq, topk - 1, d] partial outputs (normalised)
+  float* plse;            // [B, T, Hq, topk - 1] their log2-sum-exp
+  unsigned* err;
+  int B, T, Hq, Hkv, m, topk, nfull, NB;
+  float c;                // softmax scale * log2(e)
+};
+
+__device__ __forceinline__ unsigned char* align1024(unsigned char* p) {
+  return (unsigned char*)(((uintptr_t)p + 1023) & ~(uintptr_t)1023);
+}
+
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                              unsigned* err) {
+  if (*abort) return false;
+  if (ptx::mbar_wait(bar, parity, kWaitNs)) return true;
+  *abort = 1;
+  atomicOr(err, kErrTimeout);
+  return false;
+}
+
+__device__ __forceinline__ uint64_t kmaj(uint32_t base, int ks) {
+  return tc::sdesc(base + (ks >> 2) * ATOM + (ks & 3) * 32, 16, 1024, tc::kSw128);
+}
+
+__device__ __forceinline__ uint64_t mnmaj(uint32_t base, int ks) {
+  return tc::sdesc(base + ks * 2048, ATOM, 1024, tc::kSw128);
+}
+
+// ============================================================================
+// gate, scan, fill
+// ============================================================================
+
+// One thread per (token, head); 128 tokens of one head per CTA. Past blocks
+// j < t / m are scored with q . kbar[j] in fp32 and the top_k - 1 best kept
+// (higher score first, ties to the lower block: blocks arrive in increasing
+// order and only a strictly higher score displaces a kept one).
+__global__ void __launch_bounds__(128) moba_gate_kernel(MobaTcArgs a) {
+  __shared__ float kb[kGateChunk * D];
+  const int t0 = blockIdx.x * 128, h = blockIdx.y, b = blockIdx.z;
+  const int g = h / (a.Hq / a.Hkv);
+  const int t = t0 + threadIdx.x;
+  const bool ok = t < a.T;
+  const int own = ok ? t / a.m : 0;
+  const int own_max = min(t0 + 127, a.T - 1) / a.m;
+  const int want = a.topk - 1;
+  float q[D];
+  if (ok) {
+    const uint4* qr = reinterpret_cast<const uint4*>(a.q + ((size_t)(b * a.T + t) * a.Hq + h) * D);
+#pragma unroll
+    for (int c8 = 0; c8 < D / 8; ++c8) {
+      const uint4 v = __ldg(qr + c8);
+      const __nv_bfloat162* e = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 f = __bfloat1622float2(e[k]);
+        q[c8 * 8 + 2 * k] = f.x;
+        q[c8 * 8 + 2 * k + 1] = f.y;
+      }
+    }
+  }
+  float bs[kMaxTopk];
+  int bj[kMaxTopk];
+#pragma unroll
+  for (int i = 0; i < kMaxTopk; ++i) {
+    bs[i] = -INFINITY;
+    bj[i] = -1;
+  }
+  for (int c0 = 0; c0 < own_max; c0 += kGateChunk) {
+    const int nb = min(kGateChunk, own_max - c0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < nb * D / 4; i += 128) {
+      const int j = i / (D / 4), e4 = i % (D / 4);
+      reinterpret_cast<float4*>(kb)[i] = __ldg(reinterpret_cast<const float4*>(
+          a.kbar + (((size_t)b * a.nfull + c0 + j) * a.Hkv + g) * D) + e4);
+    }
+    __syncthreads();
+    const int jend = ok ? min(nb, own - c0) : 0;
+    for (int jj = 0; jj < jend; ++jj) {
+      const float4* kr = reinterpret_cast<const float4*>(kb + jj * D);
+      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+      for (int e4 = 0; e4 < D / 4; ++e4) {
+        const float4 kv = kr[e4];
+        s0 = fmaf(q[4 * e4], kv.x, s0);
+        s1 = fmaf(q[4 * e4 + 1], kv.y, s1);
+        s2 = fmaf(q[4 * e4 + 2], kv.z, s2);
+        s3 = fmaf(q[4 * e4 + 3], kv.w, s3);
+      }
+      float s = (s0 + s1) + (s2 + s3);
+      int j = c0 + jj;
+      // insert into the descending list (strictly better only)
+#pragma unroll
+      for (int i = 0; i < kMaxTopk; ++i) {
+        if (i < want && s > bs[i]) {
+          const float ts = bs[i];
+          const int tj = bj[i];
+          bs[i] = s;
+          bj[i] = j;
+          s = ts;
+          j = tj;
+        }
+      }
+    }
+  }
+  if (!ok) return;
+  // the row: the picks (or every earlier block) and the own block, ascending
+  int row[kMaxTopk];
+  int n = 0;
+  if (own <= want) {
+    for (int j = 0; j <= own; ++j) row[n++] = j;
+  } else {
+#pragma unroll
+    for (int i = 0; i < kMaxTopk; ++i)
+      if (i < want) row[n++] = bj[i];
+    for (int i = 1; i < n; ++i) {  // insertion sort, n <= 7
+      const int x = row[i];
+      int p = i - 1;
+      while (p >= 0 && row[p] > x) {
+        row[p + 1] = row[p];
+        --p;
+      }
+      row[p + 1] = x;
+    }
+    row[n++] = own;
+  }
+  int32_t* dst = a.sel + ((size_t)(b * a.T + t) * a.Hq + h) * a.topk;
+  for (int i = 0; i < a.topk; ++i) dst[i] = i < n ? row[i] : -1;
+  for (int i = 0; i + 1 < n; ++i)  // every entry but the own block is a past pick
+    atomicAdd(a.cnt + ((size_t)b * a.Hq + h) * a.nfull + row[i], 1);
+}
+
+// Exclusive prefix sums of the bucket counts (rows) and of their 128-row
+// tiles, in one CTA.
+__global__ void __launch_bounds__(1024) moba_scan_kernel(MobaTcArgs a) {
+  __shared__ int wsum[2][32];
+  __shared__ int carry[2];
+  if (threadIdx.x == 0) carry[0] = carry[1] = 0;
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int base = 0; base < a.NB; base += 1024) {
+    const int i = base + threadIdx.x;
+    const int c = i < a.NB ? a.cnt[i] : 0;
+    int v0 = c, v1 = (c + KT - 1) / KT;
+    int x0 = v0, x1 = v1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y0 = __shfl_up_sync(0xffffffffu, x0, o), y1 = __shfl_up_sync(0xffffffffu, x1, o);
+      if (lane >= o) {
+        x0 += y0;
+        x1 += y1;
+      }
+    }
+    if (lane == 31) {
+      wsum[0][warp] = x0;
+      wsum[1][warp] = x1;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      int s0 = wsum[0][lane], s1 = wsum[1][lane];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y0 = __shfl_up_sync(0xffffffffu, s0, o), y1 = __shfl_up_sync(0xffffffffu, s1, o);
+        if (lane >= o) {
+          s0 += y0;
+          s1 += y1;
+        }
+      }
+      wsum[0][lane] = s0;
+      wsum[1][lane] = s1;
+    }
+    __syncthreads();
+    const int pre0 = carry[0] + (warp ? wsum[0][warp - 1] : 0) + x0 - v0;
+    const int pre1 = carry[1] + (warp ? wsum[1][warp - 1] : 0) + x1 - v1;
+    if (i < a.NB) {
+      a.off[i] = pre0;
+      a.toff[i] = pre1;
+      a.cur[i] = 0;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      carry[0] += wsum[0][31];
+      carry[1] += wsum[1][31];
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) a.toff[a.NB] = carry[1];
+}
+
+// Rows into buckets: list[off[bucket] + k] = t * 8 + slot.
+__global__ void moba_fill_kernel(MobaTcArgs a) {
+  const long long n = (long long)a.B * a.T * a.Hq;
+  for (long long r = blockIdx.x * (long long)blockDim.x + threadIdx.x; r < n;
+       r += (long long)gridDim.x * blockDim.x) {
+    const int h = (int)(r % a.Hq);
+    const long long bt = r / a.Hq;
+    const int b = (int)(bt / a.T), t = (int)(bt % a.T);
+    const int32_t* s = a.sel + r * a.topk;
+    const int own = t / a.m;
+    int slot = 0;
+    for (int i = 0; i < a.topk; ++i) {
+      const int j = s[i];
+      if (j < 0 || j == own) continue;
+      const int bk = (b * a.Hq + h) * a.nfull + j;
+      const int pos = atomicAdd(a.cur + bk, 1);
+      a.list[a.off[bk] + pos] = t * 8 + slot;
+      ++slot;
+    }
+  }
+}
+
+// ============================================================================
+// the attention kernels: shared pieces
+// ============================================================================
+
+struct Bars {
+  uint64_t full[kStages], empty[kStages];
+  uint64_t q_full[2], q_free[2], s_full[2], p_full[2], o_done[2], fin;
+  uint32_t tmem;
+  int abort;
+};
+
+constexpr uint32_t kO = 0, kS0 = 128;  // TMEM: O at 0, S buffers at 128 and 256
+
+__device__ void init_bars(Bars* bars, int q_full_count) {
+  for (int i = 0; i < kStages; ++i) {
+    ptx::mbar_init(&bars->full[i], 1);
+    ptx::mbar_init(&bars->empty[i], 1);
+  }
+  for (int i = 0; i < 2; ++i) {
+    ptx::mbar_init(&bars->q_full[i], q_full_count);
+    ptx::mbar_init(&bars->q_free[i], 1);
+    ptx::mbar_init(&bars->s_full[i], 1);
+    ptx::mbar_init(&bars->p_full[i], 128);
+    ptx::mbar_init(&bars->o_done[i], 1);
+  }
+  ptx::mbar_init(&bars->fin, 1);
+  bars->abort = 0;
+  ptx::fence_mbar_init();
+}
+
+// One K or V tile (128 keys x 128 d) from lane `lane` of the producer warp:
+// loads c = lane (mod kStages) go to stage `lane`.
+struct Producer {
+  unsigned char* ring;
+  Bars* bars;
+  volatile int* abort;
+  unsigned* err;
+  int lane, c = 0, mine = 0;
+  bool ok = true;
+  __device__ void load(const CUtensorMap* m, int g, int z, uint64_t pol) {
+    const int cc = c++;
+    if (!ok || cc % kStages != lane) return;
+    if (cc >= kStages &&
+        !wait_or_abort(&bars->empty[lane], (uint32_t)(((cc / kStages) - 1) & 1), abort, err)) {
+      ok = false;
+      return;
+    }
+    unsigned char* dst = ring + lane * TILE;
+    ptx::mbar_arrive_expect_tx(&bars->full[lane], TILE);
+    ptx::tma_load_3d(dst, m, &bars->full[lane], 0, g, z, pol);
+    ptx::tma_load_3d(dst + ATOM, m, &bars->full[lane], 64, g, z, pol);
+    ++mine;
+  }
+  __device__ void drain() {
+    if (mine > 0) {
+      const int last = lane + (mine - 1) * kStages;
+      if (!ptx::mbar_wait(&bars->full[lane], (uint32_t)((last / kStages) & 1), kWaitNs))
+        atomicOr(err, kErrTimeout);
+    }
+  }
+};
+
+// MMA side of one query tile with `nk` key tiles: S_u = Q K_u^T into S buffer
+// (j & 1), O += P_u V_u with P from TMEM; j and c are the running tile and
+// load counters of the CTA.
+struct Mma {
+  Bars* bars;
+  volatile int* abort;
+  unsigned* err;
+  uint32_t tmem, r0;
+  int j = 0, c = 0;
+  bool ok = true;
+  __device__ int take() {
+    const int st = c % kStages;
+    if (ok) ok = wait_or_abort(&bars->full[st], (uint32_t)((c / kStages) & 1), abort, err);
+    tc::fence_after_sync();
+    return st;
+  }
+  __device__ void tile(uint32_t q0, int nk, int qbuf) {
+    const uint32_t iss = tc::idesc_bf16(128, 128, false, false);
+    const uint32_t its = tc::idesc_bf16(128, 128, false, true);
+    const int j0 = j;
+    for (int u = 0; ok && u <= nk; ++u) {
+      if (u < nk) {
+        const int jj = j0 + u, bs = jj & 1;
+        if (jj >= 2)
+          ok = ok && wait_or_abort(&bars->p_full[bs], (uint32_t)(((jj - 2) >> 1) & 1), abort, err);
+        const int st = take();
+        if (!ok) break;
+        const uint32_t kb = r0 + st * TILE;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          tc::mma_ss(tmem + kS0 + bs * 128, kmaj(q0, ks), kmaj(kb, ks), iss, ks > 0);
+        tc::commit(&bars->empty[st]);
+        tc::commit(&bars->s_full[bs]);
+        ++c;
+        if (u == nk - 1) tc::commit(&bars->q_free[qbuf]);
+      }
+      if (u >= 1) {
+        const int pj = j0 + u - 1, pb = pj & 1;
+        ok = ok && wait_or_abort(&bars->p_full[pb], (uint32_t)((pj >> 1) & 1), abort, err);
+        tc::fence_after_sync();
+        const int st = take();
+        if (!ok) break;
+        const uint32_t vb = r0 + st * TILE;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          tc::mma_ts(tmem + kO, tmem + kS0 + pb * 128 + ks * 8, mnmaj(vb, ks), its,
+                     (u > 1 || ks > 0));
+        tc::commit(&bars->empty[st]);
+        tc::commit(&bars->o_done[pj & 1]);
+        ++c;
+      }
+    }
+    j = j0 + nk;
+  }
+};
+
+// Softmax side: thread `row` of the query tile, one S tile at a time; keys at
+// index >= klim are masked (the causal edge). m is kept in the log2 domain.
+struct Softmax {
+  Bars* bars;
+  volatile int* abort;
+  unsigned* err;
+  uint32_t tl;
+  float cs;
+  int j = 0;
+  __device__ void tile(int kb, int klim, float& m, float& l) {
+    const int bs = j & 1;
+    wait_or_abort(&bars->s_full[bs], (uint32_t)((j >> 1) & 1), abort, err);
+    tc::fence_after_sync();
+    uint32_t u[128];
+    tc::ld128_sync(tl + kS0 + bs * 128, u);
+    if (kb + KT > klim) {
+#pragma unroll
+      for (int e = 0; e < 128; ++e)
+        if (kb + e >= klim) u[e] = kNegInf;
+    }
+    float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+    for (int e = 0; e < 128; e += 4) {
+      mx0 = fmaxf(mx0, __uint_as_float(u[e]));
+      mx1 = fmaxf(mx1, __uint_as_float(u[e + 1]));
+      mx2 = fmaxf(mx2, __uint_as_float(u[e + 2]));
+      mx3 = fmaxf(mx3, __uint_as_float(u[e + 3]));
+    }
+    const float mt = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * cs;
+    const float mn = fmaxf(m, mt);
+    if (mn != -INFINITY && (m == -INFINITY || mn > m + 8.f)) {
+      if (m != -INFINITY) {
+        const float f = exp2f(m - mn);
+        l *= f;
+        wait_or_abort(&bars->o_done[(j - 1) & 1], (uint32_t)(((j - 1) >> 1) & 1), abort, err);
+        tc::fence_after_sync();
+#pragma unroll 1
+        for (int q4 = 0; q4 < 8; ++q4) {
+          uint32_t w[16];
+          tc::ld16_sync(tl + kO + q4 * 16, w);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) w[e] = __float_as_uint(__uint_as_float(w[e]) * f);
+          tc::st16(tl + kO + q4 * 16, w);
+        }
+        tc::st_wait();
+      }
+      m = mn;
+    }
+    const float nm = m == -INFINITY ? 0.f : -m;
+    float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) {
+      uint32_t pk[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const float p0 = ptx::ex2(fmaf(__uint_as_float(u[q4 * 32 + 2 * e]), cs, nm));
+        const float p1 = ptx::ex2(fmaf(__uint_as_float(u[q4 * 32 + 2 * e + 1]), cs, nm));
+        ls0 += p0;
+        ls1 += p1;
+        pk[e] = ptx::pack_bf16(p0, p1);
+      }
+      tc::st16(tl + kS0 + bs * 128 + q4 * 16, pk);
+    }
+    l += ls0 + ls1;
+    tc::st_wait();
+    tc::fence_before_sync();
+    ptx::mbar_arrive(&bars->p_full[bs]);
+    ++j;
+  }
+};
+
+// ============================================================================
+// moba_blk: bucket tiles (gathered rows x one earlier block)
+// ============================================================================
+
+__device__ __forceinline__ int tile_bucket(const MobaTcArgs& a, int i) {
+  int lo = 0, hi = a.NB - 1;  // largest bucket with toff <= i
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (a.toff[mid] <= i) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+struct BlkTile {
+  int b, h, j, first, nrow;  // rows list[first .. first + nrow)
+};
+
+__device__ __forceinline__ BlkTile blk_tile(const MobaTcArgs& a, int i) {
+  BlkTile w;
+  const int bk = tile_bucket(a, i);
+  w.j = bk % a.nfull;
+  const int bh = bk / a.nfull;
+  w.h = bh % a.Hq;
+  w.b = bh / a.Hq;
+  const int k = i - a.toff[bk];
+  w.first = a.off[bk] + k * KT;
+  w.nrow = min(KT, a.cnt[bk] - k * KT);
+  return w;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    moba_blk_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+                    const MobaTcArgs a) {
+  extern __shared__ unsigned char smraw[];
+  unsigned char* base = align1024(smraw);
+  unsigned char* sQ = base;              // 2 x 32 KB
+  unsigned char* ring = base + 2 * TILE;
+  Bars* bars = reinterpret_cast<Bars*>(ring + kStages * TILE);
+  volatile int* abort = &bars->abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntile = a.toff[a.NB];
+  const int G = a.Hq / a.Hkv;
+  const int nk = a.m / KT;
+
+  if (threadIdx.x == 0) init_bars(bars, 128);
+  if (warp == 1) {
+    tc::tmem_alloc(&bars->tmem, 512);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = bars->tmem;
+
+  if (warp == 0) {
+    if (lane < kStages) {
+      if (lane == 0) {
+        ptx::prefetch_tmap(&tk);
+        ptx::prefetch_tmap(&tv);
+      }
+      Producer pr{ring, bars, abort, a.err, lane};
+      const uint64_t keep = ptx::policy_evict_last();
+      for (int i = blockIdx.x; pr.ok && i < ntile; i += gridDim.x) {
+        const BlkTile w = blk_tile(a, i);
+        const int g = w.h / G;
+        const int z0 = w.b * a.T + w.j * a.m;
+        for (int u = 0; u < nk; ++u) {
+          pr.load(&tk, g, z0 + u * KT, keep);
+          if (u >= 1) pr.load(&tv, g, z0 + (u - 1) * KT, keep);
+        }
+        pr.load(&tv, g, z0 + (nk - 1) * KT, keep);
+      }
+      pr.drain();
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      Mma mm{bars, abort, a.err, tmem, ptx::smem_u32(ring)};
+      int k = 0;
+      for (int i = blockIdx.x; mm.ok && i < ntile; i += gridDim.x, ++k) {
+        const int qb = k & 1;
+        mm.ok = wait_or_abort(&bars->q_full[qb], (uint32_t)((k >> 1) & 1), abort, a.err);
+        tc::fence_after_sync();
+        mm.tile(ptx::smem_u32(sQ + qb * TILE), nk, qb);
+      }
+      tc::commit(&bars->fin);
+      if (!ptx::mbar_wait(&bars->fin, 0, kWaitNs)) atomicOr(a.err, kErrTimeout);
+    }
+  } else {
+    const int qd = warp & 3;
+    const int row = qd * 32 + lane;
+    Softmax sm{bars, abort, a.err, tmem + ((uint32_t)(qd * 32) << 16), a.c};
+    // gather 128 query rows of tile i into Q buffer qb (zeros past the bucket)
+    auto gather = [&](int i, int kq) {
+      const int qb = kq & 1;
+      if (kq >= 2) wait_or_abort(&bars->q_free[qb], (uint32_t)(((kq >> 1) - 1) & 1), abort, a.err);
+      const BlkTile w = blk_tile(a, i);
+      unsigned char* dq = sQ + qb * TILE;
+      uint4 v[16];
+      if (row < w.nrow) {
+        const int e = a.list[w.first + row];
+        const uint4* src = reinterpret_cast<const uint4*>(
+            a.q + ((size_t)(w.b * a.T + (e >> 3)) * a.Hq + w.h) * D);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) v[c] = __ldg(src + c);
+      } else {
+#pragma unroll
+        for (int c = 0; c < 16; ++c) v[c] = make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int c = 0; c < 16; ++c)
+        *reinterpret_cast<uint4*>(dq + (c >> 3) * ATOM + row * 128 + (((c & 7) ^ (row & 7)) << 4)) =
+            v[c];
+      ptx::fence_proxy_async();
+      ptx::mbar_arrive(&bars->q_full[qb]);
+    };
+    int k = 0;
+    if (blockIdx.x < (unsigned)ntile) gather(blockIdx.x, 0);
+    for (int i = blockIdx.x; i < ntile; i += gridDim.x, ++k) {
+      if (i + (int)gridDim.x < ntile) gather(i + gridDim.x, k + 1);
+      const BlkTile w = blk_tile(a, i);
+      float m = -INFINITY, l = 0.f;
+      for (int u = 0; u < nk; ++u) sm.tile(u * KT, 1 << 30, m, l);
+      wait_or_abort(&bars->o_done[(sm.j - 1) & 1], (uint32_t)(((sm.j - 1) >> 1) & 1), abort,
+                    a.err);
+      tc::fence_after_sync();
+      const bool live = row < w.nrow;
+      const int e = live ? a.list[w.first + row] : 0;
+      const size_t pr = ((size_t)(w.b * a.T + (e >> 3)) * a.Hq + w.h) * (a.topk - 1) + (e & 7);
+      const float il = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll 1
+      for (int c16 = 0; c16 < 8; ++c16) {
+        uint32_t o[16];
+        tc::ld16_sync(sm.tl + kO + c16 * 16, o);
+        if (live) {
+          float4* dst = reinterpret_cast<float4*>(a.po + pr * D + c16 * 16);
+#pragma unroll
+          for (int x = 0; x < 4; ++x)
+            dst[x] = make_float4(__uint_as_float(o[4 * x]) * il, __uint_as_float(o[4 * x + 1]) * il,
+                                 __uint_as_float(o[4 * x + 2]) * il,
+                                 __uint_as_float(o[4 * x + 3]) * il);
+        }
+      }
+      if (live) a.plse[pr] = m + __log2f(l);
+      tc::fence_before_sync();
+    }
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == 1) tc::tmem_dealloc(tmem, 512);
+}
+
+// ============================================================================
+// moba_own: own block, causal, merged with the partials
+// ============================================================================
+
+__global__ void __launch_bounds__(kThreads, 1)
+    moba_own_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                    const __grid_constant__ CUtensorMap tv, const MobaTcArgs a) {
+  extern __shared__ unsigned char smraw[];
+  unsigned char* base = align1024(smraw);
+  unsigned char* sQ = base;
+  unsigned char* ring = base + TILE;
+  Bars* bars = reinterpret_cast<Bars*>(ring + kStages * TILE);
+  volatile int* abort = &bars->abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ntq = (a.T + KT - 1) / KT;
+  const int bh = blockIdx.x % (a.B * a.Hq);
+  const int r = blockIdx.x / (a.B * a.Hq);
+  const int b = bh / a.Hq, h = bh % a.Hq, g = h / (a.Hq / a.Hkv);
+  const int t0 = r * KT;
+  const int tlast = min(t0 + KT - 1, a.T - 1);
+  const int c0 = (t0 / a.m) * a.m;  // own block start (a 128-token tile never straddles blocks)
+  const int nk = (tlast - c0) / KT + 1;
+  (void)ntq;
+
+  if (threadIdx.x == 0) init_bars(bars, 1);
+  if (warp == 1) {
+    tc::tmem_alloc(&bars->tmem, 512);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = bars->tmem;
+
+  if (warp == 0) {
+    if (lane < kStages) {
+      if (lane == 0) {
+        ptx::prefetch_tmap(&tq);
+        ptx::prefetch_tmap(&tk);
+        ptx::prefetch_tmap(&tv);
+        ptx::mbar_arrive_expect_tx(&bars->q_full[0], TILE);
+        ptx::tma_load_3d(sQ, &tq, &bars->q_full[0], 0, h, b * a.T + t0, ptx::policy_evict_first());
+        ptx::tma_load_3d(sQ + ATOM, &tq, &bars->q_full[0], 64, h, b * a.T + t0,
+                         ptx::policy_evict_first());
+      }
+      Producer pr{ring, bars, abort, a.err, lane};
+      const uint64_t keep = ptx::policy_evict_last();
+      const int z0 = b * a.T + c0;
+      for (int u = 0; u < nk; ++u) {
+        pr.load(&tk, g, z0 + u * KT, keep);
+        if (u >= 1) pr.load(&tv, g, z0 + (u - 1) * KT, keep);
+      }
+      pr.load(&tv, g, z0 + (nk - 1) * KT, keep);
+      pr.drain();
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      Mma mm{bars, abort, a.err, tmem, ptx::smem_u32(ring)};
+      mm.ok = wait_or_abort(&bars->q_full[0], 0, abort, a.err);
+      tc::fence_after_sync();
+      mm.tile(ptx::smem_u32(sQ), nk, 0);
+      tc::commit(&bars->fin);
+      if (!ptx::mbar_wait(&bars->fin, 0, kWaitNs)) atomicOr(a.err, kErrTimeout);
+    }
+  } else {
+    const int qd = warp & 3;
+    const int row = qd * 32 + lane;
+    const int t = min(t0 + row, a.T - 1);
+    const bool live = t0 + row < a.T;
+    Softmax sm{bars, abort, a.err, tmem + ((uint32_t)(qd * 32) << 16), a.c};
+    float m = -INFINITY, l = 0.f;
+    for (int u = 0; u < nk; ++u) sm.tile(c0 + u * KT, t + 1, m, l);
+    wait_or_abort(&bars->o_done[(nk - 1) & 1], (uint32_t)(((nk - 1) >> 1) & 1), abort, a.err);
+    tc::fence_after_sync();
+    // merge: own (o / l, lse = m + log2 l) with the row's partials
+    const int npast = min(a.topk - 1, t / a.m);
+    const size_t prow = ((size_t)(b * a.T + t) * a.Hq + h) * (a.topk - 1);
+    float lse[kMaxTopk];
+    float M = m + __log2f(l);  // key t itself is always visible: l > 0
+    const float lown = M;
+#pragma unroll
+    for (int s = 0; s < kMaxTopk - 1; ++s) {
+      lse[s] = (live && s < npast) ? a.plse[prow + s] : -INFINITY;
+      M = fmaxf(M, lse[s]);
+    }
+    const float wown = exp2f(lown - M) / l;
+    float wsum = exp2f(lown - M);
+    float wp[kMaxTopk];
+#pragma unroll
+    for (int s = 0; s < kMaxTopk - 1; ++s) {
+      wp[s] = s < npast ? exp2f(lse[s] - M) : 0.f;
+      wsum += wp[s];
+    }
+    const float inv = 1.f / wsum;
+    __nv_bfloat16* dst = a.out + ((size_t)(b * a.T + t) * a.Hq + h) * D;
+#pragma unroll 1
+    for (int c16 = 0; c16 < 8; ++c16) {
+      uint32_t o[16];
+      tc::ld16_sync(sm.tl + kO + c16 * 16, o);
+      float acc[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) acc[e] = __uint_as_float(o[e]) * wown;
+      for (int s = 0; s < npast; ++s) {
+        const float4* ps = reinterpret_cast<const float4*>(a.po + (prow + s) * D + c16 * 16);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+          const float4 pv = __ldg(ps + x);
+          acc[4 * x] = fmaf(wp[s], pv.x, acc[4 * x]);
+          acc[4 * x + 1] = fmaf(wp[s], pv.y, acc[4 * x + 1]);
+          acc[4 * x + 2] = fmaf(wp[s], pv.z, acc[4 * x + 2]);
+          acc[4 * x + 3] = fmaf(wp[s], pv.w, acc[4 * x + 3]);
+        }
+      }
+      if (live) {
+        uint4 pk[2];
+        uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) pw[e] = ptx::pack_bf16(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+        reinterpret_cast<uint4*>(dst + c16 * 16)[0] = pk[0];
+        reinterpret_cast<uint4*>(dst + c16 * 16)[1] = pk[1];
+      }
+    }
+  }
+
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == 1) tc::tmem_dealloc(tmem, 512);
+}
+
+size_t attn_smem(int qbufs) { return 1024 + (size_t)(qbufs + kStages) * TILE + sizeof(Bars); }
+
+bool first_use(int id) {
+  static bool seen[2][64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return true;
+  const bool f = !seen[id][dev];
+  seen[id][dev] = true;
+  return f;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
+
+bool moba_tc_eligible(const nsa_params& p) {
+  if (p.dtype != NSA_DTYPE_BF16 || p.d != D || p.Hkv < 1 || p.Hq % p.Hkv != 0) return false;
+  if (p.sel_block < KT || p.sel_block % KT != 0 || p.sel_block > 2048) return false;
+  if (p.top_n < 1 || p.top_n > kMaxTopk) return false;
+  return (long long)p.B * p.T * p.Hq < (1ll << 31) / D && (long long)p.B * p.T < (1ll << 30) / 8;
+}
+
+// Workspace after the block means: selection (when the caller passes none),
+// bucket counts / offsets / tile offsets / cursors, the bucket rows, the
+// partial outputs and their log-sum-exp.
+size_t moba_tc_ws_bytes(const nsa_params& p, size_t kbar_bytes) {
+  const size_t rows = (size_t)p.B * p.T * p.Hq;
+  const size_t NB = (size_t)p.B * p.Hq * (p.T / p.sel_block);
+  const size_t np = (size_t)(p.top_n - 1);
+  return align256(kbar_bytes) + align256(rows * p.top_n * 4) + 4 * align256((NB + 1) * 4) +
+         align256(rows * np * 4 + 4) + align256(rows * np * D * 4 + 4) + align256(rows * np * 4 + 4);
+}
+
+cudaError_t launch_moba_tc(const nsa_params& p, const void* q, const void* k, const void* v,
+                           void* out, int32_t* sel_out, void* ws, size_t kbar_bytes,
+                           unsigned* err, cudaStream_t stream) {
+  MobaTcArgs a{};
+  const size_t rows = (size_t)p.B * p.T * p.Hq;
+  a.B = p.B;
+  a.T = p.T;
+  a.Hq = p.Hq;
+  a.Hkv = p.Hkv;
+  a.m = p.sel_block;
+  a.topk = p.top_n;
+  a.nfull = p.T / p.sel_block;
+  a.NB = p.B * p.Hq * a.nfull;
+  const size_t np = (size_t)(p.top_n - 1);
+  unsigned char* w = static_cast<unsigned char*>(ws);
+  a.kbar = reinterpret_cast<const float*>(w);
+  w += align256(kbar_bytes);
+  int32_t* selws = reinterpret_cast<int32_t*>(w);
+  w += align256(rows * p.top_n * 4);
+  a.sel = sel_out ? sel_out : selws;
+  a.cnt = reinterpret_cast<int32_t*>(w);
+  w += align256(((size_t)a.NB + 1) * 4);
+  a.off = reinterpret_cast<int32_t*>(w);
+  w += align256(((size_t)a.NB + 1) * 4);
+  a.toff = reinterpret_cast<int32_t*>(w);
+  w += align256(((size_t)a.NB + 1) * 4);
+  a.cur = reinterpret_cast<int32_t*>(w);
+  w += align256(((size_t)a.NB + 1) * 4);
+  a.list = reinterpret_cast<int32_t*>(w);
+  w += align256(rows * np * 4 + 4);
+  a.po = reinterpret_cast<float*>(w);
+  w += align256(rows * np * D * 4 + 4);
+  a.plse = reinterpret_cast<float*>(w);
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.out = static_cast<__nv_bfloat16*>(out);
+  a.err = err;
+  const float scale = p.softmax_scale > 0.f ? p.softmax_scale : 1.f / sqrtf((float)p.d);
+  a.c = scale * 1.4426950408889634f;
+
+  const uint64_t BT = (uint64_t)p.B * p.T;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap_bf16_3d(&tq, q, D, p.Hq, BT, 64, 1, KT, true) ||
+      !make_tmap_bf16_3d(&tk, k, D, p.Hkv, BT, 64, 1, KT, true) ||
+      !make_tmap_bf16_3d(&tv, v, D, p.Hkv, BT, 64, 1, KT, true))
+    return cudaErrorInvalidValue;
+
+  cudaError_t e;
+  if (a.NB > 0 && (e = cudaMemsetAsync(a.cnt, 0, (size_t)a.NB * 4, stream)) != cudaSuccess) return e;
+  {
+    TraceScope trace("moba_gate", stream);
+    dim3 grid((p.T + 127) / 128, p.Hq, p.B);
+    moba_gate_kernel<<<grid, 128, 0, stream>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if (a.NB > 0 && p.top_n > 1) {
+    {
+      TraceScope trace("moba_scan", stream);
+      moba_scan_kernel<<<1, 1024, 0, stream>>>(a);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    {
+      TraceScope trace("moba_fill", stream);
+      const long long n = (long long)rows;
+      const int grid = (int)std::min<long long>((n + 255) / 256, (long long)device_sm_count() * 8);
+      moba_fill_kernel<<<grid, 256, 0, stream>>>(a);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    {
+      const size_t sm = attn_smem(2);
+      if (first_use(0))
+        cudaFuncSetAttribute(moba_blk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+      TraceScope trace("moba_blk", stream);
+      moba_blk_kernel<<<device_sm_count(), kThreads, sm, stream>>>(tk, tv, a);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+  }
+  {
+    const size_t sm = attn_smem(1);
+    if (first_use(1))
+      cudaFuncSetAttribute(moba_own_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    TraceScope trace("moba_own", stream);
+    const long long grid = (long long)p.B * p.Hq * ((p.T + KT - 1) / KT);
+    moba_own_kernel<<<(unsigned)grid, kThreads, sm, stream>>>(tq, tk, tv, a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace nsa

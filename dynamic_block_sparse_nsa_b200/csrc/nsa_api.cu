@@ -118,9 +118,14 @@ NsaRowArgs row_args(const nsa_params* p) {
   return a;
 }
 
-size_t moba_ws_bytes(const nsa_params* p) {
+size_t moba_kbar_bytes(const nsa_params* p) {
   const size_t nfull = (size_t)(p->T / p->sel_block);
   return round_up((size_t)p->B * nfull * p->Hkv * p->d * sizeof(float), 256);
+}
+
+size_t moba_ws_bytes(const nsa_params* p) {
+  const size_t kb = moba_kbar_bytes(p);
+  return moba_tc_eligible(*p) ? moba_tc_ws_bytes(*p, kb) : kb;
 }
 
 nsa_status check_workspace(void* ws, size_t have, size_t need) {
@@ -279,6 +284,13 @@ nsa_status moba_prefill(const nsa_params* p, const void* q, const void* k, const
   a.err = err;
   a.B = p->B; a.T = p->T; a.Hq = p->Hq; a.Hkv = p->Hkv; a.d = p->d; a.m = p->sel_block;
   a.topk = p->top_n; a.scale = eff_scale(p); a.dtype = p->dtype;
+  if (moba_tc_eligible(*p)) {
+    cudaError_t e = launch_moba_block_mean(a, (cudaStream_t)stream);
+    if (e == cudaSuccess)
+      e = launch_moba_tc(*p, q, k, v, out, sel_idx, workspace, moba_kbar_bytes(p), err,
+                         (cudaStream_t)stream);
+    return e == cudaSuccess ? NSA_OK : cuda_fail(e, "moba launch");
+  }
   if (moba_simt_smem(a) > (size_t)max_smem_optin())
     return fail(NSA_ERR_UNSUPPORTED, "MoBA shape needs too much shared memory");
   cudaError_t e = launch_moba_simt(a, (cudaStream_t)stream);

@@ -501,7 +501,7 @@ size_t moba_simt_smem(const MobaArgs& a) {
   return ctx_bytes(1, a.d, nblk, a.topk);
 }
 
-cudaError_t launch_moba_simt(const MobaArgs& a, cudaStream_t stream) {
+cudaError_t launch_moba_block_mean(const MobaArgs& a, cudaStream_t stream) {
   const int nfull = a.T / a.m;
   const long total = (long)a.B * nfull * a.Hkv * a.d;
   if (total > 0) {
@@ -515,9 +515,14 @@ cudaError_t launch_moba_simt(const MobaArgs& a, cudaStream_t stream) {
     else
       moba_block_mean_kernel<float><<<(unsigned)blocks, 256, 0, stream>>>(
           (const float*)a.k, a.kbar, a.B, a.T, a.Hkv, a.d, a.m);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
   }
+  return cudaSuccess;
+}
+
+cudaError_t launch_moba_simt(const MobaArgs& a, cudaStream_t stream) {
+  cudaError_t e = launch_moba_block_mean(a, stream);
+  if (e != cudaSuccess) return e;
   const size_t smem = moba_simt_smem(a);
   dim3 grid(a.T, a.Hq, a.B);
   TraceScope trace("moba_rows_simt", stream);

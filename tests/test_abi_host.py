@@ -4,6 +4,8 @@
 * argument validation happens on the host before any CUDA call.
 """
 import ctypes
+
+import torch
 import os
 import re
 
@@ -56,8 +58,20 @@ def test_workspace_size_validation():
     assert nsa.LIB.nsa_workspace_size(ctypes.byref(bad), nsa.OP_PREFILL, ctypes.byref(n)) == 1
     bad = nsa.params(1, 1024, 4, 1, 64, cmp_block=8, cmp_stride=16)
     assert nsa.LIB.nsa_workspace_size(ctypes.byref(bad), nsa.OP_PREFILL, ctypes.byref(n)) == 1
-    moba = nsa.params(2, 131072, 32, 32, 128, sel_block=512, top_n=3)
-    assert nsa.workspace_size(moba, nsa.OP_MOBA_PREFILL) == 2 * 256 * 32 * 128 * 4
+    # MoBA: block means [B, T/m, Hkv, d] fp32; the tensor-core path (bf16,
+    # d = 128) adds the selection, bucket counts / offsets / tile offsets /
+    # cursors, bucket rows, partial outputs and their log-sum-exp
+    def a256(x):
+        return (x + 255) // 256 * 256
+    B, T, H, m, k = 2, 131072, 32, 512, 3
+    kbar = a256(B * (T // m) * H * 128 * 4)
+    rows, nb = B * T * H, B * H * (T // m)
+    moba = nsa.params(B, T, H, H, 128, sel_block=m, top_n=k)
+    assert nsa.workspace_size(moba, nsa.OP_MOBA_PREFILL) == (
+        kbar + a256(rows * k * 4) + 4 * a256((nb + 1) * 4) + a256(rows * (k - 1) * 4 + 4) +
+        a256(rows * (k - 1) * 128 * 4 + 4) + a256(rows * (k - 1) * 4 + 4))
+    moba32 = nsa.params(B, T, H, H, 128, sel_block=m, top_n=k, dtype=torch.float32)
+    assert nsa.workspace_size(moba32, nsa.OP_MOBA_PREFILL) == kbar  # CUDA-core path
 
 
 def test_calls_reject_null_pointers_before_launching():

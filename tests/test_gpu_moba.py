@@ -35,3 +35,29 @@ def test_moba_bf16_top1_and_all_blocks():
 def test_moba_bf16_full_size_sampled():
     w = inputs.workload("moba_prefill_bf16_t131072")
     gc.run_moba(w, rows=gc.sample_rows(w["T"], 24), heads=[0, 13, 31])
+
+
+# Tensor-core MoBA path (bf16, d = 128, block a multiple of 128): bucket tiles,
+# ragged query tiles, a sequence shorter than one block, GQA, up to 7 picks.
+@pytest.mark.parametrize("over", [
+    dict(T=1000, Hq=2, Hkv=2, block=128, top_k=4),
+    dict(T=300, Hq=2, Hkv=2),
+    dict(B=2, T=1536, Hq=4, Hkv=1, block=256, top_k=2),
+    dict(T=4096, Hq=2, Hkv=2, block=512, top_k=8),
+])
+def test_moba_bf16_tensor_core_edges(over):
+    w = inputs.workload("moba_prefill_bf16_t131072", **over)
+    gc.run_moba(w, seed=9)
+
+
+def test_moba_bf16_runs_the_tensor_core_kernels():
+    from dynamic_block_sparse_nsa_b200 import nsa
+    w = inputs.workload("moba_prefill_bf16_t131072", T=2048, Hq=2, Hkv=2, block=256, top_k=3)
+    nsa.trace_enable(True, 64)
+    try:
+        gc.run_moba(w, rows=gc.sample_rows(2048, 100))
+        recs, _ = nsa.trace_records()
+        names = {nm for nm, _ in recs}
+    finally:
+        nsa.trace_enable(False)
+    assert {"moba_gate", "moba_blk", "moba_own"} <= names, names
