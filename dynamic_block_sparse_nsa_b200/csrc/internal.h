@@ -15,6 +15,7 @@ namespace nsa {
 enum : unsigned {
   kErrTimeout = 1u,     // a bounded wait gave up
   kErrSeqLen = 2u,      // a decode sequence length outside [1, T]
+  kErrAppendPos = 4u,   // an append position outside [0, T)
 };
 
 // Arguments of the generic (CUDA-core) NSA row kernel, used for prefill and
@@ -119,6 +120,9 @@ bool make_tmap_bf16_3d(CUtensorMap* m, const void* base, uint64_t dim0, uint64_t
 
 cudaError_t launch_compress(const nsa_params& p, const void* k, const void* v, const float* w,
                             void* kc, void* vc, cudaStream_t stream);
+cudaError_t launch_append(const nsa_params& p, const void* k_new, const void* v_new,
+                          const int32_t* pos, void* k_cache, void* v_cache, const float* w,
+                          void* k_cmp, void* v_cmp, unsigned* err, cudaStream_t stream);
 
 // Shared-memory bytes the generic row kernel needs (0 if unsupported).
 size_t nsa_rows_simt_smem(const NsaRowArgs& a);

@@ -312,7 +312,26 @@ nsa_status nsa_check(void* stream) {
   if (word & kErrTimeout) return fail(NSA_ERR_DEVICE_TIMEOUT, "a bounded device wait gave up");
   if (word & kErrSeqLen)
     return fail(NSA_ERR_INVALID_ARGUMENT, "a decode sequence length was outside [1, T]");
+  if (word & kErrAppendPos)
+    return fail(NSA_ERR_INVALID_ARGUMENT, "an append position was outside [0, T)");
   return NSA_OK;
+}
+
+nsa_status nsa_append_kv(const nsa_params* p, const void* k_new, const void* v_new,
+                         const int32_t* pos, void* k_cache, void* v_cache, const float* w_cmp,
+                         void* k_cmp, void* v_cmp, void* stream) {
+  g_detail.clear();
+  nsa_status s = check_nsa(p);
+  if (s != NSA_OK) return s;
+  const int Nc = nsa_num_cmp_blocks(p->T, p->cmp_block, p->cmp_stride);
+  if (!k_new || !v_new || !pos || !k_cache || !v_cache || (Nc > 0 && (!w_cmp || !k_cmp || !v_cmp)))
+    return fail(NSA_ERR_INVALID_ARGUMENT,
+                "k_new, v_new, pos, k_cache, v_cache, w_cmp, k_cmp, v_cmp must be non-NULL");
+  unsigned* err = err_word(&s);
+  if (!err) return s;
+  cudaError_t e = launch_append(*p, k_new, v_new, pos, k_cache, v_cache, w_cmp, k_cmp, v_cmp, err,
+                                (cudaStream_t)stream);
+  return e == cudaSuccess ? NSA_OK : cuda_fail(e, "append launch");
 }
 
 nsa_status nsa_debug_bounded_wait(const int32_t* flag, int max_iters, void* stream) {

@@ -28,7 +28,7 @@ _TORCH_DTYPE = {DTYPE_F32: torch.float32, DTYPE_BF16: torch.bfloat16}
 # Every symbol include/nsa.h declares.
 EXPORTS = (
     "nsa_workspace_size", "nsa_num_cmp_blocks", "nsa_compress_kv", "nsa_prefill", "nsa_decode",
-    "moba_prefill", "nsa_decode_noalloc", "nsa_check", "nsa_debug_bounded_wait", "nsa_status_string",
+    "moba_prefill", "nsa_decode_noalloc", "nsa_append_kv", "nsa_check", "nsa_debug_bounded_wait", "nsa_status_string",
     "nsa_last_error_detail", "nsa_trace_enable", "nsa_trace_set_filter", "nsa_trace_count",
     "nsa_trace_timed", "nsa_trace_get",
 )
@@ -69,6 +69,7 @@ def _load():
         "nsa_decode": [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
         "moba_prefill": [P, vp, vp, vp, vp, vp, vp, sz, vp],
         "nsa_decode_noalloc": [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
+        "nsa_append_kv": [P, vp, vp, vp, vp, vp, vp, vp, vp, vp],
         "nsa_check": [vp],
         "nsa_debug_bounded_wait": [vp, ctypes.c_int, vp],
         "nsa_status_string": [ctypes.c_int],
@@ -230,6 +231,19 @@ def nsa_decode_noalloc(p, q, k_cache, v_cache, seq_lens, k_cmp, v_cmp, w_gate=No
                                   _ptr(seq_lens), _ptr(k_cmp), _ptr(v_cmp), _ptr(w_gate),
                                   _ptr(out), _ptr(sel_idx), _stream(stream)))
     return out, sel_idx
+
+
+def nsa_append_kv(p, k_new, v_new, pos, k_cache, v_cache, w_cmp, k_cmp, v_cmp, stream=None):
+    """Write one token per sequence at pos[b] into the caches; complete
+    compressed blocks are written into k_cmp / v_cmp (see include/nsa.h)."""
+    dt = p.torch_dtype
+    for t, nm in ((k_new, "k_new"), (v_new, "v_new"), (k_cache, "k_cache"), (v_cache, "v_cache"),
+                  (k_cmp, "k_cmp"), (v_cmp, "v_cmp")):
+        _dev(t, nm, dt)
+    _dev(pos, "pos", torch.int32)
+    _dev(w_cmp, "w_cmp", torch.float32)
+    _raise(LIB.nsa_append_kv(ctypes.byref(p), _ptr(k_new), _ptr(v_new), _ptr(pos), _ptr(k_cache),
+                             _ptr(v_cache), _ptr(w_cmp), _ptr(k_cmp), _ptr(v_cmp), _stream(stream)))
 
 
 def moba_prefill(p, q, k, v, out=None, sel_idx=None, ws=None, stream=None, want_sel=True):

@@ -137,6 +137,25 @@ NSA_API nsa_status nsa_decode(const nsa_params* p, const void* q, const void* k_
                       const void* v_cmp, const float* w_gate, void* out, int32_t* sel_idx,
                       void* workspace, size_t ws_bytes, void* stream);
 
+/* Streaming decode: appends one token per sequence to the caches (lchairun NSA
+ * article: decode reads the compressed cache, which gains one block every s
+ * tokens, plus the selected and most recent tokens; EP94 notes §五).
+ *   k_new, v_new      [B, Hkv, d] dtype: the new token's keys and values.
+ *   pos               [B] int32, device: where to write, the sequence's length
+ *                     before the append (0 <= pos < T).
+ *   k_cache, v_cache  [B, T, Hkv, d] dtype, written at [b, pos[b]].
+ *   w_cmp             [cmp_block] fp32 (the weights given to nsa_compress_kv).
+ *   k_cmp, v_cmp      [B, Nc, Hkv, d] dtype. When pos + 1 completes compressed
+ *                     block i = (pos + 1 - l) / s (pos + 1 >= l and
+ *                     (pos + 1 - l) % s == 0), entry i is written exactly as
+ *                     nsa_compress_kv computes it; no other entry is touched.
+ *   A position outside [0, T) writes nothing for that sequence and sets the
+ *   device error word (nsa_check then returns NSA_ERR_INVALID_ARGUMENT). The
+ *   caller passes seq_lens = pos + 1 to the next nsa_decode. */
+NSA_API nsa_status nsa_append_kv(const nsa_params* p, const void* k_new, const void* v_new,
+                                 const int32_t* pos, void* k_cache, void* v_cache,
+                                 const float* w_cmp, void* k_cmp, void* v_cmp, void* stream);
+
 /* nsa_decode without a workspace argument, for callers that cannot allocate
  * device memory: code that runs while a stream capture is in progress
  * (cudaMalloc is not permitted during a global-mode capture), real-time or
