@@ -46,7 +46,7 @@ constexpr uint32_t TILE = 32768;  // a 128 x 128 bf16 tile
 constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr int kMaxSel = 16;       // top_n bound: 8 tiles of two blocks in pf_slc
 constexpr int kMainStagesMax = 4;
-constexpr int kMainThreads = 192; // TMA, MMA, 4 softmax warps
+constexpr int kMainThreads = 320; // TMA, MMA, 8 softmax warps
 constexpr int kSlcThreads = 256;  // K TMA, V TMA, MMA, TMEM owner, 4 softmax warps
 constexpr int kSlcKStages = 3, kSlcVStages = 2;
 constexpr uint32_t kQ16 = 4096;   // 16 rows x 128 d bf16
@@ -147,6 +147,8 @@ struct MainBars {
   uint64_t q_full, s_full[2], p_full[2], o_done[2], fin;
   uint32_t tmem;
   int abort;
+  float xm[2][2][128];  // per tile parity, column half, row: partial row maxima
+  float xl[2][2][128];  // per branch, column half, row: partial row sums
 };
 
 // TMEM columns of pf_main.
@@ -192,7 +194,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     ptx::mbar_init(&bars->q_full, 1);
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&bars->s_full[i], 1);
-      ptx::mbar_init(&bars->p_full[i], 128);
+      ptx::mbar_init(&bars->p_full[i], 256);  // the eight softmax warps
       ptx::mbar_init(&bars->o_done[i], 1);
     }
     ptx::mbar_init(&bars->fin, 1);
@@ -332,63 +334,72 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     }
   } else {
     // ---------------- softmax / scores / selection / epilogue ----------------
+    // Eight warps: two per TMEM lane quarter, splitting each row's 128 columns
+    // (keys in steps 1-2, query rows in step 3) into halves.
+    const int sw = warp - 2;           // 0..7
+    const int half = sw >> 2;          // column half
     const int qd = warp & 3;
-    const int row = qd * 32 + lane;  // TMEM lane: query row in steps 1-2, key in step 3
+    const int row = qd * 32 + lane;    // TMEM lane: query row in steps 1-2, key in step 3
+    const int sid = half * 128 + row;  // 0..255 among the softmax threads
     const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
+    const uint32_t hc = half * 64;     // this thread's first column of a 128-column tile
     const int tt = row >> 4, h = row & 15;
     const int t = min(t0 + tt, a.T - 1);
     const bool row_ok = t0 + tt < a.T;
     const int nv_t = t >= CL - 1 ? min(a.Nc, (t - (CL - 1)) / CS + 1) : 0;
     const int wlo = max(0, t - a.w + 1);
-    for (int i = row; i < TQ * a.nblk; i += 128) sc[i] = 0.f;
-    if (row < TQ) scarry[row] = 0.f;
+    for (int i = sid; i < TQ * a.nblk; i += 256) sc[i] = 0.f;
+    if (sid < TQ) scarry[sid] = 0.f;
     if (a.gate_mode == 0)
-      for (int i = row; i < D * 3; i += 128) swg[i] = __ldg(a.w_gate + i);
+      for (int i = sid; i < D * 3; i += 256) swg[i] = __ldg(a.w_gate + i);
 
-    float m1 = -INFINITY, l1 = 0.f, m2 = -INFINITY, l2 = 0.f;
+    float m1 = -INFINITY, l1 = 0.f, m2 = -INFINITY, l2 = 0.f;  // l: this half's sum
     for (int j = 0; j < A; ++j) {
       const int bs = j & 1;
       wait_or_abort(&bars->s_full[bs], (uint32_t)((j >> 1) & 1), abort, a.err);
       tc::fence_after_sync();
       const bool cmp = j < J1;
-      const int kb = cmp ? j * KT : ks0 + (j - J1) * KT;
+      const int kb = (cmp ? j * KT : ks0 + (j - J1) * KT) + (int)hc;
       const int lo = cmp ? 0 : wlo, hi = cmp ? nv_t - 1 : t;
-      uint32_t u[128];
-      tc::ld128_sync(tl + kS0 + bs * 128, u);
-      if (kb < lo || kb + KT - 1 > hi) {  // the tile straddles this row's key range
+      uint32_t u[64];
+      tc::ld64_sync(tl + kS0 + bs * 128 + hc, u);
+      if (kb < lo || kb + 63 > hi) {  // these columns straddle the row's key range
 #pragma unroll
-        for (int e = 0; e < 128; ++e) {
+        for (int e = 0; e < 64; ++e) {
           const int key = kb + e;
           if (key < lo || key > hi) u[e] = kNegInf;
         }
       }
       float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-      for (int e = 0; e < 128; e += 4) {
+      for (int e = 0; e < 64; e += 4) {
         mx0 = fmaxf(mx0, __uint_as_float(u[e]));
         mx1 = fmaxf(mx1, __uint_as_float(u[e + 1]));
         mx2 = fmaxf(mx2, __uint_as_float(u[e + 2]));
         mx3 = fmaxf(mx3, __uint_as_float(u[e + 3]));
       }
-      const float mt = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * a.c;
+      // the row maximum over both halves (exchange buffers alternate by tile)
+      bars->xm[bs][half][row] = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+      ptx::named_bar_sync(1, 256);
+      const float mt = fmaxf(bars->xm[bs][0][row], bars->xm[bs][1][row]) * a.c;
       float& m = cmp ? m1 : m2;
       float& l = cmp ? l1 : l2;
       const float mn = fmaxf(m, mt);
       if (mn != -INFINITY && (m == -INFINITY || mn > m + 8.f)) {
         if (m != -INFINITY) {
-          // rescale this row of O once the previous PV MMA has finished
+          // rescale this half of the row of O once the previous PV MMA finished
           const float f = exp2f(m - mn);
           l *= f;
           wait_or_abort(&bars->o_done[(j - 1) & 1], (uint32_t)(((j - 1) >> 1) & 1), abort, a.err);
           tc::fence_after_sync();
-          const uint32_t oc = tl + (cmp ? kO1 : kO2);
+          const uint32_t oc = tl + (cmp ? kO1 : kO2) + hc;
+#pragma unroll 1
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint32_t w[16];
+            tc::ld16_sync(oc + q4 * 16, w);
 #pragma unroll
-          for (int q4 = 0; q4 < 8; ++q4) {
-            uint32_t u[16];
-            tc::ld16_sync(oc + q4 * 16, u);
-#pragma unroll
-            for (int e = 0; e < 16; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * f);
-            tc::st16(oc + q4 * 16, u);
+            for (int e = 0; e < 16; ++e) w[e] = __float_as_uint(__uint_as_float(w[e]) * f);
+            tc::st16(oc + q4 * 16, w);
           }
           tc::st_wait();
         }
@@ -399,7 +410,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       const float nm = m == -INFINITY ? 0.f : -m;
       float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
+      for (int q4 = 0; q4 < 2; ++q4) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
@@ -409,139 +420,120 @@ __global__ void __launch_bounds__(kMainThreads, 1)
           ls1 += p1;
           pk[e] = ptx::pack_bf16(p0, p1);
         }
-        tc::st16(tl + kS0 + bs * 128 + q4 * 16, pk);
+        tc::st16(tl + kS0 + bs * 128 + half * 32 + q4 * 16, pk);
       }
       l += ls0 + ls1;
       tc::st_wait();
       tc::fence_before_sync();
       ptx::mbar_arrive(&bars->p_full[bs]);
     }
+    // row sums over both halves
+    bars->xl[0][half][row] = l1;
+    bars->xl[1][half][row] = l2;
+    ptx::named_bar_sync(1, 256);
+    l1 = bars->xl[0][0][row] + bars->xl[0][1][row];
+    l2 = bars->xl[1][0][row] + bars->xl[1][1][row];
 
     // log-sum-exp (log2 domain) of the compressed branch for step 3
-    slse[row] = l1 > 0.f ? -(m1 + __log2f(l1)) : -INFINITY;  // negated, for fma
-    ptx::named_bar_sync(1, 128);
+    if (half == 0) slse[row] = l1 > 0.f ? -(m1 + __log2f(l1)) : -INFINITY;  // negated, for fma
+    ptx::named_bar_sync(1, 256);
 
-    // step 3: block scores, thread = compressed key `row` of each tile
+    // step 3: block scores; thread = compressed key `row` of each tile, tokens
+    // 4 half .. 4 half + 3
     for (int jj = 0; jj < J3; ++jj) {
       const int j = A + jj, bs = j & 1;
       wait_or_abort(&bars->s_full[bs], (uint32_t)((j >> 1) & 1), abort, a.err);
       tc::fence_after_sync();
-      uint32_t u[128];
-      tc::ld128_sync(tl + kS0 + bs * 128, u);
+      uint32_t u[64];
+      tc::ld64_sync(tl + kS0 + bs * 128 + hc, u);
       tc::fence_before_sync();
       ptx::mbar_arrive(&bars->p_full[bs]);
       const int kk = jj * KT + row;
-      float pt[TQ];
 #pragma unroll
-      for (int x = 0; x < TQ; ++x) {
-        const int tok = t0 + x;
+      for (int xx = 0; xx < TQ / 2; ++xx) {
+        const int x = half * (TQ / 2) + xx, tok = t0 + x;
         float acc0 = 0.f, acc1 = 0.f;
         if (tok < a.T && kk < a.Nc && kk * CS + CL - 1 <= tok) {
           const float4* nl = reinterpret_cast<const float4*>(slse + x * G);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const float4 l4 = nl[q];
-            acc0 += ptx::ex2(fmaf(__uint_as_float(u[x * G + 4 * q]), a.c, l4.x));
-            acc1 += ptx::ex2(fmaf(__uint_as_float(u[x * G + 4 * q + 1]), a.c, l4.y));
-            acc0 += ptx::ex2(fmaf(__uint_as_float(u[x * G + 4 * q + 2]), a.c, l4.z));
-            acc1 += ptx::ex2(fmaf(__uint_as_float(u[x * G + 4 * q + 3]), a.c, l4.w));
+            acc0 += ptx::ex2(fmaf(__uint_as_float(u[xx * G + 4 * q]), a.c, l4.x));
+            acc1 += ptx::ex2(fmaf(__uint_as_float(u[xx * G + 4 * q + 1]), a.c, l4.y));
+            acc0 += ptx::ex2(fmaf(__uint_as_float(u[xx * G + 4 * q + 2]), a.c, l4.z));
+            acc1 += ptx::ex2(fmaf(__uint_as_float(u[xx * G + 4 * q + 3]), a.c, l4.w));
           }
         }
-        pt[x] = acc0 + acc1;
+        spk[x * KT + row] = acc0 + acc1;
       }
       // selection block q of this tile collects compressed keys 4q-1 .. 4q+3
       // (key 4q-1 of block 0 comes from the previous tile)
-#pragma unroll
-      for (int x = 0; x < TQ; ++x) spk[x * KT + row] = pt[x];
-      ptx::named_bar_sync(1, 128);
+      ptx::named_bar_sync(1, 256);
       {
-        const int x = row >> 4, q0 = (row & 15) * 2;
+        const int x = sid >> 5, q = sid & 31;
         const float* px = spk + x * KT;
-        float nc = 0.f;
-        if ((row & 15) == 15) nc = px[KT - 1];
-#pragma unroll
-        for (int qq = 0; qq < 2; ++qq) {
-          const int q = q0 + qq;
-          const int jb = jj * (KT / 4) + q;
-          const float prev = q > 0 ? px[4 * q - 1] : scarry[x];
-          const float v = prev + px[4 * q] + px[4 * q + 1] + px[4 * q + 2] + px[4 * q + 3];
-          if (jb < a.nblk) sc[x * a.nblk + jb] = v;
-        }
-        ptx::named_bar_sync(1, 128);
-        if ((row & 15) == 15) {
+        const float nc = q == 31 ? px[KT - 1] : 0.f;
+        const int jb = jj * (KT / 4) + q;
+        const float prev = q > 0 ? px[4 * q - 1] : scarry[x];
+        const float v = prev + px[4 * q] + px[4 * q + 1] + px[4 * q + 2] + px[4 * q + 3];
+        if (jb < a.nblk) sc[x * a.nblk + jb] = v;
+        ptx::named_bar_sync(1, 256);
+        if (q == 31) {
           scarry[x] = nc;
           // the block after the last tile holds only the carried key
           if (jj == J1 - 1 && J1 * (KT / 4) < a.nblk) sc[x * a.nblk + J1 * (KT / 4)] = nc;
         }
       }
     }
-    ptx::named_bar_sync(1, 128);
+    ptx::named_bar_sync(1, 256);
 
-    // step 4: top-n per token, one warp per two tokens (processed together).
-    // A candidate's key is (score bits + 1, ~index): unique, ordered by score
-    // and then by the lower index; a taken block gets key 0.
+    // step 4: top-n of token `sw`, one warp per token. A candidate's key is
+    // (score bits + 1, ~index): unique, ordered by score and then by the lower
+    // index; a taken block gets key 0.
     if (a.need_sel) {
-      int tokx[2], ncand[2], mine[2];
-      uint32_t bh[2], bl[2];
-      int32_t* dst[2];
-#pragma unroll
-      for (int z = 0; z < 2; ++z) {
-        const int x = 2 * qd + z, tok = t0 + x;
-        tokx[z] = x;
-        ncand[z] = tok < a.T ? tok / SB + 1 : 0;
-        dst[z] = a.sel + ((size_t)(b * a.T + min(tok, a.T - 1)) * a.Hkv + g) * a.n;
-        mine[z] = lane == 0 ? 0 : 0x7fffffff;
-        bh[z] = 0;
-        bl[z] = 0;
-        if (tok < a.T && ncand[z] <= a.n) {
-          for (int i = lane; i < a.n; i += 32) dst[z][i] = i < ncand[z] ? i : -1;
-          ncand[z] = 0;  // done
-        }
-      }
-      auto rescan = [&](int z) {
-        const float* scx = sc + tokx[z] * a.nblk;
-        uint32_t h = 0, l = 0;
-        for (int jb = 1 + lane; jb < ncand[z]; jb += 32) {
-          const float v = scx[jb];
-          const uint32_t kh = v < 0.f ? 0u : __float_as_uint(v) + 1u;
-          const uint32_t kl = ~(uint32_t)jb;
-          if (kh > h || (kh == h && kl > l)) {
-            h = kh;
-            l = kl;
+      const int x = sw, tok = t0 + x;
+      if (tok < a.T) {  // warp-uniform
+        const int ncand = tok / SB + 1;
+        int32_t* dst = a.sel + ((size_t)(b * a.T + tok) * a.Hkv + g) * a.n;
+        if (ncand <= a.n) {
+          for (int i = lane; i < a.n; i += 32) dst[i] = i < ncand ? i : -1;
+        } else {
+          float* scx = sc + x * a.nblk;
+          uint32_t bh = 0, bl = 0;
+          auto rescan = [&]() {
+            uint32_t hh = 0, ll = 0;
+            for (int jb = 1 + lane; jb < ncand; jb += 32) {
+              const float vv = scx[jb];
+              const uint32_t kh = vv < 0.f ? 0u : __float_as_uint(vv) + 1u;
+              const uint32_t kl = ~(uint32_t)jb;
+              if (kh > hh || (kh == hh && kl > ll)) {
+                hh = kh;
+                ll = kl;
+              }
+            }
+            bh = hh;
+            bl = ll;
+          };
+          rescan();
+          int mine = lane == 0 ? 0 : 0x7fffffff;
+          for (int k = 0; k < a.n - 1; ++k) {
+            const uint32_t mh = __reduce_max_sync(0xffffffffu, bh);
+            const uint32_t ml = __reduce_max_sync(0xffffffffu, bh == mh ? bl : 0u);
+            const int pick = (int)~ml;
+            if (lane == k + 1) mine = pick;
+            if (((pick - 1) & 31) == lane) {
+              scx[pick] = -1.f;
+              rescan();
+            }
           }
+          int rank = 0;
+          for (int o = 0; o < 32; ++o) rank += (__shfl_sync(0xffffffffu, mine, o) < mine) ? 1 : 0;
+          if (lane < a.n) dst[rank] = mine;
         }
-        bh[z] = h;
-        bl[z] = l;
-      };
-      rescan(0);
-      rescan(1);
-      for (int k = 0; k < a.n - 1; ++k) {
-        int pick[2];
-#pragma unroll
-        for (int z = 0; z < 2; ++z) {
-          const uint32_t mh = __reduce_max_sync(0xffffffffu, bh[z]);
-          const uint32_t ml = __reduce_max_sync(0xffffffffu, bh[z] == mh ? bl[z] : 0u);
-          pick[z] = (int)~ml;
-          if (lane == k + 1) mine[z] = pick[z];
-        }
-#pragma unroll
-        for (int z = 0; z < 2; ++z) {
-          if (ncand[z] > 0 && ((pick[z] - 1) & 31) == lane) {
-            sc[tokx[z] * a.nblk + pick[z]] = -1.f;
-            rescan(z);
-          }
-        }
-      }
-#pragma unroll
-      for (int z = 0; z < 2; ++z) {
-        if (ncand[z] == 0) continue;  // warp-uniform
-        int rank = 0;
-        for (int o = 0; o < 32; ++o) rank += (__shfl_sync(0xffffffffu, mine[z], o) < mine[z]) ? 1 : 0;
-        if (lane < a.n) dst[z][rank] = mine[z];
       }
     }
 
-    // step 5: gated compressed + window outputs, and g_slc
+    // step 5: gated compressed + window outputs (this half's 64 columns), g_slc
     if (A >= 1)
       wait_or_abort(&bars->o_done[(A - 1) & 1], (uint32_t)(((A - 1) >> 1) & 1), abort, a.err);
     tc::fence_after_sync();
@@ -549,14 +541,14 @@ __global__ void __launch_bounds__(kMainThreads, 1)
     row_gates(a, sQ, swg, row, ATOM, gt);
     const float i1 = l1 > 0.f ? gt[0] / l1 : 0.f;
     const float i2 = l2 > 0.f ? gt[2] / l2 : 0.f;
-    const size_t orow = ((size_t)(b * a.T + t) * a.Hq + g * G + h) * D;
+    const size_t orow = ((size_t)(b * a.T + t) * a.Hq + g * G + h) * D + hc;
     // An accumulator a branch never wrote (no visible key, or the branch
     // skipped) has l = 0, so i = 0 keeps its unwritten columns out.
 #pragma unroll 1
-    for (int c16 = 0; c16 < 8; ++c16) {  // runs once per row: kept compact
+    for (int c16 = 0; c16 < 4; ++c16) {  // runs once per row: kept compact
       uint32_t u1[16], u2[16];
-      tc::ld16_sync(tl + kO1 + c16 * 16, u1);
-      tc::ld16_sync(tl + kO2 + c16 * 16, u2);
+      tc::ld16_sync(tl + kO1 + hc + c16 * 16, u1);
+      tc::ld16_sync(tl + kO2 + hc + c16 * 16, u2);
       float o[16];
 #pragma unroll
       for (int e = 0; e < 16; ++e)
@@ -578,7 +570,8 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         }
       }
     }
-    if (row_ok && !a.direct_out) a.gslc[(size_t)(b * a.T + t) * a.Hq + g * G + h] = gt[1];
+    if (row_ok && !a.direct_out && half == 0)
+      a.gslc[(size_t)(b * a.T + t) * a.Hq + g * G + h] = gt[1];
   }
 
   tc::fence_before_sync();
@@ -635,12 +628,30 @@ __device__ __forceinline__ float xreduce16(const float (&v)[G], int lane) {
   return op(w1, __shfl_xor_sync(0xffffffffu, w1, 1));
 }
 
-// Number of valid (non-negative) entries of a sorted selection row.
-__device__ __forceinline__ int count_sel(const int32_t* s, int n) {
-  int c = 0;
-  for (int i = 0; i < n; ++i) c += s[i] >= 0 ? 1 : 0;
-  return c;
-}
+// A unit's selection row packed two block indices per word (0xffff = unused
+// slot; blocks stay below 65535 for the supported T). Loaded one unit ahead so
+// the latency of the global reads overlaps the current unit's work.
+struct SelRow {
+  uint32_t w[kMaxSel / 2];
+  __device__ __forceinline__ void load(const int32_t* sl, int n) {
+#pragma unroll
+    for (int i = 0; i < kMaxSel / 2; ++i) {
+      const int s0 = 2 * i < n ? __ldg(sl + 2 * i) : -1;
+      const int s1 = 2 * i + 1 < n ? __ldg(sl + 2 * i + 1) : -1;
+      w[i] = ((uint32_t)s0 & 0xffffu) | (((uint32_t)s1 & 0xffffu) << 16);
+    }
+  }
+  __device__ __forceinline__ int blk(int i) const {  // -1 when unused
+    const uint32_t x = (w[i >> 1] >> (16 * (i & 1))) & 0xffffu;
+    return x == 0xffffu ? -1 : (int)x;
+  }
+  __device__ __forceinline__ int count() const {
+    int c = 0;
+#pragma unroll
+    for (int i = 0; i < kMaxSel; ++i) c += blk(i) >= 0 ? 1 : 0;
+    return c;
+  }
+};
 
 __global__ void __launch_bounds__(kSlcThreads, 1)
     pf_slc_kernel(const __grid_constant__ CUtensorMap tq16, const __grid_constant__ CUtensorMap tk64,
@@ -719,11 +730,18 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
       const int hb = lane >> 1, dh = lane & 1;
       int c = 0, k = 0;
       bool ok = true;
+      SelRow cur, nxt;
+      auto row_of = [&](long long uu) {
+        int b, t, g;
+        unit_of(uu, b, t, g);
+        return a.sel + ((size_t)(b * a.T + t) * a.Hkv + g) * a.n;
+      };
+      if (blockIdx.x < U) cur.load(row_of(blockIdx.x), a.n);
       for (long long u = blockIdx.x; ok && u < U; u += gridDim.x, ++k) {
         int b, t, g;
         unit_of(u, b, t, g);
-        const int32_t* sl = a.sel + ((size_t)(b * a.T + t) * a.Hkv + g) * a.n;
-        const int nsel = count_sel(sl, a.n);
+        if (u + gridDim.x < U) nxt.load(row_of(u + gridDim.x), a.n);
+        const int nsel = cur.count();
         if (isk && lane == 0) {
           const int qs = k & 1;
           if (k >= 2 && !wait_or_abort(&bars->q_empty[qs], (uint32_t)(((k >> 1) - 1) & 1), abort,
@@ -755,11 +773,12 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
           }
           unsigned char* dst = ringp + st * TILE + dh * ATOM + hb * (ATOM / 2);
           // a missing second block reads past the tensor: zero fill
-          const int z = (2 * i + hb < nsel) ? b * a.T + SB * __ldg(sl + 2 * i + hb) : (int)BT;
+          const int z = (2 * i + hb < nsel) ? b * a.T + SB * cur.blk(2 * i + hb) : (int)BT;
           ptx::mbar_arrive_expect_tx(&full[st], ATOM / 2);
           ptx::tma_load_3d(dst, m, &full[st], dh * 64, g, z, keep);
           ++c;
         }
+        cur = nxt;
       }
       for (int kq = max(0, c - NS); kq < c; ++kq)
         if (!ptx::mbar_wait(&full[kq % NS], (uint32_t)((kq / NS) & 1), kWaitNs))
@@ -803,11 +822,16 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
         }
         tc::commit(&bars->o_full[pp]);
       };
-      for (long long u = blockIdx.x; ok && u < U; u += gridDim.x, ++k) {
+      SelRow cur, nxt;
+      auto row_of = [&](long long uu) {
         int b, t, g;
-        unit_of(u, b, t, g);
-        const int32_t* sl = a.sel + ((size_t)(b * a.T + t) * a.Hkv + g) * a.n;
-        const int ntile = (count_sel(sl, a.n) + 1) / 2;
+        unit_of(uu, b, t, g);
+        return a.sel + ((size_t)(b * a.T + t) * a.Hkv + g) * a.n;
+      };
+      if (blockIdx.x < U) cur.load(row_of(blockIdx.x), a.n);
+      for (long long u = blockIdx.x; ok && u < U; u += gridDim.x, ++k) {
+        if (u + gridDim.x < U) nxt.load(row_of(u + gridDim.x), a.n);
+        const int ntile = (cur.count() + 1) / 2;
         const int pk = k & 1;
         ok = wait_or_abort(&bars->q_full[pk], (uint32_t)((k >> 1) & 1), abort, a.err);
         tc::fence_after_sync();
@@ -829,6 +853,7 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
         tc::commit(&bars->s_full[pk]);
         if (k >= 1 && ok) pv(k - 1, prev_tiles);
         prev_tiles = ntile;
+        cur = nxt;
       }
       if (k >= 1 && ok) pv(k - 1, prev_tiles);
       tc::commit(&bars->fin);
@@ -858,16 +883,18 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
       ptx::mbar_arrive(&bars->o_free[pp]);
       ptx::mbar_arrive(&bars->a_empty[pp]);
     };
+    SelRow cur, nxt;
+    auto row_of = [&](long long uu) {
+      int b, t, g;
+      unit_of(uu, b, t, g);
+      return a.sel + ((size_t)(b * a.T + t) * a.Hkv + g) * a.n;
+    };
+    if (blockIdx.x < U) cur.load(row_of(blockIdx.x), a.n);
     for (long long u = blockIdx.x; u < U; u += gridDim.x, ++k) {
       int b, t, g;
       unit_of(u, b, t, g);
-      const int32_t* sl = a.sel + ((size_t)(b * a.T + t) * a.Hkv + g) * a.n;
-      int selv[kMaxSel];
-#pragma unroll
-      for (int i = 0; i < kMaxSel; ++i) selv[i] = i < a.n ? __ldg(sl + i) : -1;
-      int nsel = 0;
-#pragma unroll
-      for (int i = 0; i < kMaxSel; ++i) nsel += selv[i] >= 0 ? 1 : 0;
+      if (u + gridDim.x < U) nxt.load(row_of(u + gridDim.x), a.n);
+      const int nsel = cur.count();
       const int pk = k & 1;
       wait_or_abort(&bars->s_full[pk], (uint32_t)((k >> 1) & 1), abort, a.err);
       tc::fence_after_sync();
@@ -880,7 +907,7 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
       for (int hh = 0; hh < G; ++hh) mh[hh] = -INFINITY;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const int blk = half ? selv[2 * i + 1] : selv[2 * i];
+        const int blk = cur.blk(2 * i + half);
         if (!(2 * i + half < nsel && blk * SB + kr <= t)) {
 #pragma unroll
           for (int hh = 0; hh < G; ++hh) uu[i * G + hh] = kNegInf;
@@ -961,6 +988,7 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
       pb = b;
       pt = t;
       pg = g;
+      cur = nxt;
     }
     if (k >= 1) {
       wait_or_abort(&bars->o_full[(k - 1) & 1], (uint32_t)(((k - 1) >> 1) & 1), abort, a.err);
