@@ -250,20 +250,27 @@ def barrier(ws):
         dist.barrier()
 
 
+def _dist_device():
+    import torch.distributed as dist
+    return "cuda" if dist.get_backend() == "nccl" else "cpu"
+
+
 def reduce_max(x, ws):
+    """Max over ranks (the step time every rank waits for)."""
     if ws == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=_dist_device())
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
 def reduce_sum(x, ws):
+    """Sum over ranks (the work of the whole job)."""
     if ws == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=_dist_device())
     dist.all_reduce(t, op=dist.ReduceOp.SUM)
     return float(t.item())
 
