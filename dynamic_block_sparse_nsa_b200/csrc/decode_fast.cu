@@ -666,16 +666,20 @@ constexpr int MP = 64;  // partials staged per chunk
 
 // Online merge of the softmax partials in slots [first, first + np): per head
 // M = max m_p and L = sum_p exp2(m_p - M) l_p (left in sM / sL), and
-//   acc[h][e0 .. e0+7] += scale_h / L_h * sum_p exp2(m_p - M_h) o_p[h][e].
+//   acc[h][e0 .. e0+E-1] += scale_h / L_h * sum_p exp2(m_p - M_h) o_p[h][e].
 // Partials are staged MP at a time with a running max and sum, so any count
-// works; one chunk costs two load-dependent steps. Threads (h, 8 dims): the
-// first 256 threads of the block accumulate; all NT take part in staging.
+// works; one chunk costs two load-dependent steps. Every thread owns E =
+// 2048 / NT output values (head h, dims e0 ..) and keeps the loads of up to 8
+// partials in flight.
 template <int NT>
 __device__ void merge_online(const float* part, long long first, int np, const float* scale,
                              float* pm, float* pl, float* sM, float* sL, float* sR, int h, int e0,
-                             float (&acc)[8]) {
+                             float (&acc)[2048 / NT]) {
+  constexpr int E = 2048 / NT;
   const int tid = threadIdx.x;
-  float run[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  float run[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) run[e] = 0.f;
   if (tid < 16) {
     sM[tid] = -INFINITY;
     sL[tid] = 0.f;
@@ -709,33 +713,30 @@ __device__ void merge_online(const float* part, long long first, int np, const f
       pm[x] = mm == -INFINITY ? 0.f : exp2f(mm - sM[x & 15]);
     }
     __syncthreads();
-    if (tid < 256) {
+    {
       const float r = sR[h];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) run[e] *= r;
-#pragma unroll 4
+      for (int e = 0; e < E; ++e) run[e] *= r;
+#pragma unroll 8
       for (int pp = 0; pp < pc; ++pp) {
         const float f = pm[pp * 16 + h];
         const float4* src =
             reinterpret_cast<const float4*>(part + (first + p0 + pp) * PART + 2 * G + h * D + e0);
-        const float4 v0 = __ldcg(src), v1 = __ldcg(src + 1);
-        run[0] += f * v0.x;
-        run[1] += f * v0.y;
-        run[2] += f * v0.z;
-        run[3] += f * v0.w;
-        run[4] += f * v1.x;
-        run[5] += f * v1.y;
-        run[6] += f * v1.z;
-        run[7] += f * v1.w;
+#pragma unroll
+        for (int q4 = 0; q4 < E / 4; ++q4) {
+          const float4 v = __ldcg(src + q4);
+          run[4 * q4] += f * v.x;
+          run[4 * q4 + 1] += f * v.y;
+          run[4 * q4 + 2] += f * v.z;
+          run[4 * q4 + 3] += f * v.w;
+        }
       }
     }
   }
   __syncthreads();
-  if (tid < 256) {
-    const float sc = sL[h] > 0.f ? scale[h] / sL[h] : 0.f;
+  const float sc = sL[h] > 0.f ? scale[h] / sL[h] : 0.f;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] += sc * run[e];
-  }
+  for (int e = 0; e < E; ++e) acc[e] += sc * run[e];
 }
 
 // ---------------------------------------------------------------------------
@@ -744,6 +745,7 @@ __device__ void merge_online(const float* part, long long first, int np, const f
 
 constexpr int SEL_THREADS = 512;
 constexpr int SEL_WARPS = SEL_THREADS / 32;
+constexpr int kRecIssuers = 8;   // threads issuing the bulk copies of the score records
 constexpr int MAXSEL = 64;       // top_n bound of the fast path
 constexpr int MAXCAND = 4096;    // selection blocks bound of the fast path (T <= 262144)
 constexpr size_t kSelDynSmemMax = 192 * 1024;  // dec_select dynamic shared memory (+ ~18 KB static)
@@ -805,15 +807,21 @@ __global__ void __launch_bounds__(SEL_THREADS) dec_select_kernel(const __grid_co
   const int ncand = t / a.bs + 1;
   const int rtiles_u = (nvis + WK - 1) / WK;  // 32-key record sub-tiles
 
-  // The unit's score records, in one bulk copy that lands while the partials merge.
+  // The unit's score records, in bulk copies that land while the partials
+  // merge: kRecIssuers threads each copy a share of the sub-tiles (one thread's
+  // copies alone move too few bytes at a time).
   if (tid == 0) {
-    ptx::mbar_init(&rec_bar, 1);
+    ptx::mbar_init(&rec_bar, kRecIssuers);
     ptx::fence_mbar_init();
-    if (rtiles_u > 0) {
-      const uint32_t bytes = (uint32_t)rtiles_u * rec_floats * 4;
-      ptx::mbar_arrive_expect_tx(&rec_bar, bytes);
-      ptx::bulk_load(recs, a.trec + (long)u * a.tiles_max * rec_floats, bytes, &rec_bar);
-    }
+  }
+  __syncthreads();
+  if (tid < kRecIssuers) {
+    const int r0 = rtiles_u * tid / kRecIssuers, r1 = rtiles_u * (tid + 1) / kRecIssuers;
+    const uint32_t bytes = (uint32_t)(r1 - r0) * rec_floats * 4;
+    ptx::mbar_arrive_expect_tx(&rec_bar, bytes);
+    if (bytes > 0)
+      ptx::bulk_load(recs + (size_t)r0 * rec_floats,
+                     a.trec + ((long)u * a.tiles_max + r0) * rec_floats, bytes, &rec_bar);
   }
   const __nv_bfloat16* qg =
       reinterpret_cast<const __nv_bfloat16*>(a.q) + ((long)b * a.Hq + g * G) * D;
@@ -845,16 +853,12 @@ __global__ void __launch_bounds__(SEL_THREADS) dec_select_kernel(const __grid_co
 
   if (nvis > 0) {
     if (tid < 16) scl[tid] = gate[tid * 3];
-    const int h = (tid & 255) >> 4, e0 = (tid & 15) * 8;
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const int h = tid >> 5, e0 = (tid & 31) * 4;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
     merge_online<SEL_THREADS>(a.part1, 2 * ((long long)rg.x + u), 2 * (rg.y - rg.x + 1), scl, pm,
                               pl, mS, lS, sR, h, e0, acc);
     if (tid < 16) lse2[tid] = mS[tid] + log2f(lS[tid]);
-    if (tid < 256) {
-      float4* dst = reinterpret_cast<float4*>(oacc + h * D + e0);
-      dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-      dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
-    }
+    *reinterpret_cast<float4*>(oacc + h * D + e0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
     // records landed? then factors exp2(m_ref - lse) per (sub-tile, head)
     if (!ptx::mbar_wait(&rec_bar, 0, kWaitNs) && tid == 0) atomicOr(a.err, kErrTimeout);
     __syncthreads();
