@@ -52,7 +52,7 @@ struct MobaTcArgs {
   int32_t* toff;          // [NB + 1] first tile of each bucket
   int32_t* cur;           // [NB] fill cursors
   int32_t* list;          // rows: t * 8 + slot
-  float* po;              // [B, T, Hq, topk - 1, d] partial outputs (normalised)
+  __nv_bfloat16* po;      // [B, T, Hq, topk - 1, d] partial outputs (normalised, bf16)
   float* plse;            // [B, T, Hq, topk - 1] their log2-sum-exp
   unsigned* err;
   int B, T, Hq, Hkv, m, topk, nfull, NB;
@@ -586,12 +586,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t o[16];
         tc::ld16_sync(sm.tl + kO + c16 * 16, o);
         if (live) {
-          float4* dst = reinterpret_cast<float4*>(a.po + pr * D + c16 * 16);
+          uint4 pk[2];
+          uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
 #pragma unroll
-          for (int x = 0; x < 4; ++x)
-            dst[x] = make_float4(__uint_as_float(o[4 * x]) * il, __uint_as_float(o[4 * x + 1]) * il,
-                                 __uint_as_float(o[4 * x + 2]) * il,
-                                 __uint_as_float(o[4 * x + 3]) * il);
+          for (int x = 0; x < 8; ++x)
+            pw[x] = ptx::pack_bf16(__uint_as_float(o[2 * x]) * il, __uint_as_float(o[2 * x + 1]) * il);
+          uint4* dst = reinterpret_cast<uint4*>(a.po + pr * D + c16 * 16);
+          dst[0] = pk[0];
+          dst[1] = pk[1];
         }
       }
       if (live) a.plse[pr] = m + __log2f(l);
@@ -708,14 +710,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int e = 0; e < 16; ++e) acc[e] = __uint_as_float(o[e]) * wown;
       for (int s = 0; s < npast; ++s) {
-        const float4* ps = reinterpret_cast<const float4*>(a.po + (prow + s) * D + c16 * 16);
+        const uint4* ps = reinterpret_cast<const uint4*>(a.po + (prow + s) * D + c16 * 16);
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
-          const float4 pv = __ldg(ps + x);
-          acc[4 * x] = fmaf(wp[s], pv.x, acc[4 * x]);
-          acc[4 * x + 1] = fmaf(wp[s], pv.y, acc[4 * x + 1]);
-          acc[4 * x + 2] = fmaf(wp[s], pv.z, acc[4 * x + 2]);
-          acc[4 * x + 3] = fmaf(wp[s], pv.w, acc[4 * x + 3]);
+        for (int x = 0; x < 2; ++x) {
+          const uint4 pv = __ldg(ps + x);
+          const __nv_bfloat162* e2 = reinterpret_cast<const __nv_bfloat162*>(&pv);
+#pragma unroll
+          for (int y = 0; y < 4; ++y) {
+            const float2 f = __bfloat1622float2(e2[y]);
+            acc[8 * x + 2 * y] = fmaf(wp[s], f.x, acc[8 * x + 2 * y]);
+            acc[8 * x + 2 * y + 1] = fmaf(wp[s], f.y, acc[8 * x + 2 * y + 1]);
+          }
         }
       }
       if (live) {
@@ -766,7 +771,7 @@ size_t moba_tc_ws_bytes(const nsa_params& p, size_t kbar_bytes) {
   const size_t NB = (size_t)p.B * p.Hq * (p.T / p.sel_block);
   const size_t np = (size_t)(p.top_n - 1);
   return align256(kbar_bytes) + align256(rows * p.top_n * 4) + 4 * align256((NB + 1) * 4) +
-         align256(rows * np * 4 + 4) + align256(rows * np * D * 4 + 4) + align256(rows * np * 4 + 4);
+         align256(rows * np * 4 + 4) + align256(rows * np * D * 2 + 4) + align256(rows * np * 4 + 4);
 }
 
 cudaError_t launch_moba_tc(const nsa_params& p, const void* q, const void* k, const void* v,
@@ -799,8 +804,8 @@ cudaError_t launch_moba_tc(const nsa_params& p, const void* q, const void* k, co
   w += align256(((size_t)a.NB + 1) * 4);
   a.list = reinterpret_cast<int32_t*>(w);
   w += align256(rows * np * 4 + 4);
-  a.po = reinterpret_cast<float*>(w);
-  w += align256(rows * np * D * 4 + 4);
+  a.po = reinterpret_cast<__nv_bfloat16*>(w);
+  w += align256(rows * np * D * 2 + 4);
   a.plse = reinterpret_cast<float*>(w);
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.out = static_cast<__nv_bfloat16*>(out);
