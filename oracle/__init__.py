@@ -29,7 +29,7 @@ class _NsaCfg(ctypes.Structure):
         ("sel_block", ctypes.c_int), ("top_n", ctypes.c_int), ("window", ctypes.c_int),
         ("scale", ctypes.c_double), ("gate_mode", ctypes.c_int),
         ("fixed_gates", ctypes.c_double * 3), ("store", ctypes.c_int),
-        ("score_mode", ctypes.c_int),
+        ("score_mode", ctypes.c_int), ("top_p", ctypes.c_double),
     ]
 
 
@@ -93,6 +93,7 @@ def _nsa_cfg(p):
         c.fixed_gates[i] = float(fg[i])
     c.store = STORE[p.get("store", "none")] if isinstance(p.get("store", "none"), str) else int(p["store"])
     c.score_mode = int(p.get("score_mode", 0))
+    c.top_p = float(p.get("top_p", 0.0))
     return c
 
 

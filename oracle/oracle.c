@@ -43,6 +43,9 @@ typedef struct {
   int score_mode;              /* compressed-to-selection block mapping:
                                   0 unweighted sum over overlapping compressed
                                   blocks; 1 weighted by overlap / l              */
+  double top_p;                /* 0: top-n; in (0, 1]: adaptive selection that
+                                  stops once the selected blocks hold top_p of
+                                  the total score (at most n blocks)            */
 } oracle_nsa_cfg;
 
 typedef struct {
@@ -248,13 +251,36 @@ void oracle_nsa_rows(const oracle_nsa_cfg* c, int nrows, const int* rows_b, cons
 
       /* Step 4 [EP94 §五 branch two, §十六; LCH selection squad]: the top-n
        * blocks by score, block 0 always kept and counted in n. With n or fewer
-       * candidates all of them are kept. */
+       * candidates all of them are kept.
+       * Adaptive variant (top_p > 0) [LCH, adaptive sparsification: choose
+       * from the most important block on until the chosen scores add up to
+       * p times the total]: block 0 first, then the others by score (higher
+       * first, ties to the lower index), stopping at the first prefix whose
+       * score sum reaches top_p times the sum over all candidates, or at n
+       * blocks. */
       int* S = (int*)malloc(sizeof(int) * (n > 0 ? n : 1));
       int ns = 0;
       if (forced_sel) {
         const int* fr = forced_sel + ((long)r * Hkv + g) * n;
         for (int a = 0; a < n; ++a)
           if (fr[a] >= 0) S[ns++] = fr[a];
+      } else if (c->top_p > 0.0) {
+        double total = 0.0;
+        for (int j = 0; j < ncand; ++j) total += blk[j];
+        const double goal = c->top_p * total;
+        char* taken = (char*)calloc(ncand > 0 ? ncand : 1, 1);
+        S[ns++] = 0;
+        taken[0] = 1;
+        double cum = blk[0];
+        while (ns < n && ns < ncand && cum < goal) {
+          int best = -1;
+          for (int j = 1; j < ncand; ++j)
+            if (!taken[j] && (best < 0 || better(blk[j], j, blk[best], best))) best = j;
+          taken[best] = 1;
+          S[ns++] = best;
+          cum += blk[best];
+        }
+        free(taken);
       } else if (ncand <= n) {
         for (int j = 0; j < ncand; ++j) S[ns++] = j;
       } else {

@@ -375,3 +375,46 @@ def test_moba_block_means():
     kbar = oracle.moba_block_means(p, k)
     want = k[0, :192].reshape(12, 16, p["Hkv"], p["d"]).mean(axis=1)
     np.testing.assert_allclose(kbar[0], want, rtol=0, atol=1e-14)
+
+
+# --------------------------------------------------------------------------
+# adaptive (top-p) selection: lchairun NSA article, adaptive sparsification
+# (choose from the most important block on until the chosen scores reach p
+# times the total). Properties that fix the rule given the block scores:
+# --------------------------------------------------------------------------
+
+def _topp_rows(p):
+    q, k, v, w, wg = rand_inputs(p, rng=np.random.default_rng(77), qscale=3.0)
+    return oracle.nsa_prefill(p, q, k, v, w, wg)
+
+
+@pytest.mark.parametrize("top_p", [0.3, 0.6, 0.9])
+def test_topp_selection_is_the_shortest_best_prefix(top_p):
+    n = 12
+    p = base_params(T=256, sel_block=8, top_n=n, cmp_block=4, cmp_stride=2, top_p=top_p)
+    got = _topp_rows(p)
+    for t in range(0, 256, 5):
+        for g in range(p["Hkv"]):
+            nc = t // 8 + 1
+            sc = got["scores"][t, g, :nc]
+            S = [int(j) for j in got["sel"][t, g] if j >= 0]
+            assert S[0] == 0 and len(S) <= min(n, nc)          # block 0 kept, at most n
+            others = sorted(range(1, nc), key=lambda j: (-sc[j], j))
+            m = len(S) - 1
+            assert sorted(S[1:]) == sorted(others[:m])          # the m best of the others
+            total = sc.sum()
+            chosen = sc[0] + sum(sc[j] for j in others[:m])
+            if len(S) < min(n, nc):
+                assert chosen >= top_p * total - 1e-12         # reaches p of the total
+            if m > 0:                                           # and is the shortest such prefix
+                assert chosen - sc[others[m - 1]] < top_p * total + 1e-12
+
+
+def test_topp_grows_with_p_and_tiny_p_keeps_block_zero():
+    base = dict(T=256, sel_block=8, top_n=16, cmp_block=4, cmp_stride=2)
+    sels = [_topp_rows(base_params(**base, top_p=tp))["sel"] for tp in (1e-12, 0.4, 0.8, 1.0)]
+    for t in range(0, 256, 3):
+        for g in range(2):
+            a = [set(int(j) for j in s[t, g] if j >= 0) for s in sels]
+            assert a[0] == {0}
+            assert a[0] <= a[1] <= a[2] <= a[3]
