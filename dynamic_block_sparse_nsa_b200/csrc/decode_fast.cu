@@ -409,13 +409,17 @@ __device__ __forceinline__ TileSrc tile_source(const DecFastArgs& a, const Walke
   } else {
     const int t = wk.L - 1;
     int start;
+    bool unused = false;
     if (wk.tile < wk.ns) {
-      start = __ldg(a.sel + (long)(wk.b * a.Hkv + wk.g) * a.n + wk.tile) * a.bs;
+      // adaptive selection may keep fewer than n blocks: unused slots hold -1
+      const int blk = __ldg(a.sel + (long)(wk.b * a.Hkv + wk.g) * a.n + wk.tile);
+      unused = blk < 0;
+      start = unused ? 0 : blk * a.bs;
     } else {
       start = t - min(a.w, wk.L) + 1 + (wk.tile - wk.ns) * TK;
     }
     ts.row = wk.b * a.T + start;
-    ts.nvalid = min(TK, t - start + 1);
+    ts.nvalid = unused ? 0 : min(TK, t - start + 1);
   }
   return ts;
 }
@@ -981,6 +985,55 @@ __global__ void __launch_bounds__(SEL_THREADS) dec_select_kernel(const __grid_co
     ns = a.n;
   }
   __syncthreads();
+  if (a.top_p > 0.f) {
+    // Adaptive selection (lchairun NSA article, adaptive sparsification): the
+    // top-p set is a best-first prefix of at most n blocks, so it is cut from
+    // the top-n set above: block 0, then the kept blocks by key (score desc,
+    // index asc) until their scores reach top_p of the total over all
+    // candidates (fp64 sums).
+    __shared__ double wtot[SEL_WARPS];
+    __shared__ int ord[MAXSEL];
+    double part = 0.0;
+    for (int j = tid; j < ncand; j += SEL_THREADS)
+      part += (double)__uint_as_float((unsigned)(keys[j] >> 32));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+    if (lane == 0) wtot[warp] = part;
+    // the kept blocks other than 0, ordered by key (descending)
+    const int nk = ns - 1;
+    if (tid < nk) {
+      const int j = sel[1 + tid];
+      const unsigned long long kj = keys[j];
+      int rank = 0;
+      for (int i = 0; i < nk; ++i) rank += keys[sel[1 + i]] > kj ? 1 : 0;
+      ord[rank] = j;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      double tot = 0.0;
+      for (int w = 0; w < SEL_WARPS; ++w) tot += wtot[w];
+      const double goal = (double)a.top_p * tot;
+      double cum = (double)__uint_as_float((unsigned)(keys[0] >> 32));
+      int m = 0;
+      while (m < nk && cum < goal) {
+        cum += (double)__uint_as_float((unsigned)(keys[ord[m]] >> 32));
+        ++m;
+      }
+      nsel_s = m + 1;
+    }
+    __syncthreads();
+    ns = nsel_s;
+    // ascending: block 0 first, then ord[0 .. ns - 1) sorted
+    int v = -1, rank = 0;
+    if (tid < ns) {
+      v = tid == 0 ? 0 : ord[tid - 1];
+      for (int i = 1; i < ns; ++i) rank += ord[i - 1] < v ? 1 : 0;
+      rank += tid == 0 ? 0 : 1;  // block 0 precedes every other block
+    }
+    __syncthreads();
+    if (tid < ns) sel[rank] = v;
+    __syncthreads();
+  }
   for (int x = tid; x < a.n; x += SEL_THREADS) {
     const int v = x < ns ? sel[x] : -1;
     a.sel[(long)u * a.n + x] = v;
@@ -1091,6 +1144,7 @@ DecFastArgs base_args(const nsa_params& p) {
   a.scale_log2 = scale * 1.4426950408889634f;
   a.gate_mode = p.gate_mode;
   for (int i = 0; i < 3; ++i) a.fixed_gates[i] = p.fixed_gates[i];
+  a.top_p = p.top_p;
   return a;
 }
 

@@ -38,6 +38,7 @@ struct NsaRowArgs {
   float fixed_gates[3];
   int decode;               // 0 prefill (row per token), 1 decode (row per sequence)
   nsa_dtype dtype;
+  float top_p;              // 0: top-n; else adaptive selection
 };
 
 struct MobaArgs {
@@ -71,6 +72,7 @@ struct DecFastArgs {
   float scale_log2;
   int gate_mode;
   float fixed_gates[3];
+  float top_p;    // 0: top-n; else adaptive selection
   int8_t klo[kDecMaxNbt], khi[kDecMaxNbt];  // per block of a tile: its key range
   float* part1;   // compressed-branch partials, slot = 2 * (stream + unit) + half
   float* trec;    // per-tile block-score records

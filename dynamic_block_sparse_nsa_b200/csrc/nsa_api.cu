@@ -94,6 +94,8 @@ nsa_status check_nsa(const nsa_params* p) {
   if (p->top_n > 1024) return fail(NSA_ERR_UNSUPPORTED, "top_n must be <= 1024");
   if (p->gate_mode != 0 && p->gate_mode != 1)
     return fail(NSA_ERR_INVALID_ARGUMENT, "gate_mode must be 0 or 1");
+  if (!(p->top_p >= 0.f && p->top_p <= 1.f))
+    return fail(NSA_ERR_INVALID_ARGUMENT, "top_p must be in [0, 1] (0: top-n selection)");
   if (p->Hkv > 65535) return fail(NSA_ERR_UNSUPPORTED, "Hkv must be <= 65535");
   return NSA_OK;
 }
@@ -114,6 +116,7 @@ NsaRowArgs row_args(const nsa_params* p) {
   a.scale = eff_scale(p);
   a.gate_mode = p->gate_mode;
   for (int i = 0; i < 3; ++i) a.fixed_gates[i] = p->fixed_gates[i];
+  a.top_p = p->top_p;
   a.dtype = p->dtype;
   return a;
 }

@@ -68,6 +68,7 @@ struct PfArgs {
   int need_sel;    // block scores and top-n (pass 3, step 4)
   int run_win;     // window attention (pass 2)
   int direct_out;  // no selected branch: pf_main writes the bf16 output itself
+  float top_p;     // 0: top-n; else adaptive selection
 };
 
 __device__ __forceinline__ unsigned char* align1024(unsigned char* p) {
@@ -495,7 +496,51 @@ __global__ void __launch_bounds__(kMainThreads, 1)
       if (tok < a.T) {  // warp-uniform
         const int ncand = tok / SB + 1;
         int32_t* dst = a.sel + ((size_t)(b * a.T + tok) * a.Hkv + g) * a.n;
-        if (ncand <= a.n) {
+        if (a.top_p > 0.f) {
+          // adaptive: block 0, then the best others until their scores reach
+          // top_p of the total over all candidates (fp64 sums), at most n
+          float* scx = sc + x * a.nblk;
+          double part = 0.0;
+          for (int jb = lane; jb < ncand; jb += 32) part += (double)scx[jb];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+          const double goal = (double)a.top_p * part;
+          double cum = (double)scx[0];
+          uint32_t bh = 0, bl = 0;
+          auto rescan = [&]() {
+            uint32_t hh = 0, ll = 0;
+            for (int jb = 1 + lane; jb < ncand; jb += 32) {
+              const float vv = scx[jb];
+              const uint32_t kh = vv < 0.f ? 0u : __float_as_uint(vv) + 1u;
+              const uint32_t kl = ~(uint32_t)jb;
+              if (kh > hh || (kh == hh && kl > ll)) {
+                hh = kh;
+                ll = kl;
+              }
+            }
+            bh = hh;
+            bl = ll;
+          };
+          rescan();
+          int mine = lane == 0 ? 0 : 0x7fffffff;
+          int cnt = 1;
+          while (cnt < a.n && cnt < ncand && cum < goal) {  // warp-uniform
+            const uint32_t mh = __reduce_max_sync(0xffffffffu, bh);
+            const uint32_t ml = __reduce_max_sync(0xffffffffu, bh == mh ? bl : 0u);
+            const int pick = (int)~ml;
+            cum += (double)__uint_as_float(mh - 1u);
+            if (lane == cnt) mine = pick;
+            ++cnt;
+            if (((pick - 1) & 31) == lane) {
+              scx[pick] = -1.f;
+              rescan();
+            }
+          }
+          int rank = 0;
+          for (int o = 0; o < 32; ++o) rank += (__shfl_sync(0xffffffffu, mine, o) < mine) ? 1 : 0;
+          if (lane < cnt) dst[rank] = mine;
+          for (int i = cnt + lane; i < a.n; i += 32) dst[i] = -1;
+        } else if (ncand <= a.n) {
           for (int i = lane; i < a.n; i += 32) dst[i] = i < ncand ? i : -1;
         } else {
           float* scx = sc + x * a.nblk;
@@ -1081,6 +1126,7 @@ cudaError_t launch_prefill_tc(const nsa_params& p, const void* q, const void* k,
   a.run_cmp = !(fixed && p.fixed_gates[0] == 0.f) || a.need_sel;
   a.run_win = !(fixed && p.fixed_gates[2] == 0.f);
   a.direct_out = !slc_branch;
+  a.top_p = p.top_p;
 
   const uint64_t BT = (uint64_t)p.B * p.T;
   CUtensorMap tq, tq16, tk, tv, tk64, tv64, tkc, tvc;

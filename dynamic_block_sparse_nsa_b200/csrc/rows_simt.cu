@@ -245,6 +245,87 @@ __device__ inline int select_top(const Ctx& c, int lo, int ncand, int forced, in
   return ns;
 }
 
+// Adaptive selection over scores[0, ncand) (lchairun NSA article, adaptive
+// sparsification): block 0, then the best others by (score desc, index asc)
+// until the chosen scores reach top_p times the sum over all candidates, at
+// most n blocks. Sums in fp64. Writes sel[0..) ascending; returns the count.
+__device__ inline int select_top_p(const Ctx& c, int ncand, int n, float top_p) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ double tot_s, cum_s;
+  __shared__ int stop_s;
+  double part = 0.0;
+  for (int j = threadIdx.x; j < ncand; j += kThreads) part += (double)c.scores[j];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+  __shared__ double wpart[kWarps];
+  if (lane == 0) wpart[warp] = part;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double t = 0.0;
+    for (int w = 0; w < kWarps; ++w) t += wpart[w];
+    tot_s = t;
+    cum_s = (double)c.scores[0];
+    c.sel[0] = 0;
+    c.scores[0] = -INFINITY;
+    stop_s = (1 >= n || 1 >= ncand || cum_s >= (double)top_p * t) ? 1 : 0;
+  }
+  __syncthreads();
+  int ns = 1;
+  while (!stop_s) {
+    float bs = -INFINITY;
+    int bj = INT_MAX;
+    for (int j = 1 + threadIdx.x; j < ncand; j += kThreads) {
+      const float sj = c.scores[j];
+      if (sj != -INFINITY && sel_better(sj, j, bs, bj)) {
+        bs = sj;
+        bj = j;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float os = __shfl_xor_sync(0xffffffffu, bs, o);
+      const int oj = __shfl_xor_sync(0xffffffffu, bj, o);
+      if (sel_better(os, oj, bs, bj)) {
+        bs = os;
+        bj = oj;
+      }
+    }
+    if (lane == 0) {
+      c.red_s[warp] = bs;
+      c.red_j[warp] = bj;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float s0 = c.red_s[0];
+      int j0 = c.red_j[0];
+      for (int w = 1; w < kWarps; ++w)
+        if (sel_better(c.red_s[w], c.red_j[w], s0, j0)) {
+          s0 = c.red_s[w];
+          j0 = c.red_j[w];
+        }
+      c.sel[ns] = j0;
+      cum_s += (double)s0;
+      c.scores[j0] = -INFINITY;
+      stop_s = (ns + 1 >= n || ns + 1 >= ncand || cum_s >= (double)top_p * tot_s) ? 1 : 0;
+    }
+    __syncthreads();
+    ++ns;
+  }
+  if (threadIdx.x == 0) {
+    for (int x = 1; x < ns; ++x) {  // insertion sort, ascending
+      const int v = c.sel[x];
+      int q = x - 1;
+      while (q >= 0 && c.sel[q] > v) {
+        c.sel[q + 1] = c.sel[q];
+        --q;
+      }
+      c.sel[q + 1] = v;
+    }
+  }
+  __syncthreads();
+  return ns;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads) nsa_rows_kernel(NsaRowArgs a) {
   extern __shared__ float sm[];
@@ -363,7 +444,9 @@ __global__ void __launch_bounds__(kThreads) nsa_rows_kernel(NsaRowArgs a) {
 
   // ---- top-n selection (block 0 forced) ----
   int ns;
-  if (ncand <= a.n) {
+  if (a.top_p > 0.f) {
+    ns = select_top_p(c, ncand, a.n, a.top_p);
+  } else if (ncand <= a.n) {
     for (int j = threadIdx.x; j < ncand; j += kThreads) c.sel[j] = j;
     __syncthreads();
     ns = ncand;

@@ -46,7 +46,7 @@ class NsaParams(ctypes.Structure):
         ("d", ctypes.c_int), ("cmp_block", ctypes.c_int), ("cmp_stride", ctypes.c_int),
         ("sel_block", ctypes.c_int), ("top_n", ctypes.c_int), ("window", ctypes.c_int),
         ("softmax_scale", ctypes.c_float), ("gate_mode", ctypes.c_int),
-        ("fixed_gates", ctypes.c_float * 3), ("dtype", ctypes.c_int),
+        ("fixed_gates", ctypes.c_float * 3), ("dtype", ctypes.c_int), ("top_p", ctypes.c_float),
     ]
 
     @property
@@ -119,7 +119,8 @@ def _dev(t, name, dtype=None):
 
 
 def params(B, T, Hq, Hkv, d, cmp_block=32, cmp_stride=16, sel_block=64, top_n=16, window=512,
-           softmax_scale=0.0, gate_mode=0, fixed_gates=(0.0, 0.0, 0.0), dtype=torch.bfloat16):
+           softmax_scale=0.0, gate_mode=0, fixed_gates=(0.0, 0.0, 0.0), dtype=torch.bfloat16,
+           top_p=0.0):
     p = NsaParams()
     p.B, p.T, p.Hq, p.Hkv, p.d = B, T, Hq, Hkv, d
     p.cmp_block, p.cmp_stride, p.sel_block, p.top_n, p.window = (
@@ -129,6 +130,7 @@ def params(B, T, Hq, Hkv, d, cmp_block=32, cmp_stride=16, sel_block=64, top_n=16
     for i in range(3):
         p.fixed_gates[i] = fixed_gates[i]
     p.dtype = DTYPE_BF16 if dtype == torch.bfloat16 else DTYPE_F32
+    p.top_p = top_p
     return p
 
 

@@ -81,6 +81,11 @@ typedef enum {
  *   gate_mode  0: g = sigmoid(q . Wg) per branch (Wg [d,3], order cmp, slc,
  *              win, raw unscaled q); 1: g = fixed_gates for every query.
  *   dtype      element type of q, k, v, compressed k/v and out.
+ *   top_p      0: keep top_n blocks. In (0, 1]: adaptive selection (lchairun
+ *              NSA article, adaptive sparsification): block 0, then the other
+ *              blocks by score (ties to the lower index) up to the first prefix
+ *              whose score sum reaches top_p times the sum over all candidate
+ *              blocks, at most top_n blocks; unused sel_idx slots hold -1.
  * MoBA uses B, T, Hq, Hkv, d, sel_block, top_n, softmax_scale and dtype. */
 typedef struct {
   int B, T, Hq, Hkv, d;
@@ -90,6 +95,7 @@ typedef struct {
   int gate_mode;
   float fixed_gates[3];
   nsa_dtype dtype;
+  float top_p;
 } nsa_params;
 
 /* Bytes of caller-provided device workspace `op` needs for `p` (0 is

@@ -60,6 +60,37 @@ def check_selection(gpu_sel, ora_sel, ora_scores, ncand, n_keep, forced_first=Tr
     return False
 
 
+def check_selection_topp(gpu_sel, ora_sel, ora_scores, ncand, n_keep, top_p):
+    """Compare one row of adaptive (top-p) selection. True if the sets are
+    equal; False if they differ only within the tolerances (near-equal scores
+    at the cut, or a cumulative sum within SEL_REL of top_p times the total);
+    raises otherwise. The GPU set must be block 0 plus a best-first prefix of
+    the others that reaches top_p of the total (unless n blocks are taken) and
+    is the shortest such prefix."""
+    g = sorted(int(x) for x in gpu_sel if x >= 0)
+    o = sorted(int(x) for x in ora_sel if x >= 0)
+    if g == o:
+        return True
+    sc = np.asarray(ora_scores[:ncand], dtype=np.float64)
+    assert 0 in g, f"block 0 missing from gpu selection {g}"
+    assert len(g) <= min(n_keep, ncand), f"gpu kept {len(g)} blocks (n {n_keep}, {ncand} candidates)"
+    total = float(sc.sum())
+    goal = top_p * total
+    tol = SEL_REL * max(abs(total), 1e-30)
+    free = [j for j in g if j != 0]
+    chosen = float(sc[0] + sc[free].sum()) if free else float(sc[0])
+    if free:
+        s_min = float(sc[free].min())
+        for j in range(1, ncand):
+            if j not in free:
+                assert sc[j] <= s_min + SEL_REL * abs(s_min), (
+                    f"gpu dropped block {j} ({sc[j]:.9e}) above kept {s_min:.9e}: gpu {g} oracle {o}")
+        assert chosen - s_min < goal + tol, f"gpu selection {g} is longer than needed (oracle {o})"
+    if len(g) < min(n_keep, ncand):
+        assert chosen >= goal - tol, f"gpu selection {g} stops short of top_p (oracle {o})"
+    return False
+
+
 def check_output(gpu, ref, dtype, what="out"):
     gpu = np.asarray(gpu, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)

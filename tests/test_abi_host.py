@@ -56,6 +56,9 @@ def test_workspace_size_validation():
     assert b"head dim" in nsa.LIB.nsa_last_error_detail()
     bad = nsa.params(1, 1024, 6, 4, 64)
     assert nsa.LIB.nsa_workspace_size(ctypes.byref(bad), nsa.OP_PREFILL, ctypes.byref(n)) == 1
+    bad = nsa.params(1, 1024, 4, 1, 64, top_p=1.5)
+    assert nsa.LIB.nsa_workspace_size(ctypes.byref(bad), nsa.OP_PREFILL, ctypes.byref(n)) == 1
+    assert b"top_p" in nsa.LIB.nsa_last_error_detail()
     bad = nsa.params(1, 1024, 4, 1, 64, cmp_block=8, cmp_stride=16)
     assert nsa.LIB.nsa_workspace_size(ctypes.byref(bad), nsa.OP_PREFILL, ctypes.byref(n)) == 1
     # MoBA: block means [B, T/m, Hkv, d] fp32; the tensor-core path (bf16,

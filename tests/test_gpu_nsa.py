@@ -181,3 +181,42 @@ def test_prefill_bf16_dense_closed_form(want_sel):
         for t in range(T):
             row = s[t][s[t] >= 0]
             assert len(row) == min(w["top_n"], t // 64 + 1) and (np.diff(row) > 0).all()
+
+
+# Adaptive (top-p) selection on every selection implementation. Unit-variance
+# queries and keys make the block scores uneven enough that the cumulative
+# rule stops before n blocks for many rows.
+@pytest.mark.parametrize("top_p", [0.2, 0.5, 0.95])
+def test_prefill_bf16_top_p_tensor_core(top_p):
+    w = inputs.workload("nsa_prefill_bf16_t8192", T=1500, Hq=16, Hkv=1, qkv_scale=1.0, top_p=top_p)
+    gc.run_nsa_prefill(w, seed=31)
+
+
+def test_prefill_f32_top_p_generic():
+    w = inputs.workload("nsa_prefill_f32_t1024", top_n=8, top_p=0.4)
+    gc.run_nsa_prefill(w, seed=32)
+
+
+@pytest.mark.parametrize("top_p", [0.3, 0.7])
+def test_decode_bf16_top_p_fast(top_p):
+    w = inputs.workload("nsa_decode_bf16_b32_l65536", B=4, T=5000, top_p=top_p)
+    gc.run_nsa_decode(w, [5000, 3001, 700, 64])
+
+
+def test_decode_f32_top_p_generic():
+    w = inputs.workload("nsa_decode_bf16_b32_l65536", B=3, T=3000, dtype="f32", Hq=8, Hkv=2,
+                        d=64, top_n=6, window=100, top_p=0.5)
+    gc.run_nsa_decode(w, [2999, 1500, 200])
+
+
+def test_prefill_top_p_stops_before_n():
+    from dynamic_block_sparse_nsa_b200 import nsa
+    w = inputs.workload("nsa_prefill_bf16_t8192", T=1500, Hq=16, Hkv=1, qkv_scale=1.0, top_p=0.2)
+    inp = inputs.make_prefill(w, 31)
+    p = gc.nsa_params_for(w)
+    dev = {k_: v_.cuda() for k_, v_ in inp.items()}
+    kc, vc = nsa.nsa_compress_kv(p, dev["k"], dev["v"], dev["w_cmp"])
+    _, sel = nsa.nsa_prefill(p, dev["q"], dev["k"], dev["v"], kc, vc, dev["w_gate"])
+    nsa.nsa_check()
+    counts = (sel[0, 1100:, 0] >= 0).sum(-1)
+    assert int(counts.min()) < w["top_n"] and int(counts.max()) >= 2
