@@ -6,26 +6,26 @@
 // (EP94 notes §六; lchairun.cn NSA article, decode paragraph). Four kernels:
 //
 //  dec_cmp_partial  stream kernel over the compressed keys (see below); also
-//                   writes, per 64-key tile and head, the running max it used
-//                   and the exp-sums of its keys per overlapped selection
+//                   writes, per 32-key sub-tile and head, the running max it
+//                   used and the exp-sums of its keys per overlapped selection
 //                   block, because block scores need probabilities normalised
 //                   by the final lse, which is known only at the end.
-//  dec_select       one CTA per (sequence, KV head): merges the partials into
-//                   lse and o_cmp, rescales the tile records into block scores
-//                   summed over the group's heads, keeps block 0 plus the top
-//                   n-1 others (ties to the lower index), computes the gates.
+//  dec_select       one CTA per (sequence, KV head): merges the partials' (m, l)
+//                   into the lse, rescales the sub-tile records into block
+//                   scores summed over the group's heads, keeps block 0 plus
+//                   the top n-1 others (ties to the lower index).
 //  dec_sel_win      stream kernel over the selected blocks, then the window.
-//  dec_combine      one CTA per unit: out = g0 o_cmp + g1 o_slc + g2 o_win.
+//  dec_combine      merges the partials of all three branches, computes the
+//                   gates: out = g0 o_cmp + g1 o_slc + g2 o_win.
 //
-// Stream kernel: persistent, one CTA per SM, 1 TMA producer warp + 3 pairs of
-// consumer warps (7 warps: at most two per SM sub-partition, whose register
-// file then holds up to 255 registers a thread). The global sequence of 64-key
-// tiles (sequence-major, then KV head, then tile) is split evenly over the
-// SMs x 3 pair streams; each pair has a private ring of four 16 KB slots (K or
-// V of a tile, 128B-swizzled TMA boxes, L2 evict-first) so no stream waits on
-// another's slot. The two warps of a pair take 32 keys each of every tile and
-// keep online-softmax partials (m, l, O), written once per segment they touch
-// (segment = unit, or unit and branch).
+// Stream kernel: persistent, one CTA per SM, 1 TMA producer warp + 4 pairs of
+// consumer warps. The global sequence of 64-key tiles (sequence-major, then KV
+// head, then tile) is split evenly over the SMs x 4 pair streams; each pair has
+// a private ring of three 16 KB slots (K or V of a tile, 128B-swizzled TMA
+// boxes, L2 evict-first) so no stream waits on another's slot. The two warps
+// of a pair take 32 keys each of every tile and keep online-softmax partials
+// (m, l, O), written once per segment they touch (segment = unit, or unit and
+// branch).
 // Softmax runs in the log2 domain: z2 = (q . k) * scale * log2(e).
 #include <algorithm>
 #include <climits>
@@ -663,87 +663,6 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
 }
 
 // ---------------------------------------------------------------------------
-// merging stream partials (dec_select, dec_combine)
-// ---------------------------------------------------------------------------
-
-constexpr int MP = 64;  // partials staged per chunk
-
-// Online merge of the softmax partials in slots [first, first + np): per head
-// M = max m_p and L = sum_p exp2(m_p - M) l_p (left in sM / sL), and
-//   acc[h][e0 .. e0+E-1] += scale_h / L_h * sum_p exp2(m_p - M_h) o_p[h][e].
-// Partials are staged MP at a time with a running max and sum, so any count
-// works; one chunk costs two load-dependent steps. Every thread owns E =
-// 2048 / NT output values (head h, dims e0 ..) and keeps the loads of up to 8
-// partials in flight.
-template <int NT>
-__device__ void merge_online(const float* part, long long first, int np, const float* scale,
-                             float* pm, float* pl, float* sM, float* sL, float* sR, int h, int e0,
-                             float (&acc)[2048 / NT]) {
-  constexpr int E = 2048 / NT;
-  const int tid = threadIdx.x;
-  float run[E];
-#pragma unroll
-  for (int e = 0; e < E; ++e) run[e] = 0.f;
-  if (tid < 16) {
-    sM[tid] = -INFINITY;
-    sL[tid] = 0.f;
-  }
-  for (int p0 = 0; p0 < np; p0 += MP) {
-    const int pc = min(MP, np - p0);
-    __syncthreads();
-    for (int x = tid; x < pc * 16; x += NT) {
-      const float* src = part + (first + p0 + (x >> 4)) * PART;
-      pm[x] = __ldcg(src + (x & 15));
-      pl[x] = __ldcg(src + G + (x & 15));
-    }
-    __syncthreads();
-    if (tid < 16) {
-      float Mc = -INFINITY;
-      for (int pp = 0; pp < pc; ++pp) Mc = fmaxf(Mc, pm[pp * 16 + tid]);
-      const float Mo = sM[tid], Mn = fmaxf(Mo, Mc);
-      const float r = Mo == -INFINITY ? 0.f : exp2f(Mo - Mn);
-      float Lc = 0.f;
-      for (int pp = 0; pp < pc; ++pp) {
-        const float mm = pm[pp * 16 + tid];
-        if (mm != -INFINITY) Lc += exp2f(mm - Mn) * pl[pp * 16 + tid];
-      }
-      sL[tid] = sL[tid] * r + Lc;
-      sM[tid] = Mn;
-      sR[tid] = r;
-    }
-    __syncthreads();
-    for (int x = tid; x < pc * 16; x += NT) {
-      const float mm = pm[x];
-      pm[x] = mm == -INFINITY ? 0.f : exp2f(mm - sM[x & 15]);
-    }
-    __syncthreads();
-    {
-      const float r = sR[h];
-#pragma unroll
-      for (int e = 0; e < E; ++e) run[e] *= r;
-#pragma unroll 8
-      for (int pp = 0; pp < pc; ++pp) {
-        const float f = pm[pp * 16 + h];
-        const float4* src =
-            reinterpret_cast<const float4*>(part + (first + p0 + pp) * PART + 2 * G + h * D + e0);
-#pragma unroll
-        for (int q4 = 0; q4 < E / 4; ++q4) {
-          const float4 v = __ldcg(src + q4);
-          run[4 * q4] += f * v.x;
-          run[4 * q4 + 1] += f * v.y;
-          run[4 * q4 + 2] += f * v.z;
-          run[4 * q4 + 3] += f * v.w;
-        }
-      }
-    }
-  }
-  __syncthreads();
-  const float sc = sL[h] > 0.f ? scale[h] / sL[h] : 0.f;
-#pragma unroll
-  for (int e = 0; e < E; ++e) acc[e] += sc * run[e];
-}
-
-// ---------------------------------------------------------------------------
 // dec_select
 // ---------------------------------------------------------------------------
 
@@ -758,7 +677,7 @@ constexpr size_t kSelDynSmemMax = 192 * 1024;  // dec_select dynamic shared memo
 // and two per-(sub-tile, head) arrays.
 __host__ __device__ inline size_t sel_dyn_smem(int T, int sel_block, int tiles_max, int nbt) {
   const int nblk = (T + sel_block - 1) / sel_block;
-  int npow = 1;
+  int npow = 2;  // >= 2 keeps the float arrays after the keys 16-byte aligned
   while (npow < nblk) npow <<= 1;
   return (size_t)tiles_max * 16 * (1 + nbt) * 4 + (size_t)npow * 8 + 2 * (size_t)tiles_max * 16 * 4 +
          16;
@@ -775,10 +694,7 @@ __global__ void __launch_bounds__(SEL_THREADS) dec_select_kernel(const __grid_co
   // dynamic: records [tiles_max][16 (1 + nbt)] | keys [npow] u64 | fac [tiles_max][16]
   //          | tsum [tiles_max][16]
   extern __shared__ __align__(128) unsigned char dyn_raw[];
-  __shared__ float mS[G], lS[G], sR[G], lse2[G], gate[3 * G], scl[G];
-  __shared__ __align__(16) float pm[MP * G], pl[MP * G];
-  __shared__ float wg_s[D * 3];
-  __shared__ float q_s[G * D];
+  __shared__ float lse2[G];
   __shared__ int sel[MAXSEL];
   __shared__ unsigned hist[256];
   __shared__ int cut_bin, cut_above, nsel_s;
@@ -786,8 +702,12 @@ __global__ void __launch_bounds__(SEL_THREADS) dec_select_kernel(const __grid_co
 
   const int u = blockIdx.x, b = u / a.Hkv, g = u - b * a.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  if (tid == 0) {
+    ptx::mbar_init(&rec_bar, kRecIssuers);
+    ptx::fence_mbar_init();
+  }
   const int nblk = (a.T + a.bs - 1) / a.bs;
-  int npow = 1;
+  int npow = 2;  // as in sel_dyn_smem
   while (npow < nblk) npow <<= 1;
   const int rec_floats = G * (1 + a.nbt);
   float* recs = reinterpret_cast<float*>(dyn_raw);
@@ -796,7 +716,6 @@ __global__ void __launch_bounds__(SEL_THREADS) dec_select_kernel(const __grid_co
   float* tsum = fac + (size_t)a.tiles_max * G;
 
   const int L = __ldg(a.seq_lens + b);
-  float* oacc = a.oacc + (long)u * G * D;
   if (!len_ok(L, a)) {
     for (int x = tid; x < G * D; x += SEL_THREADS)
       reinterpret_cast<__nv_bfloat16*>(a.out)[((long)b * a.Hq + g * G) * D + x] =
@@ -810,59 +729,41 @@ __global__ void __launch_bounds__(SEL_THREADS) dec_select_kernel(const __grid_co
   const int nvis = n_visible(L, a.l, a.s, a.Nc);
   const int ncand = t / a.bs + 1;
   const int rtiles_u = (nvis + WK - 1) / WK;  // 32-key record sub-tiles
-
-  // The unit's score records, in bulk copies that land while the partials
-  // merge: kRecIssuers threads each copy a share of the sub-tiles (one thread's
-  // copies alone move too few bytes at a time).
-  if (tid == 0) {
-    ptx::mbar_init(&rec_bar, kRecIssuers);
-    ptx::fence_mbar_init();
-  }
-  __syncthreads();
-  if (tid < kRecIssuers) {
-    const int r0 = rtiles_u * tid / kRecIssuers, r1 = rtiles_u * (tid + 1) / kRecIssuers;
-    const uint32_t bytes = (uint32_t)(r1 - r0) * rec_floats * 4;
-    ptx::mbar_arrive_expect_tx(&rec_bar, bytes);
-    if (bytes > 0)
-      ptx::bulk_load(recs + (size_t)r0 * rec_floats,
-                     a.trec + ((long)u * a.tiles_max + r0) * rec_floats, bytes, &rec_bar);
-  }
-  const __nv_bfloat16* qg =
-      reinterpret_cast<const __nv_bfloat16*>(a.q) + ((long)b * a.Hq + g * G) * D;
-  for (int x = tid; x < G * D; x += SEL_THREADS) q_s[x] = __bfloat162float(qg[x]);
-  if (a.gate_mode == 0)
-    for (int x = tid; x < D * 3; x += SEL_THREADS) wg_s[x] = __ldg(a.w_gate + x);
-  const int2 rg = *reinterpret_cast<const int2*>(a.rng1 + 2 * u);
-  __syncthreads();
-
-  // gates (EP94 notes §五 gating), from the raw query: a warp per dot product
-  for (int x = warp; x < 3 * G; x += SEL_WARPS) {
-    const int h = x / 3, br = x - h * 3;
-    float gv;
-    if (a.gate_mode == 1) {
-      gv = a.fixed_gates[br];
-    } else {
-      float dot = 0.f;
-#pragma unroll
-      for (int e = lane; e < D; e += 32) dot = fmaf(q_s[h * D + e], wg_s[e * 3 + br], dot);
-      dot = warp_sum(dot);
-      gv = 1.f / (1.f + expf(-dot));
-    }
-    if (lane == 0) {
-      gate[x] = gv;
-      a.gates[(long)u * 3 * G + x] = gv;
-    }
-  }
-  __syncthreads();
+  __syncthreads();  // rec_bar initialised
 
   if (nvis > 0) {
-    if (tid < 16) scl[tid] = gate[tid * 3];
-    const int h = tid >> 5, e0 = (tid & 31) * 4;
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-    merge_online<SEL_THREADS>(a.part1, 2 * ((long long)rg.x + u), 2 * (rg.y - rg.x + 1), scl, pm,
-                              pl, mS, lS, sR, h, e0, acc);
-    if (tid < 16) lse2[tid] = mS[tid] + log2f(lS[tid]);
-    *reinterpret_cast<float4*>(oacc + h * D + e0) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    // The unit's score records, in bulk copies that land while the lse is
+    // merged: kRecIssuers threads each copy a share of the sub-tiles (one
+    // thread's copies alone move too few bytes at a time).
+    if (tid < kRecIssuers) {
+      const int r0 = rtiles_u * tid / kRecIssuers, r1 = rtiles_u * (tid + 1) / kRecIssuers;
+      const uint32_t bytes = (uint32_t)(r1 - r0) * rec_floats * 4;
+      ptx::mbar_arrive_expect_tx(&rec_bar, bytes);
+      if (bytes > 0)
+        ptx::bulk_load(recs + (size_t)r0 * rec_floats,
+                       a.trec + ((long)u * a.tiles_max + r0) * rec_floats, bytes, &rec_bar);
+    }
+    // lse of the compressed branch per head (warp h): log2 of sum_p 2^m_p l_p
+    // over the unit's partials, each lane merging a strided share first
+    {
+      const int2 rg = *reinterpret_cast<const int2*>(a.rng1 + 2 * u);
+      const long long first = 2 * ((long long)rg.x + u);
+      const int np = 2 * (rg.y - rg.x + 1);
+      const int h = warp;  // SEL_WARPS == G
+      float M = -INFINITY, Ls = 0.f;
+      for (int pp = lane; pp < np; pp += 32) {
+        const float* src = a.part1 + (first + pp) * PART;
+        const float m = __ldcg(src + h), l = __ldcg(src + G + h);
+        if (m == -INFINITY) continue;
+        const float Mn = fmaxf(M, m);
+        Ls = Ls * exp2f(M - Mn) + l * exp2f(m - Mn);  // exp2f(-inf) = 0 on the first
+        M = Mn;
+      }
+      const float Mw = warp_max(M);
+      const float c = M == -INFINITY ? 0.f : Ls * exp2f(M - Mw);
+      const float Lw = warp_sum(c);
+      if (lane == 0) lse2[h] = Mw + log2f(Lw);
+    }
     // records landed? then factors exp2(m_ref - lse) per (sub-tile, head)
     if (!ptx::mbar_wait(&rec_bar, 0, kWaitNs) && tid == 0) atomicOr(a.err, kErrTimeout);
     __syncthreads();
@@ -871,24 +772,30 @@ __global__ void __launch_bounds__(SEL_THREADS) dec_select_kernel(const __grid_co
       fac[x] = exp2f(recs[tau * rec_floats + h] - lse2[h]);
     }
     __syncthreads();
-    // per (sub-tile, block slot): the head-weighted sum of the record, as a
-    // 16-wide dot product of two contiguous shared-memory rows
-    for (int x = tid; x < rtiles_u * 16; x += SEL_THREADS) {
-      const int tau = x >> 4, jl = x & 15;
-      float v = 0.f;
-      if (jl < a.nbt) {
-        const float4* rt = reinterpret_cast<const float4*>(recs + tau * rec_floats + G * (1 + jl));
-        const float4* f = reinterpret_cast<const float4*>(fac + tau * G);
-        float v0 = 0.f, v1 = 0.f;
-#pragma unroll
-        for (int q4 = 0; q4 < 4; q4 += 2) {
-          const float4 r0 = rt[q4], f0 = f[q4], r1 = rt[q4 + 1], f1 = f[q4 + 1];
-          v0 += r0.x * f0.x + r0.y * f0.y + r0.z * f0.z + r0.w * f0.w;
-          v1 += r1.x * f1.x + r1.y * f1.y + r1.z * f1.z + r1.w * f1.w;
+    // per (sub-tile, block slot): the head-weighted sum of the record. Four
+    // threads share a 16-wide dot product, one float4 each, so a warp reads
+    // consecutive 16-byte words of the record rows (no bank conflicts).
+    {
+      const int per_tau = a.nbt * 4;
+      const int nitems = rtiles_u * per_tau;
+      for (int x0 = 0; x0 < nitems; x0 += SEL_THREADS) {
+        const int x = x0 + tid;  // warps stay converged for the shuffles below
+        float v = 0.f;
+        int tau = 0, jl = 0;
+        if (x < nitems) {
+          tau = x / per_tau;
+          const int r = x - tau * per_tau;
+          jl = r >> 2;
+          const int q4 = r & 3;
+          const float4 rv =
+              *reinterpret_cast<const float4*>(recs + tau * rec_floats + G * (1 + jl) + 4 * q4);
+          const float4 fv = *reinterpret_cast<const float4*>(fac + tau * G + 4 * q4);
+          v = rv.x * fv.x + rv.y * fv.y + rv.z * fv.z + rv.w * fv.w;
         }
-        v = v0 + v1;
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        if (x < nitems && (x & 3) == 0) tsum[tau * 16 + jl] = v;
       }
-      tsum[x] = v;
     }
     __syncthreads();
     // block j collects the slots of the sub-tiles whose block ranges include it
@@ -904,7 +811,6 @@ __global__ void __launch_bounds__(SEL_THREADS) dec_select_kernel(const __grid_co
       keys[j] = sel_key(v, j);
     }
   } else {
-    for (int x = tid; x < G * D; x += SEL_THREADS) oacc[x] = 0.f;
     for (int j = tid; j < ncand; j += SEL_THREADS) keys[j] = sel_key(0.f, j);
   }
   if (tid == 0) nsel_s = 0;
@@ -926,9 +832,15 @@ __global__ void __launch_bounds__(SEL_THREADS) dec_select_kernel(const __grid_co
     for (int shift = 56; shift >= 0; shift -= 8) {
       if (tid < 256) hist[tid] = 0u;
       __syncthreads();
-      for (int j = 1 + tid; j < ncand; j += SEL_THREADS) {
-        const unsigned long long k = keys[j];
-        if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+      // one shared-memory atomic per distinct digit of a warp (the leading
+      // digits are mostly equal across all candidates)
+      for (int j0 = 1; j0 < ncand; j0 += SEL_THREADS) {
+        const int j = j0 + tid;
+        const unsigned long long k = j < ncand ? keys[j] : 0ull;
+        const bool in = j < ncand && (k & mask) == prefix;
+        const unsigned bin = in ? (unsigned)((k >> shift) & 255u) : 256u;
+        const unsigned peers = __match_any_sync(0xffffffffu, bin);
+        if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (unsigned)__popc(peers));
       }
       __syncthreads();
       if (warp == 0) {
@@ -1045,35 +957,133 @@ __global__ void __launch_bounds__(SEL_THREADS) dec_select_kernel(const __grid_co
 // dec_combine
 // ---------------------------------------------------------------------------
 
-constexpr int CMB_THREADS = 256;
+constexpr int CMB_HEADS = 4;                   // heads per CTA
+constexpr int CMB_GROUP = CMB_HEADS * 16;      // threads per branch: 16 per head, 8 dims each
+constexpr int CMB_THREADS = 3 * CMB_GROUP;     // one group per branch
+constexpr int CMB_CHUNK = 4;                   // partials whose loads are in flight together
 
+// Per thread: the online merge of partials [first, first + np) for head h,
+// dims e0 .. e0 + 7: M = max m_p, Ls = sum_p 2^(m_p - M) l_p,
+// run = sum_p 2^(m_p - M) o_p. Partials with m = -inf (no valid key) add nothing.
+__device__ __forceinline__ void merge_thread(const float* part, long long first, int np, int h,
+                                             int e0, float& M, float& Ls, float (&run)[8]) {
+  for (int p0 = 0; p0 < np; p0 += CMB_CHUNK) {
+    float m[CMB_CHUNK], l[CMB_CHUNK];
+    float4 o[CMB_CHUNK][2];
+#pragma unroll
+    for (int i = 0; i < CMB_CHUNK; ++i) {
+      if (p0 + i < np) {
+        const float* src = part + (first + p0 + i) * PART;
+        m[i] = __ldcg(src + h);
+        l[i] = __ldcg(src + G + h);
+        const float4* ov = reinterpret_cast<const float4*>(src + 2 * G + h * D + e0);
+        o[i][0] = __ldcg(ov);
+        o[i][1] = __ldcg(ov + 1);
+      } else {
+        m[i] = -INFINITY;
+      }
+    }
+    float Mn = M;
+#pragma unroll
+    for (int i = 0; i < CMB_CHUNK; ++i) Mn = fmaxf(Mn, m[i]);
+    if (Mn == -INFINITY) continue;
+    const float r = exp2f(M - Mn);  // 0 while nothing was merged (M = -inf)
+    Ls *= r;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) run[e] *= r;
+#pragma unroll
+    for (int i = 0; i < CMB_CHUNK; ++i) {
+      if (m[i] == -INFINITY) continue;
+      const float f = exp2f(m[i] - Mn);
+      Ls = fmaf(f, l[i], Ls);
+      run[0] = fmaf(f, o[i][0].x, run[0]);
+      run[1] = fmaf(f, o[i][0].y, run[1]);
+      run[2] = fmaf(f, o[i][0].z, run[2]);
+      run[3] = fmaf(f, o[i][0].w, run[3]);
+      run[4] = fmaf(f, o[i][1].x, run[4]);
+      run[5] = fmaf(f, o[i][1].y, run[5]);
+      run[6] = fmaf(f, o[i][1].z, run[6]);
+      run[7] = fmaf(f, o[i][1].w, run[7]);
+    }
+    M = Mn;
+  }
+}
+
+// CTA (unit, head quarter): three thread groups merge the compressed,
+// selected and window partials of four heads at once, each thread on its own
+// (no block-wide steps inside the merge); the gates come from the raw query;
+// out = sum over branches of g_c o_c.
 __global__ void __launch_bounds__(CMB_THREADS) dec_combine_kernel(const __grid_constant__ DecFastArgs a) {
   const int u = blockIdx.x, b = u / a.Hkv, g = u - b * a.Hkv;
-  const int tid = threadIdx.x;
-  __shared__ float mS[G], lS[G], sR[G], scl[2][G];
-  __shared__ __align__(16) float pm[MP * G], pl[MP * G];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int br = tid / CMB_GROUP, hl = (tid % CMB_GROUP) >> 4, e0 = (tid & 15) * 8;
+  const int h = blockIdx.y * CMB_HEADS + hl;
+  __shared__ float gate_s[CMB_HEADS * 3];
+  __shared__ __align__(16) float contrib[3][CMB_HEADS][D];
   const int L = __ldg(a.seq_lens + b);
   if (!len_ok(L, a)) return;  // output zeroed by dec_select
-  const int4 rg = *reinterpret_cast<const int4*>(a.rng3 + (long)u * 4);  // written by dec_sel_win
-  const int h = tid >> 4, e0 = (tid & 15) * 8;
-  float acc[8];
-  {
-    const float4* oc = reinterpret_cast<const float4*>(a.oacc + (long)u * G * D + h * D + e0);
-    const float4 v0 = oc[0], v1 = oc[1];
-    acc[0] = v0.x; acc[1] = v0.y; acc[2] = v0.z; acc[3] = v0.w;
-    acc[4] = v1.x; acc[5] = v1.y; acc[6] = v1.z; acc[7] = v1.w;
-  }
-  if (tid < 2 * G) scl[tid >> 4][tid & 15] = a.gates[(long)u * 3 * G + (tid & 15) * 3 + 1 + (tid >> 4)];
-  // selected branch (segment 2u), then window branch (segment 2u + 1)
-  merge_online<CMB_THREADS>(a.part3, 2 * ((long long)rg.x + 2 * u), 2 * (rg.y - rg.x + 1), scl[0],
-                            pm, pl, mS, lS, sR, h, e0, acc);
-  merge_online<CMB_THREADS>(a.part3, 2 * ((long long)rg.z + 2 * u + 1), 2 * (rg.w - rg.z + 1),
-                            scl[1], pm, pl, mS, lS, sR, h, e0, acc);
-  __nv_bfloat16* orow =
-      reinterpret_cast<__nv_bfloat16*>(a.out) + ((long)b * a.Hq + g * G + h) * D + e0;
+
+  // gates (EP94 notes §五 gating): sigmoid(q_h . Wg[:, c]), a warp per dot product
+  const __nv_bfloat16* qg =
+      reinterpret_cast<const __nv_bfloat16*>(a.q) + ((long)b * a.Hq + g * G) * D;
+  for (int x = warp; x < CMB_HEADS * 3; x += CMB_THREADS / 32) {
+    const int hh = blockIdx.y * CMB_HEADS + x / 3, c = x % 3;
+    float gv;
+    if (a.gate_mode == 1) {
+      gv = a.fixed_gates[c];
+    } else {
+      float dot = 0.f;
 #pragma unroll
-  for (int e = 0; e < 8; e += 2)
-    *reinterpret_cast<__nv_bfloat162*>(orow + e) = __floats2bfloat162_rn(acc[e], acc[e + 1]);
+      for (int e = lane; e < D; e += 32)
+        dot = fmaf(__bfloat162float(qg[hh * D + e]), __ldg(a.w_gate + e * 3 + c), dot);
+      dot = warp_sum(dot);
+      gv = 1.f / (1.f + expf(-dot));
+    }
+    if (lane == 0) gate_s[x] = gv;
+  }
+
+  const float* part;
+  long long first;
+  int np;
+  if (br == 0) {  // compressed branch: absent while no compressed block is complete
+    part = a.part1;
+    if (n_visible(L, a.l, a.s, a.Nc) > 0) {
+      const int2 rg = *reinterpret_cast<const int2*>(a.rng1 + 2 * u);
+      first = 2 * ((long long)rg.x + u);
+      np = 2 * (rg.y - rg.x + 1);
+    } else {
+      first = 0;
+      np = 0;
+    }
+  } else {  // selected (segment 2u), window (segment 2u + 1)
+    part = a.part3;
+    const int2 rg = *reinterpret_cast<const int2*>(a.rng3 + (long)u * 4 + 2 * (br - 1));
+    first = 2 * ((long long)rg.x + 2 * u + (br - 1));
+    np = 2 * (rg.y - rg.x + 1);
+  }
+  float M = -INFINITY, Ls = 0.f, run[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) run[e] = 0.f;
+  merge_thread(part, first, np, h, e0, M, Ls, run);
+  __syncthreads();  // gates
+  const float sc = Ls > 0.f ? gate_s[hl * 3 + br] / Ls : 0.f;
+  float4* dst = reinterpret_cast<float4*>(&contrib[br][hl][e0]);
+  dst[0] = make_float4(sc * run[0], sc * run[1], sc * run[2], sc * run[3]);
+  dst[1] = make_float4(sc * run[4], sc * run[5], sc * run[6], sc * run[7]);
+  __syncthreads();
+  for (int x = tid; x < CMB_HEADS * D / 4; x += CMB_THREADS) {
+    const int hh = x / (D / 4), e = (x % (D / 4)) * 4;
+    const float4 c0 = *reinterpret_cast<const float4*>(&contrib[0][hh][e]);
+    const float4 c1 = *reinterpret_cast<const float4*>(&contrib[1][hh][e]);
+    const float4 c2 = *reinterpret_cast<const float4*>(&contrib[2][hh][e]);
+    __nv_bfloat16* orow = reinterpret_cast<__nv_bfloat16*>(a.out) +
+                          ((long)b * a.Hq + g * G + blockIdx.y * CMB_HEADS + hh) * D + e;
+    // the same branch order as the oracle: cmp, then slc, then win
+    const float o0 = (c0.x + c1.x) + c2.x, o1 = (c0.y + c1.y) + c2.y;
+    const float o2 = (c0.z + c1.z) + c2.z, o3 = (c0.w + c1.w) + c2.w;
+    *reinterpret_cast<__nv_bfloat162*>(orow) = __floats2bfloat162_rn(o0, o1);
+    *reinterpret_cast<__nv_bfloat162*>(orow + 2) = __floats2bfloat162_rn(o2, o3);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -1094,7 +1104,7 @@ bool first_use(int id) {
 }
 
 struct WsLayout {
-  size_t part1, trec, oacc, gates, sel, part3, rng1, rng3, total;
+  size_t part1, trec, sel, part3, rng1, rng3, total;
 };
 
 WsLayout ws_layout(const DecFastArgs& a) {
@@ -1103,8 +1113,6 @@ WsLayout ws_layout(const DecFastArgs& a) {
   size_t off = 0;
   w.part1 = off; off = align256(off + 2 * (size_t)(a.grid1 + units) * PART * 4);
   w.trec = off; off = align256(off + units * a.tiles_max * G * (1 + a.nbt) * 4);
-  w.oacc = off; off = align256(off + units * G * D * 4);
-  w.gates = off; off = align256(off + units * 3 * G * 4);
   w.sel = off; off = align256(off + units * a.n * 4);
   w.part3 = off; off = align256(off + 2 * (size_t)(a.grid3 + 2 * units) * PART * 4);
   w.rng1 = off; off = align256(off + units * 2 * 4);
@@ -1187,8 +1195,6 @@ cudaError_t launch_decode_fast(const nsa_params& p, const void* q, const void* k
   a.err = err;
   a.part1 = reinterpret_cast<float*>(w + L.part1);
   a.trec = reinterpret_cast<float*>(w + L.trec);
-  a.oacc = reinterpret_cast<float*>(w + L.oacc);
-  a.gates = reinterpret_cast<float*>(w + L.gates);
   a.sel = reinterpret_cast<int*>(w + L.sel);
   a.part3 = reinterpret_cast<float*>(w + L.part3);
   a.rng1 = reinterpret_cast<int*>(w + L.rng1);
@@ -1236,7 +1242,7 @@ cudaError_t launch_decode_fast(const nsa_params& p, const void* q, const void* k
   }
   {
     TraceScope trace("dec_combine", stream);
-    dec_combine_kernel<<<p.B * p.Hkv, CMB_THREADS, 0, stream>>>(a);
+    dec_combine_kernel<<<dim3(p.B * p.Hkv, G / CMB_HEADS), CMB_THREADS, 0, stream>>>(a);
     return cudaGetLastError();
   }
 }

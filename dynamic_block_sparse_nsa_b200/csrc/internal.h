@@ -76,8 +76,6 @@ struct DecFastArgs {
   int8_t klo[kDecMaxNbt], khi[kDecMaxNbt];  // per block of a tile: its key range
   float* part1;   // compressed-branch partials, slot = 2 * (stream + unit) + half
   float* trec;    // per-tile block-score records
-  float* oacc;    // g0 * o_cmp per unit
-  float* gates;   // per unit [16][3]
   int* sel;       // per unit [n]
   float* part3;   // selected / window partials, slot = 2 * (stream + 2 * unit + branch) + half
   int* rng1;      // per unit: first/last stream of its compressed tiles

@@ -281,7 +281,8 @@ def trace_enable(on=True, capacity=4096, only=None):
 
 
 def trace_records():
-    """[(kernel name, device ms)] of the launches traced since trace_enable."""
+    """([(kernel name, device ms)] of the timed launches, count of all launches)
+    since trace_enable."""
     out = []
     n = LIB.nsa_trace_count()
     for i in range(LIB.nsa_trace_timed()):

@@ -115,6 +115,30 @@ def test_decode_bf16_many_units_ragged():
     gc.run_nsa_decode(w, lens, check_b=[0, 3, 7, 11, 15])
 
 
+# Fast decode path (bf16, d = 128, 16 heads per KV head): small caches and the
+# degenerate selections and gates; the trace shows the four fast kernels ran.
+@pytest.mark.parametrize("over,lens", [
+    (dict(B=4, T=64), [64, 40, 20, 1]),                         # a cache of one selection block
+    (dict(B=3, T=33, window=1, top_n=1), [33, 32, 31]),         # one compressed block at most
+    (dict(B=2, T=200, gate_mode=1, fixed_gates=(0.0, 1.0, 0.0)), [200, 129]),
+    (dict(B=2, T=130, top_n=64, window=3000), [130, 65]),       # n above the candidates
+])
+def test_decode_bf16_fast_path_edges(over, lens):
+    from dynamic_block_sparse_nsa_b200 import nsa
+    w = inputs.workload("nsa_decode_bf16_b32_l65536", **over)
+    nsa.trace_enable(True, 64)
+    try:
+        gc.run_nsa_decode(w, lens)
+        recs, _ = nsa.trace_records()
+        names = {nm for nm, _ in recs}
+    finally:
+        nsa.trace_enable(False)
+    want = {"dec_select", "dec_sel_win", "dec_combine"}
+    if max(lens) >= w["cmp_block"]:
+        want.add("dec_cmp_partial")
+    assert want <= names, names
+
+
 def test_decode_bf16_group_of_8_generic_path():
     w = inputs.workload("nsa_decode_bf16_b32_l65536", B=3, T=4000, Hq=32, Hkv=4)
     gc.run_nsa_decode(w, [4000, 1234, 64])
