@@ -3,7 +3,9 @@
 // blocks of 64 tokens.
 //
 // Decode moves the group's one shared KV subset and is bound by HBM bytes
-// (EP94 notes §六; lchairun.cn NSA article, decode paragraph). Four kernels:
+// (EP94 notes §六; lchairun.cn NSA article, decode paragraph). Four kernels,
+// each launched to be scheduled while its predecessor drains (programmatic
+// dependent launch; each waits for the predecessor's writes first):
 //
 //  dec_cmp_partial  stream kernel over the compressed keys (see below); also
 //                   writes, per 32-key sub-tile and head, the running max it
@@ -29,6 +31,7 @@
 // Softmax runs in the log2 domain: z2 = (q . k) * scale * log2(e).
 #include <algorithm>
 #include <climits>
+#include <utility>
 
 #include "device_common.cuh"
 #include "internal.h"
@@ -267,6 +270,50 @@ __device__ __forceinline__ void softmax_step_lazy(float (&s)[NT][4], float (&o)[
   l1 += quad_sum(sum1);
 }
 
+// Score record of a warp's 32-key compressed sub-tile straight from the
+// probabilities in registers, for a compressed block of two strides and a
+// selection block of four (l = 2s, bs = 4s): selection block jl of the
+// sub-tile then takes keys 4jl-1 .. 4jl+3 (key -1 and keys past 31 absent),
+// i.e. the 4-key group jl plus the last key of group jl-1 (blocks 8 and 9 keep
+// key 31 alone and nothing). In the accumulator layout lane quad q holds keys
+// 8nt + 2q, 8nt + 2q + 1 of rows r0 and r0 + 8, so a group is a lane pair and
+// the extra key one shuffle away. Writes rec[h] = m (running max) and
+// rec[16 (1 + jl) + h] = the block's exp-sum, as the shared-memory path does.
+__device__ __forceinline__ void record_regs(float* rec, const float (&p)[4][4], float m0, float m1,
+                                            int lane) {
+  const int q = lane & 3, r0 = lane >> 2, base = lane & ~3;
+  float* blk = rec + G;
+  float prev0 = 0.f, prev1 = 0.f;  // last key of group 2nt - 1 (rows r0, r0 + 8)
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt) {
+    float g0 = p[nt][0] + p[nt][1], g1 = p[nt][2] + p[nt][3];
+    g0 += __shfl_xor_sync(0xffffffffu, g0, 1);  // group 2nt + q / 2
+    g1 += __shfl_xor_sync(0xffffffffu, g1, 1);
+    const float ea0 = __shfl_sync(0xffffffffu, p[nt][1], base | 1);  // key 8nt + 3
+    const float ea1 = __shfl_sync(0xffffffffu, p[nt][3], base | 1);
+    const float eb0 = __shfl_sync(0xffffffffu, p[nt][1], base | 3);  // key 8nt + 7
+    const float eb1 = __shfl_sync(0xffffffffu, p[nt][3], base | 3);
+    if (q == 0) {
+      blk[(2 * nt) * G + r0] = g0 + prev0;
+      blk[(2 * nt) * G + r0 + 8] = g1 + prev1;
+    } else if (q == 2) {
+      blk[(2 * nt + 1) * G + r0] = g0 + ea0;
+      blk[(2 * nt + 1) * G + r0 + 8] = g1 + ea1;
+    }
+    prev0 = eb0;
+    prev1 = eb1;
+  }
+  if (q == 0) {
+    blk[8 * G + r0] = prev0;
+    blk[8 * G + r0 + 8] = prev1;
+    rec[r0] = m0;
+    rec[r0 + 8] = m1;
+  } else if (q == 2) {
+    blk[9 * G + r0] = 0.f;
+    blk[9 * G + r0 + 8] = 0.f;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // global tile order and its even split over the pair streams
 // ---------------------------------------------------------------------------
@@ -450,7 +497,7 @@ __device__ __forceinline__ void store_partial(float* dst, int lane, float m0, fl
 // Every consumer takes part in every phase of its pair's slots, so the mbarrier
 // phase parity is always unambiguous. The producer polls the three rings
 // without blocking on any one of them.
-template <int MODE>
+template <int MODE, bool RF>
 __global__ void __launch_bounds__((NCW + 1) * 32, 1)
     dec_stream_kernel(const __grid_constant__ DecFastArgs a, const __grid_constant__ CUtensorMap tk,
                       const __grid_constant__ CUtensorMap tv) {
@@ -469,6 +516,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
   int* lens_s = abort_flag + 1;  // [LENS_CAP]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  ptx::grid_dep_wait();  // the previous kernel's writes (inputs, this kernel's workspace)
   if (warp == NCW) {
     // the slot ring is idle until the pipeline starts: use it as plan scratch
     make_plans<MODE, NPAIR>(a, plans, lens_s, reinterpret_cast<long long*>(slots),
@@ -613,9 +661,18 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
     const int nvalid = ok ? min(WK, info[slk] - WK * hw) : 0;
     float s[4][4];
     if (nvalid > 0) qk_tile_q<4>(s, qbase, ptx::smem_u32(slots + slk * SLOT_BYTES), WK * hw, lane);
+    constexpr bool early = MODE != MODE_CMP || RF;  // K slot not needed after QK
+    if (early) {
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&empty[slk]);
+    }
     if (nvalid > 0) {
       softmax_step_lazy<4>(s, o, m0, m1, l0, l1, nvalid, a.scale_log2, lane);
-      if (MODE == MODE_CMP) {
+      if (MODE == MODE_CMP && RF) {
+        const int u = wk.b * a.Hkv + wk.g;
+        record_regs(a.trec + ((long)u * a.tiles_max + 2 * wk.tile + hw) * (G * (1 + a.nbt)), s, m0,
+                    m1, lane);
+      } else if (MODE == MODE_CMP) {
         // record of this 32-key sub-tile: running max per head, and per
         // overlapped selection block the exp-sum of its keys. Scratch: this
         // warp's own 32 key rows of the K slot (first TMA box), already read.
@@ -645,8 +702,10 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
         ptx::fence_proxy_async();  // scratch writes before the slot's next TMA fill
       }
     }
-    __syncwarp();
-    if (lane == 0) ptx::mbar_arrive(&empty[slk]);
+    if (!early) {
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&empty[slk]);
+    }
     if (ok && !ptx::mbar_wait(&full[slv], (uint32_t)((hv / PSLOTS) & 1), kWaitNs)) {
       if (lane == 0) {
         atomicOr(a.err, kErrTimeout);
@@ -706,6 +765,7 @@ __global__ void __launch_bounds__(SEL_THREADS) dec_select_kernel(const __grid_co
     ptx::mbar_init(&rec_bar, kRecIssuers);
     ptx::fence_mbar_init();
   }
+  ptx::grid_dep_wait();  // partials, records and stream ranges of dec_cmp_partial
   const int nblk = (a.T + a.bs - 1) / a.bs;
   int npow = 2;  // as in sel_dyn_smem
   while (npow < nblk) npow <<= 1;
@@ -776,25 +836,28 @@ __global__ void __launch_bounds__(SEL_THREADS) dec_select_kernel(const __grid_co
     // threads share a 16-wide dot product, one float4 each, so a warp reads
     // consecutive 16-byte words of the record rows (no bank conflicts).
     {
+      // item x = (tau, r = 4 jl + q4); (tau, r) advances by a fixed step
       const int per_tau = a.nbt * 4;
       const int nitems = rtiles_u * per_tau;
+      const int dtau = SEL_THREADS / per_tau, dr = SEL_THREADS - dtau * per_tau;
+      int tau = tid / per_tau, r = tid - tau * per_tau;
       for (int x0 = 0; x0 < nitems; x0 += SEL_THREADS) {
-        const int x = x0 + tid;  // warps stay converged for the shuffles below
+        const bool in = x0 + tid < nitems;  // warps stay converged for the shuffles below
         float v = 0.f;
-        int tau = 0, jl = 0;
-        if (x < nitems) {
-          tau = x / per_tau;
-          const int r = x - tau * per_tau;
-          jl = r >> 2;
-          const int q4 = r & 3;
-          const float4 rv =
-              *reinterpret_cast<const float4*>(recs + tau * rec_floats + G * (1 + jl) + 4 * q4);
-          const float4 fv = *reinterpret_cast<const float4*>(fac + tau * G + 4 * q4);
+        if (in) {
+          const float4 rv = *reinterpret_cast<const float4*>(recs + tau * rec_floats + G + 4 * r);
+          const float4 fv = *reinterpret_cast<const float4*>(fac + tau * G + 4 * (r & 3));
           v = rv.x * fv.x + rv.y * fv.y + rv.z * fv.z + rv.w * fv.w;
         }
         v += __shfl_xor_sync(0xffffffffu, v, 1);
         v += __shfl_xor_sync(0xffffffffu, v, 2);
-        if (x < nitems && (x & 3) == 0) tsum[tau * 16 + jl] = v;
+        if (in && (r & 3) == 0) tsum[tau * 16 + (r >> 2)] = v;
+        tau += dtau;
+        r += dr;
+        if (r >= per_tau) {
+          r -= per_tau;
+          ++tau;
+        }
       }
     }
     __syncthreads();
@@ -832,15 +895,21 @@ __global__ void __launch_bounds__(SEL_THREADS) dec_select_kernel(const __grid_co
     for (int shift = 56; shift >= 0; shift -= 8) {
       if (tid < 256) hist[tid] = 0u;
       __syncthreads();
-      // one shared-memory atomic per distinct digit of a warp (the leading
-      // digits are mostly equal across all candidates)
+      // a warp whose candidates all share the digit adds them with one atomic
+      // (the leading digits are mostly equal across all candidates)
       for (int j0 = 1; j0 < ncand; j0 += SEL_THREADS) {
         const int j = j0 + tid;
         const unsigned long long k = j < ncand ? keys[j] : 0ull;
         const bool in = j < ncand && (k & mask) == prefix;
-        const unsigned bin = in ? (unsigned)((k >> shift) & 255u) : 256u;
-        const unsigned peers = __match_any_sync(0xffffffffu, bin);
-        if (in && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (unsigned)__popc(peers));
+        const unsigned bin = (unsigned)((k >> shift) & 255u);
+        const unsigned inset = __ballot_sync(0xffffffffu, in);
+        if (inset == 0u) continue;
+        const unsigned b0 = __shfl_sync(0xffffffffu, bin, __ffs(inset) - 1);
+        if (__all_sync(0xffffffffu, !in || bin == b0)) {
+          if (lane == 0) atomicAdd(&hist[b0], (unsigned)__popc(inset));
+        } else if (in) {
+          atomicAdd(&hist[bin], 1u);
+        }
       }
       __syncthreads();
       if (warp == 0) {
@@ -1020,6 +1089,7 @@ __global__ void __launch_bounds__(CMB_THREADS) dec_combine_kernel(const __grid_c
   const int h = blockIdx.y * CMB_HEADS + hl;
   __shared__ float gate_s[CMB_HEADS * 3];
   __shared__ __align__(16) float contrib[3][CMB_HEADS][D];
+  ptx::grid_dep_wait();  // partials and stream ranges of dec_cmp_partial / dec_sel_win
   const int L = __ldg(a.seq_lens + b);
   if (!len_ok(L, a)) return;  // output zeroed by dec_select
 
@@ -1094,7 +1164,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // True the first time kernel `id` is launched on the current device.
 bool first_use(int id) {
-  static bool seen[3][64] = {};
+  static bool seen[4][64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev < 0 || dev >= 64) return true;
@@ -1157,6 +1227,26 @@ DecFastArgs base_args(const nsa_params& p) {
 }
 
 
+// Launch with programmatic stream serialization: the grid is scheduled as the
+// previous kernel in the stream drains instead of after it has fully retired;
+// every decode kernel calls grid_dep_wait before it touches global memory, so
+// the order of memory effects is that of plain launches.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 }  // namespace
 
 bool decode_fast_eligible(const nsa_params& p) {
@@ -1216,11 +1306,14 @@ cudaError_t launch_decode_fast(const nsa_params& p, const void* q, const void* k
   if (a.Nc > 0) {
     TraceScope trace("dec_cmp_partial", stream);
     constexpr size_t smem = StreamCfg<MODE_CMP>::SMEM;
-    if (first_use(0))
-      cudaFuncSetAttribute(dec_stream_kernel<MODE_CMP>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    dec_stream_kernel<MODE_CMP><<<a.grid1 / NPAIR, (NCW + 1) * 32, smem, stream>>>(a, tkc, tvc);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // score records from registers when l = 2s and bs = 4s
+    const bool rf = p.cmp_block == 2 * p.cmp_stride && p.sel_block == 4 * p.cmp_stride;
+    auto kern = rf ? dec_stream_kernel<MODE_CMP, true> : dec_stream_kernel<MODE_CMP, false>;
+    if (first_use(rf ? 0 : 3))
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if ((e = launch_pdl(kern, dim3(a.grid1 / NPAIR), dim3((NCW + 1) * 32), smem, stream, a, tkc,
+                        tvc)) != cudaSuccess)
+      return e;
   }
   {
     const size_t smem = sel_dyn_smem(p.T, p.sel_block, a.tiles_max, a.nbt);
@@ -1228,22 +1321,24 @@ cudaError_t launch_decode_fast(const nsa_params& p, const void* q, const void* k
     if (first_use(2))
       cudaFuncSetAttribute(dec_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)kSelDynSmemMax);
-    dec_select_kernel<<<p.B * p.Hkv, SEL_THREADS, smem, stream>>>(a);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = launch_pdl(dec_select_kernel, dim3(p.B * p.Hkv), dim3(SEL_THREADS), smem, stream,
+                        a)) != cudaSuccess)
+      return e;
   }
   {
     TraceScope trace("dec_sel_win", stream);
     constexpr size_t smem = StreamCfg<MODE_SW>::SMEM;
     if (first_use(1))
-      cudaFuncSetAttribute(dec_stream_kernel<MODE_SW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)smem);
-    dec_stream_kernel<MODE_SW><<<a.grid3 / NPAIR, (NCW + 1) * 32, smem, stream>>>(a, tk, tv);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      cudaFuncSetAttribute(dec_stream_kernel<MODE_SW, false>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if ((e = launch_pdl(dec_stream_kernel<MODE_SW, false>, dim3(a.grid3 / NPAIR),
+                        dim3((NCW + 1) * 32), smem, stream, a, tk, tv)) != cudaSuccess)
+      return e;
   }
   {
     TraceScope trace("dec_combine", stream);
-    dec_combine_kernel<<<dim3(p.B * p.Hkv, G / CMB_HEADS), CMB_THREADS, 0, stream>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(dec_combine_kernel, dim3(p.B * p.Hkv, G / CMB_HEADS), dim3(CMB_THREADS), 0,
+                      stream, a);
   }
 }
 
