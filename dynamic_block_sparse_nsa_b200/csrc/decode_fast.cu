@@ -20,8 +20,8 @@
 //  dec_combine      merges the partials of all three branches, computes the
 //                   gates: out = g0 o_cmp + g1 o_slc + g2 o_win.
 //
-// Stream kernel: persistent, one CTA per SM, 1 TMA producer warp + 4 pairs of
-// consumer warps. The global sequence of 64-key tiles (sequence-major, then KV
+// Stream kernel: persistent, one CTA per SM, 4 pairs of consumer warps, each
+// pair fed by its own TMA producer warp. The global sequence of 64-key tiles (sequence-major, then KV
 // head, then tile) is split evenly over the SMs x 4 pair streams; each pair has
 // a private ring of three 16 KB slots (K or V of a tile, 128B-swizzled TMA
 // boxes, L2 evict-first) so no stream waits on another's slot. The two warps
@@ -431,15 +431,17 @@ __device__ void make_plans(const DecFastArgs& a, StreamPlan* plans, int* lens_s,
 constexpr int NPAIR = 4;              // consumer warp pairs = tile streams per CTA
 constexpr int PSLOTS = 3;             // ring slots per pair: K and V of a tile + one ahead
 constexpr int SLOTS = NPAIR * PSLOTS;
-constexpr int NCW = 2 * NPAIR;        // consumer warps; + 1 producer = 9 warps
+constexpr int NCW = 2 * NPAIR;        // consumer warps
+constexpr int NPW = NPAIR;            // producer warps, one per pair
+constexpr int STREAM_THREADS = (NCW + NPW) * 32;
 constexpr int RPITCH = WK + 2;        // record scratch pitch (floats)
 constexpr int QBYTES = G * D * 2;     // query block of a pair
 
 template <int MODE>
 struct StreamCfg {
   static constexpr size_t SMEM = 1024 + (size_t)SLOTS * SLOT_BYTES + NPAIR * QBYTES +
-                                 2 * SLOTS * 8 + SLOTS * 4 + NPAIR * sizeof(StreamPlan) +
-                                 NPAIR * 6 * 4 + 64 + LENS_CAP * 4;
+                                 2 * SLOTS * 8 + SLOTS * 4 + NPAIR * sizeof(StreamPlan) + 64 +
+                                 LENS_CAP * 4;
 };
 
 struct TileSrc {
@@ -489,16 +491,15 @@ __device__ __forceinline__ void store_partial(float* dst, int lane, float m0, fl
   }
 }
 
-// One CTA per SM: warps 0..5 are three pairs of consumers, warp 6 the TMA
-// producer. Pair p streams its own range of 64-key tiles through its own ring
-// of four 16 KB slots (K and V of the current and the next tile); warp h of
-// the pair handles keys [32h, 32h + 32) of every tile, with its own online
-// softmax state, and writes its partial to slot 2 * (stream + segment) + h.
-// Every consumer takes part in every phase of its pair's slots, so the mbarrier
-// phase parity is always unambiguous. The producer polls the three rings
-// without blocking on any one of them.
+// One CTA per SM: warps 0..7 are four pairs of consumers, warps 8..11 the TMA
+// producers (one per pair). Pair p streams its own range of 64-key tiles
+// through its own ring of three 16 KB slots (K and V of the current tile and
+// the K of the next); warp h of the pair handles keys [32h, 32h + 32) of every
+// tile, with its own online softmax state, and writes its partial to slot
+// 2 * (stream + segment) + h. Every consumer takes part in every phase of its
+// pair's slots, so the mbarrier phase parity is always unambiguous.
 template <int MODE, bool RF>
-__global__ void __launch_bounds__((NCW + 1) * 32, 1)
+__global__ void __launch_bounds__(STREAM_THREADS, 1)
     dec_stream_kernel(const __grid_constant__ DecFastArgs a, const __grid_constant__ CUtensorMap tk,
                       const __grid_constant__ CUtensorMap tv) {
   using C = StreamCfg<MODE>;
@@ -511,8 +512,7 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
   uint64_t* empty = full + SLOTS;
   int* info = reinterpret_cast<int*>(empty + SLOTS);
   StreamPlan* plans = reinterpret_cast<StreamPlan*>(info + SLOTS);
-  Walker<MODE>* pwk = reinterpret_cast<Walker<MODE>*>(plans + NPAIR);
-  int* abort_flag = reinterpret_cast<int*>(pwk + NPAIR);
+  int* abort_flag = reinterpret_cast<int*>(plans + NPAIR);
   int* lens_s = abort_flag + 1;  // [LENS_CAP]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -536,36 +536,39 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
   const int* lens_p = a.B <= LENS_CAP ? lens_s : a.seq_lens;
   float* part = MODE == MODE_CMP ? a.part1 : a.part3;
 
-  if (warp == NCW) {
-    // ---------------- producer ----------------
-    if (lane != 0) return;
+  if (warp >= NCW) {
+    // ---------------- producers: warp NCW + p fills pair p's ring ----------------
+    // Lanes 0 and 1 each issue one 8 KB box of every half-tile: TMA ingest
+    // grows with the number of issuing threads, and one thread for all rings
+    // is slower than the HBM share of an SM.
+    const int p = warp - NCW;
+    if (lane >= 2) return;
     const uint64_t pol = ptx::policy_evict_first();
-    int h[NPAIR], hend[NPAIR];
-    TileSrc ts[NPAIR];
-    long long remaining = 0;
-#pragma unroll
-    for (int p = 0; p < NPAIR; ++p) {
-      h[p] = 0;
-      hend[p] = 2 * plans[p].len;
-      remaining += hend[p];
-      if (hend[p] > 0) {
-        pwk[p].init(a, lens_p, plans[p]);
-        ts[p] = tile_source<MODE>(a, pwk[p]);
+    const int hend = 2 * plans[p].len;
+    if (hend == 0) return;
+    Walker<MODE> wk;
+    wk.init(a, lens_p, plans[p]);
+    TileSrc ts = tile_source<MODE>(a, wk);
+    int h = 0;
+    for (; h < hend; ++h) {
+      const int sl = p * PSLOTS + h % PSLOTS;
+      const int use = h / PSLOTS;
+      // both lanes wait for the slot; they go on only together
+      const bool freed = use == 0 || ptx::mbar_wait(&empty[sl], (uint32_t)((use - 1) & 1), kWaitNs);
+      const bool aborted = lane == 0 && *(volatile int*)abort_flag;
+      const unsigned fb = __ballot_sync(0x3u, freed), ab = __ballot_sync(0x3u, aborted);
+      if (fb != 0x3u) {
+        if (lane == 0) {
+          atomicOr(a.err, kErrTimeout);
+          atomicExch(abort_flag, 1);
+        }
+        break;
       }
-    }
-    uint64_t t_last = ptx::globaltimer();
-    while (remaining > 0) {
-      bool progressed = false;
-#pragma unroll
-      for (int p = 0; p < NPAIR; ++p) {
-        if (h[p] >= hend[p]) continue;
-        const int sl = p * PSLOTS + h[p] % PSLOTS;
-        const int use = h[p] / PSLOTS;
-        if (use > 0 && !ptx::mbar_try_wait(&empty[sl], (uint32_t)((use - 1) & 1))) continue;
-        const bool isv = h[p] & 1;
+      if (ab) break;
+      const bool isv = h & 1;
+      if (lane == 0) {
         if (!isv) {
           // first / last stream of each segment, for the merging kernels
-          const Walker<MODE>& wk = pwk[p];
           const int u = wk.b * a.Hkv + wk.g;
           const int v = blockIdx.x * NPAIR + p;
           if (MODE == MODE_CMP) {
@@ -578,35 +581,23 @@ __global__ void __launch_bounds__((NCW + 1) * 32, 1)
             if (wk.tile == wk.ntiles - 1) a.rng3[4 * u + 3] = v;
           }
         }
-        info[sl] = ts[p].nvalid;
-        unsigned char* dst = slots + sl * SLOT_BYTES;
-        const CUtensorMap* m = isv ? &tv : &tk;
+        info[sl] = ts.nvalid;
         ptx::mbar_arrive_expect_tx(&full[sl], SLOT_BYTES);
-        ptx::tma_load_3d(dst, m, &full[sl], 0, pwk[p].g, ts[p].row, pol);
-        ptx::tma_load_3d(dst + HALF_BYTES, m, &full[sl], 64, pwk[p].g, ts[p].row, pol);
-        if (isv) {
-          pwk[p].advance(a, lens_p);
-          if (h[p] + 1 < hend[p]) ts[p] = tile_source<MODE>(a, pwk[p]);  // next tile, early
-        }
-        ++h[p];
-        --remaining;
-        progressed = true;
       }
-      if (progressed) {
-        t_last = ptx::globaltimer();
-      } else if (ptx::globaltimer() - t_last > kWaitNs || *(volatile int*)abort_flag) {
-        atomicOr(a.err, kErrTimeout);
-        atomicExch(abort_flag, 1);
-        break;
+      __syncwarp(0x3u);
+      ptx::tma_load_3d(slots + sl * SLOT_BYTES + lane * HALF_BYTES, isv ? &tv : &tk, &full[sl],
+                       64 * lane, wk.g, ts.row, pol);
+      if (isv) {
+        wk.advance(a, lens_p);
+        if (h + 1 < hend) ts = tile_source<MODE>(a, wk);  // next tile, early
       }
     }
     // every issued load must have landed before the CTA exits
-#pragma unroll
-    for (int p = 0; p < NPAIR; ++p)
-      for (int k = 0; k < PSLOTS && k < h[p]; ++k) {
-        const int last = h[p] - 1 - ((h[p] - 1 - k) % PSLOTS);  // last half-tile in slot k
-        if (!ptx::mbar_wait(&full[p * PSLOTS + last % PSLOTS],
-                            (uint32_t)((last / PSLOTS) & 1), kWaitNs))
+    if (lane == 0)
+      for (int k = 0; k < PSLOTS && k < h; ++k) {
+        const int last = h - 1 - ((h - 1 - k) % PSLOTS);  // last half-tile in slot k
+        if (!ptx::mbar_wait(&full[p * PSLOTS + last % PSLOTS], (uint32_t)((last / PSLOTS) & 1),
+                            kWaitNs))
           atomicOr(a.err, kErrTimeout);
       }
     return;
@@ -1311,7 +1302,7 @@ cudaError_t launch_decode_fast(const nsa_params& p, const void* q, const void* k
     auto kern = rf ? dec_stream_kernel<MODE_CMP, true> : dec_stream_kernel<MODE_CMP, false>;
     if (first_use(rf ? 0 : 3))
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if ((e = launch_pdl(kern, dim3(a.grid1 / NPAIR), dim3((NCW + 1) * 32), smem, stream, a, tkc,
+    if ((e = launch_pdl(kern, dim3(a.grid1 / NPAIR), dim3(STREAM_THREADS), smem, stream, a, tkc,
                         tvc)) != cudaSuccess)
       return e;
   }
@@ -1332,7 +1323,7 @@ cudaError_t launch_decode_fast(const nsa_params& p, const void* q, const void* k
       cudaFuncSetAttribute(dec_stream_kernel<MODE_SW, false>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if ((e = launch_pdl(dec_stream_kernel<MODE_SW, false>, dim3(a.grid3 / NPAIR),
-                        dim3((NCW + 1) * 32), smem, stream, a, tk, tv)) != cudaSuccess)
+                        dim3(STREAM_THREADS), smem, stream, a, tk, tv)) != cudaSuccess)
       return e;
   }
   {
