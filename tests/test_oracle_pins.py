@@ -418,3 +418,91 @@ def test_topp_grows_with_p_and_tiny_p_keeps_block_zero():
             a = [set(int(j) for j in s[t, g] if j >= 0) for s in sels]
             assert a[0] == {0}
             assert a[0] <= a[1] <= a[2] <= a[3]
+
+
+# --------------------------------------------------------------------------
+# backward oracle (oracle/backward.py)
+# --------------------------------------------------------------------------
+
+def _bwd_case(seed, **kw):
+    p = base_params(B=2, T=70, Hq=4, Hkv=2, d=8, window=12, **kw)
+    rng = np.random.default_rng(seed)
+    B, T, Hq, Hkv, d = p["B"], p["T"], p["Hq"], p["Hkv"], p["d"]
+    q = rng.standard_normal((B, T, Hq, d))
+    k = rng.standard_normal((B, T, Hkv, d))
+    v = rng.standard_normal((B, T, Hkv, d))
+    w = rng.standard_normal(p["cmp_block"]) / math.sqrt(p["cmp_block"])
+    wg = rng.standard_normal((d, 3)) / math.sqrt(d)
+    dout = rng.standard_normal((B, T, Hq, d))
+    fwd = oracle.nsa_prefill(p, q, k, v, w, wg)
+    sel = fwd["sel"].reshape(B, T, Hkv, p["top_n"])
+    return p, q, k, v, w, wg, dout, fwd, sel
+
+
+def test_backward_matches_finite_differences_of_the_forward():
+    """Central differences of the C forward oracle (selection held at the
+    forward's choice) against the analytic gradient of every input."""
+    from oracle import backward
+    p, q, k, v, w, wg, dout, fwd, sel = _bwd_case(5)
+    B, T, Hq, d = q.shape
+    grads = backward.nsa_prefill_backward(p, q, k, v, w, wg, dout, sel)
+    np.testing.assert_allclose(grads["out"], fwd["out"].reshape(B, T, Hq, d), atol=1e-12)
+    forced = sel.reshape(B * T, p["Hkv"], p["top_n"])
+
+    def loss(q, k, v, w, wg):
+        r = oracle.nsa_prefill(p, q, k, v, w, wg, forced_sel=forced)
+        return float(np.sum(dout.reshape(-1, Hq, d) * r["out"]))
+
+    args = {"q": q, "k": k, "v": v, "w": w, "wg": wg}
+    names = {"q": "dq", "k": "dk", "v": "dv", "w": "dw_cmp", "wg": "dwg"}
+    rng = np.random.default_rng(6)
+    eps = 1e-6
+    for name, arr in args.items():
+        for _ in range(10):
+            idx = tuple(int(rng.integers(0, n)) for n in arr.shape)
+            plus = {a: b.copy() for a, b in args.items()}
+            minus = {a: b.copy() for a, b in args.items()}
+            plus[name][idx] += eps
+            minus[name][idx] -= eps
+            fd = (loss(**plus) - loss(**minus)) / (2 * eps)
+            an = grads[names[name]][idx]
+            assert abs(fd - an) <= 1e-6 * (1.0 + abs(an)), (name, idx, fd, an)
+
+
+def test_backward_window_only_equals_autograd_of_softmax_attention():
+    """Gates (0, 0, 1): the output is sliding-window attention, whose gradient
+    torch autograd gives for a plain masked-softmax formulation in fp64."""
+    from oracle import backward
+    p, q, k, v, w, wg, dout, _, sel = _bwd_case(7, gate_mode=1, fixed_gates=(0.0, 0.0, 1.0))
+    B, T, Hq, d = q.shape
+    G = Hq // p["Hkv"]
+    grads = backward.nsa_prefill_backward(p, q, k, v, w, wg, dout, sel)
+    qt, kt, vt = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    kh = kt.repeat_interleave(G, dim=2)  # [B, T, Hq, d]: head h reads KV head h // G
+    vh = vt.repeat_interleave(G, dim=2)
+    s = torch.einsum("bthe,buhe->bhtu", qt, kh) / math.sqrt(d)
+    t_idx = torch.arange(T)
+    allowed = (t_idx[None, :] <= t_idx[:, None]) & (t_idx[None, :] > t_idx[:, None] - p["window"])
+    s = s.masked_fill(~allowed, float("-inf"))
+    o = torch.einsum("bhtu,buhe->bthe", torch.softmax(s, dim=-1), vh)
+    (o * torch.tensor(dout)).sum().backward()
+    np.testing.assert_allclose(grads["dq"], qt.grad.numpy(), atol=1e-12)
+    np.testing.assert_allclose(grads["dk"], kt.grad.numpy(), atol=1e-12)
+    np.testing.assert_allclose(grads["dv"], vt.grad.numpy(), atol=1e-12)
+    assert np.all(grads["dw_cmp"] == 0.0) and np.all(grads["dwg"] == 0.0)
+
+
+def test_backward_value_gradient_sums_to_the_gated_upstream():
+    """Softmax weights sum to one, so the value gradients of a branch sum to
+    its gated upstream gradient: sum_u dv[u] = sum over rows and the group's
+    heads of (g_slc + g_win + g_cmp sum_j w_j [a compressed block is visible]) dout."""
+    from oracle import backward
+    p, q, k, v, w, wg, dout, fwd, sel = _bwd_case(9)
+    B, T, Hq, d = q.shape
+    G = Hq // p["Hkv"]
+    grads = backward.nsa_prefill_backward(p, q, k, v, w, wg, dout, sel)
+    gates = fwd["gates"].reshape(B, T, Hq, 3)
+    vis = (np.arange(T) + 1 >= p["cmp_block"]).astype(np.float64)
+    coef = gates[..., 1] + gates[..., 2] + gates[..., 0] * w.sum() * vis[None, :, None]
+    want = (coef[..., None] * dout).reshape(B, T, p["Hkv"], G, d).sum(axis=(1, 3))
+    np.testing.assert_allclose(grads["dv"].sum(axis=1), want, atol=1e-10)
