@@ -715,6 +715,61 @@ def prefill_summary(ws, rank, local, peaks, K=5, W=3):
                     "a step is nsa_compress_kv + nsa_prefill on device-resident inputs"}
 
 
+def backward_summary(ws, rank, peaks, clk_max_mhz, K=2, W=1):
+    """The prefill backward at 8192 tokens (64 / 4 heads, d = 128, bf16):
+    forward once for the selection, then K timed backward steps. Algorithmic
+    flops: 10 d per (query head, attended key) over the three branches (the
+    logits again, dO . v, and the dq, dk, dv products). The path runs on CUDA
+    cores in fp32, so its roofline is the fp32 FMA rate: SMs x 128 lanes x 2
+    flops x the maximum SM clock."""
+    from dynamic_block_sparse_nsa_b200 import nsa
+    name = "nsa_prefill_bf16_t8192"
+    w = inputs.workload(name)
+    inp = inputs.make_prefill(w, seed=w["seed"] + rank, device="cuda")
+    dt = inputs.DTYPES[w["dtype"]]
+    p = nsa.params(w["B"], w["T"], w["Hq"], w["Hkv"], w["d"], cmp_block=w["cmp_block"],
+                   cmp_stride=w["cmp_stride"], sel_block=w["sel_block"], top_n=w["top_n"],
+                   window=w["window"], dtype=dt)
+    kc, vc = nsa.nsa_compress_kv(p, inp["k"], inp["v"], inp["w_cmp"])
+    _, sel = nsa.nsa_prefill(p, inp["q"], inp["k"], inp["v"], kc, vc, inp["w_gate"])
+    gen = torch.Generator(device="cuda").manual_seed(w["seed"] + 7 + rank)
+    dout = torch.randn(inp["q"].shape, generator=gen, device="cuda").to(dt)
+    ws_buf = nsa.workspace(p, nsa.OP_PREFILL_BACKWARD)
+
+    def step():
+        nsa.nsa_prefill_backward(p, inp["q"], inp["k"], inp["v"], kc, vc, inp["w_cmp"],
+                                 inp["w_gate"], sel, dout, ws=ws_buf)
+
+    for _ in range(W):
+        step()
+    nsa.nsa_check()
+    ms = reduce_max(_run_steps(step, K, False)[0] / K, ws)
+    nsa.nsa_check()
+    # attended keys per (token, KV head): visible compressed blocks, selected
+    # tokens up to t, window
+    T, bs, l, s_ = w["T"], w["sel_block"], w["cmp_block"], w["cmp_stride"]
+    t = np.arange(T)
+    nvis = np.where(t + 1 >= l, (t + 1 - l) // s_ + 1, 0)
+    sl = sel.cpu().numpy().astype(np.int64)  # [B, T, Hkv, n]
+    tt = t[None, :, None, None]
+    ok = (sl >= 0) & (sl <= tt // bs)
+    nslc = np.where(ok, np.minimum(bs, tt + 1 - sl * bs), 0).sum(axis=-1)  # [B, T, Hkv]
+    nwin = np.minimum(w["window"], t + 1)
+    keys = nslc.sum() + w["B"] * w["Hkv"] * (nvis.sum() + nwin.sum())
+    G = w["Hq"] // w["Hkv"]
+    flops = 10.0 * w["d"] * G * float(keys)
+    tflops = flops / (ms / 1000.0) / 1e12
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    peak = sms * 128 * 2 * clk_max_mhz * 1e6 / 1e12
+    return {"workload": name, "value": tflops, "unit": "TFLOP/s", "ms_per_step": ms,
+            "steps": K, "warmup": W, "flops_per_step": flops,
+            "roofline": {"bound": "alu", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                         "frac": tflops / peak,
+                         "peak_from": f"{sms} SMs x 128 fp32 lanes x 2 flops x {clk_max_mhz} MHz"},
+            "note": "nsa_prefill_backward (CUDA-core fp32 path): dq, dk, dv, dw_cmp, dw_gate "
+                    "of sum(dout * out), selection from the forward"}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -793,9 +848,11 @@ def main():
                     "timing": "events around each launch of this kernel over a second "
                               "timed region of the same K steps"}
 
-    pf = None
+    pf = bw = None
     if kind == "decode" and not args.set and not args.no_prefill and args.workload == DEFAULT_WORKLOAD:
         pf = prefill_summary(ws, rank, local, peaks)
+        clk_max = (res.get("clk") or {}).get("sm_max_mhz") or 1965
+        bw = backward_summary(ws, rank, peaks, clk_max)
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -842,6 +899,8 @@ def main():
             line["kernel_tflops"] = per
         if pf is not None:
             line["prefill_64k"] = pf
+        if bw is not None:
+            line["prefill_backward_8k"] = bw
         print(json.dumps(line), flush=True)
     if ws > 1:
         import torch.distributed as dist

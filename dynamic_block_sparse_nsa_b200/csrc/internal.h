@@ -41,6 +41,37 @@ struct NsaRowArgs {
   float top_p;              // 0: top-n; else adaptive selection
 };
 
+struct NsaBwdArgs {
+  const void* q;
+  const void* k;
+  const void* v;
+  const void* kc;
+  const void* vc;
+  const float* w_cmp;
+  const float* w_gate;
+  const int32_t* sel;       // [B, T, Hkv, n] the forward's selected blocks
+  const void* dout;
+  float* dq;                // [B, T, Hq, d]
+  float* dk;                // [B, T, Hkv, d]
+  float* dv;
+  float* dw_cmp;            // [l]
+  float* dw_gate;           // [d, 3]
+  float* dkc;               // workspace [B, Nc, Hkv, d]
+  float* dvc;
+  float* dz;                // workspace [B, T, Hq, 3]
+  int B, T, Hq, Hkv, d;
+  int l, s, bs, n, w, Nc;
+  float scale;
+  int gate_mode;
+  float fixed_gates[3];
+  nsa_dtype dtype;
+};
+
+// Prefill backward (generic CUDA-core path).
+size_t nsa_bwd_smem(int G, int d);
+size_t nsa_bwd_ws_bytes(const nsa_params& p);
+cudaError_t launch_nsa_backward(NsaBwdArgs a, void* ws, cudaStream_t stream);
+
 struct MobaArgs {
   const void* q;
   const void* k;

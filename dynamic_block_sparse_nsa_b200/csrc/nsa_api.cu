@@ -178,6 +178,12 @@ nsa_status nsa_workspace_size(const nsa_params* p, int op, size_t* bytes) {
       *bytes = decode_fast_ws_bytes(*p);
       return NSA_OK;
     }
+    case NSA_OP_PREFILL_BACKWARD: {
+      nsa_status s = check_nsa(p);
+      if (s != NSA_OK) return s;
+      *bytes = nsa_bwd_ws_bytes(*p);
+      return NSA_OK;
+    }
     case NSA_OP_MOBA_PREFILL: {
       nsa_status s = check_common(p);
       if (s != NSA_OK) return s;
@@ -231,6 +237,43 @@ nsa_status nsa_prefill(const nsa_params* p, const void* q, const void* k, const 
                 p->Hq / p->Hkv, p->d, smem);
   cudaError_t e = launch_nsa_rows_simt(a, (cudaStream_t)stream);
   return e == cudaSuccess ? NSA_OK : cuda_fail(e, "prefill launch");
+}
+
+nsa_status nsa_prefill_backward(const nsa_params* p, const void* q, const void* k, const void* v,
+                                const void* k_cmp, const void* v_cmp, const float* w_cmp,
+                                const float* w_gate, const int32_t* sel_idx, const void* dout,
+                                float* dq, float* dk, float* dv, float* dw_cmp, float* dw_gate,
+                                void* workspace, size_t ws_bytes, void* stream) {
+  g_detail.clear();
+  nsa_status s = check_nsa(p);
+  if (s != NSA_OK) return s;
+  const int Nc = nsa_num_cmp_blocks(p->T, p->cmp_block, p->cmp_stride);
+  if (!q || !k || !v || !w_cmp || !sel_idx || !dout || !dq || !dk || !dv || !dw_cmp ||
+      (Nc > 0 && (!k_cmp || !v_cmp)))
+    return fail(NSA_ERR_INVALID_ARGUMENT,
+                "q, k, v, k_cmp, v_cmp, w_cmp, sel_idx, dout, dq, dk, dv, dw_cmp must be non-NULL");
+  if (p->gate_mode == 0 && (!w_gate || !dw_gate))
+    return fail(NSA_ERR_INVALID_ARGUMENT, "w_gate and dw_gate must be non-NULL when gate_mode == 0");
+  if (p->top_n > 64) return fail(NSA_ERR_UNSUPPORTED, "the backward supports top_n <= 64");
+  const size_t smem = nsa_bwd_smem(p->Hq / p->Hkv, p->d);
+  if (smem > (size_t)max_smem_optin())
+    return fail(NSA_ERR_UNSUPPORTED, "group size %d x head dim %d needs %zu bytes of shared memory",
+                p->Hq / p->Hkv, p->d, smem);
+  s = check_workspace(workspace, ws_bytes, nsa_bwd_ws_bytes(*p));
+  if (s != NSA_OK) return s;
+  NsaBwdArgs a{};
+  a.q = q; a.k = k; a.v = v; a.kc = k_cmp; a.vc = v_cmp;
+  a.w_cmp = w_cmp; a.w_gate = w_gate; a.sel = sel_idx; a.dout = dout;
+  a.dq = dq; a.dk = dk; a.dv = dv; a.dw_cmp = dw_cmp; a.dw_gate = dw_gate;
+  a.B = p->B; a.T = p->T; a.Hq = p->Hq; a.Hkv = p->Hkv; a.d = p->d;
+  a.l = p->cmp_block; a.s = p->cmp_stride; a.bs = p->sel_block; a.n = p->top_n; a.w = p->window;
+  a.Nc = Nc;
+  a.scale = eff_scale(p);
+  a.gate_mode = p->gate_mode;
+  for (int i = 0; i < 3; ++i) a.fixed_gates[i] = p->fixed_gates[i];
+  a.dtype = p->dtype;
+  cudaError_t e = launch_nsa_backward(a, workspace, (cudaStream_t)stream);
+  return e == cudaSuccess ? NSA_OK : cuda_fail(e, "prefill backward launch");
 }
 
 nsa_status nsa_decode(const nsa_params* p, const void* q, const void* k_cache, const void* v_cache,

@@ -21,13 +21,14 @@ STATUS = {
     0: "NSA_OK", 1: "NSA_ERR_INVALID_ARGUMENT", 2: "NSA_ERR_UNSUPPORTED",
     3: "NSA_ERR_WORKSPACE_TOO_SMALL", 4: "NSA_ERR_CUDA", 5: "NSA_ERR_DEVICE_TIMEOUT",
 }
-OP_COMPRESS, OP_PREFILL, OP_DECODE, OP_MOBA_PREFILL = 0, 1, 2, 3
+OP_COMPRESS, OP_PREFILL, OP_DECODE, OP_MOBA_PREFILL, OP_PREFILL_BACKWARD = 0, 1, 2, 3, 4
 DTYPE_F32, DTYPE_BF16 = 0, 1
 _TORCH_DTYPE = {DTYPE_F32: torch.float32, DTYPE_BF16: torch.bfloat16}
 
 # Every symbol include/nsa.h declares.
 EXPORTS = (
-    "nsa_workspace_size", "nsa_num_cmp_blocks", "nsa_compress_kv", "nsa_prefill", "nsa_decode",
+    "nsa_workspace_size", "nsa_num_cmp_blocks", "nsa_compress_kv", "nsa_prefill",
+    "nsa_prefill_backward", "nsa_decode",
     "moba_prefill", "nsa_decode_noalloc", "nsa_append_kv", "nsa_check", "nsa_debug_bounded_wait", "nsa_status_string",
     "nsa_last_error_detail", "nsa_trace_enable", "nsa_trace_set_filter", "nsa_trace_count",
     "nsa_trace_timed", "nsa_trace_get",
@@ -67,6 +68,7 @@ def _load():
         "nsa_compress_kv": [P, vp, vp, vp, vp, vp, vp],
         "nsa_prefill": [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
         "nsa_decode": [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
+        "nsa_prefill_backward": [P] + [vp] * 15 + [sz, vp],
         "moba_prefill": [P, vp, vp, vp, vp, vp, vp, sz, vp],
         "nsa_decode_noalloc": [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
         "nsa_append_kv": [P, vp, vp, vp, vp, vp, vp, vp, vp, vp],
@@ -186,6 +188,32 @@ def nsa_prefill(p, q, k, v, k_cmp, v_cmp, w_gate=None, out=None, sel_idx=None, w
                            _ptr(w_gate), _ptr(out), _ptr(sel_idx), _ptr(ws), nbytes,
                            _stream(stream)))
     return out, sel_idx
+
+
+def nsa_prefill_backward(p, q, k, v, k_cmp, v_cmp, w_cmp, w_gate, sel_idx, dout, ws=None,
+                         stream=None):
+    """Gradients of sum(dout * out) of nsa_prefill: (dq, dk, dv, dw_cmp, dw_gate), fp32."""
+    dt = p.torch_dtype
+    for t, nm in ((q, "q"), (k, "k"), (v, "v"), (k_cmp, "k_cmp"), (v_cmp, "v_cmp"),
+                  (dout, "dout")):
+        _dev(t, nm, dt)
+    _dev(w_cmp, "w_cmp", torch.float32)
+    _dev(w_gate, "w_gate", torch.float32)
+    _dev(sel_idx, "sel_idx", torch.int32)
+    f32 = dict(dtype=torch.float32, device=q.device)
+    dq = torch.empty(p.B, p.T, p.Hq, p.d, **f32)
+    dk = torch.empty(p.B, p.T, p.Hkv, p.d, **f32)
+    dv = torch.empty(p.B, p.T, p.Hkv, p.d, **f32)
+    dw_cmp = torch.empty(p.cmp_block, **f32)
+    dw_gate = torch.empty(p.d, 3, **f32)
+    if ws is None:
+        ws = workspace(p, OP_PREFILL_BACKWARD, q.device)
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _raise(LIB.nsa_prefill_backward(
+        ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(k_cmp), _ptr(v_cmp), _ptr(w_cmp),
+        _ptr(w_gate), _ptr(sel_idx), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dw_cmp),
+        _ptr(dw_gate), _ptr(ws), nbytes, _stream(stream)))
+    return dq, dk, dv, dw_cmp, dw_gate
 
 
 def nsa_decode(p, q, k_cache, v_cache, seq_lens, k_cmp, v_cmp, w_gate=None, out=None,

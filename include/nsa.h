@@ -62,7 +62,8 @@ typedef enum {
   NSA_OP_COMPRESS = 0,
   NSA_OP_PREFILL = 1,
   NSA_OP_DECODE = 2,
-  NSA_OP_MOBA_PREFILL = 3
+  NSA_OP_MOBA_PREFILL = 3,
+  NSA_OP_PREFILL_BACKWARD = 4
 } nsa_op;
 
 /* Problem description shared by all calls.
@@ -127,6 +128,34 @@ NSA_API nsa_status nsa_compress_kv(const nsa_params* p, const void* k, const voi
 NSA_API nsa_status nsa_prefill(const nsa_params* p, const void* q, const void* k, const void* v,
                        const void* k_cmp, const void* v_cmp, const float* w_gate, void* out,
                        int32_t* sel_idx, void* workspace, size_t ws_bytes, void* stream);
+
+/* NSA prefill backward: gradients of L = sum(dout * out) of nsa_prefill
+ * (EP94 notes §五: the compressed branch carries the gradient that trains the
+ * selection; lchairun.cn NSA article, the paragraph on trainability). The
+ * selected blocks are constants of the backward (the top-n choice is
+ * discrete); gradients flow through the gates, the three attentions and the
+ * compression, whose storage rounding is taken as the identity.
+ *   q, k, v, k_cmp, v_cmp, w_gate  as passed to nsa_prefill; k_cmp, v_cmp are
+ *              nsa_compress_kv(k, v, w_cmp).
+ *   w_cmp      [cmp_block] fp32, the compression weights.
+ *   sel_idx    [B, T, Hkv, top_n] int32: the forward's selected blocks (as
+ *              nsa_prefill writes them); entries < 0, repeated, or past the
+ *              row's own block are ignored.
+ *   dout       [B, T, Hq, d] dtype.
+ *   dq         [B, T, Hq, d] fp32 output.
+ *   dk, dv     [B, T, Hkv, d] fp32 outputs (overwritten).
+ *   dw_cmp     [cmp_block] fp32 output.
+ *   dw_gate    [d, 3] fp32 output; zeros when gate_mode == 1 (may be NULL then).
+ *   workspace  device scratch of nsa_workspace_size(NSA_OP_PREFILL_BACKWARD)
+ *              bytes (caller-owned; contents need not be initialised).
+ * Runs on CUDA cores in fp32; dk, dv and the compressed-branch gradients are
+ * summed with atomics, so their last bits can vary between runs. top_n > 64
+ * returns NSA_ERR_UNSUPPORTED. */
+NSA_API nsa_status nsa_prefill_backward(const nsa_params* p, const void* q, const void* k,
+                                const void* v, const void* k_cmp, const void* v_cmp,
+                                const float* w_cmp, const float* w_gate, const int32_t* sel_idx,
+                                const void* dout, float* dq, float* dk, float* dv, float* dw_cmp,
+                                float* dw_gate, void* workspace, size_t ws_bytes, void* stream);
 
 /* NSA single-token decode over a KV cache (EP94 notes §六; lchairun.cn NSA
  * article: decode moves the group's one shared KV subset).

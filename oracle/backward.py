@@ -57,8 +57,12 @@ def _attention_backward(q, keys, vals, scale, d_o):
     return o, dq, dk, dv
 
 
-def nsa_prefill_backward(p, q, k, v, w_cmp, wg, dout, sel):
+def nsa_prefill_backward(p, q, k, v, w_cmp, wg, dout, sel, kc=None, vc=None):
     """Gradients of L = sum(dout * out) of the causal NSA prefill.
+
+    ``kc``, ``vc``: the compressed keys and values the forward attended to,
+    when it stored them rounded (bf16); the rounding is taken as the identity
+    in the gradient of the compression. Default: the exact compression.
 
     Returns a dict with ``dq`` ``[B, T, Hq, d]``, ``dk``, ``dv`` ``[B, T, Hkv,
     d]`` (through the selected and window branches and, via the compression,
@@ -80,12 +84,16 @@ def nsa_prefill_backward(p, q, k, v, w_cmp, wg, dout, sel):
     Nc = (T - l) // s + 1 if T >= l else 0
 
     # compression (its output is what the compressed branch attends to)
-    kc = np.zeros((B, Nc, Hkv, d))
-    vc = np.zeros((B, Nc, Hkv, d))
-    for i in range(Nc):
-        for j in range(l):
-            kc[:, i] += w_cmp[j] * k[:, i * s + j]
-            vc[:, i] += w_cmp[j] * v[:, i * s + j]
+    if kc is None:
+        kc = np.zeros((B, Nc, Hkv, d))
+        vc = np.zeros((B, Nc, Hkv, d))
+        for i in range(Nc):
+            for j in range(l):
+                kc[:, i] += w_cmp[j] * k[:, i * s + j]
+                vc[:, i] += w_cmp[j] * v[:, i * s + j]
+    else:
+        kc = np.asarray(kc, dtype=np.float64)
+        vc = np.asarray(vc, dtype=np.float64)
 
     dq = np.zeros_like(q)
     dk = np.zeros_like(k)

@@ -103,3 +103,22 @@ def test_moba_rejects_small_workspace_before_launching():
     st = nsa.LIB.moba_prefill(ctypes.byref(p), fake, fake, fake, fake, None, ctypes.c_void_p(264),
                               need, None)
     assert st == 1  # misaligned workspace
+
+
+def test_backward_workspace_and_argument_checks():
+    """Backward scratch: dK~ and dV~ fp32 [B, Nc, Hkv, d] and the gate
+    gradients dz fp32 [B, T, Hq, 3], each 256-byte aligned; the calls reject
+    NULL pointers and top_n > 64 before touching the device."""
+    def a256(x):
+        return (x + 255) // 256 * 256
+    B, T, Hq, Hkv, d = 2, 8192, 64, 4, 128
+    p = nsa.params(B, T, Hq, Hkv, d)
+    Nc = nsa.LIB.nsa_num_cmp_blocks(T, 32, 16)
+    assert nsa.workspace_size(p, nsa.OP_PREFILL_BACKWARD) == (
+        2 * a256(B * Nc * Hkv * d * 4) + a256(B * T * Hq * 3 * 4))
+    L = nsa.LIB
+    assert L.nsa_prefill_backward(ctypes.byref(p), *([None] * 15), 0, None) == 1
+    fake = ctypes.c_void_p(256)
+    big = nsa.params(1, 1024, 4, 1, 64, top_n=65)
+    assert L.nsa_prefill_backward(ctypes.byref(big), *([fake] * 15), 1 << 30, None) == 2
+    assert b"top_n" in L.nsa_last_error_detail()
