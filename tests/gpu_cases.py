@@ -163,3 +163,38 @@ def sample_rows(T, n, seed=0, B=1):
     extra = list(rng.integers(0, T, max(0, n - len(fixed))))
     ts = sorted(set(fixed + [int(x) for x in extra]))
     return [(b, t) for b in range(B) for t in ts]
+
+
+def run_backward(w, seed, tol):
+    """GPU prefill backward against the fp64 backward oracle (selection and
+    compressed cache from the oracle's forward); asserts every gradient within
+    tol of its largest magnitude and returns the relative errors."""
+    from oracle import backward as obwd
+    inp = inputs.make_prefill(w, seed)
+    p = nsa_params_for(w)
+    op = oracle_params_for(w)
+    B, T, Hq, d = inp["q"].shape
+    dev = {k_: v_.cuda() for k_, v_ in inp.items()}
+    kc, vc = nsa.nsa_compress_kv(p, dev["k"], dev["v"], dev["w_cmp"])
+    q64, k64, v64 = f64(inp["q"]), f64(inp["k"]), f64(inp["v"])
+    wc64, wg64 = f64(inp["w_cmp"]), f64(inp["w_gate"])
+    kc64, vc64 = oracle.compress(op, k64, v64, wc64)
+    np.testing.assert_array_equal(f64(kc), kc64)
+    fwd = oracle.nsa_prefill(op, q64, k64, v64, wc64, wg64)
+    sel = fwd["sel"].reshape(B, T, p.Hkv, p.top_n)
+    gen = torch.Generator().manual_seed(seed + 1)
+    dout = torch.randn(B, T, Hq, d, generator=gen).to(inp["q"].dtype)
+    got = nsa.nsa_prefill_backward(p, dev["q"], dev["k"], dev["v"], kc, vc, dev["w_cmp"],
+                                   dev["w_gate"], torch.from_numpy(sel).cuda(), dout.cuda())
+    nsa.nsa_check()
+    ref = obwd.nsa_prefill_backward(op, q64, k64, v64, wc64, wg64, f64(dout), sel,
+                                    kc=kc64, vc=vc64)
+    stats = {}
+    for name, g in zip(("dq", "dk", "dv", "dw_cmp", "dwg"), got):
+        r = ref[name]
+        err = float(np.abs(f64(g) - r).max()) if r.size else 0.0
+        scale = max(float(np.abs(r).max()) if r.size else 0.0, 1e-6)
+        stats[name] = (err, scale)
+    for name, (err, scale) in stats.items():
+        assert err <= tol * scale, (name, err, scale)
+    return {k_: e / s for k_, (e, s) in stats.items()}
