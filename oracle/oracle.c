@@ -40,9 +40,11 @@ typedef struct {
   double fixed_gates[3];       /* (cmp, slc, win) when gate_mode == 1            */
   int store;                   /* rounding of stored compressed K/V:
                                   0 none (keep fp64), 1 fp32, 2 bf16             */
-  int score_mode;              /* compressed-to-selection block mapping:
-                                  0 unweighted sum over overlapping compressed
-                                  blocks; 1 weighted by overlap / l              */
+  int score_mode;              /* block scores for the selection:
+                                  0 compressed-branch mass, unweighted sum over
+                                  overlapping compressed blocks; 1 the same
+                                  weighted by overlap / l; 2 the Quest-style
+                                  block bound (see step 3')                      */
   double top_p;                /* 0: top-n; in (0, 1]: adaptive selection that
                                   stops once the selected blocks hold top_p of
                                   the total score (at most n blocks)            */
@@ -243,6 +245,41 @@ void oracle_nsa_rows(const oracle_nsa_cfg* c, int nrows, const int* rows_b, cons
             blk[j] += wgt * p[i];
           }
         }
+      }
+      /* Step 3' (score_mode 2) [EP94 §八: the Quest-style heuristic block
+       * score of the selection ablation; the pages print no formula, so the
+       * one of the Quest paper they cite is used]: per selection block j the
+       * element-wise minimum and maximum of its keys up to t, and the bound
+       * sum_e max(q_e kmin_e, q_e kmax_e) >= max_u q . k_u over the block,
+       * summed over the query heads of the GQA group. It replaces the
+       * compressed-branch scores; the compressed branch itself is unchanged. */
+      if (c->score_mode == 2) {
+        double* kmin = (double*)malloc(sizeof(double) * d);
+        double* kmax = (double*)malloc(sizeof(double) * d);
+        for (int j = 0; j < ncand; ++j) {
+          const int u1 = (j + 1) * bs - 1 < t ? (j + 1) * bs - 1 : t;
+          for (int e = 0; e < d; ++e) {
+            kmin[e] = INFINITY;
+            kmax[e] = -INFINITY;
+          }
+          for (int u = j * bs; u <= u1; ++u)
+            for (int e = 0; e < d; ++e) {
+              const double x = kb[(long)u * tok + e];
+              if (x < kmin[e]) kmin[e] = x;
+              if (x > kmax[e]) kmax[e] = x;
+            }
+          double sc = 0.0;
+          for (int hh = 0; hh < G; ++hh) {
+            const double* qh = q_rows + ((long)r * Hq + g * G + hh) * d;
+            for (int e = 0; e < d; ++e) {
+              const double lo = qh[e] * kmin[e], hi = qh[e] * kmax[e];
+              sc += lo > hi ? lo : hi;
+            }
+          }
+          blk[j] = sc;
+        }
+        free(kmin);
+        free(kmax);
       }
       if (scores) {
         double* srow = scores + ((long)r * Hkv + g) * nblk_max;

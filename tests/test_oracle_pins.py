@@ -506,3 +506,56 @@ def test_backward_value_gradient_sums_to_the_gated_upstream():
     coef = gates[..., 1] + gates[..., 2] + gates[..., 0] * w.sum() * vis[None, :, None]
     want = (coef[..., None] * dout).reshape(B, T, p["Hkv"], G, d).sum(axis=(1, 3))
     np.testing.assert_allclose(grads["dv"].sum(axis=1), want, atol=1e-10)
+
+
+# --------------------------------------------------------------------------
+# Quest-style block bound (score_mode 2)
+# --------------------------------------------------------------------------
+
+def test_quest_bound_is_the_box_maximum_and_bounds_every_key():
+    """The largest q . x over the axis-aligned box of a block's keys is attained
+    at a corner; brute force over all 2^d corners (d = 4) must give the score,
+    summed over the group's heads, and it bounds q . k of every key."""
+    p = base_params(T=90, Hq=4, Hkv=2, d=4, sel_block=8, score_mode=2)
+    q, k, v, w, wg = rand_inputs(p, rng=np.random.default_rng(41))
+    res = oracle.nsa_prefill(p, q, k, v, w, wg)
+    G, bs, d = 2, p["sel_block"], p["d"]
+    corners = np.array(list(itertools.product([0, 1], repeat=d)))
+    for t in (0, 3, 7, 8, 40, 89):
+        for g in range(p["Hkv"]):
+            for j in range(t // bs + 1):
+                keys = k[0, j * bs:min(j * bs + bs, t + 1), g]
+                box = np.where(corners == 0, keys.min(axis=0), keys.max(axis=0))
+                want = best = 0.0
+                for hh in range(G):
+                    qh = q[0, t, g * G + hh]
+                    want += (box @ qh).max()
+                    best += (keys @ qh).max()
+                got = res["scores"][t, g, j]
+                assert abs(got - want) <= 1e-12 * (1 + abs(want)), (t, g, j)
+                assert got >= best - 1e-12
+
+
+def test_quest_with_one_token_blocks_selects_by_summed_logits():
+    """Blocks of one token: the bound is q . k itself, so the score of token j is
+    the group's summed logits and the selection is token 0 plus the n-1 best."""
+    p = base_params(T=60, Hq=4, Hkv=2, d=16, sel_block=1, top_n=5, score_mode=2)
+    q, k, v, w, wg = rand_inputs(p, rng=np.random.default_rng(42))
+    res = oracle.nsa_prefill(p, q, k, v, w, wg)
+    G = 2
+    for t in (4, 5, 30, 59):
+        for g in range(p["Hkv"]):
+            logit = sum(k[0, :t + 1, g] @ q[0, t, g * G + hh] for hh in range(G))
+            np.testing.assert_allclose(res["scores"][t, g, :t + 1], logit, rtol=0, atol=1e-12)
+            order = [j for j in np.argsort(-logit[1:], kind="stable") + 1][:p["top_n"] - 1]
+            assert sorted(int(x) for x in res["sel"][t, g]) == sorted([0] + order)
+
+
+def test_quest_ignores_future_tokens_of_the_current_block():
+    p = base_params(T=70, sel_block=16, score_mode=2)
+    q, k, v, w, wg = rand_inputs(p, rng=np.random.default_rng(43))
+    base = oracle.nsa_prefill(p, q, k, v, w, wg, rows=[(0, 37)])
+    k2 = k.copy()
+    k2[0, 38:48] += 5.0  # later tokens of block 2, which holds t = 37
+    moved = oracle.nsa_prefill(p, q, k2, v, w, wg, rows=[(0, 37)])
+    np.testing.assert_array_equal(base["scores"], moved["scores"])
