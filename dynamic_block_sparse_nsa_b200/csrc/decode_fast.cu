@@ -1241,6 +1241,7 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 }  // namespace
 
 bool decode_fast_eligible(const nsa_params& p) {
+  if (p.sel_mode != 0) return false;  // Quest-bound selection: CUDA-core path
   if (!(p.dtype == NSA_DTYPE_BF16 && p.d == D && p.Hq == G * p.Hkv && p.sel_block == TK &&
         p.top_n <= MAXSEL && p.T >= 1 && (p.T + p.sel_block - 1) / p.sel_block <= MAXCAND))
     return false;

@@ -39,6 +39,7 @@ struct NsaRowArgs {
   int decode;               // 0 prefill (row per token), 1 decode (row per sequence)
   nsa_dtype dtype;
   float top_p;              // 0: top-n; else adaptive selection
+  int sel_mode;             // 0: compressed-branch scores; 1: Quest block bound
 };
 
 struct NsaBwdArgs {

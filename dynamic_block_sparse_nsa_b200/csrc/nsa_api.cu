@@ -96,6 +96,10 @@ nsa_status check_nsa(const nsa_params* p) {
     return fail(NSA_ERR_INVALID_ARGUMENT, "gate_mode must be 0 or 1");
   if (!(p->top_p >= 0.f && p->top_p <= 1.f))
     return fail(NSA_ERR_INVALID_ARGUMENT, "top_p must be in [0, 1] (0: top-n selection)");
+  if (p->sel_mode != 0 && p->sel_mode != 1)
+    return fail(NSA_ERR_INVALID_ARGUMENT, "sel_mode must be 0 (compressed scores) or 1 (Quest bound)");
+  if (p->sel_mode == 1 && p->top_p != 0.f)
+    return fail(NSA_ERR_INVALID_ARGUMENT, "sel_mode 1 (Quest bound) needs top_p == 0");
   if (p->Hkv > 65535) return fail(NSA_ERR_UNSUPPORTED, "Hkv must be <= 65535");
   return NSA_OK;
 }
@@ -117,6 +121,7 @@ NsaRowArgs row_args(const nsa_params* p) {
   a.gate_mode = p->gate_mode;
   for (int i = 0; i < 3; ++i) a.fixed_gates[i] = p->fixed_gates[i];
   a.top_p = p->top_p;
+  a.sel_mode = p->sel_mode;
   a.dtype = p->dtype;
   return a;
 }

@@ -1080,6 +1080,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 bool prefill_tc_eligible(const nsa_params& p) {
   if (p.dtype != NSA_DTYPE_BF16 || p.d != D || p.Hkv < 1 || p.Hq != G * p.Hkv) return false;
+  if (p.sel_mode != 0) return false;  // Quest-bound selection: CUDA-core path
   if (p.cmp_block != CL || p.cmp_stride != CS || p.sel_block != SB) return false;
   if (p.top_n < 1 || p.top_n > kMaxSel || p.window < 1) return false;
   if ((long long)p.B * p.T >= (1ll << 30)) return false;

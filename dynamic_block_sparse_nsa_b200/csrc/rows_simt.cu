@@ -10,6 +10,7 @@
 //      each selection block j = sum over the group's heads of the p mass on the
 //      compressed blocks that overlap j;
 //   3. top-n: block 0 kept, the n-1 best others (ties to the lower index);
+//      with sel_mode 1 the scores are the Quest-style block bound instead;
 //   4. selected branch: softmax over the tokens of the chosen blocks up to t;
 //   5. window branch: softmax over [max(0, t-w+1), t];
 //   6. gates g = sigmoid(q . Wg) (or fixed), out = g0 o_cmp + g1 o_slc + g2 o_win.
@@ -441,6 +442,33 @@ __global__ void __launch_bounds__(kThreads) nsa_rows_kernel(NsaRowArgs a) {
     add_branch(c, 0, false);
   }
   __syncthreads();
+
+  // ---- Quest-style block bound (sel_mode 1; EP94 notes §八, the selection
+  // ablation): per block j the element-wise min / max of its keys up to t and
+  // the sum over the group's heads of sum_e max(q_e kmin_e, q_e kmax_e); it
+  // replaces the compressed-branch scores as the selection's ranking. ----
+  if (a.sel_mode == 1) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int j = warp; j < ncand; j += kWarps) {
+      const int u1 = min(j * a.bs + a.bs - 1, t);
+      float acc = 0.f;
+      for (int e = lane; e < d; e += 32) {
+        float mn = INFINITY, mx = -INFINITY;
+        for (int u = j * a.bs; u <= u1; ++u) {
+          const float x = to_f32(kb[(long)u * tok + e]);
+          mn = fminf(mn, x);
+          mx = fmaxf(mx, x);
+        }
+        for (int h = 0; h < G; ++h) {
+          const float qe = c.qs[h * d + e];
+          acc += fmaxf(qe * mn, qe * mx);
+        }
+      }
+      acc = warp_sum(acc);
+      if (lane == 0) c.scores[j] = acc;
+    }
+    __syncthreads();
+  }
 
   // ---- top-n selection (block 0 forced) ----
   int ns;

@@ -48,6 +48,7 @@ class NsaParams(ctypes.Structure):
         ("sel_block", ctypes.c_int), ("top_n", ctypes.c_int), ("window", ctypes.c_int),
         ("softmax_scale", ctypes.c_float), ("gate_mode", ctypes.c_int),
         ("fixed_gates", ctypes.c_float * 3), ("dtype", ctypes.c_int), ("top_p", ctypes.c_float),
+        ("sel_mode", ctypes.c_int),
     ]
 
     @property
@@ -122,7 +123,7 @@ def _dev(t, name, dtype=None):
 
 def params(B, T, Hq, Hkv, d, cmp_block=32, cmp_stride=16, sel_block=64, top_n=16, window=512,
            softmax_scale=0.0, gate_mode=0, fixed_gates=(0.0, 0.0, 0.0), dtype=torch.bfloat16,
-           top_p=0.0):
+           top_p=0.0, sel_mode=0):
     p = NsaParams()
     p.B, p.T, p.Hq, p.Hkv, p.d = B, T, Hq, Hkv, d
     p.cmp_block, p.cmp_stride, p.sel_block, p.top_n, p.window = (
@@ -133,6 +134,7 @@ def params(B, T, Hq, Hkv, d, cmp_block=32, cmp_stride=16, sel_block=64, top_n=16
         p.fixed_gates[i] = fixed_gates[i]
     p.dtype = DTYPE_BF16 if dtype == torch.bfloat16 else DTYPE_F32
     p.top_p = top_p
+    p.sel_mode = sel_mode
     return p
 
 

@@ -87,6 +87,13 @@ typedef enum {
  *              blocks by score (ties to the lower index) up to the first prefix
  *              whose score sum reaches top_p times the sum over all candidate
  *              blocks, at most top_n blocks; unused sel_idx slots hold -1.
+ *   sel_mode   block scores the NSA selection ranks: 0 the compressed-branch
+ *              probability mass on each block, summed over the GQA group
+ *              (EP94 notes §五); 1 the Quest-style block bound of the pages'
+ *              selection ablation (EP94 notes §八): with kmin, kmax the
+ *              element-wise min and max of the block's keys up to the query,
+ *              sum over the group's heads of sum_e max(q_e kmin_e, q_e kmax_e).
+ *              Mode 1 needs top_p == 0 and runs on the CUDA-core path.
  * MoBA uses B, T, Hq, Hkv, d, sel_block, top_n, softmax_scale and dtype. */
 typedef struct {
   int B, T, Hq, Hkv, d;
@@ -97,6 +104,7 @@ typedef struct {
   float fixed_gates[3];
   nsa_dtype dtype;
   float top_p;
+  int sel_mode;
 } nsa_params;
 
 /* Bytes of caller-provided device workspace `op` needs for `p` (0 is

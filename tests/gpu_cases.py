@@ -18,7 +18,8 @@ def nsa_params_for(w, **kw):
                       cmp_stride=w["cmp_stride"], sel_block=w["sel_block"], top_n=w["top_n"],
                       window=w["window"], gate_mode=w.get("gate_mode", 0),
                       fixed_gates=w.get("fixed_gates", (0.0, 0.0, 0.0)),
-                      dtype=inputs.DTYPES[w["dtype"]], top_p=w.get("top_p", 0.0), **kw)
+                      dtype=inputs.DTYPES[w["dtype"]], top_p=w.get("top_p", 0.0),
+                      sel_mode=w.get("sel_mode", 0), **kw)
 
 
 def oracle_params_for(w):
@@ -26,7 +27,8 @@ def oracle_params_for(w):
                 cmp_block=w["cmp_block"], cmp_stride=w["cmp_stride"], sel_block=w["sel_block"],
                 top_n=w["top_n"], window=w["window"], scale=0.0,
                 gate_mode=w.get("gate_mode", 0), fixed_gates=w.get("fixed_gates", (0.0, 0.0, 0.0)),
-                store=w["dtype"], score_mode=0, top_p=w.get("top_p", 0.0))
+                store=w["dtype"], score_mode=2 if w.get("sel_mode", 0) == 1 else 0,
+                top_p=w.get("top_p", 0.0))
 
 
 def compare_nsa_rows(w, op, rows_b, rows_t, q_rows, k64, v64, kc64, vc64, wg64, gpu_out, gpu_sel):
@@ -40,8 +42,13 @@ def compare_nsa_rows(w, op, rows_b, rows_t, q_rows, k64, v64, kc64, vc64, wg64, 
                 same = parity.check_selection_topp(gpu_sel[r, g], res["sel"][r, g],
                                                    res["scores"][r, g], t // bs + 1, n, w["top_p"])
             else:
-                same = parity.check_selection(gpu_sel[r, g], res["sel"][r, g], res["scores"][r, g],
-                                              t // bs + 1, n)
+                # Quest bounds can sit near zero: their near-tie scale is the
+                # row's largest score magnitude
+                sc = res["scores"][r, g]
+                abs_scale = (float(np.abs(sc[:t // bs + 1]).max())
+                             if w.get("sel_mode", 0) == 1 else 0.0)
+                same = parity.check_selection(gpu_sel[r, g], res["sel"][r, g], sc, t // bs + 1, n,
+                                              abs_scale=abs_scale)
             differ[r] |= not same
     if differ.any():
         idx = np.nonzero(differ)[0]

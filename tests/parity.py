@@ -21,12 +21,13 @@ def _ranked(scores, lo, hi):
 
 
 def check_selection(gpu_sel, ora_sel, ora_scores, ncand, n_keep, forced_first=True,
-                    forced_block=None):
+                    forced_block=None, abs_scale=0.0):
     """Compare one row's selection. Returns True if the sets are equal, False if
     they differ but the difference is allowed (a near tie); raises otherwise.
 
     ncand: candidate blocks are 0..ncand-1 (NSA) -- for MoBA pass the number of
-    earlier blocks and forced_block = own block.
+    earlier blocks and forced_block = own block. abs_scale: a floor for the
+    scale the relative near-tie gap is taken of (scores that can be near zero).
     """
     g = sorted(int(x) for x in gpu_sel if x >= 0)
     o = sorted(int(x) for x in ora_sel if x >= 0)
@@ -42,7 +43,7 @@ def check_selection(gpu_sel, ora_sel, ora_scores, ncand, n_keep, forced_first=Tr
     s_last = ora_scores[ranked[want - 1]]
     s_next = ora_scores[ranked[want]]
     gap = abs(s_last - s_next)
-    if gap > SEL_REL * abs(s_last):
+    if gap > SEL_REL * max(abs(s_last), abs_scale):
         raise AssertionError(
             f"selection differs beyond the tie tolerance: gpu {g} oracle {o} "
             f"(gap {gap:.3e}, last kept {s_last:.9e})")
@@ -51,7 +52,7 @@ def check_selection(gpu_sel, ora_sel, ora_scores, ncand, n_keep, forced_first=Tr
     if forced is not None:
         assert forced in g, f"forced block {forced} missing from gpu selection {g}"
     assert len(free) == want, f"gpu kept {len(free)} blocks, expected {want}"
-    tol = SEL_REL * abs(s_last)
+    tol = SEL_REL * max(abs(s_last), abs_scale)
     for j in free:
         assert ora_scores[j] >= s_last - tol, f"gpu kept block {j} well below the cut"
     dropped = [j for j in ranked if j not in free]

@@ -122,3 +122,20 @@ def test_backward_workspace_and_argument_checks():
     big = nsa.params(1, 1024, 4, 1, 64, top_n=65)
     assert L.nsa_prefill_backward(ctypes.byref(big), *([fake] * 15), 1 << 30, None) == 2
     assert b"top_n" in L.nsa_last_error_detail()
+
+
+def test_selection_mode_checks():
+    """sel_mode: 0 or 1; the Quest bound (1) ranks raw bounds, not a probability
+    mass, so it takes no top-p threshold."""
+    n = ctypes.c_size_t()
+    ok = nsa.params(1, 1024, 4, 1, 64, sel_mode=1)
+    assert nsa.LIB.nsa_workspace_size(ctypes.byref(ok), nsa.OP_PREFILL, ctypes.byref(n)) == 0
+    bad = nsa.params(1, 1024, 4, 1, 64, sel_mode=2)
+    assert nsa.LIB.nsa_workspace_size(ctypes.byref(bad), nsa.OP_PREFILL, ctypes.byref(n)) == 1
+    bad = nsa.params(1, 1024, 4, 1, 64, sel_mode=1, top_p=0.5)
+    assert nsa.LIB.nsa_workspace_size(ctypes.byref(bad), nsa.OP_PREFILL, ctypes.byref(n)) == 1
+    assert b"top_p" in nsa.LIB.nsa_last_error_detail()
+    # the fast paths leave the Quest bound to the CUDA-core path
+    fast = nsa.params(1, 8192, 64, 4, 128)
+    assert nsa.workspace_size(fast, nsa.OP_PREFILL) > 0
+    assert nsa.workspace_size(nsa.params(1, 8192, 64, 4, 128, sel_mode=1), nsa.OP_PREFILL) == 0

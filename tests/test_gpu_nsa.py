@@ -139,6 +139,32 @@ def test_decode_bf16_fast_path_edges(over, lens):
     assert want <= names, names
 
 
+# Quest-style block-bound selection (sel_mode 1, the pages' selection ablation):
+# the CUDA-core path for prefill and decode against the oracle's score_mode 2.
+@pytest.mark.parametrize("name,over", [
+    ("nsa_prefill_bf16_t8192", dict(T=300, Hq=16, Hkv=1, sel_mode=1)),
+    ("nsa_prefill_f32_t1024", dict(T=400, sel_mode=1)),
+    ("nsa_prefill_f32_t1024", dict(B=2, T=130, Hq=8, Hkv=2, cmp_block=8, cmp_stride=4,
+                                   sel_block=16, top_n=3, window=20, sel_mode=1)),
+])
+def test_prefill_quest_selection(name, over):
+    from dynamic_block_sparse_nsa_b200 import nsa
+    w = inputs.workload(name, **over)
+    nsa.trace_enable(True, 64)
+    try:
+        gc.run_nsa_prefill(w)
+        recs, _ = nsa.trace_records()
+        names = {nm for nm, _ in recs}
+    finally:
+        nsa.trace_enable(False)
+    assert "nsa_rows_simt" in names and "pf_cmp_win" not in names, names
+
+
+def test_decode_quest_selection():
+    w = inputs.workload("nsa_decode_bf16_b32_l65536", B=3, T=3000, sel_mode=1)
+    gc.run_nsa_decode(w, [3000, 1777, 65])
+
+
 def test_decode_bf16_group_of_8_generic_path():
     w = inputs.workload("nsa_decode_bf16_b32_l65536", B=3, T=4000, Hq=32, Hkv=4)
     gc.run_nsa_decode(w, [4000, 1234, 64])
