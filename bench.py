@@ -653,7 +653,7 @@ def config_of(w):
 # --------------------------------------------------------------------------
 
 def run_dense(w, K, W, rank):
-    """Dense causal attention of the prefill's shape, in this build: nsa_prefill
+    """Dense causal attention of the prefill's shape, with this library: nsa_prefill
     with gates fixed to (0, 0, 1) and a window covering the sequence (the
     closed form in which NSA is dense attention; the zero-gated branches are
     skipped). Returns (ms per step, algorithmic flops per step)."""
