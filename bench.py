@@ -782,6 +782,8 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-prefill", action="store_true",
                     help="skip the 65536-token prefill measured beside the default decode line")
+    ap.add_argument("--only-backward", action="store_true",
+                    help="time only the 8192-token prefill backward (for profiling it)")
     ap.add_argument("--no-graph", action="store_true",
                     help="time decode steps as separate launches instead of one CUDA graph")
     ap.add_argument("--set", action="append", default=[], metavar="KEY=VALUE",
@@ -808,6 +810,11 @@ def main():
 
     ws, rank, local = dist_setup()
     import dynamic_block_sparse_nsa_b200.nsa  # noqa: F401  (fails loudly if unbuilt)
+    if args.only_backward:
+        bw = backward_summary(ws, rank, load_peaks(), 1965)
+        if rank == 0:
+            print(json.dumps({"prefill_backward_8k": bw}), flush=True)
+        return
     runner = {"decode": run_decode, "prefill": run_prefill, "moba": run_moba}[kind]
     kw = {"use_graph": not args.no_graph} if kind == "decode" else {}
     res = runner(w, args.steps, args.warmup, ws, rank, local, e2e=not args.no_e2e, **kw)
