@@ -1081,7 +1081,11 @@ __global__ void __launch_bounds__(CMB_THREADS) dec_combine_kernel(const __grid_c
   __shared__ float gate_s[CMB_HEADS * 3];
   __shared__ __align__(16) float contrib[3][CMB_HEADS][D];
   ptx::grid_dep_wait();  // partials and stream ranges of dec_cmp_partial / dec_sel_win
+  // the length and this branch's stream range in one round trip (the range
+  // words are in bounds whatever the length; they are used only when valid)
   const int L = __ldg(a.seq_lens + b);
+  const int2 rg = br == 0 ? *reinterpret_cast<const int2*>(a.rng1 + 2 * u)
+                          : *reinterpret_cast<const int2*>(a.rng3 + (long)u * 4 + 2 * (br - 1));
   if (!len_ok(L, a)) return;  // output zeroed by dec_select
 
   // gates (EP94 notes §五 gating): sigmoid(q_h . Wg[:, c]), a warp per dot product
@@ -1109,7 +1113,6 @@ __global__ void __launch_bounds__(CMB_THREADS) dec_combine_kernel(const __grid_c
   if (br == 0) {  // compressed branch: absent while no compressed block is complete
     part = a.part1;
     if (n_visible(L, a.l, a.s, a.Nc) > 0) {
-      const int2 rg = *reinterpret_cast<const int2*>(a.rng1 + 2 * u);
       first = 2 * ((long long)rg.x + u);
       np = 2 * (rg.y - rg.x + 1);
     } else {
@@ -1118,7 +1121,6 @@ __global__ void __launch_bounds__(CMB_THREADS) dec_combine_kernel(const __grid_c
     }
   } else {  // selected (segment 2u), window (segment 2u + 1)
     part = a.part3;
-    const int2 rg = *reinterpret_cast<const int2*>(a.rng3 + (long)u * 4 + 2 * (br - 1));
     first = 2 * ((long long)rg.x + 2 * u + (br - 1));
     np = 2 * (rg.y - rg.x + 1);
   }
