@@ -7,9 +7,9 @@
 // [c m, t] and to top_k - 1 earlier blocks chosen by q . mean(K_block). With
 // independent per-row choices no two rows share much, so the work is grouped
 // by key block instead of by query (the gather / re-index view of the pages):
-//   moba_gate  scores and picks per row on CUDA cores in fp32 (block means
-//              staged in shared memory), the selection row, and per-(head,
-//              block) pick counts;
+//   moba_gate  scores per row on the tensor cores at fp32 accuracy (block
+//              means split into three bf16 parts), the picks, the selection
+//              row, and per-(head, block) pick counts;
 //   moba_scan  offsets of each (sequence, head, block) bucket and of its
 //              128-row tiles;
 //   moba_fill  the rows of every bucket (token, slot);
@@ -40,7 +40,6 @@ constexpr int kMaxTopk = 8;
 constexpr int kStages = 4;
 constexpr int kThreads = 192;     // TMA lanes, MMA thread, 4 softmax warps
 constexpr uint32_t kNegInf = 0xff800000u;
-constexpr int kGateChunk = 64;    // block means staged per round in moba_gate
 
 struct MobaTcArgs {
   const __nv_bfloat16* q;
@@ -88,76 +87,163 @@ __device__ __forceinline__ uint64_t mnmaj(uint32_t base, int ks) {
 // j < t / m are scored with q . kbar[j] in fp32 and the top_k - 1 best kept
 // (higher score first, ties to the lower block: blocks arrive in increasing
 // order and only a strictly higher score displaces a kept one).
-__global__ void __launch_bounds__(128) moba_gate_kernel(MobaTcArgs a) {
-  __shared__ float kb[kGateChunk * D];
-  const int t0 = blockIdx.x * 128, h = blockIdx.y, b = blockIdx.z;
-  const int g = h / (a.Hq / a.Hkv);
-  const int t = t0 + threadIdx.x;
-  const bool ok = t < a.T;
-  const int own = ok ? t / a.m : 0;
-  const int own_max = min(t0 + 127, a.T - 1) / a.m;
-  const int want = a.topk - 1;
-  float q[D];
-  if (ok) {
-    const uint4* qr = reinterpret_cast<const uint4*>(a.q + ((size_t)(b * a.T + t) * a.Hq + h) * D);
-#pragma unroll
-    for (int c8 = 0; c8 < D / 8; ++c8) {
-      const uint4 v = __ldg(qr + c8);
-      const __nv_bfloat162* e = reinterpret_cast<const __nv_bfloat162*>(&v);
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float2 f = __bfloat1622float2(e[k]);
-        q[c8 * 8 + 2 * k] = f.x;
-        q[c8 * 8 + 2 * k + 1] = f.y;
-      }
-    }
-  }
-  float bs[kMaxTopk];
-  int bj[kMaxTopk];
+// Block scores q . kbar_j on the tensor cores without losing fp32 accuracy:
+// q is bf16, and each fp32 block mean is split into three bf16 parts
+// (hi + mid + lo, 24 significant bits), so every product q_e * part_e is exact
+// in fp32 and the three m16n8k16 passes accumulate them in fp32, like the fp32
+// dot product on CUDA cores. A CTA takes 128 tokens of one (sequence, head)
+// (8 warps x 16 rows; the tokens share one own block, m being a multiple of
+// 128); block means are staged kGateBlk at a time, split, in a padded layout
+// whose fragment loads hit distinct banks.
+constexpr int kGateTok = 128;
+constexpr int kGateBlk = 64;
+constexpr int kGatePitch = D + 8;  // bf16 elements per staged row
+constexpr size_t kGateSmem = 3 * (size_t)kGateBlk * kGatePitch * 2;
+
+__device__ __forceinline__ uint32_t ld_b32(const __nv_bfloat16* p) {
+  return *reinterpret_cast<const uint32_t*>(p);
+}
+
+// Keep the best `want` (score, block) of one row: higher score first, equal
+// scores to the lower block (candidates arrive in ascending block order and
+// only a strictly better one moves ahead). `worst` is the want-th kept score
+// (-inf until the list is full): most candidates fail that one comparison.
+__device__ __forceinline__ void keep_best(float (&bs)[kMaxTopk], int (&bj)[kMaxTopk], int want,
+                                          float& worst, float s, int j) {
+  if (!(s > worst)) return;
 #pragma unroll
   for (int i = 0; i < kMaxTopk; ++i) {
-    bs[i] = -INFINITY;
-    bj[i] = -1;
+    if (i < want && s > bs[i]) {
+      const float ts = bs[i];
+      const int tj = bj[i];
+      bs[i] = s;
+      bj[i] = j;
+      s = ts;
+      j = tj;
+    }
   }
-  for (int c0 = 0; c0 < own_max; c0 += kGateChunk) {
-    const int nb = min(kGateChunk, own_max - c0);
+#pragma unroll
+  for (int i = 0; i < kMaxTopk; ++i)
+    if (i == want - 1) worst = bs[i];
+}
+
+// Merge the four lane lists of a quad (disjoint blocks) into the best `want`,
+// in order: repeatedly the quad-wide best head (score desc, block asc).
+__device__ __forceinline__ void quad_merge(const float (&bs)[kMaxTopk], const int (&bj)[kMaxTopk],
+                                           int want, int (&out)[kMaxTopk]) {
+  int head = 0;
+#pragma unroll
+  for (int i = 0; i < kMaxTopk; ++i) {
+    if (i >= want) break;
+    float s = -INFINITY;
+    int j = 0x7fffffff;
+#pragma unroll
+    for (int x = 0; x < kMaxTopk; ++x)
+      if (x == head && bj[x] >= 0) {
+        s = bs[x];
+        j = bj[x];
+      }
+    const int mine = j;
+#pragma unroll
+    for (int o = 1; o <= 2; o <<= 1) {
+      const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+      const int j2 = __shfl_xor_sync(0xffffffffu, j, o);
+      if (s2 > s || (s2 == s && j2 < j)) {
+        s = s2;
+        j = j2;
+      }
+    }
+    out[i] = j == 0x7fffffff ? -1 : j;
+    if (mine == j && j != 0x7fffffff) ++head;
+  }
+}
+
+__global__ void __launch_bounds__(256) moba_gate_kernel(MobaTcArgs a) {
+  extern __shared__ __align__(16) unsigned char gate_raw[];
+  __nv_bfloat16* kbs = reinterpret_cast<__nv_bfloat16*>(gate_raw);  // [3][kGateBlk][kGatePitch]
+  const int t0 = blockIdx.x * kGateTok, h = blockIdx.y, b = blockIdx.z;
+  const int g = h / (a.Hq / a.Hkv);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int r0 = lane >> 2, q2 = (lane & 3) * 2;
+  const int own = t0 / a.m;  // the own block of every token of the tile
+  const int want = a.topk - 1;
+  const int ta = t0 + warp * 16 + r0, tb = ta + 8;  // this lane's rows
+  uint32_t qa[D / 16][4];
+  {
+    const __nv_bfloat16* qr0 = a.q + ((size_t)(b * a.T + ta) * a.Hq + h) * D;
+    const __nv_bfloat16* qr1 = a.q + ((size_t)(b * a.T + tb) * a.Hq + h) * D;
+#pragma unroll
+    for (int ks = 0; ks < D / 16; ++ks) {
+      qa[ks][0] = ta < a.T ? __ldg(reinterpret_cast<const unsigned*>(qr0 + ks * 16 + q2)) : 0u;
+      qa[ks][1] = tb < a.T ? __ldg(reinterpret_cast<const unsigned*>(qr1 + ks * 16 + q2)) : 0u;
+      qa[ks][2] = ta < a.T ? __ldg(reinterpret_cast<const unsigned*>(qr0 + ks * 16 + 8 + q2)) : 0u;
+      qa[ks][3] = tb < a.T ? __ldg(reinterpret_cast<const unsigned*>(qr1 + ks * 16 + 8 + q2)) : 0u;
+    }
+  }
+  float bs0[kMaxTopk], bs1[kMaxTopk];
+  int bj0[kMaxTopk], bj1[kMaxTopk];
+  float worst0 = -INFINITY, worst1 = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < kMaxTopk; ++i) {
+    bs0[i] = bs1[i] = -INFINITY;
+    bj0[i] = bj1[i] = -1;
+  }
+  // the scores of 8-block tile nt (c[0], c[1]: row r0; c[2], c[3]: row r0 + 8)
+  auto take = [&](const float (&c)[4], int j0) {
+    if (j0 < own) {
+      keep_best(bs0, bj0, want, worst0, c[0], j0);
+      keep_best(bs1, bj1, want, worst1, c[2], j0);
+    }
+    if (j0 + 1 < own) {
+      keep_best(bs0, bj0, want, worst0, c[1], j0 + 1);
+      keep_best(bs1, bj1, want, worst1, c[3], j0 + 1);
+    }
+  };
+  for (int c0 = 0; c0 < own; c0 += kGateBlk) {
+    const int nb = min(kGateBlk, own - c0);
     __syncthreads();
-    for (int i = threadIdx.x; i < nb * D / 4; i += 128) {
-      const int j = i / (D / 4), e4 = i % (D / 4);
-      reinterpret_cast<float4*>(kb)[i] = __ldg(reinterpret_cast<const float4*>(
-          a.kbar + (((size_t)b * a.nfull + c0 + j) * a.Hkv + g) * D) + e4);
+    for (int i = threadIdx.x; i < nb * D; i += 256) {
+      const int j = i / D, e = i - j * D;
+      const float x = __ldg(a.kbar + (((size_t)b * a.nfull + c0 + j) * a.Hkv + g) * D + e);
+      const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+      const float r1 = x - __bfloat162float(hi);
+      const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+      kbs[(0 * kGateBlk + j) * kGatePitch + e] = hi;
+      kbs[(1 * kGateBlk + j) * kGatePitch + e] = mid;
+      kbs[(2 * kGateBlk + j) * kGatePitch + e] = lo;
     }
     __syncthreads();
-    const int jend = ok ? min(nb, own - c0) : 0;
-    for (int jj = 0; jj < jend; ++jj) {
-      const float4* kr = reinterpret_cast<const float4*>(kb + jj * D);
-      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+    // two 8-block tiles at a time: two independent accumulator chains. B
+    // fragment column n = r0 is block c0 + 8 nt + r0; rows past nb are stale
+    // and their columns are discarded by take().
+    const int ntl = (nb + 7) / 8;
+    for (int nt = 0; nt < ntl; nt += 2) {
+      const bool two = nt + 1 < ntl;
+      float ca[4] = {0.f, 0.f, 0.f, 0.f}, cb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int e4 = 0; e4 < D / 4; ++e4) {
-        const float4 kv = kr[e4];
-        s0 = fmaf(q[4 * e4], kv.x, s0);
-        s1 = fmaf(q[4 * e4 + 1], kv.y, s1);
-        s2 = fmaf(q[4 * e4 + 2], kv.z, s2);
-        s3 = fmaf(q[4 * e4 + 3], kv.w, s3);
-      }
-      float s = (s0 + s1) + (s2 + s3);
-      int j = c0 + jj;
-      // insert into the descending list (strictly better only)
+      for (int pp = 0; pp < 3; ++pp) {
+        const __nv_bfloat16* ka = kbs + ((size_t)pp * kGateBlk + nt * 8 + r0) * kGatePitch;
+        const __nv_bfloat16* kb2 = ka + 8 * kGatePitch;
 #pragma unroll
-      for (int i = 0; i < kMaxTopk; ++i) {
-        if (i < want && s > bs[i]) {
-          const float ts = bs[i];
-          const int tj = bj[i];
-          bs[i] = s;
-          bj[i] = j;
-          s = ts;
-          j = tj;
+        for (int ks = 0; ks < D / 16; ++ks) {
+          ptx::mma_16816(ca, qa[ks], ld_b32(ka + ks * 16 + q2), ld_b32(ka + ks * 16 + 8 + q2));
+          if (two)
+            ptx::mma_16816(cb, qa[ks], ld_b32(kb2 + ks * 16 + q2),
+                           ld_b32(kb2 + ks * 16 + 8 + q2));
         }
       }
+      take(ca, c0 + nt * 8 + q2);  // blocks of c[0], c[2] and, + 1, of c[1], c[3]
+      if (two) take(cb, c0 + nt * 8 + 8 + q2);
     }
   }
-  if (!ok) return;
-  // the row: the picks (or every earlier block) and the own block, ascending
+  int pick0[kMaxTopk], pick1[kMaxTopk];
+  quad_merge(bs0, bj0, want, pick0);
+  quad_merge(bs1, bj1, want, pick1);
+  // lane q = 0 writes row r0, q = 1 row r0 + 8
+  if ((lane & 3) > 1) return;
+  const int t = (lane & 3) == 0 ? ta : tb;
+  if (t >= a.T) return;
   int row[kMaxTopk];
   int n = 0;
   if (own <= want) {
@@ -165,7 +251,7 @@ __global__ void __launch_bounds__(128) moba_gate_kernel(MobaTcArgs a) {
   } else {
 #pragma unroll
     for (int i = 0; i < kMaxTopk; ++i)
-      if (i < want) row[n++] = bj[i];
+      if (i < want) row[n++] = (lane & 3) == 0 ? pick0[i] : pick1[i];
     for (int i = 1; i < n; ++i) {  // insertion sort, n <= 7
       const int x = row[i];
       int p = i - 1;
@@ -824,8 +910,16 @@ cudaError_t launch_moba_tc(const nsa_params& p, const void* q, const void* k, co
   if (a.NB > 0 && (e = cudaMemsetAsync(a.cnt, 0, (size_t)a.NB * 4, stream)) != cudaSuccess) return e;
   {
     TraceScope trace("moba_gate", stream);
-    dim3 grid((p.T + 127) / 128, p.Hq, p.B);
-    moba_gate_kernel<<<grid, 128, 0, stream>>>(a);
+    static bool attr_set[64] = {};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+      cudaFuncSetAttribute(moba_gate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kGateSmem);
+      attr_set[dev] = true;
+    }
+    dim3 grid((p.T + kGateTok - 1) / kGateTok, p.Hq, p.B);
+    moba_gate_kernel<<<grid, 256, kGateSmem, stream>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (a.NB > 0 && p.top_n > 1) {
