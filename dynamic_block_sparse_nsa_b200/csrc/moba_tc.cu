@@ -202,16 +202,37 @@ __global__ void __launch_bounds__(256) moba_gate_kernel(MobaTcArgs a) {
   for (int c0 = 0; c0 < own; c0 += kGateBlk) {
     const int nb = min(kGateBlk, own - c0);
     __syncthreads();
-    for (int i = threadIdx.x; i < nb * D; i += 256) {
-      const int j = i / D, e = i - j * D;
-      const float x = __ldg(a.kbar + (((size_t)b * a.nfull + c0 + j) * a.Hkv + g) * D + e);
-      const __nv_bfloat16 hi = __float2bfloat16_rn(x);
-      const float r1 = x - __bfloat162float(hi);
-      const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-      const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
-      kbs[(0 * kGateBlk + j) * kGatePitch + e] = hi;
-      kbs[(1 * kGateBlk + j) * kGatePitch + e] = mid;
-      kbs[(2 * kGateBlk + j) * kGatePitch + e] = lo;
+    // every thread's eight float4 loads in flight at once, then the split
+    constexpr int kLd = kGateBlk * D / 4 / 256;
+    float4 xv[kLd];
+#pragma unroll
+    for (int r = 0; r < kLd; ++r) {
+      const int i4 = threadIdx.x + r * 256, j = i4 / (D / 4), e4 = i4 - j * (D / 4);
+      xv[r] = j < nb ? __ldg(reinterpret_cast<const float4*>(
+                           a.kbar + (((size_t)b * a.nfull + c0 + j) * a.Hkv + g) * D) + e4)
+                     : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int r = 0; r < kLd; ++r) {
+      const int i4 = threadIdx.x + r * 256, j = i4 / (D / 4), e = 4 * (i4 - j * (D / 4));
+      // hi = bf16(x), mid = bf16(x - hi), lo = bf16(x - hi - mid), two values a word
+      uint2 hv, mv, lv;
+      auto split2 = [](float x0, float x1, uint32_t& h, uint32_t& m, uint32_t& l) {
+        const __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
+        const float2 hf = __bfloat1622float2(hb);
+        const float r0 = x0 - hf.x, r1 = x1 - hf.y;
+        const __nv_bfloat162 mb = __floats2bfloat162_rn(r0, r1);
+        const float2 mf = __bfloat1622float2(mb);
+        const __nv_bfloat162 lb = __floats2bfloat162_rn(r0 - mf.x, r1 - mf.y);
+        h = *reinterpret_cast<const uint32_t*>(&hb);
+        m = *reinterpret_cast<const uint32_t*>(&mb);
+        l = *reinterpret_cast<const uint32_t*>(&lb);
+      };
+      split2(xv[r].x, xv[r].y, hv.x, mv.x, lv.x);
+      split2(xv[r].z, xv[r].w, hv.y, mv.y, lv.y);
+      *reinterpret_cast<uint2*>(kbs + (0 * kGateBlk + j) * kGatePitch + e) = hv;
+      *reinterpret_cast<uint2*>(kbs + (1 * kGateBlk + j) * kGatePitch + e) = mv;
+      *reinterpret_cast<uint2*>(kbs + (2 * kGateBlk + j) * kGatePitch + e) = lv;
     }
     __syncthreads();
     // two 8-block tiles at a time: two independent accumulator chains. B
