@@ -559,3 +559,65 @@ def test_quest_ignores_future_tokens_of_the_current_block():
     k2[0, 38:48] += 5.0  # later tokens of block 2, which holds t = 37
     moved = oracle.nsa_prefill(p, q, k2, v, w, wg, rows=[(0, 37)])
     np.testing.assert_array_equal(base["scores"], moved["scores"])
+
+
+# --------------------------------------------------------------------------
+# exact token top-k (oracle/variants.py; oracle-level variant only)
+# --------------------------------------------------------------------------
+
+def _topk_case(seed, **kw):
+    p = base_params(T=80, Hq=4, Hkv=2, d=8, sel_block=4, top_n=3, window=10, **kw)
+    q, k, v, w, wg = rand_inputs(p, rng=np.random.default_rng(seed))
+    return p, q, k, v, w, wg
+
+
+def test_exact_topk_with_every_token_is_dense_causal_attention():
+    from oracle import variants
+    p, q, k, v, w, wg = _topk_case(51)
+    rows = [(0, t) for t in (0, 5, 11, 40, 79)]
+    res = variants.exact_topk_rows(p, q, k, v, w, wg, rows, ktok=p["T"])
+    G = 2
+    for r, (_, t) in enumerate(rows):
+        for h in range(p["Hq"]):
+            z = k[0, :t + 1, h // G] @ q[0, t, h] / math.sqrt(p["d"])
+            pr = np.exp(z - z.max())
+            pr /= pr.sum()
+            np.testing.assert_allclose(res["o_slc"][r, h], pr @ v[0, :t + 1, h // G], atol=1e-12)
+
+
+def test_exact_topk_of_one_is_the_value_of_the_heaviest_token():
+    from oracle import variants
+    p, q, k, v, w, wg = _topk_case(52, gate_mode=1, fixed_gates=(0.0, 1.0, 0.0))
+    rows = [(0, t) for t in (3, 20, 79)]
+    res = variants.exact_topk_rows(p, q, k, v, w, wg, rows, ktok=1)
+    G = 2
+    for r, (_, t) in enumerate(rows):
+        for g in range(p["Hkv"]):
+            mass = np.zeros(t + 1)
+            for hh in range(G):
+                z = k[0, :t + 1, g] @ q[0, t, g * G + hh] / math.sqrt(p["d"])
+                e = np.exp(z - z.max())
+                mass += e / e.sum()
+            u = int(np.argmax(mass))  # first maximum: the lower index on a tie
+            assert res["sel"][r, g, 0] == u
+            for hh in range(G):
+                np.testing.assert_allclose(res["out"][r, g * G + hh], v[0, u, g], atol=1e-12)
+
+
+def test_exact_topk_set_is_the_heaviest_tokens():
+    from oracle import variants
+    p, q, k, v, w, wg = _topk_case(53)
+    rows = [(0, t) for t in (12, 50, 79)]
+    res = variants.exact_topk_rows(p, q, k, v, w, wg, rows)
+    ktok = p["top_n"] * p["sel_block"]
+    G = 2
+    for r, (_, t) in enumerate(rows):
+        for g in range(p["Hkv"]):
+            mass = np.zeros(t + 1)
+            for hh in range(G):
+                z = k[0, :t + 1, g] @ q[0, t, g * G + hh] / math.sqrt(p["d"])
+                e = np.exp(z - z.max())
+                mass += e / e.sum()
+            want = sorted(np.lexsort((np.arange(t + 1), -mass))[:ktok].tolist())
+            got = [int(x) for x in res["sel"][r, g] if x >= 0]
+            assert got == want
