@@ -715,6 +715,46 @@ def prefill_summary(ws, rank, local, peaks, K=5, W=3):
                     "a step is nsa_compress_kv + nsa_prefill on device-resident inputs"}
 
 
+def backward_oracle_sample(budget_s=6.0):
+    """The fp64 backward oracle, as it stands, on the host: whole backward
+    passes of a bounded sample with the benchmark's heads and head dim (bf16
+    values, 64 / 4 heads, d = 128, top-16, window 512) and fewer tokens,
+    repeated until the budget is spent. Returns a cpu_baseline dict in the
+    bench's flop count (10 d per query head and attended key)."""
+    import oracle
+    from oracle import backward as obwd
+    T = 128
+    w = inputs.workload("nsa_prefill_bf16_t8192", T=T)
+    inp = inputs.make_prefill(w, seed=5)
+    op = dict(B=1, T=T, Hq=w["Hq"], Hkv=w["Hkv"], d=w["d"], cmp_block=w["cmp_block"],
+              cmp_stride=w["cmp_stride"], sel_block=w["sel_block"], top_n=w["top_n"],
+              window=w["window"], scale=0.0, gate_mode=0, fixed_gates=(0.0, 0.0, 0.0),
+              store="bf16", score_mode=0, top_p=0.0)
+    f64 = {k_: v_.double().numpy() for k_, v_ in inp.items()}
+    fwd = oracle.nsa_prefill(op, f64["q"], f64["k"], f64["v"], f64["w_cmp"], f64["w_gate"])
+    sel = fwd["sel"].reshape(1, T, w["Hkv"], w["top_n"])
+    dout = np.random.default_rng(6).standard_normal(f64["q"].shape)
+    bs, l, s_ = w["sel_block"], w["cmp_block"], w["cmp_stride"]
+    t = np.arange(T)
+    tt = t[None, :, None, None]
+    ok = (sel >= 0) & (sel <= tt // bs)
+    nslc = np.where(ok, np.minimum(bs, tt + 1 - sel * bs), 0).sum()
+    keys = nslc + w["Hkv"] * (np.where(t + 1 >= l, (t + 1 - l) // s_ + 1, 0).sum() +
+                              np.minimum(w["window"], t + 1).sum())
+    flops_per = 10.0 * w["d"] * (w["Hq"] // w["Hkv"]) * float(keys)
+    done, used = 0, 0.0
+    while used < budget_s:
+        t0 = time.perf_counter()
+        obwd.nsa_prefill_backward(op, f64["q"], f64["k"], f64["v"], f64["w_cmp"], f64["w_gate"],
+                                  dout, sel, kc=fwd["k_cmp"], vc=fwd["v_cmp"])
+        used += time.perf_counter() - t0
+        done += 1
+    return {"value": done * flops_per / used / 1e12, "unit": "TFLOP/s", "cores": 1,
+            "kind": "oracle", "seconds": used,
+            "sample": f"{done} whole backward passes of a {T}-token sequence (64 / 4 heads, "
+                      f"d = 128, top-16, window 512)"}
+
+
 def backward_summary(ws, rank, peaks, clk_max_mhz, K=2, W=1):
     """The prefill backward at 8192 tokens (64 / 4 heads, d = 128, bf16):
     forward once for the selection, then K timed backward steps. Algorithmic
@@ -761,8 +801,9 @@ def backward_summary(ws, rank, peaks, clk_max_mhz, K=2, W=1):
     tflops = flops / (ms / 1000.0) / 1e12
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     peak = sms * 128 * 2 * clk_max_mhz * 1e6 / 1e12
+    cpu = backward_oracle_sample() if rank == 0 else None
     return {"workload": name, "value": tflops, "unit": "TFLOP/s", "ms_per_step": ms,
-            "steps": K, "warmup": W, "flops_per_step": flops,
+            "steps": K, "warmup": W, "flops_per_step": flops, "cpu_baseline": cpu,
             "roofline": {"bound": "alu", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
                          "frac": tflops / peak,
                          "peak_from": f"{sms} SMs x 128 fp32 lanes x 2 flops x {clk_max_mhz} MHz"},
