@@ -619,7 +619,7 @@ def run_reference(args, w):
     sample each, sized so the whole run stays within a few minutes."""
     kind = w["kind"]
     unit, scale = unit_of(kind)
-    per_step = max(0.02, 150.0 / max(1, args.steps + args.warmup))
+    per_step = max(0.02, args.ref_seconds / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
         oracle_sample(w, per_step)
     work = secs = 0.0
@@ -820,6 +820,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(inputs.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--ref-seconds", type=float, default=150.0,
+                    help="host seconds the reference arm spends over all its steps")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-prefill", action="store_true",
                     help="skip the 65536-token prefill measured beside the default decode line")
