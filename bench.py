@@ -382,8 +382,10 @@ def run_decode(w, K, W, ws, rank, local, e2e=True, use_graph=True):
     res.update(work=step_bytes, union=union_bytes, parts=parts)
     if e2e:
         # through the public call with host buffers: H2D of the step's query and
-        # lengths, D2H of the output and selection; the KV caches are device-
-        # resident state (as in serving), not per-step inputs.
+        # lengths from pinned memory, D2H of the output and selection, every
+        # step; the KV caches are device-resident state (as in serving), not
+        # per-step inputs. The copies are captured with the call into the same
+        # CUDA graph as the device-only timing (one graph of K steps).
         q_h = q.cpu().pin_memory()
         lens_h = lens.cpu().pin_memory()
         out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
@@ -400,8 +402,10 @@ def run_decode(w, K, W, ws, rank, local, e2e=True, use_graph=True):
             e2e_step()
         torch.cuda.synchronize()
         barrier(ws)
-        res["e2e_ms"] = _run_steps(e2e_step, K, False)[0]
+        res["e2e_ms"] = _run_steps(e2e_step, K, use_graph)[0]
         barrier(ws)
+        res["e2e_how"] = ("K steps of (H2D query + lengths, nsa_decode, D2H output + selection) "
+                          + ("captured in one CUDA graph" if use_graph else "as eager launches"))
         res["h2d"] = q_h.numel() * q_h.element_size() + lens_h.numel() * 4
         res["d2h"] = out_h.numel() * out_h.element_size() + sel_h_p.numel() * 4
     return res
@@ -573,14 +577,14 @@ def oracle_sample(w, budget_s):
                   gate_mode=0, store=w["dtype"], score_mode=0)
         k64, v64 = inp["k"].double().numpy(), inp["v"].double().numpy()
         kc, vc = oracle.compress(op, k64, v64, inp["w_cmp"].double().numpy())
-        q64 = inp["q"].double().numpy()
+        wg64 = inp["w_gate"].double().numpy()
         rng = np.random.default_rng(0)
         fl, t_used, done = 0, 0.0, 0
         while t_used < budget_s:
             rows = np.sort(rng.integers(0, w["T"], cores))
+            q_rows = np.ascontiguousarray(inp["q"][0, torch.from_numpy(rows)].double().numpy())
             t0 = time.perf_counter()
-            res = oracle.nsa_rows(op, [0] * len(rows), rows, q64[0, rows], k64, v64, kc, vc,
-                                  inp["w_gate"].double().numpy())
+            res = oracle.nsa_rows(op, [0] * len(rows), rows, q_rows, k64, v64, kc, vc, wg64)
             t_used += time.perf_counter() - t0
             for i, t in enumerate(rows):
                 nv = n_cmp(t + 1, w["cmp_block"], w["cmp_stride"])
@@ -683,36 +687,79 @@ def run_dense(w, K, W, rank):
     return ms, flops
 
 
-def prefill_summary(ws, rank, local, peaks, K=5, W=3):
-    """The 65536-token bf16 prefill (the metric's prefill half), timed like the
-    main line: whole-step TFLOP/s and every kernel against the bf16 peak."""
-    name = "nsa_prefill_bf16_t65536"
-    w = inputs.workload(name)
-    res = run_prefill(w, K, W, ws, rank, local, e2e=False)
-    ms_max = reduce_max(res["ms"], ws)
-    work_all = reduce_sum(res["work"] * K, ws)
+def kernel_entries(kind, res, w, K, peaks):
+    """Every traced kernel of a prefill-like step against the bf16 peak
+    (burst, and sustained beside it), from the first timed region's events."""
     per = {}
     for n, e in res["table0"].items():
-        wk, _ = kernel_work("prefill", n, res, w)
+        wk, _ = kernel_work(kind, n, res, w)
         if wk is None or not e["launches"]:
             continue
         per_launch = wk / (e["launches"] / min(K, 50))
-        ach = per_launch / (e["total_ms"] / e["launches"] / 1000.0) / 1e12
-        per[n] = {"tflops": ach, "frac": ach / peaks["bf16"], "peak": peaks["bf16"],
-                  "mean_launch_us": 1000.0 * e["total_ms"] / e["launches"]}
-    dms, dfl = run_dense(w, 2, 1, rank)
-    dms = reduce_max(dms, ws)
-    dense = {"ms_per_step": dms, "tflops": dfl / (dms / 1000.0) / 1e12, "flops_per_step": dfl,
-             "frac": dfl / (dms / 1000.0) / 1e12 / peaks["bf16"],
-             "nsa_speedup": dms / (ms_max / K),
-             "how": "nsa_prefill with gates fixed to (0, 0, 1) and window = T (dense causal "
-                    "attention, same shape), 2 timed steps after 1 warm-up"}
-    return {"workload": name, "value": work_all / (ms_max / 1000.0) / 1e12, "unit": "TFLOP/s",
-            "ms_per_step": ms_max / K, "steps": K, "warmup": W, "dense_causal": dense,
-            "flops_per_step": res["parts"], "kernel_tflops": per,
-            "peak_source": peaks["src"], "clocks": res["clk"],
-            "note": "algorithmic flops (4 d per query head and attended key); "
-                    "a step is nsa_compress_kv + nsa_prefill on device-resident inputs"}
+        mean_s = e["total_ms"] / e["launches"] / 1000.0
+        ach = per_launch / mean_s / 1e12
+        ent = {"tflops": ach, "frac": ach / peaks["bf16"], "peak": peaks["bf16"],
+               "frac_sustained": ach / peaks["bf16_sus"], "mean_launch_us": 1e6 * mean_s,
+               "flops_per_launch": per_launch}
+        g = gather_bytes(kind, n, res, w)
+        if g is not None:
+            ent["gathered_bytes_per_launch"] = g
+            ent["gather_gbs"] = g / mean_s / 1e9
+        per[n] = ent
+    return per
+
+
+def gather_bytes(kind, name, res, w):
+    """Bytes a kernel moves into shared memory per launch by design (not its
+    DRAM traffic): the selected-branch prefill kernel reads every selected
+    block's K and V once per (token, KV head), so this is its ingest figure."""
+    if kind == "prefill" and name == "pf_slc_attn":
+        return res["parts"]["slc"] / (4 * w["d"]) / (w["Hq"] // w["Hkv"]) * 2 * w["d"] * 2
+    return None
+
+
+def side_summary(name, ws, rank, local, peaks, K, W, cpu_budget, dense=False, e2e=True):
+    """One more workload timed like the main line (prefill or MoBA): whole-step
+    TFLOP/s, every kernel against the bf16 peak, the end-to-end figure with
+    host copies, and the oracle timed on a bounded sample (rank 0, one GPU)."""
+    w = inputs.workload(name)
+    kind = w["kind"]
+    runner = {"prefill": run_prefill, "moba": run_moba}[kind]
+    res = runner(w, K, W, ws, rank, local, e2e=e2e)
+    ms_max = reduce_max(res["ms"], ws)
+    work_all = reduce_sum(res["work"] * K, ws)
+    out = {"workload": name, "config": config_of(w), "value": work_all / (ms_max / 1000.0) / 1e12,
+           "unit": "TFLOP/s", "ms_per_step": ms_max / K, "steps": K, "warmup": W,
+           "flops_per_step": res["parts"], "kernel_tflops": kernel_entries(kind, res, w, K, peaks),
+           "peak_source": peaks["src"], "clocks": res["clk"]}
+    out["value_frac"] = out["value"] / peaks["bf16"]
+    if "e2e_ms" in res:
+        e_ms = reduce_max(res["e2e_ms"], ws)
+        out["e2e"] = {"value": work_all / (e_ms / 1000.0) / 1e12, "unit": "TFLOP/s",
+                      "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"],
+                      "ms_per_step": e_ms / K,
+                      "how": "H2D of q, k, v from pinned memory, the call(s), D2H of the "
+                             "output, every step"}
+    if dense:
+        dms, dfl = run_dense(w, 2, 1, rank)
+        dms = reduce_max(dms, ws)
+        out["dense_causal"] = {
+            "ms_per_step": dms, "tflops": dfl / (dms / 1000.0) / 1e12, "flops_per_step": dfl,
+            "frac": dfl / (dms / 1000.0) / 1e12 / peaks["bf16"],
+            "nsa_speedup": dms / (ms_max / K),
+            "how": "nsa_prefill with gates fixed to (0, 0, 1) and window = T (dense causal "
+                   "attention, same shape), 2 timed steps after 1 warm-up"}
+    if rank == 0 and ws == 1 and cpu_budget > 0:
+        wk, secs, cores, desc = oracle_sample(w, cpu_budget)
+        out["cpu_baseline"] = {"value": wk / secs / 1e12, "unit": "TFLOP/s", "cores": cores,
+                               "kind": "oracle", "sample": desc, "seconds": secs}
+    if kind == "prefill":
+        out["note"] = ("algorithmic flops (4 d per query head and attended key); a step is "
+                       "nsa_compress_kv + nsa_prefill on device-resident inputs")
+    else:
+        out["note"] = ("algorithmic flops: 4 d per (query head, attended key) plus the gate's "
+                       "2 d per (query head, earlier block); a step is one moba_prefill")
+    return out
 
 
 def backward_oracle_sample(budget_s=6.0):
@@ -820,11 +867,14 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(inputs.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--side-cpu-budget", type=float, default=8.0,
+                    help="host seconds of oracle timing for each workload beside the main one")
     ap.add_argument("--ref-seconds", type=float, default=150.0,
                     help="host seconds the reference arm spends over all its steps")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-prefill", action="store_true",
-                    help="skip the 65536-token prefill measured beside the default decode line")
+                    help="skip the prefill, MoBA and backward workloads measured beside the "
+                         "default decode line")
     ap.add_argument("--only-backward", action="store_true",
                     help="time only the 8192-token prefill backward (for profiling it)")
     ap.add_argument("--no-graph", action="store_true",
@@ -873,6 +923,8 @@ def main():
         e2e = {"value": work_all / (e_ms / 1000.0) / scale, "unit": unit,
                "h2d_bytes_per_step": res["h2d"], "d2h_bytes_per_step": res["d2h"],
                "ms_per_step": e_ms / K}
+        if "e2e_how" in res:
+            e2e["how"] = res["e2e_how"]
 
     tab = kernel_table(res["recs"], K)
     peaks = load_peaks()
@@ -890,19 +942,29 @@ def main():
             else:
                 ach = per_launch / mean_s / 1e12
                 pk, u = peaks["bf16"], "TFLOP/s"
-            roof = {"kernel": dom, "bound": bound, "achieved": ach, "peak": pk, "unit": u,
-                    "frac": ach / pk, "peak_source": peaks["src"],
+            roof = {"scope": "kernel", "kernel": dom, "bound": bound, "achieved": ach, "peak": pk,
+                    "unit": u, "frac": ach / pk, "peak_source": peaks["src"],
                     "traffic": kernel_traffic(dom, args.workload),
                     "algorithmic_per_launch": per_launch,
                     "mean_launch_us": mean_s * 1e6,
                     "timing": "events around each launch of this kernel over a second "
-                              "timed region of the same K steps"}
+                              "timed region of the same K steps",
+                    # the whole step against the same peak (the line's value)
+                    "step": {"achieved": value, "frac": value / pk,
+                             **({"frac_nominal_8tbs": value / 8000.0} if bound == "hbm" else {})}}
 
-    pf = bw = None
+    sides = {}
     if kind == "decode" and not args.set and not args.no_prefill and args.workload == DEFAULT_WORKLOAD:
-        pf = prefill_summary(ws, rank, local, peaks)
+        cb = 0.0 if args.no_cpu_baseline else args.side_cpu_budget
+        sides["prefill_64k"] = side_summary("nsa_prefill_bf16_t65536", ws, rank, local, peaks,
+                                            K=5, W=3, cpu_budget=cb, dense=True,
+                                            e2e=not args.no_e2e)
+        sides["prefill_8k"] = side_summary("nsa_prefill_bf16_t8192", ws, rank, local, peaks,
+                                           K=20, W=3, cpu_budget=cb, e2e=not args.no_e2e)
+        sides["moba_128k"] = side_summary("moba_prefill_bf16_t131072", ws, rank, local, peaks,
+                                          K=5, W=3, cpu_budget=cb, e2e=not args.no_e2e)
         clk_max = (res.get("clk") or {}).get("sm_max_mhz") or 1965
-        bw = backward_summary(ws, rank, peaks, clk_max)
+        sides["prefill_backward_8k"] = backward_summary(ws, rank, peaks, clk_max)
 
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
@@ -937,20 +999,9 @@ def main():
         else:
             line["flops_per_step"] = {k: v for k, v in res["parts"].items()}
             # every traced kernel against the bf16 peak (first timed region's events)
-            per = {}
-            for n, e in res["table0"].items():
-                wk, _ = kernel_work(kind, n, res, w)
-                if wk is None or not e["launches"]:
-                    continue
-                per_launch = wk / (e["launches"] / min(K, 50))
-                ach = per_launch / (e["total_ms"] / e["launches"] / 1000.0) / 1e12
-                per[n] = {"tflops": ach, "frac": ach / peaks["bf16"],
-                          "mean_launch_us": 1000.0 * e["total_ms"] / e["launches"]}
+            per = kernel_entries(kind, res, w, K, peaks)
             line["kernel_tflops"] = per
-        if pf is not None:
-            line["prefill_64k"] = pf
-        if bw is not None:
-            line["prefill_backward_8k"] = bw
+        line.update(sides)
         print(json.dumps(line), flush=True)
     if ws > 1:
         import torch.distributed as dist

@@ -1155,17 +1155,6 @@ __global__ void __launch_bounds__(CMB_THREADS) dec_combine_kernel(const __grid_c
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-// True the first time kernel `id` is launched on the current device.
-bool first_use(int id) {
-  static bool seen[4][64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) return true;
-  const bool f = !seen[id][dev];
-  seen[id][dev] = true;
-  return f;
-}
-
 struct WsLayout {
   size_t part1, trec, sel, part3, rng1, rng3, total;
 };
@@ -1303,8 +1292,7 @@ cudaError_t launch_decode_fast(const nsa_params& p, const void* q, const void* k
     // score records from registers when l = 2s and bs = 4s
     const bool rf = p.cmp_block == 2 * p.cmp_stride && p.sel_block == 4 * p.cmp_stride;
     auto kern = rf ? dec_stream_kernel<MODE_CMP, true> : dec_stream_kernel<MODE_CMP, false>;
-    if (first_use(rf ? 0 : 3))
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if ((e = ensure_dyn_smem((const void*)kern, (int)smem)) != cudaSuccess) return e;
     if ((e = launch_pdl(kern, dim3(a.grid1 / NPAIR), dim3(STREAM_THREADS), smem, stream, a, tkc,
                         tvc)) != cudaSuccess)
       return e;
@@ -1312,9 +1300,8 @@ cudaError_t launch_decode_fast(const nsa_params& p, const void* q, const void* k
   {
     const size_t smem = sel_dyn_smem(p.T, p.sel_block, a.tiles_max, a.nbt);
     TraceScope trace("dec_select", stream);
-    if (first_use(2))
-      cudaFuncSetAttribute(dec_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)kSelDynSmemMax);
+    if ((e = ensure_dyn_smem((const void*)dec_select_kernel, (int)kSelDynSmemMax)) != cudaSuccess)
+      return e;
     if ((e = launch_pdl(dec_select_kernel, dim3(p.B * p.Hkv), dim3(SEL_THREADS), smem, stream,
                         a)) != cudaSuccess)
       return e;
@@ -1322,9 +1309,9 @@ cudaError_t launch_decode_fast(const nsa_params& p, const void* q, const void* k
   {
     TraceScope trace("dec_sel_win", stream);
     constexpr size_t smem = StreamCfg<MODE_SW>::SMEM;
-    if (first_use(1))
-      cudaFuncSetAttribute(dec_stream_kernel<MODE_SW, false>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if ((e = ensure_dyn_smem((const void*)dec_stream_kernel<MODE_SW, false>, (int)smem)) !=
+        cudaSuccess)
+      return e;
     if ((e = launch_pdl(dec_stream_kernel<MODE_SW, false>, dim3(a.grid3 / NPAIR),
                         dim3(STREAM_THREADS), smem, stream, a, tk, tv)) != cudaSuccess)
       return e;

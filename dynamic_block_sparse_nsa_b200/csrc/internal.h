@@ -145,6 +145,11 @@ void set_last_error(nsa_status s, const char* msg);
 // Multiprocessor count of the current device (cached per device).
 int device_sm_count();
 
+// Raises the dynamic shared-memory limit of kernel `func` to `bytes` on the
+// current device (once per kernel and device; safe from several host threads:
+// a caller returns only after the limit is in place).
+cudaError_t ensure_dyn_smem(const void* func, int bytes);
+
 // 3-D TMA map over a contiguous bf16 array [dim2][dim1][dim0] with a box of
 // (box0, box1, box2) elements; false if the driver rejects it.
 bool make_tmap_bf16_3d(CUtensorMap* m, const void* base, uint64_t dim0, uint64_t dim1,

@@ -849,15 +849,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 size_t attn_smem(int qbufs) { return 1024 + (size_t)(qbufs + kStages) * TILE + sizeof(Bars); }
 
-bool first_use(int id) {
-  static bool seen[2][64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) return true;
-  const bool f = !seen[id][dev];
-  seen[id][dev] = true;
-  return f;
-}
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -931,14 +922,8 @@ cudaError_t launch_moba_tc(const nsa_params& p, const void* q, const void* k, co
   if (a.NB > 0 && (e = cudaMemsetAsync(a.cnt, 0, (size_t)a.NB * 4, stream)) != cudaSuccess) return e;
   {
     TraceScope trace("moba_gate", stream);
-    static bool attr_set[64] = {};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-      cudaFuncSetAttribute(moba_gate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)kGateSmem);
-      attr_set[dev] = true;
-    }
+    if ((e = ensure_dyn_smem((const void*)moba_gate_kernel, (int)kGateSmem)) != cudaSuccess)
+      return e;
     dim3 grid((p.T + kGateTok - 1) / kGateTok, p.Hq, p.B);
     moba_gate_kernel<<<grid, 256, kGateSmem, stream>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -958,8 +943,7 @@ cudaError_t launch_moba_tc(const nsa_params& p, const void* q, const void* k, co
     }
     {
       const size_t sm = attn_smem(2);
-      if (first_use(0))
-        cudaFuncSetAttribute(moba_blk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+      if ((e = ensure_dyn_smem((const void*)moba_blk_kernel, (int)sm)) != cudaSuccess) return e;
       TraceScope trace("moba_blk", stream);
       moba_blk_kernel<<<device_sm_count(), kThreads, sm, stream>>>(tk, tv, a);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -967,8 +951,7 @@ cudaError_t launch_moba_tc(const nsa_params& p, const void* q, const void* k, co
   }
   {
     const size_t sm = attn_smem(1);
-    if (first_use(1))
-      cudaFuncSetAttribute(moba_own_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if ((e = ensure_dyn_smem((const void*)moba_own_kernel, (int)sm)) != cudaSuccess) return e;
     TraceScope trace("moba_own", stream);
     const long long grid = (long long)p.B * p.Hq * ((p.T + KT - 1) / KT);
     moba_own_kernel<<<(unsigned)grid, kThreads, sm, stream>>>(tq, tk, tv, a);

@@ -1064,16 +1064,6 @@ int main_stages(int nblk) {
   return 0;
 }
 
-bool first_use(int id) {
-  static bool seen[2][64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) return true;
-  const bool f = !seen[id][dev];
-  seen[id][dev] = true;
-  return f;
-}
-
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
@@ -1148,8 +1138,7 @@ cudaError_t launch_prefill_tc(const nsa_params& p, const void* q, const void* k,
 
   cudaError_t e;
   const size_t sm1 = main_smem(a.stages, a.nblk);
-  if (first_use(0))
-    cudaFuncSetAttribute(pf_main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+  if ((e = ensure_dyn_smem((const void*)pf_main_kernel, 227 * 1024)) != cudaSuccess) return e;
   {
     TraceScope trace("pf_cmp_win", stream);
     const long long grid = (long long)p.B * p.Hkv * ((p.T + TQ - 1) / TQ);
@@ -1158,8 +1147,7 @@ cudaError_t launch_prefill_tc(const nsa_params& p, const void* q, const void* k,
   }
   if (a.direct_out) return cudaSuccess;
   const size_t sm2 = slc_smem();
-  if (first_use(1))
-    cudaFuncSetAttribute(pf_slc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
+  if ((e = ensure_dyn_smem((const void*)pf_slc_kernel, (int)sm2)) != cudaSuccess) return e;
   {
     TraceScope trace("pf_slc_attn", stream);
     const long long U = (long long)p.B * p.T * p.Hkv;

@@ -23,14 +23,43 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 int device_sm_count() {
+  static std::mutex mu;
   static int cache[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(mu);
   if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (dev >= 0 && dev < 64) cache[dev] = sms;
   return sms;
+}
+
+cudaError_t ensure_dyn_smem(const void* func, int bytes) {
+  struct Entry {
+    const void* f;
+    int dev, bytes;
+  };
+  static std::mutex mu;
+  static Entry done[256];
+  static int ndone = 0;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  // The lock is held across the attribute call, so no caller can see the
+  // kernel as prepared before the limit is raised.
+  std::lock_guard<std::mutex> lk(mu);
+  for (int i = 0; i < ndone; ++i)
+    if (done[i].f == func && done[i].dev == dev && done[i].bytes >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  for (int i = 0; i < ndone; ++i)
+    if (done[i].f == func && done[i].dev == dev) {
+      done[i].bytes = bytes;
+      return cudaSuccess;
+    }
+  if (ndone < 256) done[ndone++] = Entry{func, dev, bytes};
+  return cudaSuccess;
 }
 
 namespace {

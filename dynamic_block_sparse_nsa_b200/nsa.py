@@ -105,12 +105,17 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream):
-    s = stream if stream is not None else torch.cuda.current_stream()
-    return ctypes.c_void_p(s.cuda_stream)
+def _stream(stream, device=None):
+    """The stream to enqueue on: `stream`, else the current stream of `device`
+    (of the current device when None). A given stream must live on `device`."""
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    elif device is not None and stream.device != torch.device(device):
+        raise ValueError(f"stream is on {stream.device}, the tensors on {device}")
+    return ctypes.c_void_p(stream.cuda_stream)
 
 
-def _dev(t, name, dtype=None):
+def _dev(t, name, dtype=None, device=None):
     if t is None:
         return
     if not t.is_cuda:
@@ -119,6 +124,24 @@ def _dev(t, name, dtype=None):
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device} (all tensors of a call "
+                         f"must share one device)")
+
+
+class _on:
+    """Makes the tensors' device current for the call: the library reads the
+    current device for its per-device state (error word, cached tensor maps,
+    the no-allocation scratch), so it must be the device the data lives on."""
+
+    def __init__(self, device):
+        self.ctx = torch.cuda.device(device)
+
+    def __enter__(self):
+        self.ctx.__enter__()
+
+    def __exit__(self, *a):
+        self.ctx.__exit__(*a)
 
 
 def params(B, T, Hq, Hkv, d, cmp_block=32, cmp_stride=16, sel_block=64, top_n=16, window=512,
@@ -155,40 +178,46 @@ def workspace(p, op, device="cuda"):
 
 def nsa_compress_kv(p, k, v, w_cmp, k_cmp=None, v_cmp=None, stream=None):
     dt = p.torch_dtype
-    for t, nm in ((k, "k"), (v, "v")):
-        _dev(t, nm, dt)
-    _dev(w_cmp, "w_cmp", torch.float32)
+    _dev(k, "k", dt)
+    dev = k.device
+    _dev(v, "v", dt, dev)
+    _dev(w_cmp, "w_cmp", torch.float32, dev)
     Nc = num_cmp_blocks(p.T, p.cmp_block, p.cmp_stride)
     shape = (p.B, Nc, p.Hkv, p.d)
     if k_cmp is None:
-        k_cmp = torch.empty(shape, dtype=dt, device=k.device)
+        k_cmp = torch.empty(shape, dtype=dt, device=dev)
     if v_cmp is None:
-        v_cmp = torch.empty(shape, dtype=dt, device=k.device)
-    _dev(k_cmp, "k_cmp", dt)
-    _dev(v_cmp, "v_cmp", dt)
-    _raise(LIB.nsa_compress_kv(ctypes.byref(p), _ptr(k), _ptr(v), _ptr(w_cmp), _ptr(k_cmp),
-                               _ptr(v_cmp), _stream(stream)))
+        v_cmp = torch.empty(shape, dtype=dt, device=dev)
+    _dev(k_cmp, "k_cmp", dt, dev)
+    _dev(v_cmp, "v_cmp", dt, dev)
+    with _on(dev):
+        _raise(LIB.nsa_compress_kv(ctypes.byref(p), _ptr(k), _ptr(v), _ptr(w_cmp), _ptr(k_cmp),
+                                   _ptr(v_cmp), _stream(stream, dev)))
     return k_cmp, v_cmp
 
 
 def nsa_prefill(p, q, k, v, k_cmp, v_cmp, w_gate=None, out=None, sel_idx=None, ws=None,
                 stream=None, want_sel=True):
     dt = p.torch_dtype
-    for t, nm in ((q, "q"), (k, "k"), (v, "v"), (k_cmp, "k_cmp"), (v_cmp, "v_cmp")):
-        _dev(t, nm, dt)
-    _dev(w_gate, "w_gate", torch.float32)
+    _dev(q, "q", dt)
+    dev = q.device
+    for t, nm in ((k, "k"), (v, "v"), (k_cmp, "k_cmp"), (v_cmp, "v_cmp")):
+        _dev(t, nm, dt, dev)
+    _dev(w_gate, "w_gate", torch.float32, dev)
     if out is None:
-        out = torch.empty(p.B, p.T, p.Hq, p.d, dtype=dt, device=q.device)
+        out = torch.empty(p.B, p.T, p.Hq, p.d, dtype=dt, device=dev)
     if sel_idx is None and want_sel:
-        sel_idx = torch.empty(p.B, p.T, p.Hkv, p.top_n, dtype=torch.int32, device=q.device)
-    _dev(out, "out", dt)
-    _dev(sel_idx, "sel_idx", torch.int32)
+        sel_idx = torch.empty(p.B, p.T, p.Hkv, p.top_n, dtype=torch.int32, device=dev)
+    _dev(out, "out", dt, dev)
+    _dev(sel_idx, "sel_idx", torch.int32, dev)
     if ws is None:
-        ws = workspace(p, OP_PREFILL, q.device)
+        ws = workspace(p, OP_PREFILL, dev)
+    _dev(ws, "ws", None, dev)
     nbytes = 0 if ws is None else ws.numel() * ws.element_size()
-    _raise(LIB.nsa_prefill(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(k_cmp), _ptr(v_cmp),
-                           _ptr(w_gate), _ptr(out), _ptr(sel_idx), _ptr(ws), nbytes,
-                           _stream(stream)))
+    with _on(dev):
+        _raise(LIB.nsa_prefill(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(k_cmp),
+                               _ptr(v_cmp), _ptr(w_gate), _ptr(out), _ptr(sel_idx), _ptr(ws),
+                               nbytes, _stream(stream, dev)))
     return out, sel_idx
 
 
@@ -196,48 +225,65 @@ def nsa_prefill_backward(p, q, k, v, k_cmp, v_cmp, w_cmp, w_gate, sel_idx, dout,
                          stream=None):
     """Gradients of sum(dout * out) of nsa_prefill: (dq, dk, dv, dw_cmp, dw_gate), fp32."""
     dt = p.torch_dtype
-    for t, nm in ((q, "q"), (k, "k"), (v, "v"), (k_cmp, "k_cmp"), (v_cmp, "v_cmp"),
-                  (dout, "dout")):
-        _dev(t, nm, dt)
-    _dev(w_cmp, "w_cmp", torch.float32)
-    _dev(w_gate, "w_gate", torch.float32)
-    _dev(sel_idx, "sel_idx", torch.int32)
-    f32 = dict(dtype=torch.float32, device=q.device)
+    _dev(q, "q", dt)
+    dev = q.device
+    for t, nm in ((k, "k"), (v, "v"), (k_cmp, "k_cmp"), (v_cmp, "v_cmp"), (dout, "dout")):
+        _dev(t, nm, dt, dev)
+    _dev(w_cmp, "w_cmp", torch.float32, dev)
+    _dev(w_gate, "w_gate", torch.float32, dev)
+    _dev(sel_idx, "sel_idx", torch.int32, dev)
+    f32 = dict(dtype=torch.float32, device=dev)
     dq = torch.empty(p.B, p.T, p.Hq, p.d, **f32)
     dk = torch.empty(p.B, p.T, p.Hkv, p.d, **f32)
     dv = torch.empty(p.B, p.T, p.Hkv, p.d, **f32)
     dw_cmp = torch.empty(p.cmp_block, **f32)
     dw_gate = torch.empty(p.d, 3, **f32)
     if ws is None:
-        ws = workspace(p, OP_PREFILL_BACKWARD, q.device)
+        ws = workspace(p, OP_PREFILL_BACKWARD, dev)
+    _dev(ws, "ws", None, dev)
     nbytes = 0 if ws is None else ws.numel() * ws.element_size()
-    _raise(LIB.nsa_prefill_backward(
-        ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(k_cmp), _ptr(v_cmp), _ptr(w_cmp),
-        _ptr(w_gate), _ptr(sel_idx), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dw_cmp),
-        _ptr(dw_gate), _ptr(ws), nbytes, _stream(stream)))
+    with _on(dev):
+        _raise(LIB.nsa_prefill_backward(
+            ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(k_cmp), _ptr(v_cmp), _ptr(w_cmp),
+            _ptr(w_gate), _ptr(sel_idx), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dw_cmp),
+            _ptr(dw_gate), _ptr(ws), nbytes, _stream(stream, dev)))
     return dq, dk, dv, dw_cmp, dw_gate
+
+
+def _decode_args(p, q, k_cache, v_cache, seq_lens, k_cmp, v_cmp, w_gate, out, sel_idx,
+                 want_sel):
+    """Checks of the decode arguments (one device for all); allocates the
+    outputs that are not given."""
+    dt = p.torch_dtype
+    _dev(q, "q", dt)
+    dev = q.device
+    for t, nm in ((k_cache, "k_cache"), (v_cache, "v_cache"), (k_cmp, "k_cmp"),
+                  (v_cmp, "v_cmp")):
+        _dev(t, nm, dt, dev)
+    _dev(seq_lens, "seq_lens", torch.int32, dev)
+    _dev(w_gate, "w_gate", torch.float32, dev)
+    if out is None:
+        out = torch.empty(p.B, p.Hq, p.d, dtype=dt, device=dev)
+    if sel_idx is None and want_sel:
+        sel_idx = torch.empty(p.B, p.Hkv, p.top_n, dtype=torch.int32, device=dev)
+    _dev(out, "out", dt, dev)
+    _dev(sel_idx, "sel_idx", torch.int32, dev)
+    return out, sel_idx
 
 
 def nsa_decode(p, q, k_cache, v_cache, seq_lens, k_cmp, v_cmp, w_gate=None, out=None,
                sel_idx=None, ws=None, stream=None, want_sel=True):
-    dt = p.torch_dtype
-    for t, nm in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"), (k_cmp, "k_cmp"),
-                  (v_cmp, "v_cmp")):
-        _dev(t, nm, dt)
-    _dev(seq_lens, "seq_lens", torch.int32)
-    _dev(w_gate, "w_gate", torch.float32)
-    if out is None:
-        out = torch.empty(p.B, p.Hq, p.d, dtype=dt, device=q.device)
-    if sel_idx is None and want_sel:
-        sel_idx = torch.empty(p.B, p.Hkv, p.top_n, dtype=torch.int32, device=q.device)
-    _dev(out, "out", dt)
-    _dev(sel_idx, "sel_idx", torch.int32)
+    out, sel_idx = _decode_args(p, q, k_cache, v_cache, seq_lens, k_cmp, v_cmp, w_gate, out,
+                                sel_idx, want_sel)
+    dev = q.device
     if ws is None:
-        ws = workspace(p, OP_DECODE, q.device)
+        ws = workspace(p, OP_DECODE, dev)
+    _dev(ws, "ws", None, dev)
     nbytes = 0 if ws is None else ws.numel() * ws.element_size()
-    _raise(LIB.nsa_decode(ctypes.byref(p), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens),
-                          _ptr(k_cmp), _ptr(v_cmp), _ptr(w_gate), _ptr(out), _ptr(sel_idx),
-                          _ptr(ws), nbytes, _stream(stream)))
+    with _on(dev):
+        _raise(LIB.nsa_decode(ctypes.byref(p), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                              _ptr(seq_lens), _ptr(k_cmp), _ptr(v_cmp), _ptr(w_gate), _ptr(out),
+                              _ptr(sel_idx), _ptr(ws), nbytes, _stream(stream, dev)))
     return out, sel_idx
 
 
@@ -247,21 +293,14 @@ def nsa_decode_noalloc(p, q, k_cache, v_cache, seq_lens, k_cmp, v_cmp, w_gate=No
     callers that cannot allocate device memory (include/nsa.h gives the limits;
     calls must not overlap on the GPU). The C call allocates nothing; this
     wrapper allocates `out` / `sel_idx` only when they are not given."""
-    dt = p.torch_dtype
-    for t, nm in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache"), (k_cmp, "k_cmp"),
-                  (v_cmp, "v_cmp")):
-        _dev(t, nm, dt)
-    _dev(seq_lens, "seq_lens", torch.int32)
-    _dev(w_gate, "w_gate", torch.float32)
-    if out is None:
-        out = torch.empty(p.B, p.Hq, p.d, dtype=dt, device=q.device)
-    if sel_idx is None and want_sel:
-        sel_idx = torch.empty(p.B, p.Hkv, p.top_n, dtype=torch.int32, device=q.device)
-    _dev(out, "out", dt)
-    _dev(sel_idx, "sel_idx", torch.int32)
-    _raise(LIB.nsa_decode_noalloc(ctypes.byref(p), _ptr(q), _ptr(k_cache), _ptr(v_cache),
-                                  _ptr(seq_lens), _ptr(k_cmp), _ptr(v_cmp), _ptr(w_gate),
-                                  _ptr(out), _ptr(sel_idx), _stream(stream)))
+    out, sel_idx = _decode_args(p, q, k_cache, v_cache, seq_lens, k_cmp, v_cmp, w_gate, out,
+                                sel_idx, want_sel)
+    dev = q.device
+    # the device current during the call selects which GPU's static scratch is used
+    with _on(dev):
+        _raise(LIB.nsa_decode_noalloc(ctypes.byref(p), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                      _ptr(seq_lens), _ptr(k_cmp), _ptr(v_cmp), _ptr(w_gate),
+                                      _ptr(out), _ptr(sel_idx), _stream(stream, dev)))
     return out, sel_idx
 
 
@@ -269,30 +308,38 @@ def nsa_append_kv(p, k_new, v_new, pos, k_cache, v_cache, w_cmp, k_cmp, v_cmp, s
     """Write one token per sequence at pos[b] into the caches; complete
     compressed blocks are written into k_cmp / v_cmp (see include/nsa.h)."""
     dt = p.torch_dtype
-    for t, nm in ((k_new, "k_new"), (v_new, "v_new"), (k_cache, "k_cache"), (v_cache, "v_cache"),
+    _dev(k_new, "k_new", dt)
+    dev = k_new.device
+    for t, nm in ((v_new, "v_new"), (k_cache, "k_cache"), (v_cache, "v_cache"),
                   (k_cmp, "k_cmp"), (v_cmp, "v_cmp")):
-        _dev(t, nm, dt)
-    _dev(pos, "pos", torch.int32)
-    _dev(w_cmp, "w_cmp", torch.float32)
-    _raise(LIB.nsa_append_kv(ctypes.byref(p), _ptr(k_new), _ptr(v_new), _ptr(pos), _ptr(k_cache),
-                             _ptr(v_cache), _ptr(w_cmp), _ptr(k_cmp), _ptr(v_cmp), _stream(stream)))
+        _dev(t, nm, dt, dev)
+    _dev(pos, "pos", torch.int32, dev)
+    _dev(w_cmp, "w_cmp", torch.float32, dev)
+    with _on(dev):
+        _raise(LIB.nsa_append_kv(ctypes.byref(p), _ptr(k_new), _ptr(v_new), _ptr(pos),
+                                 _ptr(k_cache), _ptr(v_cache), _ptr(w_cmp), _ptr(k_cmp),
+                                 _ptr(v_cmp), _stream(stream, dev)))
 
 
 def moba_prefill(p, q, k, v, out=None, sel_idx=None, ws=None, stream=None, want_sel=True):
     dt = p.torch_dtype
-    for t, nm in ((q, "q"), (k, "k"), (v, "v")):
-        _dev(t, nm, dt)
+    _dev(q, "q", dt)
+    dev = q.device
+    _dev(k, "k", dt, dev)
+    _dev(v, "v", dt, dev)
     if out is None:
-        out = torch.empty(p.B, p.T, p.Hq, p.d, dtype=dt, device=q.device)
+        out = torch.empty(p.B, p.T, p.Hq, p.d, dtype=dt, device=dev)
     if sel_idx is None and want_sel:
-        sel_idx = torch.empty(p.B, p.T, p.Hq, p.top_n, dtype=torch.int32, device=q.device)
-    _dev(out, "out", dt)
-    _dev(sel_idx, "sel_idx", torch.int32)
+        sel_idx = torch.empty(p.B, p.T, p.Hq, p.top_n, dtype=torch.int32, device=dev)
+    _dev(out, "out", dt, dev)
+    _dev(sel_idx, "sel_idx", torch.int32, dev)
     if ws is None:
-        ws = workspace(p, OP_MOBA_PREFILL, q.device)
+        ws = workspace(p, OP_MOBA_PREFILL, dev)
+    _dev(ws, "ws", None, dev)
     nbytes = 0 if ws is None else ws.numel() * ws.element_size()
-    _raise(LIB.moba_prefill(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(sel_idx),
-                            _ptr(ws), nbytes, _stream(stream)))
+    with _on(dev):
+        _raise(LIB.moba_prefill(ctypes.byref(p), _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                _ptr(sel_idx), _ptr(ws), nbytes, _stream(stream, dev)))
     return out, sel_idx
 
 

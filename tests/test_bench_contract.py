@@ -36,3 +36,10 @@ def test_reference_arm_on_a_prefill_workload():
     line = _run("--impl", "reference", "--workload", "nsa_prefill_bf16_t8192", "--steps", "1",
                 "--warmup", "3", "--ref-seconds", "2")
     assert line["unit"] == "TFLOP/s" and line["value"] > 0
+
+
+def test_reference_arm_on_the_moba_workload():
+    line = _run("--impl", "reference", "--workload", "moba_prefill_bf16_t131072", "--steps", "1",
+                "--warmup", "3", "--ref-seconds", "2")
+    assert line["unit"] == "TFLOP/s" and line["value"] > 0
+    assert line["config"]["workload"] == "moba_prefill_bf16_t131072"

@@ -72,6 +72,24 @@ def test_prefill_bf16_tensor_core_edges(over):
     gc.run_nsa_prefill(w, seed=7)
 
 
+# Each branch alone on the tensor-core path, with unit-variance q, k, v so the
+# outputs are O(1) and the absolute bf16 bounds are tight: a late-row error in
+# one branch cannot hide behind the others or behind a small output scale.
+@pytest.mark.parametrize("gates", [(1.0, 0.0, 0.0), (0.0, 1.0, 0.0), (0.0, 0.0, 1.0)])
+def test_prefill_bf16_tensor_core_branch_alone(gates):
+    w = inputs.workload("nsa_prefill_bf16_t8192", T=1403, Hq=16, Hkv=1, qkv_scale=1.0,
+                        gate_mode=1, fixed_gates=gates, top_n=6, window=300)
+    rows = [(0, t) for t in list(range(0, 1403, 7)) + list(range(1350, 1403))]
+    gc.run_nsa_prefill(w, rows=rows, seed=17)
+
+
+@pytest.mark.parametrize("gates", [(1.0, 0.0, 0.0), (0.0, 1.0, 0.0), (0.0, 0.0, 1.0)])
+def test_decode_bf16_fast_path_branch_alone(gates):
+    w = inputs.workload("nsa_decode_bf16_b32_l65536", B=4, T=6000, gate_mode=1,
+                        fixed_gates=gates)
+    gc.run_nsa_decode(w, [6000, 4033, 999, 70], seed=18)
+
+
 def test_prefill_bf16_runs_the_tensor_core_kernels():
     from dynamic_block_sparse_nsa_b200 import nsa
     w = inputs.workload("nsa_prefill_bf16_t8192", T=600, Hq=16, Hkv=1)

@@ -29,13 +29,30 @@ def _c_abi_noalloc(nsa, p, dev, kc, vc, out, sel):
         P(torch.cuda.current_stream().cuda_stream))
 
 
-def test_noalloc_decode_matches_workspace_decode_twice(cuda_ok):
-    from dynamic_block_sparse_nsa_b200 import nsa
-    w = inputs.workload("nsa_decode_bf16_b32_l65536", B=6, T=12000)
-    inp = inputs.make_decode(w, seed=11, seq_lens=[12000, 9000, 4097, 777, 64, 11999])
+def _decode_case(nsa, B, T, seed, lens):
+    w = inputs.workload("nsa_decode_bf16_b32_l65536", B=B, T=T)
+    inp = inputs.make_decode(w, seed=seed, seq_lens=lens)
     p = gc.nsa_params_for(w)
     dev = {k_: v_.cuda() for k_, v_ in inp.items()}
     kc, vc = nsa.nsa_compress_kv(p, dev["k"], dev["v"], dev["w_cmp"])
+    return p, dev, kc, vc
+
+
+def test_noalloc_decode_matches_workspace_decode_twice(cuda_ok):
+    from dynamic_block_sparse_nsa_b200 import nsa
+    # A first call of another shape leaves its own contents in the static
+    # scratch: other batch size, lengths shorter than one compressed block (no
+    # compressed key at all) and a different selection count.
+    p0, dev0, kc0, vc0 = _decode_case(nsa, 3, 5000, 4, [5000, 20, 1])
+    assert nsa.workspace_size(p0, nsa.OP_DECODE) > 0
+    out0 = torch.empty(3, p0.Hq, p0.d, dtype=torch.bfloat16, device="cuda")
+    sel0 = torch.empty(3, p0.Hkv, p0.top_n, dtype=torch.int32, device="cuda")
+    assert _c_abi_noalloc(nsa, p0, dev0, kc0, vc0, out0, sel0) == 0
+    nsa.nsa_check()
+
+    p, dev, kc, vc = _decode_case(nsa, 6, 12000, 11, [12000, 9000, 4097, 777, 64, 11999])
+    # the fast decode path is the one that uses the scratch
+    assert nsa.workspace_size(p, nsa.OP_DECODE) > 0
     ref_out, ref_sel = nsa.nsa_decode(p, dev["q"], dev["k"], dev["v"], dev["seq_lens"], kc, vc,
                                       dev["w_gate"])
     nsa.nsa_check()
@@ -46,6 +63,26 @@ def test_noalloc_decode_matches_workspace_decode_twice(cuda_ok):
         nsa.nsa_check()
         parity.check_output(out.float().cpu().numpy(), ref_out.float().cpu().numpy(), "bf16")
         assert torch.equal(sel, ref_sel)
+
+    # the first shape again, after the second one wrote over the scratch
+    ref0, rsel0 = nsa.nsa_decode(p0, dev0["q"], dev0["k"], dev0["v"], dev0["seq_lens"], kc0, vc0,
+                                 dev0["w_gate"])
+    assert _c_abi_noalloc(nsa, p0, dev0, kc0, vc0, out0, sel0) == 0
+    nsa.nsa_check()
+    parity.check_output(out0.float().cpu().numpy(), ref0.float().cpu().numpy(), "bf16")
+    assert torch.equal(sel0, rsel0)
+
+
+def test_noalloc_python_wrapper(cuda_ok):
+    from dynamic_block_sparse_nsa_b200 import nsa
+    p, dev, kc, vc = _decode_case(nsa, 2, 3000, 12, [3000, 1500])
+    ref_out, ref_sel = nsa.nsa_decode(p, dev["q"], dev["k"], dev["v"], dev["seq_lens"], kc, vc,
+                                      dev["w_gate"])
+    out, sel = nsa.nsa_decode_noalloc(p, dev["q"], dev["k"], dev["v"], dev["seq_lens"], kc, vc,
+                                      dev["w_gate"])
+    nsa.nsa_check()
+    parity.check_output(out.float().cpu().numpy(), ref_out.float().cpu().numpy(), "bf16")
+    assert torch.equal(sel, ref_sel)
 
 
 def test_noalloc_rejects_shapes_beyond_the_static_scratch(cuda_ok):
