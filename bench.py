@@ -381,34 +381,97 @@ def run_decode(w, K, W, ws, rank, local, e2e=True, use_graph=True):
     step_bytes, union_bytes, parts = decode_work(w, lens_l, sel_h)
     res.update(work=step_bytes, union=union_bytes, parts=parts)
     if e2e:
-        # through the public call with host buffers: H2D of the step's query and
-        # lengths from pinned memory, D2H of the output and selection, every
-        # step; the KV caches are device-resident state (as in serving), not
-        # per-step inputs. The copies are captured with the call into the same
-        # CUDA graph as the device-only timing (one graph of K steps).
-        q_h = q.cpu().pin_memory()
-        lens_h = lens.cpu().pin_memory()
-        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        sel_h_p = torch.empty(sel.shape, dtype=sel.dtype).pin_memory()
-
-        def e2e_step():
-            q.copy_(q_h, non_blocking=True)
-            lens.copy_(lens_h, non_blocking=True)
-            step()
-            out_h.copy_(out, non_blocking=True)
-            sel_h_p.copy_(sel, non_blocking=True)
-
-        for _ in range(3):
-            e2e_step()
-        torch.cuda.synchronize()
-        barrier(ws)
-        res["e2e_ms"] = _run_steps(e2e_step, K, use_graph)[0]
-        barrier(ws)
-        res["e2e_how"] = ("K steps of (H2D query + lengths, nsa_decode, D2H output + selection) "
-                          + ("captured in one CUDA graph" if use_graph else "as eager launches"))
-        res["h2d"] = q_h.numel() * q_h.element_size() + lens_h.numel() * 4
-        res["d2h"] = out_h.numel() * out_h.element_size() + sel_h_p.numel() * 4
+        res.update(decode_e2e(p, inp, kc, vc, ws_buf, q, lens, out, sel, K, ws, use_graph))
     return res
+
+
+def decode_e2e(p, inp, kc, vc, ws_buf, q, lens, out, sel, K, ws, use_graph):
+    """End to end through the public call with host buffers, as a serving loop
+    runs it: every step copies its query and lengths from pinned host memory
+    and reads its output and selection back; the KV caches are device-resident
+    state, not per-step inputs. Query and output buffers are double-buffered so
+    the H2D of step i + 1 (one copy stream) and the D2H of step i - 1 (another)
+    overlap the decode of step i; every copy of the K steps is inside the timed
+    region. Captured as one CUDA graph (streams forked and joined with events)."""
+    from dynamic_block_sparse_nsa_b200 import nsa
+    q_h = q.cpu().pin_memory()
+    lens_h = lens.cpu().pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    sel_h = torch.empty(sel.shape, dtype=sel.dtype).pin_memory()
+    qd = [q, torch.empty_like(q)]
+    ld = [lens, torch.empty_like(lens)]
+    od = [out, torch.empty_like(out)]
+    sd = [sel, torch.empty_like(sel)]
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def run(nsteps):
+        main = torch.cuda.current_stream()  # the capture stream while capturing
+        ev_in = [torch.cuda.Event() for _ in range(nsteps)]
+        ev_done = [torch.cuda.Event() for _ in range(nsteps)]
+        ev_read = [torch.cuda.Event() for _ in range(nsteps)]
+        start = torch.cuda.Event()
+        start.record(main)
+        s_in.wait_event(start)
+        s_out.wait_event(start)
+
+        def h2d(i):
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_done[i - 2])  # buffer i % 2 no longer read
+                qd[i % 2].copy_(q_h, non_blocking=True)
+                ld[i % 2].copy_(lens_h, non_blocking=True)
+                ev_in[i].record(s_in)
+
+        h2d(0)
+        for i in range(nsteps):
+            if i + 1 < nsteps:
+                h2d(i + 1)
+            main.wait_event(ev_in[i])
+            if i >= 2:
+                main.wait_event(ev_read[i - 2])  # output buffer i % 2 read back
+            nsa.nsa_decode(p, qd[i % 2], inp["k"], inp["v"], ld[i % 2], kc, vc, inp["w_gate"],
+                           out=od[i % 2], sel_idx=sd[i % 2], ws=ws_buf)
+            ev_done[i].record(main)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_done[i])
+                out_h.copy_(od[i % 2], non_blocking=True)
+                sel_h.copy_(sd[i % 2], non_blocking=True)
+                ev_read[i].record(s_out)
+        main.wait_event(ev_read[nsteps - 1])
+        main.wait_stream(s_in)
+
+    run(4)
+    torch.cuda.synchronize()
+    g = None
+    if use_graph:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            run(K)
+        g.replay()
+        torch.cuda.synchronize()
+    barrier(ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    if g is not None:
+        g.replay()
+    else:
+        run(K)
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(ws)
+    ms = e0.elapsed_time(e1)
+    del g
+    # the last step's output read back equals the device-only run's
+    if not torch.equal(out_h, out.cpu()):
+        raise RuntimeError("decode end-to-end output differs from the device-resident run")
+    return {"e2e_ms": ms,
+            "e2e_how": ("K steps of (H2D query + lengths from pinned memory, nsa_decode, D2H "
+                        "output + selection), double-buffered: the H2D of step i + 1 and the D2H "
+                        "of step i - 1 on two copy streams overlap the decode of step i; "
+                        + ("one CUDA graph" if use_graph else "eager launches")),
+            "h2d": q_h.numel() * q_h.element_size() + lens_h.numel() * 4,
+            "d2h": out_h.numel() * out_h.element_size() + sel_h.numel() * 4}
 
 
 def run_prefill(w, K, W, ws, rank, local, e2e=True):

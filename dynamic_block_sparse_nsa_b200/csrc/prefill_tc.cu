@@ -17,7 +17,7 @@
 //              registers; a selection block j collects compressed blocks
 //              4j-1 .. 4j+3;
 //           4. top-n per token with block 0 forced (ties to the lower index);
-//           5. g_cmp * o_cmp + g_win * o_win (fp32) and g_slc to the workspace.
+//           5. g_cmp * o_cmp + g_win * o_win (bf16) and g_slc to the workspace.
 //  pf_slc   persistent; one unit per (sequence, token, KV head): the selected
 //           blocks, two per 128-key tile, give S^T = K_sel Q^T (M = 128 keys,
 //           N = 16 heads); an exact softmax over all selected keys per head;
@@ -47,14 +47,14 @@ constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr int kMaxSel = 16;       // top_n bound: 8 tiles of two blocks in pf_slc
 constexpr int kMainStagesMax = 4;
 constexpr int kMainThreads = 320; // TMA, MMA, 8 softmax warps
-constexpr int kSlcThreads = 256;  // K TMA, V TMA, MMA, TMEM owner, 4 softmax warps
-constexpr int kSlcKStages = 3, kSlcVStages = 2;
+constexpr int kSlcThreads = 256;  // K/V TMA, Q/acc loads, MMA, TMEM owner, 4 softmax warps
+constexpr int kSlcStages = 5;     // one ring of K and V tiles, in the order the MMAs use them
 constexpr uint32_t kQ16 = 4096;   // 16 rows x 128 d bf16
 constexpr uint32_t kNegInf = 0xff800000u;  // bits of -inf
 
 struct PfArgs {
   const float* w_gate;
-  float* acc;    // [B, T, Hq, d]: g_cmp * o_cmp + g_win * o_win
+  __nv_bfloat16* acc;  // [B, T, Hq, d]: g_cmp * o_cmp + g_win * o_win
   float* gslc;   // [B, T, Hq]
   int32_t* sel;  // [B, T, Hkv, n]
   __nv_bfloat16* out;
@@ -609,9 +609,13 @@ __global__ void __launch_bounds__(kMainThreads, 1)
           dst[0] = pk[0];
           dst[1] = pk[1];
         } else {
-          float4* dst = reinterpret_cast<float4*>(a.acc + orow + c16 * 16);
+          uint4 pk[2];
+          uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) dst[e] = make_float4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
+          for (int e = 0; e < 8; ++e) pw[e] = ptx::pack_bf16(o[2 * e], o[2 * e + 1]);
+          uint4* dst = reinterpret_cast<uint4*>(a.acc + orow + c16 * 16);
+          dst[0] = pk[0];
+          dst[1] = pk[1];
         }
       }
     }
@@ -630,8 +634,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
 // ============================================================================
 
 struct SlcBars {
-  uint64_t kfull[kSlcKStages], kempty[kSlcKStages];
-  uint64_t vfull[kSlcVStages], vempty[kSlcVStages];
+  uint64_t full[kSlcStages], empty[kSlcStages];
   uint64_t q_full[2], q_empty[2], s_full[2], p_full[2], o_full[2], o_free[2], fin;
   uint64_t a_full[2], a_empty[2];
   uint32_t tmem;
@@ -639,7 +642,7 @@ struct SlcBars {
   alignas(16) float red[2][4][G];
 };
 
-constexpr uint32_t kAccBytes = G * D * 4;  // one unit's acc rows
+constexpr uint32_t kAccBytes = G * D * 2;  // one unit's acc rows (bf16)
 constexpr uint32_t kAccSlot = kAccBytes + 256;  // + its 16 gates
 
 // TMEM columns of pf_slc: S^T of unit parity p at 128 p (8 tiles x 16 heads),
@@ -703,11 +706,10 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
                   const __grid_constant__ CUtensorMap tv64, const PfArgs a) {
   extern __shared__ unsigned char smraw[];
   unsigned char* base = align1024(smraw);
-  unsigned char* kring = base;                               // 3 x 32 KB
-  unsigned char* vring = kring + kSlcKStages * TILE;         // 2 x 32 KB
-  unsigned char* sP = vring + kSlcVStages * TILE;            // 32 KB: [1024 keys][16] SW32
+  unsigned char* ring = base;                                // kSlcStages x 32 KB
+  unsigned char* sP = ring + kSlcStages * TILE;              // 32 KB: [1024 keys][16] SW32
   unsigned char* sQ = sP + 32768;                            // 2 x 4 KB
-  unsigned char* sA = sQ + 2 * kQ16;                         // 2 x (acc 8 KB + gates)
+  unsigned char* sA = sQ + 2 * kQ16;                         // 2 x (acc 4 KB + gates)
   SlcBars* bars = reinterpret_cast<SlcBars*>(sA + 2 * kAccSlot);
   volatile int* abort = &bars->abort;
 
@@ -716,13 +718,9 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
   const long long U = BT * a.Hkv;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kSlcKStages; ++i) {
-      ptx::mbar_init(&bars->kfull[i], 4);  // one arrival per issuing lane
-      ptx::mbar_init(&bars->kempty[i], 1);
-    }
-    for (int i = 0; i < kSlcVStages; ++i) {
-      ptx::mbar_init(&bars->vfull[i], 4);
-      ptx::mbar_init(&bars->vempty[i], 1);
+    for (int i = 0; i < kSlcStages; ++i) {
+      ptx::mbar_init(&bars->full[i], 4);  // one arrival per issuing lane
+      ptx::mbar_init(&bars->empty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(&bars->q_full[i], 1);
@@ -755,95 +753,118 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
     t = (int)(bt % a.T);
   };
 
-  if (warp == 0 || warp == 1) {
-    // ---------------- TMA producers: warp 0 K (and Q), warp 1 V ----------------
-    // Lane L < 4 issues box L of every tile (selected block L / 2, d-half L % 2):
-    // four issuing threads keep enough bulk copies moving to reach the SM's
-    // ingest rate. A tile's full barrier takes one arrival per lane.
+  if (warp == 0) {
+    // ---------------- TMA producer of the K / V ring ----------------
+    // One ring in the order the MMA warp consumes it: the K tiles of unit k,
+    // then the V tiles of unit k - 1 (whose softmax runs meanwhile), so no
+    // slot waits for the other operand's stream. Lane L < 4 issues box L of
+    // every tile (selected block L / 2, d-half L % 2): four issuing threads
+    // keep enough bulk copies moving to reach the SM's ingest rate. A tile's
+    // full barrier takes one arrival per lane.
     if (lane < 4) {
-      const bool isk = warp == 0;
-      const CUtensorMap* m = isk ? &tk64 : &tv64;
       if (lane == 0) {
-        ptx::prefetch_tmap(m);
-        if (isk) ptx::prefetch_tmap(&tq16);
+        ptx::prefetch_tmap(&tk64);
+        ptx::prefetch_tmap(&tv64);
       }
-      const uint64_t keep = ptx::policy_evict_last(), once = ptx::policy_evict_first();
-      const int NS = isk ? kSlcKStages : kSlcVStages;
-      uint64_t* full = isk ? bars->kfull : bars->vfull;
-      uint64_t* empty = isk ? bars->kempty : bars->vempty;
-      unsigned char* ringp = isk ? kring : vring;
+      const uint64_t keep = ptx::policy_evict_last();
       const int hb = lane >> 1, dh = lane & 1;
-      int c = 0, k = 0;
+      int c = 0;
       bool ok = true;
-      SelRow cur, nxt;
+      SelRow cur, prv, nxt;
+      int pb = 0, pt = 0, pg = 0;  // unit k - 1
       auto row_of = [&](long long uu) {
         int b, t, g;
         unit_of(uu, b, t, g);
         return a.sel + ((size_t)(b * a.T + t) * a.Hkv + g) * a.n;
       };
+      // the tiles of one unit's K or V, two selected blocks per tile (a
+      // missing second block reads past the tensor: zero fill)
+      auto tiles = [&](const CUtensorMap* m, const SelRow& sr, int b, int g) {
+        const int nsel = sr.count();
+        for (int i = 0; ok && i < (nsel + 1) / 2; ++i) {
+          const int st = c % kSlcStages;
+          if (c >= kSlcStages &&
+              !wait_or_abort(&bars->empty[st], (uint32_t)(((c / kSlcStages) - 1) & 1), abort,
+                             a.err)) {
+            ok = false;
+            break;
+          }
+          unsigned char* dst = ring + st * TILE + dh * ATOM + hb * (ATOM / 2);
+          const int z = (2 * i + hb < nsel) ? b * a.T + SB * sr.blk(2 * i + hb) : (int)BT;
+          ptx::mbar_arrive_expect_tx(&bars->full[st], ATOM / 2);
+          ptx::tma_load_3d(dst, m, &bars->full[st], dh * 64, g, z, keep);
+          ++c;
+        }
+      };
       if (blockIdx.x < U) cur.load(row_of(blockIdx.x), a.n);
-      for (long long u = blockIdx.x; ok && u < U; u += gridDim.x, ++k) {
+      long long u = blockIdx.x;
+      for (int k = 0; ok && u < U; u += gridDim.x, ++k) {
         int b, t, g;
         unit_of(u, b, t, g);
         if (u + gridDim.x < U) nxt.load(row_of(u + gridDim.x), a.n);
-        const int nsel = cur.count();
-        if (isk && lane == 0) {
-          const int qs = k & 1;
-          if (k >= 2 && !wait_or_abort(&bars->q_empty[qs], (uint32_t)(((k >> 1) - 1) & 1), abort,
-                                       a.err)) {
-            ok = false;
-            break;
-          }
-          unsigned char* qd = sQ + qs * kQ16;
-          ptx::mbar_arrive_expect_tx(&bars->q_full[qs], kQ16);
-          ptx::tma_load_3d(qd, &tq16, &bars->q_full[qs], 0, g * G, b * a.T + t, once);
-          ptx::tma_load_3d(qd + kQ16 / 2, &tq16, &bars->q_full[qs], 64, g * G, b * a.T + t, once);
-          // the unit's acc rows and g_slc, for the epilogue
-          if (k >= 2 && !wait_or_abort(&bars->a_empty[qs], (uint32_t)(((k >> 1) - 1) & 1), abort,
-                                       a.err)) {
-            ok = false;
-            break;
-          }
-          const size_t row0 = (size_t)(b * a.T + t) * a.Hq + g * G;
-          unsigned char* ad = sA + qs * kAccSlot;
-          ptx::mbar_arrive_expect_tx(&bars->a_full[qs], kAccBytes + G * 4);
-          ptx::bulk_load(ad, a.acc + row0 * D, kAccBytes, &bars->a_full[qs]);
-          ptx::bulk_load(ad + kAccBytes, a.gslc + row0, G * 4, &bars->a_full[qs]);
-        }
-        for (int i = 0; i < (nsel + 1) / 2; ++i) {
-          const int st = c % NS;
-          if (c >= NS && !wait_or_abort(&empty[st], (uint32_t)(((c / NS) - 1) & 1), abort, a.err)) {
-            ok = false;
-            break;
-          }
-          unsigned char* dst = ringp + st * TILE + dh * ATOM + hb * (ATOM / 2);
-          // a missing second block reads past the tensor: zero fill
-          const int z = (2 * i + hb < nsel) ? b * a.T + SB * cur.blk(2 * i + hb) : (int)BT;
-          ptx::mbar_arrive_expect_tx(&full[st], ATOM / 2);
-          ptx::tma_load_3d(dst, m, &full[st], dh * 64, g, z, keep);
-          ++c;
-        }
+        tiles(&tk64, cur, b, g);
+        if (k >= 1) tiles(&tv64, prv, pb, pg);
+        prv = cur;
+        pb = b;
+        pt = t;
+        pg = g;
         cur = nxt;
       }
-      for (int kq = max(0, c - NS); kq < c; ++kq)
-        if (!ptx::mbar_wait(&full[kq % NS], (uint32_t)((kq / NS) & 1), kWaitNs))
+      if (ok && u != (long long)blockIdx.x) tiles(&tv64, prv, pb, pg);
+      (void)pt;
+      for (int kq = max(0, c - kSlcStages); kq < c; ++kq)
+        if (!ptx::mbar_wait(&bars->full[kq % kSlcStages], (uint32_t)((kq / kSlcStages) & 1),
+                            kWaitNs))
           atomicOr(a.err, kErrTimeout);
-      if (isk && lane == 0)
-        for (int kq = max(0, k - 2); kq < k; ++kq) {
-          if (!ptx::mbar_wait(&bars->q_full[kq & 1], (uint32_t)((kq >> 1) & 1), kWaitNs))
-            atomicOr(a.err, kErrTimeout);
-          if (!ptx::mbar_wait(&bars->a_full[kq & 1], (uint32_t)((kq >> 1) & 1), kWaitNs))
-            atomicOr(a.err, kErrTimeout);
+    }
+  } else if (warp == 1) {
+    // ---------------- Q rows, acc rows and g_slc of each unit ----------------
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tq16);
+      const uint64_t once = ptx::policy_evict_first();
+      int k = 0;
+      bool ok = true;
+      for (long long u = blockIdx.x; u < U; u += gridDim.x, ++k) {
+        int b, t, g;
+        unit_of(u, b, t, g);
+        const int qs = k & 1;
+        if (k >= 2 && !wait_or_abort(&bars->q_empty[qs], (uint32_t)(((k >> 1) - 1) & 1), abort,
+                                     a.err)) {
+          ok = false;
+          break;
         }
+        unsigned char* qd = sQ + qs * kQ16;
+        ptx::mbar_arrive_expect_tx(&bars->q_full[qs], kQ16);
+        ptx::tma_load_3d(qd, &tq16, &bars->q_full[qs], 0, g * G, b * a.T + t, once);
+        ptx::tma_load_3d(qd + kQ16 / 2, &tq16, &bars->q_full[qs], 64, g * G, b * a.T + t, once);
+        // the unit's acc rows and g_slc, for the epilogue
+        if (k >= 2 && !wait_or_abort(&bars->a_empty[qs], (uint32_t)(((k >> 1) - 1) & 1), abort,
+                                     a.err)) {
+          ok = false;
+          break;
+        }
+        const size_t row0 = (size_t)(b * a.T + t) * a.Hq + g * G;
+        unsigned char* ad = sA + qs * kAccSlot;
+        ptx::mbar_arrive_expect_tx(&bars->a_full[qs], kAccBytes + G * 4);
+        ptx::bulk_load(ad, a.acc + row0 * D, kAccBytes, &bars->a_full[qs]);
+        ptx::bulk_load(ad + kAccBytes, a.gslc + row0, G * 4, &bars->a_full[qs]);
+      }
+      (void)ok;
+      for (int kq = max(0, k - 2); kq < k; ++kq) {
+        if (!ptx::mbar_wait(&bars->q_full[kq & 1], (uint32_t)((kq >> 1) & 1), kWaitNs))
+          atomicOr(a.err, kErrTimeout);
+        if (!ptx::mbar_wait(&bars->a_full[kq & 1], (uint32_t)((kq >> 1) & 1), kWaitNs))
+          atomicOr(a.err, kErrTimeout);
+      }
     }
   } else if (warp == 2) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       const uint32_t is16 = tc::idesc_bf16(128, 16, false, false);
       const uint32_t ipv = tc::idesc_bf16(128, 16, true, true);
-      const uint32_t kr = ptx::smem_u32(kring), vr = ptx::smem_u32(vring);
+      const uint32_t rr = ptx::smem_u32(ring);
       const uint32_t pb0 = ptx::smem_u32(sP), qb = ptx::smem_u32(sQ);
-      int ck = 0, cv = 0, k = 0, prev_tiles = 0;
+      int c = 0, k = 0, prev_tiles = 0;
       bool ok = true;
       auto pv = [&](int kk, int ntile) {
         const int pp = kk & 1;
@@ -852,18 +873,18 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
           ok = ok && wait_or_abort(&bars->o_free[pp], (uint32_t)(((kk >> 1) - 1) & 1), abort, a.err);
         tc::fence_after_sync();
         for (int i = 0; ok && i < ntile; ++i) {
-          const int st = cv % kSlcVStages;
-          ok = wait_or_abort(&bars->vfull[st], (uint32_t)((cv / kSlcVStages) & 1), abort, a.err);
+          const int st = c % kSlcStages;
+          ok = wait_or_abort(&bars->full[st], (uint32_t)((c / kSlcStages) & 1), abort, a.err);
           tc::fence_after_sync();
           if (!ok) break;
-          const uint32_t vb = vr + st * TILE;
+          const uint32_t vb = rr + st * TILE;
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)
             tc::mma_ss(tmem + kSlcO + pp * 16, mnmaj(vb, ks),
                        tc::sdesc(pb0 + i * 4096 + ks * 512, 16, 256, tc::kSw32), ipv,
                        (i > 0 || ks > 0));
-          tc::commit(&bars->vempty[st]);
-          ++cv;
+          tc::commit(&bars->empty[st]);
+          ++c;
         }
         tc::commit(&bars->o_full[pp]);
       };
@@ -882,17 +903,17 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
         tc::fence_after_sync();
         const uint32_t qd = qb + pk * kQ16;
         for (int i = 0; ok && i < ntile; ++i) {
-          const int st = ck % kSlcKStages;
-          ok = wait_or_abort(&bars->kfull[st], (uint32_t)((ck / kSlcKStages) & 1), abort, a.err);
+          const int st = c % kSlcStages;
+          ok = wait_or_abort(&bars->full[st], (uint32_t)((c / kSlcStages) & 1), abort, a.err);
           tc::fence_after_sync();
           if (!ok) break;
-          const uint32_t kb = kr + st * TILE;
+          const uint32_t kb = rr + st * TILE;
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks)
             tc::mma_ss(tmem + pk * 128 + i * 16, kmaj(kb, ks, ATOM), kmaj(qd, ks, kQ16 / 2), is16,
                        ks > 0);
-          tc::commit(&bars->kempty[st]);
-          ++ck;
+          tc::commit(&bars->empty[st]);
+          ++c;
         }
         tc::commit(&bars->q_empty[pk]);
         tc::commit(&bars->s_full[pk]);
@@ -918,12 +939,13 @@ __global__ void __launch_bounds__(kSlcThreads, 1)
       uint32_t u[16];
       tc::ld16_sync(tl + kSlcO + pp * 16, u);
       wait_or_abort(&bars->a_full[pp], (uint32_t)((kk >> 1) & 1), abort, a.err);
-      const float* accs = reinterpret_cast<const float*>(sA + pp * kAccSlot);
+      const __nv_bfloat16* accs = reinterpret_cast<const __nv_bfloat16*>(sA + pp * kAccSlot);
+      const float* gsl = reinterpret_cast<const float*>(sA + pp * kAccSlot + kAccBytes);
       __nv_bfloat16* o = a.out + ((size_t)(pb * a.T + pt) * a.Hq + pg * G) * D + r;
 #pragma unroll
       for (int hh = 0; hh < G; ++hh)
         o[hh * D] = __float2bfloat16_rn(
-            fmaf(accs[G * D + hh] / pl[hh], __uint_as_float(u[hh]), accs[hh * D + r]));
+            fmaf(gsl[hh] / pl[hh], __uint_as_float(u[hh]), __bfloat162float(accs[hh * D + r])));
       tc::fence_before_sync();
       ptx::mbar_arrive(&bars->o_free[pp]);
       ptx::mbar_arrive(&bars->a_empty[pp]);
@@ -1054,7 +1076,7 @@ size_t main_smem(int stages, int nblk) {
 }
 
 size_t slc_smem() {
-  return 1024 + (kSlcKStages + kSlcVStages) * (size_t)TILE + 32768 + 2 * kQ16 + 2 * kAccSlot +
+  return 1024 + kSlcStages * (size_t)TILE + 32768 + 2 * kQ16 + 2 * kAccSlot +
          sizeof(SlcBars);
 }
 
@@ -1080,7 +1102,7 @@ bool prefill_tc_eligible(const nsa_params& p) {
 
 size_t prefill_tc_ws_bytes(const nsa_params& p) {
   const size_t rows = (size_t)p.B * p.T * p.Hq;
-  return align256(rows * D * 4) + align256(rows * 4) +
+  return align256(rows * D * 2) + align256(rows * 4) +
          align256((size_t)p.B * p.T * p.Hkv * p.top_n * 4);
 }
 
@@ -1090,8 +1112,8 @@ cudaError_t launch_prefill_tc(const nsa_params& p, const void* q, const void* k,
   PfArgs a{};
   const size_t rows = (size_t)p.B * p.T * p.Hq;
   unsigned char* w = static_cast<unsigned char*>(ws);
-  a.acc = reinterpret_cast<float*>(w);
-  w += align256(rows * D * 4);
+  a.acc = reinterpret_cast<__nv_bfloat16*>(w);
+  w += align256(rows * D * 2);
   a.gslc = reinterpret_cast<float*>(w);
   w += align256(rows * 4);
   a.sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(w);
