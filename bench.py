@@ -480,7 +480,8 @@ def run_prefill(w, K, W, ws, rank, local, e2e=True):
     dt = inputs.DTYPES[w["dtype"]]
     p = nsa.params(w["B"], w["T"], w["Hq"], w["Hkv"], w["d"], cmp_block=w["cmp_block"],
                    cmp_stride=w["cmp_stride"], sel_block=w["sel_block"], top_n=w["top_n"],
-                   window=w["window"], dtype=dt)
+                   window=w["window"], dtype=dt, sel_mode=w.get("sel_mode", 0),
+                   top_p=w.get("top_p", 0.0))
     Nc = nsa.num_cmp_blocks(w["T"], w["cmp_block"], w["cmp_stride"])
     kc = torch.empty(w["B"], Nc, w["Hkv"], w["d"], dtype=dt, device="cuda")
     vc = torch.empty_like(kc)

@@ -129,6 +129,14 @@ cudaError_t launch_prefill_tc(const nsa_params& p, const void* q, const void* k,
                               const void* kc, const void* vc, const float* w_gate, void* out,
                               int32_t* sel_out, void* ws, unsigned* err, cudaStream_t stream);
 
+// Quest-style block selection (nsa_params.sel_mode = 1) for the tensor-core
+// prefill: per-block key extremes, block scores, top-n into `sel`
+// [B, T, Hkv, n]. Its workspace follows the prefill's own.
+bool quest_tc_supported(const nsa_params& p);
+size_t quest_ws_bytes(const nsa_params& p);
+cudaError_t launch_quest_select(const nsa_params& p, const void* q, const void* k, int32_t* sel,
+                                void* ws, cudaStream_t stream);
+
 // Kernel trace: bracket a launch with events when tracing is on.
 void trace_begin(const char* name, cudaStream_t stream);
 void trace_end(cudaStream_t stream);

@@ -1092,7 +1092,8 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 bool prefill_tc_eligible(const nsa_params& p) {
   if (p.dtype != NSA_DTYPE_BF16 || p.d != D || p.Hkv < 1 || p.Hq != G * p.Hkv) return false;
-  if (p.sel_mode != 0) return false;  // Quest-bound selection: CUDA-core path
+  if (p.sel_mode == 1 && (p.top_p != 0.f || !quest_tc_supported(p))) return false;
+  if (p.sel_mode != 0 && p.sel_mode != 1) return false;
   if (p.cmp_block != CL || p.cmp_stride != CS || p.sel_block != SB) return false;
   if (p.top_n < 1 || p.top_n > kMaxSel || p.window < 1) return false;
   if ((long long)p.B * p.T >= (1ll << 30)) return false;
@@ -1103,7 +1104,8 @@ bool prefill_tc_eligible(const nsa_params& p) {
 size_t prefill_tc_ws_bytes(const nsa_params& p) {
   const size_t rows = (size_t)p.B * p.T * p.Hq;
   return align256(rows * D * 2) + align256(rows * 4) +
-         align256((size_t)p.B * p.T * p.Hkv * p.top_n * 4);
+         align256((size_t)p.B * p.T * p.Hkv * p.top_n * 4) +
+         (p.sel_mode == 1 ? quest_ws_bytes(p) : 0);
 }
 
 cudaError_t launch_prefill_tc(const nsa_params& p, const void* q, const void* k, const void* v,
@@ -1117,6 +1119,8 @@ cudaError_t launch_prefill_tc(const nsa_params& p, const void* q, const void* k,
   a.gslc = reinterpret_cast<float*>(w);
   w += align256(rows * 4);
   a.sel = sel_out ? sel_out : reinterpret_cast<int32_t*>(w);
+  w += align256((size_t)p.B * p.T * p.Hkv * p.top_n * 4);
+  const bool quest = p.sel_mode == 1;  // the selection comes from the block bounds
   a.w_gate = w_gate;
   a.out = static_cast<__nv_bfloat16*>(out);
   a.err = err;
@@ -1135,7 +1139,7 @@ cudaError_t launch_prefill_tc(const nsa_params& p, const void* q, const void* k,
   for (int i = 0; i < 3; ++i) a.fixed_gates[i] = p.fixed_gates[i];
   const bool fixed = p.gate_mode == 1;
   const bool slc_branch = !(fixed && p.fixed_gates[1] == 0.f);
-  a.need_sel = slc_branch || sel_out != nullptr;
+  a.need_sel = !quest && (slc_branch || sel_out != nullptr);
   a.run_cmp = !(fixed && p.fixed_gates[0] == 0.f) || a.need_sel;
   a.run_win = !(fixed && p.fixed_gates[2] == 0.f);
   a.direct_out = !slc_branch;
@@ -1159,6 +1163,9 @@ cudaError_t launch_prefill_tc(const nsa_params& p, const void* q, const void* k,
   if (!ok) return cudaErrorInvalidValue;
 
   cudaError_t e;
+  if (quest && (slc_branch || sel_out != nullptr) &&
+      (e = launch_quest_select(p, q, k, a.sel, w, stream)) != cudaSuccess)
+    return e;
   const size_t sm1 = main_smem(a.stages, a.nblk);
   if ((e = ensure_dyn_smem((const void*)pf_main_kernel, 227 * 1024)) != cudaSuccess) return e;
   {

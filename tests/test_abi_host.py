@@ -135,7 +135,11 @@ def test_selection_mode_checks():
     bad = nsa.params(1, 1024, 4, 1, 64, sel_mode=1, top_p=0.5)
     assert nsa.LIB.nsa_workspace_size(ctypes.byref(bad), nsa.OP_PREFILL, ctypes.byref(n)) == 1
     assert b"top_p" in nsa.LIB.nsa_last_error_detail()
-    # the fast paths leave the Quest bound to the CUDA-core path
+    # the tensor-core prefill takes the Quest bound with a block-bounds table and
+    # a score matrix in its workspace
     fast = nsa.params(1, 8192, 64, 4, 128)
-    assert nsa.workspace_size(fast, nsa.OP_PREFILL) > 0
-    assert nsa.workspace_size(nsa.params(1, 8192, 64, 4, 128, sel_mode=1), nsa.OP_PREFILL) == 0
+    base = nsa.workspace_size(fast, nsa.OP_PREFILL)
+    assert base > 0
+    nblk = 8192 // 64
+    quest = nsa.workspace_size(nsa.params(1, 8192, 64, 4, 128, sel_mode=1), nsa.OP_PREFILL)
+    assert quest >= nblk * 4 * 2 * 128 * 2 + 8192 * 4 * nblk * 4

@@ -157,25 +157,42 @@ def test_decode_bf16_fast_path_edges(over, lens):
     assert want <= names, names
 
 
-# Quest-style block-bound selection (sel_mode 1, the pages' selection ablation):
-# the CUDA-core path for prefill and decode against the oracle's score_mode 2.
-@pytest.mark.parametrize("name,over", [
-    ("nsa_prefill_bf16_t8192", dict(T=300, Hq=16, Hkv=1, sel_mode=1)),
-    ("nsa_prefill_f32_t1024", dict(T=400, sel_mode=1)),
+# Quest-style block-bound selection (sel_mode 1, the pages' selection ablation)
+# against the oracle's score_mode 2: bf16 with d = 128 and 16 heads per KV head
+# runs the block-bounds table, its scores and top-n ahead of the tensor-core
+# kernels; other shapes and fp32 run the CUDA-core row kernel.
+@pytest.mark.parametrize("name,over,tc", [
+    ("nsa_prefill_bf16_t8192", dict(T=300, Hq=16, Hkv=1, sel_mode=1), True),
+    ("nsa_prefill_bf16_t8192", dict(B=2, T=1403, Hq=32, Hkv=2, top_n=7, window=200,
+                                    sel_mode=1), True),
+    ("nsa_prefill_bf16_t8192", dict(T=2100, Hq=16, Hkv=1, qkv_scale=1.0, top_n=9,
+                                    sel_mode=1), True),
+    ("nsa_prefill_bf16_t8192", dict(T=700, Hq=16, Hkv=1, top_n=16, sel_mode=1), True),
+    ("nsa_prefill_bf16_t8192", dict(T=500, Hq=8, Hkv=1, sel_mode=1), False),
+    ("nsa_prefill_f32_t1024", dict(T=400, sel_mode=1), False),
     ("nsa_prefill_f32_t1024", dict(B=2, T=130, Hq=8, Hkv=2, cmp_block=8, cmp_stride=4,
-                                   sel_block=16, top_n=3, window=20, sel_mode=1)),
+                                   sel_block=16, top_n=3, window=20, sel_mode=1), False),
 ])
-def test_prefill_quest_selection(name, over):
+def test_prefill_quest_selection(name, over, tc):
     from dynamic_block_sparse_nsa_b200 import nsa
     w = inputs.workload(name, **over)
     nsa.trace_enable(True, 64)
     try:
-        gc.run_nsa_prefill(w)
+        gc.run_nsa_prefill(w, rows=None if w["T"] <= 1500 else gc.sample_rows(w["T"], 300))
         recs, _ = nsa.trace_records()
         names = {nm for nm, _ in recs}
     finally:
         nsa.trace_enable(False)
-    assert "nsa_rows_simt" in names and "pf_cmp_win" not in names, names
+    if tc:
+        assert {"quest_scores", "quest_select", "pf_cmp_win", "pf_slc_attn"} <= names, names
+        assert "nsa_rows_simt" not in names, names
+    else:
+        assert "nsa_rows_simt" in names and "pf_cmp_win" not in names, names
+
+
+def test_prefill_quest_t8192_sampled_rows():
+    w = inputs.workload("nsa_prefill_bf16_t8192", sel_mode=1)
+    gc.run_nsa_prefill(w, rows=gc.sample_rows(w["T"], 96))
 
 
 def test_decode_quest_selection():
