@@ -424,6 +424,52 @@ __device__ void make_plans(const DecFastArgs& a, StreamPlan* plans, int* lens_s,
   }
 }
 
+// Streams holding unit u's tiles in a stream kernel's plan, from the lengths
+// alone (the split of make_plans): with `pre` the tiles of the units before u,
+// `nt` its own, `total` all tiles and V the streams in use, stream v owns
+// [total v / V, total (v + 1) / V), so tile x lies in stream
+// ceil((x + 1) V / total) - 1.
+__device__ __forceinline__ int stream_of_tile(long long x, long long V, long long total) {
+  return (int)(((x + 1) * V - 1) / total);
+}
+
+// Block-wide: tiles (times Hkv) of the sequences before b and of all
+// sequences, for both stream kernels. `red` holds 4 * (threads / 32) entries.
+// Reads only the sequence lengths (an input of the call).
+__device__ void tile_spans(const DecFastArgs& a, int b, long long (&pre)[2], long long (&total)[2],
+                           long long* red) {
+  long long acc[4] = {0, 0, 0, 0};
+  for (int i = threadIdx.x; i < a.B; i += blockDim.x) {
+    const int L = __ldg(a.seq_lens + i);
+    const long long x0 = (long long)unit_tiles<MODE_CMP>(L, a) * a.Hkv;
+    const long long x1 = (long long)unit_tiles<MODE_SW>(L, a) * a.Hkv;
+    acc[2] += x0;
+    acc[3] += x1;
+    if (i < b) {
+      acc[0] += x0;
+      acc[1] += x1;
+    }
+  }
+  const int nw = blockDim.x >> 5, w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc[k] += __shfl_xor_sync(0xffffffffu, acc[k], o);
+    if (lane == 0) red[k * nw + w] = acc[k];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    long long v = 0;
+    for (int i = 0; i < nw; ++i) v += red[k * nw + i];
+    acc[k] = v;
+  }
+  pre[0] = acc[0];
+  pre[1] = acc[1];
+  total[0] = acc[2];
+  total[1] = acc[3];
+}
+
 // ---------------------------------------------------------------------------
 // the stream kernel
 // ---------------------------------------------------------------------------
@@ -516,7 +562,15 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1)
   int* lens_s = abort_flag + 1;  // [LENS_CAP]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  ptx::grid_dep_wait();  // the previous kernel's writes (inputs, this kernel's workspace)
+  // The compressed-branch kernel's predecessor is the caller's: it waits
+  // before reading anything. The selected/window kernel's predecessors are
+  // this library's own, which waited on the caller's writes already, so its
+  // plan (from the sequence lengths, an input) is made before the wait.
+  if (MODE == MODE_CMP) ptx::grid_dep_wait();
+  // The next decode kernel may be scheduled as this grid's CTAs finish (this
+  // grid is resident in full: one CTA per SM), so its input-only set-up
+  // overlaps this grid's tail; it waits for this grid before reading its output.
+  ptx::grid_dep_launch();
   if (warp == NCW) {
     // the slot ring is idle until the pipeline starts: use it as plan scratch
     make_plans<MODE, NPAIR>(a, plans, lens_s, reinterpret_cast<long long*>(slots),
@@ -532,6 +586,7 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1)
       ptx::prefetch_tmap(&tv);
     }
   }
+  if (MODE != MODE_CMP) ptx::grid_dep_wait();  // the selection, and this kernel's workspace
   __syncthreads();
   const int* lens_p = a.B <= LENS_CAP ? lens_s : a.seq_lens;
   float* part = MODE == MODE_CMP ? a.part1 : a.part3;
@@ -659,11 +714,11 @@ __global__ void __launch_bounds__(STREAM_THREADS, 1)
     }
     if (nvalid > 0) {
       softmax_step_lazy<4>(s, o, m0, m1, l0, l1, nvalid, a.scale_log2, lane);
-      if (MODE == MODE_CMP && RF) {
+      if (MODE == MODE_CMP && RF && a.want_rec) {
         const int u = wk.b * a.Hkv + wk.g;
         record_regs(a.trec + ((long)u * a.tiles_max + 2 * wk.tile + hw) * (G * (1 + a.nbt)), s, m0,
                     m1, lane);
-      } else if (MODE == MODE_CMP) {
+      } else if (MODE == MODE_CMP && a.want_rec) {
         // record of this 32-key sub-tile: running max per head, and per
         // overlapped selection block the exp-sum of its keys. Scratch: this
         // warp's own 32 key rows of the K slot (first TMA box), already read.
@@ -749,6 +804,7 @@ __global__ void __launch_bounds__(SEL_THREADS) dec_select_kernel(const __grid_co
   __shared__ unsigned hist[256];
   __shared__ int cut_bin, cut_above, nsel_s;
   __shared__ __align__(8) uint64_t rec_bar;
+  __shared__ long long span_red[4 * SEL_WARPS];
 
   const int u = blockIdx.x, b = u / a.Hkv, g = u - b * a.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -756,7 +812,25 @@ __global__ void __launch_bounds__(SEL_THREADS) dec_select_kernel(const __grid_co
     ptx::mbar_init(&rec_bar, kRecIssuers);
     ptx::fence_mbar_init();
   }
-  ptx::grid_dep_wait();  // partials, records and stream ranges of dec_cmp_partial
+  // the compressed-branch streams of this unit, from the lengths (before the
+  // wait when the predecessor is this library's kernel, which waited on the
+  // caller's writes)
+  if (!a.after_cmp) ptx::grid_dep_wait();
+  ptx::grid_dep_launch();  // the selected/window kernel's set-up overlaps this one
+  long long pre[2], tot[2];
+  tile_spans(a, b, pre, tot, span_red);
+  const int L = __ldg(a.seq_lens + b);
+  int v_first = 0, v_last = -1;
+  {
+    const int nt = unit_tiles<MODE_CMP>(L, a);
+    if (nt > 0) {
+      const long long V = min((long long)a.grid1, tot[0]);
+      const long long T0 = pre[0] + (long long)g * nt;
+      v_first = stream_of_tile(T0, V, tot[0]);
+      v_last = stream_of_tile(T0 + nt - 1, V, tot[0]);
+    }
+  }
+  ptx::grid_dep_wait();  // partials and records of dec_cmp_partial
   const int nblk = (a.T + a.bs - 1) / a.bs;
   int npow = 2;  // as in sel_dyn_smem
   while (npow < nblk) npow <<= 1;
@@ -766,7 +840,6 @@ __global__ void __launch_bounds__(SEL_THREADS) dec_select_kernel(const __grid_co
   float* fac = reinterpret_cast<float*>(keys + npow);
   float* tsum = fac + (size_t)a.tiles_max * G;
 
-  const int L = __ldg(a.seq_lens + b);
   if (!len_ok(L, a)) {
     for (int x = tid; x < G * D; x += SEL_THREADS)
       reinterpret_cast<__nv_bfloat16*>(a.out)[((long)b * a.Hq + g * G) * D + x] =
@@ -797,9 +870,8 @@ __global__ void __launch_bounds__(SEL_THREADS) dec_select_kernel(const __grid_co
     // lse of the compressed branch per head (warp h): log2 of sum_p 2^m_p l_p
     // over the unit's partials, each lane merging a strided share first
     {
-      const int2 rg = *reinterpret_cast<const int2*>(a.rng1 + 2 * u);
-      const long long first = 2 * ((long long)rg.x + u);
-      const int np = 2 * (rg.y - rg.x + 1);
+      const long long first = 2 * ((long long)v_first + u);
+      const int np = 2 * (v_last - v_first + 1);
       const int h = warp;  // SEL_WARPS == G
       float M = -INFINITY, Ls = 0.f;
       for (int pp = lane; pp < np; pp += 32) {
@@ -1014,6 +1086,132 @@ __global__ void __launch_bounds__(SEL_THREADS) dec_select_kernel(const __grid_co
 }
 
 // ---------------------------------------------------------------------------
+// dec_quest_select
+// ---------------------------------------------------------------------------
+
+// Order-preserving 32-bit image of a float (-0 taken as +0).
+__device__ __forceinline__ unsigned ordered_bits(float x) {
+  const unsigned u = __float_as_uint(x + 0.f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Quest-style selection (EP94 notes §八, the selection ablation; the Quest
+// bound): one CTA per (sequence, KV head). With P = sum over the group's heads
+// of max(q, 0) and N of min(q, 0), block j scores P . kmax_j + N . kmin_j from
+// the caller's block-bounds table (its entry for the block holding the query
+// covers the keys so far); block 0 and the n - 1 best others are kept (ties to
+// the lower index). Replaces dec_select; the compressed branch's partials are
+// merged by dec_combine as usual.
+__global__ void __launch_bounds__(SEL_THREADS) dec_quest_select_kernel(const __grid_constant__ DecFastArgs a) {
+  __shared__ __align__(16) float pn[2 * D];
+  __shared__ float qsc[MAXCAND];
+  __shared__ int sel[MAXSEL];
+  const int u = blockIdx.x, b = u / a.Hkv, g = u - b * a.Hkv;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  // inputs only before the wait when the predecessor is this library's
+  // kernel, which waited on the caller's writes
+  if (!a.after_cmp) ptx::grid_dep_wait();
+  ptx::grid_dep_launch();  // the selected/window kernel's set-up overlaps this one
+  const int L = __ldg(a.seq_lens + b);
+  if (tid < D) {
+    const __nv_bfloat16* qg =
+        reinterpret_cast<const __nv_bfloat16*>(a.q) + ((long)b * a.Hq + g * G) * D + tid;
+    float P = 0.f, N = 0.f;
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float x = __bfloat162float(qg[h * D]);
+      P += fmaxf(x, 0.f);
+      N += fminf(x, 0.f);
+    }
+    pn[tid] = P;
+    pn[D + tid] = N;
+  }
+  ptx::grid_dep_wait();
+  if (!len_ok(L, a)) {
+    for (int x = tid; x < G * D; x += SEL_THREADS)
+      reinterpret_cast<__nv_bfloat16*>(a.out)[((long)b * a.Hq + g * G) * D + x] =
+          __float2bfloat16_rn(0.f);
+    if (a.sel_out)
+      for (int x = tid; x < a.n; x += SEL_THREADS) a.sel_out[(long)u * a.n + x] = -1;
+    if (tid == 0) atomicOr(a.err, kErrSeqLen);
+    return;
+  }
+  __syncthreads();
+  const int ncand = (L - 1) / a.bs + 1;
+  int ns;
+  if (ncand <= a.n) {
+    for (int j = tid; j < ncand; j += SEL_THREADS) sel[j] = j;
+    ns = ncand;
+  } else {
+    // warp w scores blocks w, w + 16, ...: lane l takes table elements 8l .. 8l + 7
+    const __nv_bfloat16* kb = reinterpret_cast<const __nv_bfloat16*>(a.kbounds);
+    float pl[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) pl[i] = pn[8 * lane + i];
+    for (int j = warp; j < ncand; j += SEL_WARPS) {
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(
+                                 kb + (((size_t)b * a.nblk + j) * a.Hkv + g) * 2 * D) +
+                             lane);
+      const __nv_bfloat162* e2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+      float v = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(e2[i]);
+        v = fmaf(pl[2 * i], f.x, v);
+        v = fmaf(pl[2 * i + 1], f.y, v);
+      }
+      v = warp_sum(v);
+      if (lane == 0) qsc[j] = v;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // top n - 1 of blocks 1 .. ncand - 1: per round the warp maximum of the
+      // lanes' best (ordered score bits, ~index) keys; the owner drops it
+      auto rescan = [&](unsigned& bh, unsigned& bl) {
+        bh = 0u;
+        bl = 0u;
+        for (int j = 1 + lane; j < ncand; j += 32) {
+          const unsigned kh = ordered_bits(qsc[j]), kl = ~(unsigned)j;
+          if (kh > bh || (kh == bh && kl > bl)) {
+            bh = kh;
+            bl = kl;
+          }
+        }
+      };
+      unsigned bh, bl;
+      rescan(bh, bl);
+      for (int r = 1; r < a.n; ++r) {
+        const unsigned mh = __reduce_max_sync(0xffffffffu, bh);
+        const unsigned ml = __reduce_max_sync(0xffffffffu, bh == mh ? bl : 0u);
+        const int pick = (int)~ml;
+        if (lane == 0) sel[r] = pick;
+        if (bh == mh && bl == ml) {
+          qsc[pick] = -INFINITY;  // finite scores remain above it (n - 1 < ncand - 1)
+          rescan(bh, bl);
+        }
+      }
+      if (lane == 0) sel[0] = 0;
+    }
+    __syncthreads();
+    // ascending order
+    int v = 0, rank = 0;
+    if (tid < a.n) {
+      v = sel[tid];
+      for (int k = 0; k < a.n; ++k) rank += sel[k] < v;
+    }
+    __syncthreads();
+    if (tid < a.n) sel[rank] = v;
+    ns = a.n;
+  }
+  __syncthreads();
+  for (int x = tid; x < a.n; x += SEL_THREADS) {
+    const int v = x < ns ? sel[x] : -1;
+    a.sel[(long)u * a.n + x] = v;
+    if (a.sel_out) a.sel_out[(long)u * a.n + x] = v;
+  }
+}
+
+// ---------------------------------------------------------------------------
 // dec_combine
 // ---------------------------------------------------------------------------
 
@@ -1080,13 +1278,29 @@ __global__ void __launch_bounds__(CMB_THREADS) dec_combine_kernel(const __grid_c
   const int h = blockIdx.y * CMB_HEADS + hl;
   __shared__ float gate_s[CMB_HEADS * 3];
   __shared__ __align__(16) float contrib[3][CMB_HEADS][D];
-  ptx::grid_dep_wait();  // partials and stream ranges of dec_cmp_partial / dec_sel_win
-  // the length and this branch's stream range in one round trip (the range
-  // words are in bounds whatever the length; they are used only when valid)
+  __shared__ long long span_red[4 * (CMB_THREADS / 32)];
+  // Before the wait (the predecessors are this library's kernels, which
+  // waited on the caller's writes): the streams of this unit's three
+  // branches, from the lengths, and the gates, from the query.
+  long long pre[2], tot[2];
+  tile_spans(a, b, pre, tot, span_red);
   const int L = __ldg(a.seq_lens + b);
-  const int2 rg = br == 0 ? *reinterpret_cast<const int2*>(a.rng1 + 2 * u)
-                          : *reinterpret_cast<const int2*>(a.rng3 + (long)u * 4 + 2 * (br - 1));
-  if (!len_ok(L, a)) return;  // output zeroed by dec_select
+  if (!len_ok(L, a)) return;  // output zeroed by dec_select (uniform over the CTA)
+  int2 rg = make_int2(0, -1);
+  if (br == 0) {
+    const int nt = unit_tiles<MODE_CMP>(L, a);
+    if (nt > 0) {
+      const long long V = min((long long)a.grid1, tot[0]);
+      const long long T0 = pre[0] + (long long)g * nt;
+      rg = make_int2(stream_of_tile(T0, V, tot[0]), stream_of_tile(T0 + nt - 1, V, tot[0]));
+    }
+  } else {
+    const int nt = unit_tiles<MODE_SW>(L, a), ns = n_selected(L, a);
+    const long long V = min((long long)a.grid3, tot[1]);
+    const long long T0 = pre[1] + (long long)g * nt;
+    const long long x0 = br == 1 ? T0 : T0 + ns, x1 = br == 1 ? T0 + ns - 1 : T0 + nt - 1;
+    rg = make_int2(stream_of_tile(x0, V, tot[1]), stream_of_tile(x1, V, tot[1]));
+  }
 
   // gates (EP94 notes §五 gating): sigmoid(q_h . Wg[:, c]), a warp per dot product
   const __nv_bfloat16* qg =
@@ -1106,6 +1320,7 @@ __global__ void __launch_bounds__(CMB_THREADS) dec_combine_kernel(const __grid_c
     }
     if (lane == 0) gate_s[x] = gv;
   }
+  ptx::grid_dep_wait();  // partials of dec_cmp_partial / dec_sel_win
 
   const float* part;
   long long first;
@@ -1209,10 +1424,14 @@ DecFastArgs base_args(const nsa_params& p) {
 }
 
 
-// Launch with programmatic stream serialization: the grid is scheduled as the
-// previous kernel in the stream drains instead of after it has fully retired;
-// every decode kernel calls grid_dep_wait before it touches global memory, so
-// the order of memory effects is that of plain launches.
+// Launch with programmatic stream serialization: the grid may be scheduled
+// once the previous kernel's CTAs have called grid_dep_launch (the
+// compressed-branch, selection and selected/window kernels do so at their
+// start). Every decode kernel calls grid_dep_wait before it reads anything an
+// earlier kernel writes; before that wait it reads only the call's inputs, and
+// only when its predecessor is this library's kernel (which waited on the
+// caller's writes first), so the order of memory effects is that of plain
+// launches.
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
                        cudaStream_t stream, Args&&... args) {
@@ -1231,8 +1450,9 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 
 }  // namespace
 
-bool decode_fast_eligible(const nsa_params& p) {
-  if (p.sel_mode != 0) return false;  // Quest-bound selection: CUDA-core path
+namespace {
+// Shapes of the fast decode kernels (either selection).
+bool decode_fast_shape(const nsa_params& p) {
   if (!(p.dtype == NSA_DTYPE_BF16 && p.d == D && p.Hq == G * p.Hkv && p.sel_block == TK &&
         p.top_n <= MAXSEL && p.T >= 1 && (p.T + p.sel_block - 1) / p.sel_block <= MAXCAND))
     return false;
@@ -1247,17 +1467,28 @@ bool decode_fast_eligible(const nsa_params& p) {
   const int Nc = nsa_num_cmp_blocks(p.T, p.cmp_block, p.cmp_stride);
   return sel_dyn_smem(p.T, p.sel_block, (Nc + WK - 1) / WK, nbt) <= kSelDynSmemMax;
 }
+}  // namespace
+
+bool decode_fast_eligible(const nsa_params& p) { return p.sel_mode == 0 && decode_fast_shape(p); }
+
+bool decode_quest_fast_eligible(const nsa_params& p) {
+  return p.sel_mode == 1 && p.top_p == 0.f && decode_fast_shape(p);
+}
 
 size_t decode_fast_ws_bytes(const nsa_params& p) {
-  if (!decode_fast_eligible(p)) return 0;
+  if (!decode_fast_eligible(p) && !decode_quest_fast_eligible(p)) return 0;
   return ws_layout(base_args(p)).total;
 }
 
 cudaError_t launch_decode_fast(const nsa_params& p, const void* q, const void* k, const void* v,
                                const int32_t* seq_lens, const void* kc, const void* vc,
                                const float* w_gate, void* out, int32_t* sel_out, void* ws,
-                               unsigned* err, cudaStream_t stream) {
+                               unsigned* err, cudaStream_t stream, const void* kbounds) {
   DecFastArgs a = base_args(p);
+  a.kbounds = kbounds;
+  a.want_rec = kbounds == nullptr;
+  a.nblk = (p.T + p.sel_block - 1) / p.sel_block;
+  a.after_cmp = a.Nc > 0;
   const WsLayout L = ws_layout(a);
   char* w = static_cast<char*>(ws);
   a.q = q;
@@ -1297,7 +1528,12 @@ cudaError_t launch_decode_fast(const nsa_params& p, const void* q, const void* k
                         tvc)) != cudaSuccess)
       return e;
   }
-  {
+  if (kbounds) {
+    TraceScope trace("dec_quest_select", stream);
+    if ((e = launch_pdl(dec_quest_select_kernel, dim3(p.B * p.Hkv), dim3(SEL_THREADS), 0, stream,
+                        a)) != cudaSuccess)
+      return e;
+  } else {
     const size_t smem = sel_dyn_smem(p.T, p.sel_block, a.tiles_max, a.nbt);
     TraceScope trace("dec_select", stream);
     if ((e = ensure_dyn_smem((const void*)dec_select_kernel, (int)kSelDynSmemMax)) != cudaSuccess)

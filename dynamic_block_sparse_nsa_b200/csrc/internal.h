@@ -112,14 +112,22 @@ struct DecFastArgs {
   float* part3;   // selected / window partials, slot = 2 * (stream + 2 * unit + branch) + half
   int* rng1;      // per unit: first/last stream of its compressed tiles
   int* rng3;      // per unit: first/last stream of its selected and window tiles
+  const void* kbounds;  // Quest-style selection: block key extremes [B, nblk, Hkv, 2, d]; else NULL
+  int want_rec;         // the compressed-branch kernel writes score records (NSA selection)
+  int nblk;             // selection blocks at capacity T
+  int after_cmp;        // the selection kernel follows this library's compressed-branch
+                        // kernel (else the caller's work: it waits before any read)
 };
 
 bool decode_fast_eligible(const nsa_params& p);
+// The same kernels with the Quest-style selection from a block-bounds table
+// (nsa_decode_quest): sel_mode == 1 on the fast decode's shapes.
+bool decode_quest_fast_eligible(const nsa_params& p);
 size_t decode_fast_ws_bytes(const nsa_params& p);
 cudaError_t launch_decode_fast(const nsa_params& p, const void* q, const void* k, const void* v,
                                const int32_t* seq_lens, const void* kc, const void* vc,
                                const float* w_gate, void* out, int32_t* sel_out, void* ws,
-                               unsigned* err, cudaStream_t stream);
+                               unsigned* err, cudaStream_t stream, const void* kbounds = nullptr);
 
 // Tensor-core prefill: bf16, d = 128, 16 query heads per KV head, l = 32,
 // s = 16, selection block 64, top_n <= 16.
@@ -133,6 +141,11 @@ cudaError_t launch_prefill_tc(const nsa_params& p, const void* q, const void* k,
 // prefill: per-block key extremes, block scores, top-n into `sel`
 // [B, T, Hkv, n]. Its workspace follows the prefill's own.
 bool quest_tc_supported(const nsa_params& p);
+// Block key extremes beside a KV cache, and their update by one appended token.
+cudaError_t launch_block_bounds(const nsa_params& p, const void* k, const int32_t* seq_lens,
+                                void* kbounds, unsigned* err, cudaStream_t stream);
+cudaError_t launch_append_bounds(const nsa_params& p, const void* k_new, const int32_t* pos,
+                                 void* kbounds, unsigned* err, cudaStream_t stream);
 size_t quest_ws_bytes(const nsa_params& p);
 cudaError_t launch_quest_select(const nsa_params& p, const void* q, const void* k, int32_t* sel,
                                 void* ws, cudaStream_t stream);

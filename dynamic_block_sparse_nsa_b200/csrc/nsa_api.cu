@@ -315,6 +315,63 @@ nsa_status nsa_decode(const nsa_params* p, const void* q, const void* k_cache, c
   return e == cudaSuccess ? NSA_OK : cuda_fail(e, "decode launch");
 }
 
+nsa_status nsa_decode_quest(const nsa_params* p, const void* q, const void* k_cache,
+                            const void* v_cache, const int32_t* seq_lens, const void* k_cmp,
+                            const void* v_cmp, const void* k_bounds, const float* w_gate,
+                            void* out, int32_t* sel_idx, void* workspace, size_t ws_bytes,
+                            void* stream) {
+  g_detail.clear();
+  nsa_status s = check_nsa(p);
+  if (s != NSA_OK) return s;
+  if (p->sel_mode != 1)
+    return fail(NSA_ERR_INVALID_ARGUMENT, "nsa_decode_quest needs sel_mode == 1 (Quest bound)");
+  if (!decode_quest_fast_eligible(*p))  // other shapes: the CUDA-core path reads the keys
+    return nsa_decode(p, q, k_cache, v_cache, seq_lens, k_cmp, v_cmp, w_gate, out, sel_idx,
+                      workspace, ws_bytes, stream);
+  const int Nc = nsa_num_cmp_blocks(p->T, p->cmp_block, p->cmp_stride);
+  if (!q || !k_cache || !v_cache || !seq_lens || !out || !k_bounds ||
+      (Nc > 0 && (!k_cmp || !v_cmp)))
+    return fail(NSA_ERR_INVALID_ARGUMENT,
+                "q, k_cache, v_cache, seq_lens, k_cmp, v_cmp, k_bounds, out must be non-NULL");
+  if (p->gate_mode == 0 && !w_gate)
+    return fail(NSA_ERR_INVALID_ARGUMENT, "w_gate must be non-NULL when gate_mode == 0");
+  unsigned* err = err_word(&s);
+  if (!err) return s;
+  s = check_workspace(workspace, ws_bytes, decode_fast_ws_bytes(*p));
+  if (s != NSA_OK) return s;
+  cudaError_t e = launch_decode_fast(*p, q, k_cache, v_cache, seq_lens, k_cmp, v_cmp, w_gate, out,
+                                     sel_idx, workspace, err, (cudaStream_t)stream, k_bounds);
+  return e == cudaSuccess ? NSA_OK : cuda_fail(e, "decode launch");
+}
+
+nsa_status nsa_block_bounds(const nsa_params* p, const void* k_cache, const int32_t* seq_lens,
+                            void* k_bounds, void* stream) {
+  g_detail.clear();
+  nsa_status s = check_common(p);
+  if (s != NSA_OK) return s;
+  if (p->sel_block < 1) return fail(NSA_ERR_INVALID_ARGUMENT, "sel_block must be >= 1");
+  if (!k_cache || !seq_lens || !k_bounds)
+    return fail(NSA_ERR_INVALID_ARGUMENT, "k_cache, seq_lens, k_bounds must be non-NULL");
+  unsigned* err = err_word(&s);
+  if (!err) return s;
+  cudaError_t e = launch_block_bounds(*p, k_cache, seq_lens, k_bounds, err, (cudaStream_t)stream);
+  return e == cudaSuccess ? NSA_OK : cuda_fail(e, "block bounds launch");
+}
+
+nsa_status nsa_append_bounds(const nsa_params* p, const void* k_new, const int32_t* pos,
+                             void* k_bounds, void* stream) {
+  g_detail.clear();
+  nsa_status s = check_common(p);
+  if (s != NSA_OK) return s;
+  if (p->sel_block < 1) return fail(NSA_ERR_INVALID_ARGUMENT, "sel_block must be >= 1");
+  if (!k_new || !pos || !k_bounds)
+    return fail(NSA_ERR_INVALID_ARGUMENT, "k_new, pos, k_bounds must be non-NULL");
+  unsigned* err = err_word(&s);
+  if (!err) return s;
+  cudaError_t e = launch_append_bounds(*p, k_new, pos, k_bounds, err, (cudaStream_t)stream);
+  return e == cudaSuccess ? NSA_OK : cuda_fail(e, "append bounds launch");
+}
+
 nsa_status moba_prefill(const nsa_params* p, const void* q, const void* k, const void* v,
                         void* out, int32_t* sel_idx, void* workspace, size_t ws_bytes,
                         void* stream) {

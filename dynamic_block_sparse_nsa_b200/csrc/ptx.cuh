@@ -152,6 +152,13 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 // launched without the programmatic-serialization attribute).
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// Lets the next kernel in the stream (launched with programmatic stream
+// serialization) be scheduled now; it still waits in grid_dep_wait for this
+// grid's completion and memory before reading what this grid writes.
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }

@@ -8,7 +8,7 @@
 // heads moves inside: with P_e = sum_h max(q_he, 0) and N_e = sum_h min(q_he, 0),
 //     score(t, g, j) = P . kmax_j + N . kmin_j,
 // one dot product of length 2d per (token, group, block) against a per-block
-// table. Three kernels:
+// table. Three kernels for the prefill:
 //   quest_bounds  kmax, kmin of every full selection block (bf16: the extremes
 //                 of bf16 keys are bf16 values), [B, nblk, Hkv, 2, d];
 //   quest_scores  per 64-token chunk (one selection block of queries) and KV
@@ -18,6 +18,9 @@
 //                 up to each token; [B, T, Hkv, pitch] fp32;
 //   quest_select  a warp per (token, KV head): block 0 and the n - 1 best
 //                 others (ties to the lower index), ascending, -1 padded.
+// and, for decode, the same table kept beside the KV cache: block_bounds
+// builds it from a cache, append_bounds folds in each appended token (the
+// decode's scores are in the decode kernels).
 #include <cuda_bf16.h>
 
 #include <cstdint>
@@ -222,7 +225,92 @@ __global__ void __launch_bounds__(256) quest_select_kernel(const QuestSelArgs a)
 
 size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Keys' block extremes beside a KV cache (decode): block j of sequence b and
+// KV head g covers keys [j bs, min(j bs + bs, len_b)); blocks at or past the
+// length are left alone. One thread per head-dimension element.
+template <typename T>
+__global__ void block_bounds_kernel(const T* __restrict__ k, const int32_t* __restrict__ lens,
+                                    T* __restrict__ bounds, int T_, int Hkv, int d, int bs,
+                                    int nblk, unsigned* err) {
+  const int j = blockIdx.x, g = blockIdx.y, b = blockIdx.z, e = threadIdx.x;
+  const int L = __ldg(lens + b);
+  if (L < 1 || L > T_) {
+    if (j == 0 && g == 0 && e == 0) atomicOr(err, kErrSeqLen);
+    return;
+  }
+  const int u0 = j * bs;
+  if (u0 >= L) return;
+  const int u1 = min(u0 + bs, L);
+  const T* src = k + (((size_t)b * T_ + u0) * Hkv + g) * d + e;
+  float mx = -INFINITY, mn = INFINITY;
+  for (int u = u0; u < u1; ++u) {
+    const float x = to_f32(src[(size_t)(u - u0) * Hkv * d]);
+    mx = fmaxf(mx, x);
+    mn = fminf(mn, x);
+  }
+  T* dst = bounds + (((size_t)b * nblk + j) * Hkv + g) * 2 * d;
+  dst[e] = from_f32<T>(mx);  // exact: an element of the block
+  dst[d + e] = from_f32<T>(mn);
+}
+
+// One appended token per sequence at pos[b]: its block's extremes take it in
+// (the first token of a block starts them).
+template <typename T>
+__global__ void append_bounds_kernel(const T* __restrict__ k_new, const int32_t* __restrict__ pos,
+                                     T* __restrict__ bounds, int T_, int Hkv, int d, int bs,
+                                     int nblk, unsigned* err) {
+  const int g = blockIdx.x, b = blockIdx.y, e = threadIdx.x;
+  const int P = __ldg(pos + b);
+  if (P < 0 || P >= T_) {
+    if (g == 0 && e == 0) atomicOr(err, kErrAppendPos);
+    return;
+  }
+  const T xv = k_new[((size_t)b * Hkv + g) * d + e];
+  T* dst = bounds + (((size_t)b * nblk + P / bs) * Hkv + g) * 2 * d;
+  if (P % bs == 0) {
+    dst[e] = xv;
+    dst[d + e] = xv;
+  } else {
+    const float x = to_f32(xv);
+    if (x > to_f32(dst[e])) dst[e] = xv;
+    if (x < to_f32(dst[d + e])) dst[d + e] = xv;
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_block_bounds(const nsa_params& p, const void* k, const int32_t* seq_lens,
+                                void* kbounds, unsigned* err, cudaStream_t stream) {
+  const int nblk = (p.T + p.sel_block - 1) / p.sel_block;
+  const dim3 grid(nblk, p.Hkv, p.B);
+  TraceScope trace("block_bounds", stream);
+  if (p.dtype == NSA_DTYPE_BF16)
+    block_bounds_kernel<__nv_bfloat16><<<grid, p.d, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(k), seq_lens, static_cast<__nv_bfloat16*>(kbounds), p.T,
+        p.Hkv, p.d, p.sel_block, nblk, err);
+  else
+    block_bounds_kernel<float><<<grid, p.d, 0, stream>>>(static_cast<const float*>(k), seq_lens,
+                                                        static_cast<float*>(kbounds), p.T, p.Hkv,
+                                                        p.d, p.sel_block, nblk, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_append_bounds(const nsa_params& p, const void* k_new, const int32_t* pos,
+                                 void* kbounds, unsigned* err, cudaStream_t stream) {
+  const int nblk = (p.T + p.sel_block - 1) / p.sel_block;
+  const dim3 grid(p.Hkv, p.B);
+  TraceScope trace("append_bounds", stream);
+  if (p.dtype == NSA_DTYPE_BF16)
+    append_bounds_kernel<__nv_bfloat16><<<grid, p.d, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(k_new), pos, static_cast<__nv_bfloat16*>(kbounds), p.T,
+        p.Hkv, p.d, p.sel_block, nblk, err);
+  else
+    append_bounds_kernel<float><<<grid, p.d, 0, stream>>>(static_cast<const float*>(k_new), pos,
+                                                         static_cast<float*>(kbounds), p.T, p.Hkv,
+                                                         p.d, p.sel_block, nblk, err);
+  return cudaGetLastError();
+}
+
 
 bool quest_tc_supported(const nsa_params& p) {
   const int nblk = (p.T + QB - 1) / QB;

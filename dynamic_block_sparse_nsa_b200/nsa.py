@@ -29,7 +29,8 @@ _TORCH_DTYPE = {DTYPE_F32: torch.float32, DTYPE_BF16: torch.bfloat16}
 EXPORTS = (
     "nsa_workspace_size", "nsa_num_cmp_blocks", "nsa_compress_kv", "nsa_prefill",
     "nsa_prefill_backward", "nsa_decode",
-    "moba_prefill", "nsa_decode_noalloc", "nsa_append_kv", "nsa_check", "nsa_debug_bounded_wait", "nsa_status_string",
+    "moba_prefill", "nsa_decode_noalloc", "nsa_append_kv", "nsa_block_bounds",
+    "nsa_append_bounds", "nsa_decode_quest", "nsa_check", "nsa_debug_bounded_wait", "nsa_status_string",
     "nsa_last_error_detail", "nsa_trace_enable", "nsa_trace_set_filter", "nsa_trace_count",
     "nsa_trace_timed", "nsa_trace_get",
 )
@@ -73,6 +74,9 @@ def _load():
         "moba_prefill": [P, vp, vp, vp, vp, vp, vp, sz, vp],
         "nsa_decode_noalloc": [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp],
         "nsa_append_kv": [P, vp, vp, vp, vp, vp, vp, vp, vp, vp],
+        "nsa_block_bounds": [P, vp, vp, vp, vp],
+        "nsa_append_bounds": [P, vp, vp, vp, vp],
+        "nsa_decode_quest": [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp],
         "nsa_check": [vp],
         "nsa_debug_bounded_wait": [vp, ctypes.c_int, vp],
         "nsa_status_string": [ctypes.c_int],
@@ -319,6 +323,55 @@ def nsa_append_kv(p, k_new, v_new, pos, k_cache, v_cache, w_cmp, k_cmp, v_cmp, s
         _raise(LIB.nsa_append_kv(ctypes.byref(p), _ptr(k_new), _ptr(v_new), _ptr(pos),
                                  _ptr(k_cache), _ptr(v_cache), _ptr(w_cmp), _ptr(k_cmp),
                                  _ptr(v_cmp), _stream(stream, dev)))
+
+
+def nsa_block_bounds(p, k_cache, seq_lens, k_bounds=None, stream=None):
+    """Per selection block of the cache, the element-wise max and min of its
+    keys among the first seq_lens[b] tokens: [B, nblk, Hkv, 2, d]."""
+    dt = p.torch_dtype
+    _dev(k_cache, "k_cache", dt)
+    dev = k_cache.device
+    _dev(seq_lens, "seq_lens", torch.int32, dev)
+    nblk = -(-p.T // p.sel_block)
+    if k_bounds is None:
+        k_bounds = torch.empty(p.B, nblk, p.Hkv, 2, p.d, dtype=dt, device=dev)
+    _dev(k_bounds, "k_bounds", dt, dev)
+    with _on(dev):
+        _raise(LIB.nsa_block_bounds(ctypes.byref(p), _ptr(k_cache), _ptr(seq_lens), _ptr(k_bounds),
+                                    _stream(stream, dev)))
+    return k_bounds
+
+
+def nsa_append_bounds(p, k_new, pos, k_bounds, stream=None):
+    """Fold the keys appended at pos[b] into their blocks' bounds."""
+    dt = p.torch_dtype
+    _dev(k_new, "k_new", dt)
+    dev = k_new.device
+    _dev(pos, "pos", torch.int32, dev)
+    _dev(k_bounds, "k_bounds", dt, dev)
+    with _on(dev):
+        _raise(LIB.nsa_append_bounds(ctypes.byref(p), _ptr(k_new), _ptr(pos), _ptr(k_bounds),
+                                     _stream(stream, dev)))
+
+
+def nsa_decode_quest(p, q, k_cache, v_cache, seq_lens, k_cmp, v_cmp, k_bounds, w_gate=None,
+                     out=None, sel_idx=None, ws=None, stream=None, want_sel=True):
+    """nsa_decode ranking blocks by the Quest-style bound from k_bounds
+    (p.sel_mode must be 1)."""
+    out, sel_idx = _decode_args(p, q, k_cache, v_cache, seq_lens, k_cmp, v_cmp, w_gate, out,
+                                sel_idx, want_sel)
+    dev = q.device
+    _dev(k_bounds, "k_bounds", p.torch_dtype, dev)
+    if ws is None:
+        ws = workspace(p, OP_DECODE, dev)
+    _dev(ws, "ws", None, dev)
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    with _on(dev):
+        _raise(LIB.nsa_decode_quest(ctypes.byref(p), _ptr(q), _ptr(k_cache), _ptr(v_cache),
+                                    _ptr(seq_lens), _ptr(k_cmp), _ptr(v_cmp), _ptr(k_bounds),
+                                    _ptr(w_gate), _ptr(out), _ptr(sel_idx), _ptr(ws), nbytes,
+                                    _stream(stream, dev)))
+    return out, sel_idx
 
 
 def moba_prefill(p, q, k, v, out=None, sel_idx=None, ws=None, stream=None, want_sel=True):

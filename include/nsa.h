@@ -93,7 +93,11 @@ typedef enum {
  *              selection ablation (EP94 notes §八): with kmin, kmax the
  *              element-wise min and max of the block's keys up to the query,
  *              sum over the group's heads of sum_e max(q_e kmin_e, q_e kmax_e).
- *              Mode 1 needs top_p == 0 and runs on the CUDA-core path.
+ *              Mode 1 needs top_p == 0. Prefill (bf16, d = 128, 16 heads per
+ *              KV head, selection block 64) takes it from a block-bounds
+ *              table built inside the call; decode takes that table from the
+ *              caller through nsa_decode_quest (nsa_decode computes the bounds
+ *              from the keys, on the CUDA-core path).
  * MoBA uses B, T, Hq, Hkv, d, sel_block, top_n, softmax_scale and dtype. */
 typedef struct {
   int B, T, Hq, Hkv, d;
@@ -198,6 +202,44 @@ NSA_API nsa_status nsa_decode(const nsa_params* p, const void* q, const void* k_
 NSA_API nsa_status nsa_append_kv(const nsa_params* p, const void* k_new, const void* v_new,
                                  const int32_t* pos, void* k_cache, void* v_cache,
                                  const float* w_cmp, void* k_cmp, void* v_cmp, void* stream);
+
+/* Quest-style block bounds beside a KV cache, for nsa_decode_quest (EP94 notes
+ * §八: the selection ablation's Quest-style block score).
+ *   k_cache    [B, T, Hkv, d] dtype.
+ *   seq_lens   [B] int32, device, 1 <= seq_lens[b] <= T.
+ *   k_bounds   [B, nblk, Hkv, 2, d] dtype, nblk = ceil(T / sel_block):
+ *              k_bounds[b, j, g, 0, :] is the element-wise maximum and
+ *              k_bounds[b, j, g, 1, :] the minimum of the keys of selection
+ *              block j among the first seq_lens[b] tokens (the block holding
+ *              the last token covers the tokens so far). Entries of blocks at
+ *              or past seq_lens[b] are not written. Uses B, T, Hkv, d,
+ *              sel_block and dtype of p.
+ *   A length outside [1, T] writes nothing for that sequence and sets the
+ *   device error word (nsa_check: NSA_ERR_INVALID_ARGUMENT). */
+NSA_API nsa_status nsa_block_bounds(const nsa_params* p, const void* k_cache,
+                                    const int32_t* seq_lens, void* k_bounds, void* stream);
+
+/* Keeps k_bounds current after nsa_append_kv wrote token pos[b] (0 <= pos[b]
+ * < T): block pos[b] / sel_block then covers keys up to pos[b] (a block's
+ * first token restarts its extremes).
+ *   k_new      [B, Hkv, d] dtype (the appended keys); pos [B] int32, device. */
+NSA_API nsa_status nsa_append_bounds(const nsa_params* p, const void* k_new, const int32_t* pos,
+                                     void* k_bounds, void* stream);
+
+/* NSA decode that ranks blocks by the Quest-style bound (p->sel_mode must be
+ * 1; EP94 notes §八): for the query's group, sum over its heads of
+ * sum_e max(q_e kmin_e, q_e kmax_e), with kmin / kmax read from k_bounds as
+ * nsa_block_bounds / nsa_append_bounds keep them; block 0 and the n - 1 best
+ * others (ties to the lower index) are kept, the three branches and gates are
+ * nsa_decode's. Arguments as nsa_decode plus k_bounds; the workspace is
+ * nsa_workspace_size(NSA_OP_DECODE). On shapes other than the bf16, d = 128,
+ * 16 heads per KV head, selection block 64 fast path, the CUDA-core path
+ * computes the bounds from the keys (k_bounds unused). */
+NSA_API nsa_status nsa_decode_quest(const nsa_params* p, const void* q, const void* k_cache,
+                                    const void* v_cache, const int32_t* seq_lens,
+                                    const void* k_cmp, const void* v_cmp, const void* k_bounds,
+                                    const float* w_gate, void* out, int32_t* sel_idx,
+                                    void* workspace, size_t ws_bytes, void* stream);
 
 /* nsa_decode without a workspace argument, for callers that cannot allocate
  * device memory: code that runs while a stream capture is in progress

@@ -86,14 +86,21 @@ def run_nsa_prefill(w, rows=None, seed=None):
                             f64(inp["w_gate"]), out_h, sel_h)
 
 
-def run_nsa_decode(w, seq_lens, check_b=None, seed=None, inp=None):
+def run_nsa_decode(w, seq_lens, check_b=None, seed=None, inp=None, quest_table=False):
+    """GPU decode against the oracle. quest_table: the Quest-style selection
+    through nsa_decode_quest with a block-bounds table from nsa_block_bounds."""
     if inp is None:
         inp = inputs.make_decode(w, seed, seq_lens)
     p = nsa_params_for(w)
     dev = {k_: v_.cuda() for k_, v_ in inp.items()}
     kc, vc = nsa.nsa_compress_kv(p, dev["k"], dev["v"], dev["w_cmp"])
-    out, sel = nsa.nsa_decode(p, dev["q"], dev["k"], dev["v"], dev["seq_lens"], kc, vc,
-                              dev["w_gate"])
+    if quest_table:
+        kb = nsa.nsa_block_bounds(p, dev["k"], dev["seq_lens"])
+        out, sel = nsa.nsa_decode_quest(p, dev["q"], dev["k"], dev["v"], dev["seq_lens"], kc, vc,
+                                        kb, dev["w_gate"])
+    else:
+        out, sel = nsa.nsa_decode(p, dev["q"], dev["k"], dev["v"], dev["seq_lens"], kc, vc,
+                                  dev["w_gate"])
     nsa.nsa_check()
     if check_b is None:
         check_b = list(range(w["B"]))

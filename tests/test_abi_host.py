@@ -87,6 +87,16 @@ def test_calls_reject_null_pointers_before_launching():
                         None, 0, None) == 1
     assert L.moba_prefill(ctypes.byref(p), None, None, None, None, None, None, 0, None) == 1
     assert L.nsa_debug_bounded_wait(None, 10, None) == 1
+    assert L.nsa_block_bounds(ctypes.byref(p), None, None, None, None) == 1
+    assert L.nsa_append_bounds(ctypes.byref(p), None, None, None, None) == 1
+    # the Quest decode needs sel_mode 1, then its pointers (k_bounds included)
+    assert L.nsa_decode_quest(ctypes.byref(p), *([None] * 11), 0, None) == 1
+    assert b"sel_mode" in L.nsa_last_error_detail()
+    pq = nsa.params(2, 4096, 32, 2, 128, sel_mode=1)
+    args = [ctypes.c_void_p(256)] * 11
+    args[6] = None  # k_bounds
+    assert L.nsa_decode_quest(ctypes.byref(pq), *args, 0, None) == 1
+    assert b"k_bounds" in L.nsa_last_error_detail()
     # gate weights are required for learned gates only
     fake = ctypes.c_void_p(256)
     assert L.nsa_prefill(ctypes.byref(p), fake, fake, fake, fake, fake, None, fake, None, None,
