@@ -45,7 +45,7 @@ constexpr int D = 128;                      // head dim
 constexpr int TK = 64;                      // keys per tile
 constexpr int HALF_BYTES = TK * 64 * 2;     // 64 rows x 64 dims of bf16 (one TMA box)
 constexpr int SLOT_BYTES = 2 * HALF_BYTES;  // 64 keys x 128 dims
-constexpr int PART = 2 * G + G * D;         // m[16], l[16], o[16][128]
+constexpr int PART = 2 * G + G * D / 2;     // floats: m[16], l[16], then o[16][128] in bf16
 constexpr uint64_t kWaitNs = 2000000000ull;
 
 enum { MODE_CMP = 0, MODE_SW = 1 };
@@ -519,7 +519,9 @@ __device__ __forceinline__ TileSrc tile_source(const DecFastArgs& a, const Walke
   return ts;
 }
 
-// Write one warp's (m, l, unnormalised O) partial straight to global.
+// Write one warp's (m, l, unnormalised O) partial straight to global: m and l
+// in fp32, O in bf16 (half the bytes the merge reads back; each partial then
+// carries a relative rounding of 2^-9, the output's own precision).
 __device__ __forceinline__ void store_partial(float* dst, int lane, float m0, float m1, float l0,
                                               float l1, const float (&o)[16][4]) {
   const int r0 = lane >> 2, c = (lane & 3) * 2;
@@ -529,11 +531,13 @@ __device__ __forceinline__ void store_partial(float* dst, int lane, float m0, fl
     dst[G + r0] = l0;
     dst[G + r0 + 8] = l1;
   }
-  float* po = dst + 2 * G;
+  __nv_bfloat16* po = reinterpret_cast<__nv_bfloat16*>(dst + 2 * G);
 #pragma unroll
   for (int dt = 0; dt < 16; ++dt) {
-    *reinterpret_cast<float2*>(po + r0 * D + dt * 8 + c) = make_float2(o[dt][0], o[dt][1]);
-    *reinterpret_cast<float2*>(po + (r0 + 8) * D + dt * 8 + c) = make_float2(o[dt][2], o[dt][3]);
+    *reinterpret_cast<__nv_bfloat162*>(po + r0 * D + dt * 8 + c) =
+        __floats2bfloat162_rn(o[dt][0], o[dt][1]);
+    *reinterpret_cast<__nv_bfloat162*>(po + (r0 + 8) * D + dt * 8 + c) =
+        __floats2bfloat162_rn(o[dt][2], o[dt][3]);
   }
 }
 
@@ -1218,7 +1222,7 @@ __global__ void __launch_bounds__(SEL_THREADS) dec_quest_select_kernel(const __g
 constexpr int CMB_HEADS = 4;                   // heads per CTA
 constexpr int CMB_GROUP = CMB_HEADS * 16;      // threads per branch: 16 per head, 8 dims each
 constexpr int CMB_THREADS = 3 * CMB_GROUP;     // one group per branch
-constexpr int CMB_CHUNK = 4;                   // partials whose loads are in flight together
+constexpr int CMB_CHUNK = 8;                   // partials whose loads are in flight together
 
 // Per thread: the online merge of partials [first, first + np) for head h,
 // dims e0 .. e0 + 7: M = max m_p, Ls = sum_p 2^(m_p - M) l_p,
@@ -1227,16 +1231,15 @@ __device__ __forceinline__ void merge_thread(const float* part, long long first,
                                              int e0, float& M, float& Ls, float (&run)[8]) {
   for (int p0 = 0; p0 < np; p0 += CMB_CHUNK) {
     float m[CMB_CHUNK], l[CMB_CHUNK];
-    float4 o[CMB_CHUNK][2];
+    uint4 o[CMB_CHUNK];
 #pragma unroll
     for (int i = 0; i < CMB_CHUNK; ++i) {
       if (p0 + i < np) {
         const float* src = part + (first + p0 + i) * PART;
         m[i] = __ldcg(src + h);
         l[i] = __ldcg(src + G + h);
-        const float4* ov = reinterpret_cast<const float4*>(src + 2 * G + h * D + e0);
-        o[i][0] = __ldcg(ov);
-        o[i][1] = __ldcg(ov + 1);
+        o[i] = __ldcg(reinterpret_cast<const uint4*>(
+            reinterpret_cast<const __nv_bfloat16*>(src + 2 * G) + h * D + e0));
       } else {
         m[i] = -INFINITY;
       }
@@ -1254,14 +1257,13 @@ __device__ __forceinline__ void merge_thread(const float* part, long long first,
       if (m[i] == -INFINITY) continue;
       const float f = exp2f(m[i] - Mn);
       Ls = fmaf(f, l[i], Ls);
-      run[0] = fmaf(f, o[i][0].x, run[0]);
-      run[1] = fmaf(f, o[i][0].y, run[1]);
-      run[2] = fmaf(f, o[i][0].z, run[2]);
-      run[3] = fmaf(f, o[i][0].w, run[3]);
-      run[4] = fmaf(f, o[i][1].x, run[4]);
-      run[5] = fmaf(f, o[i][1].y, run[5]);
-      run[6] = fmaf(f, o[i][1].z, run[6]);
-      run[7] = fmaf(f, o[i][1].w, run[7]);
+      const __nv_bfloat162* ob = reinterpret_cast<const __nv_bfloat162*>(&o[i]);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 v = __bfloat1622float2(ob[k]);
+        run[2 * k] = fmaf(f, v.x, run[2 * k]);
+        run[2 * k + 1] = fmaf(f, v.y, run[2 * k + 1]);
+      }
     }
     M = Mn;
   }
