@@ -751,7 +751,7 @@ def run_dense(w, K, W, rank):
     return ms, flops
 
 
-def kernel_entries(kind, res, w, K, peaks):
+def kernel_entries(kind, res, w, K, peaks, wname):
     """Every traced kernel of a prefill-like step against the bf16 peak
     (burst, and sustained beside it), from the first timed region's events."""
     per = {}
@@ -765,6 +765,9 @@ def kernel_entries(kind, res, w, K, peaks):
         ent = {"tflops": ach, "frac": ach / peaks["bf16"], "peak": peaks["bf16"],
                "frac_sustained": ach / peaks["bf16_sus"], "mean_launch_us": 1e6 * mean_s,
                "flops_per_launch": per_launch}
+        tr = kernel_traffic(n, wname)
+        if tr is not None:
+            ent["traffic"] = tr  # DRAM bytes per launch (ncu), while the source is unchanged
         g = gather_bytes(kind, n, res, w)
         if g is not None:
             ent["gathered_bytes_per_launch"] = g
@@ -794,7 +797,8 @@ def side_summary(name, ws, rank, local, peaks, K, W, cpu_budget, dense=False, e2
     work_all = reduce_sum(res["work"] * K, ws)
     out = {"workload": name, "config": config_of(w), "value": work_all / (ms_max / 1000.0) / 1e12,
            "unit": "TFLOP/s", "ms_per_step": ms_max / K, "steps": K, "warmup": W,
-           "flops_per_step": res["parts"], "kernel_tflops": kernel_entries(kind, res, w, K, peaks),
+           "flops_per_step": res["parts"],
+           "kernel_tflops": kernel_entries(kind, res, w, K, peaks, name),
            "peak_source": peaks["src"], "clocks": res["clk"]}
     out["value_frac"] = out["value"] / peaks["bf16"]
     if "e2e_ms" in res:
@@ -1063,7 +1067,7 @@ def main():
         else:
             line["flops_per_step"] = {k: v for k, v in res["parts"].items()}
             # every traced kernel against the bf16 peak (first timed region's events)
-            per = kernel_entries(kind, res, w, K, peaks)
+            per = kernel_entries(kind, res, w, K, peaks, args.workload)
             line["kernel_tflops"] = per
         line.update(sides)
         print(json.dumps(line), flush=True)
