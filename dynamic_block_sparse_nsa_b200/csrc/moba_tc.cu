@@ -7,9 +7,11 @@
 // [c m, t] and to top_k - 1 earlier blocks chosen by q . mean(K_block). With
 // independent per-row choices no two rows share much, so the work is grouped
 // by key block instead of by query (the gather / re-index view of the pages):
-//   moba_gate  scores per row on the tensor cores at fp32 accuracy (block
-//              means split into three bf16 parts), the picks, the selection
-//              row, and per-(head, block) pick counts;
+//   moba_split each fp32 block mean split once into three bf16 parts
+//              (hi + mid + lo: 24 significant bits);
+//   moba_gate  scores per row on the tensor cores at fp32 accuracy (the
+//              parts staged by cp.async, double-buffered), the picks, the
+//              selection row, and per-(head, block) pick counts;
 //   moba_scan  offsets of each (sequence, head, block) bucket and of its
 //              128-row tiles;
 //   moba_fill  the rows of every bucket (token, slot);
@@ -44,6 +46,7 @@ constexpr uint32_t kNegInf = 0xff800000u;
 struct MobaTcArgs {
   const __nv_bfloat16* q;
   const float* kbar;      // [B, nfull, Hkv, d]
+  __nv_bfloat16* kparts;  // [B, nfull, Hkv, 3, d]: hi, mid, lo of each block mean
   __nv_bfloat16* out;
   int32_t* sel;           // [B, T, Hq, topk]
   int32_t* cnt;           // [NB] picks per bucket (b, h, j)
@@ -93,12 +96,14 @@ __device__ __forceinline__ uint64_t mnmaj(uint32_t base, int ks) {
 // in fp32 and the three m16n8k16 passes accumulate them in fp32, like the fp32
 // dot product on CUDA cores. A CTA takes 128 tokens of one (sequence, head)
 // (8 warps x 16 rows; the tokens share one own block, m being a multiple of
-// 128); block means are staged kGateBlk at a time, split, in a padded layout
-// whose fragment loads hit distinct banks.
+// 128); the parts of kGateBlk block means at a time are copied (cp.async, two
+// buffers: the next chunk lands while the current one is scored) into a
+// padded layout whose fragment loads hit distinct banks.
 constexpr int kGateTok = 128;
 constexpr int kGateBlk = 64;
 constexpr int kGatePitch = D + 8;  // bf16 elements per staged row
-constexpr size_t kGateSmem = 3 * (size_t)kGateBlk * kGatePitch * 2;
+constexpr size_t kGateBuf = 3 * (size_t)kGateBlk * kGatePitch;  // bf16 elements per buffer
+constexpr size_t kGateSmem = 2 * kGateBuf * 2;
 
 __device__ __forceinline__ uint32_t ld_b32(const __nv_bfloat16* p) {
   return *reinterpret_cast<const uint32_t*>(p);
@@ -199,40 +204,32 @@ __global__ void __launch_bounds__(256) moba_gate_kernel(MobaTcArgs a) {
       keep_best(bs1, bj1, want, worst1, c[3], j0 + 1);
     }
   };
-  for (int c0 = 0; c0 < own; c0 += kGateBlk) {
+  // chunk c0 .. c0 + 63 of the parts into buffer `buf`: 16-byte granules, a
+  // block's three part rows (768 B) are contiguous in kparts
+  auto stage = [&](int c0, int buf) {
     const int nb = min(kGateBlk, own - c0);
-    __syncthreads();
-    // every thread's eight float4 loads in flight at once, then the split
-    constexpr int kLd = kGateBlk * D / 4 / 256;
-    float4 xv[kLd];
-#pragma unroll
-    for (int r = 0; r < kLd; ++r) {
-      const int i4 = threadIdx.x + r * 256, j = i4 / (D / 4), e4 = i4 - j * (D / 4);
-      xv[r] = j < nb ? __ldg(reinterpret_cast<const float4*>(
-                           a.kbar + (((size_t)b * a.nfull + c0 + j) * a.Hkv + g) * D) + e4)
-                     : make_float4(0.f, 0.f, 0.f, 0.f);
+    __nv_bfloat16* dstb = kbs + (size_t)buf * kGateBuf;
+    constexpr int kGran = kGateBlk * 3 * (D / 8);  // granules per chunk
+#pragma unroll 1
+    for (int r = 0; r < kGran / 256; ++r) {
+      const int idx = threadIdx.x + r * 256, j = idx / (3 * D / 8), rem = idx - j * (3 * D / 8);
+      const int pp = rem / (D / 8), gr = rem - pp * (D / 8);
+      if (j < nb)
+        ptx::cp_async16(dstb + ((size_t)pp * kGateBlk + j) * kGatePitch + gr * 8,
+                        a.kparts + (((size_t)b * a.nfull + c0 + j) * a.Hkv + g) * 3 * D + pp * D +
+                            gr * 8);
     }
-#pragma unroll
-    for (int r = 0; r < kLd; ++r) {
-      const int i4 = threadIdx.x + r * 256, j = i4 / (D / 4), e = 4 * (i4 - j * (D / 4));
-      // hi = bf16(x), mid = bf16(x - hi), lo = bf16(x - hi - mid), two values a word
-      uint2 hv, mv, lv;
-      auto split2 = [](float x0, float x1, uint32_t& h, uint32_t& m, uint32_t& l) {
-        const __nv_bfloat162 hb = __floats2bfloat162_rn(x0, x1);
-        const float2 hf = __bfloat1622float2(hb);
-        const float r0 = x0 - hf.x, r1 = x1 - hf.y;
-        const __nv_bfloat162 mb = __floats2bfloat162_rn(r0, r1);
-        const float2 mf = __bfloat1622float2(mb);
-        const __nv_bfloat162 lb = __floats2bfloat162_rn(r0 - mf.x, r1 - mf.y);
-        h = *reinterpret_cast<const uint32_t*>(&hb);
-        m = *reinterpret_cast<const uint32_t*>(&mb);
-        l = *reinterpret_cast<const uint32_t*>(&lb);
-      };
-      split2(xv[r].x, xv[r].y, hv.x, mv.x, lv.x);
-      split2(xv[r].z, xv[r].w, hv.y, mv.y, lv.y);
-      *reinterpret_cast<uint2*>(kbs + (0 * kGateBlk + j) * kGatePitch + e) = hv;
-      *reinterpret_cast<uint2*>(kbs + (1 * kGateBlk + j) * kGatePitch + e) = mv;
-      *reinterpret_cast<uint2*>(kbs + (2 * kGateBlk + j) * kGatePitch + e) = lv;
+    ptx::cp_async_commit();
+  };
+  if (own > 0) stage(0, 0);
+  for (int c0 = 0, it = 0; c0 < own; c0 += kGateBlk, ++it) {
+    const int nb = min(kGateBlk, own - c0);
+    const __nv_bfloat16* kbuf = kbs + (size_t)(it & 1) * kGateBuf;
+    if (c0 + kGateBlk < own) {
+      stage(c0 + kGateBlk, (it + 1) & 1);  // its buffer was last read before the previous barrier
+      ptx::cp_async_wait<1>();
+    } else {
+      ptx::cp_async_wait<0>();
     }
     __syncthreads();
     // two 8-block tiles at a time: two independent accumulator chains. B
@@ -244,7 +241,7 @@ __global__ void __launch_bounds__(256) moba_gate_kernel(MobaTcArgs a) {
       float ca[4] = {0.f, 0.f, 0.f, 0.f}, cb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int pp = 0; pp < 3; ++pp) {
-        const __nv_bfloat16* ka = kbs + ((size_t)pp * kGateBlk + nt * 8 + r0) * kGatePitch;
+        const __nv_bfloat16* ka = kbuf + ((size_t)pp * kGateBlk + nt * 8 + r0) * kGatePitch;
         const __nv_bfloat16* kb2 = ka + 8 * kGatePitch;
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
@@ -257,6 +254,7 @@ __global__ void __launch_bounds__(256) moba_gate_kernel(MobaTcArgs a) {
       take(ca, c0 + nt * 8 + q2);  // blocks of c[0], c[2] and, + 1, of c[1], c[3]
       if (two) take(cb, c0 + nt * 8 + 8 + q2);
     }
+    __syncthreads();  // this buffer is refilled two chunks on
   }
   int pick0[kMaxTopk], pick1[kMaxTopk];
   quad_merge(bs0, bj0, want, pick0);
@@ -288,6 +286,32 @@ __global__ void __launch_bounds__(256) moba_gate_kernel(MobaTcArgs a) {
   for (int i = 0; i < a.topk; ++i) dst[i] = i < n ? row[i] : -1;
   for (int i = 0; i + 1 < n; ++i)  // every entry but the own block is a past pick
     atomicAdd(a.cnt + ((size_t)b * a.Hq + h) * a.nfull + row[i], 1);
+}
+
+// Each fp32 block mean once into three bf16 parts hi + mid + lo (hi = bf16(x),
+// mid = bf16(x - hi), lo = bf16(x - hi - mid): 24 significant bits), so every
+// product with a bf16 query element is exact in fp32.
+__global__ void __launch_bounds__(256) moba_split_kernel(MobaTcArgs a) {
+  const size_t n4 = (size_t)a.B * a.nfull * a.Hkv * (D / 4);
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const size_t row = i / (D / 4);
+    const int e = (int)(i - row * (D / 4)) * 4;
+    const float4 x = reinterpret_cast<const float4*>(a.kbar + row * D + e)[0];
+    const float xs[4] = {x.x, x.y, x.z, x.w};
+    __nv_bfloat16 hi[4], mid[4], lo[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      hi[k] = __float2bfloat16_rn(xs[k]);
+      const float r1 = xs[k] - __bfloat162float(hi[k]);
+      mid[k] = __float2bfloat16_rn(r1);
+      lo[k] = __float2bfloat16_rn(r1 - __bfloat162float(mid[k]));
+    }
+    __nv_bfloat16* dst = a.kparts + row * 3 * D + e;
+    *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(hi);
+    *reinterpret_cast<uint2*>(dst + D) = *reinterpret_cast<const uint2*>(mid);
+    *reinterpret_cast<uint2*>(dst + 2 * D) = *reinterpret_cast<const uint2*>(lo);
+  }
 }
 
 // Exclusive prefix sums of the bucket counts (rows) and of their 128-row
@@ -868,8 +892,10 @@ size_t moba_tc_ws_bytes(const nsa_params& p, size_t kbar_bytes) {
   const size_t rows = (size_t)p.B * p.T * p.Hq;
   const size_t NB = (size_t)p.B * p.Hq * (p.T / p.sel_block);
   const size_t np = (size_t)(p.top_n - 1);
+  const size_t parts = (size_t)p.B * (p.T / p.sel_block) * p.Hkv * 3 * D * 2;
   return align256(kbar_bytes) + align256(rows * p.top_n * 4) + 4 * align256((NB + 1) * 4) +
-         align256(rows * np * 4 + 4) + align256(rows * np * D * 2 + 4) + align256(rows * np * 4 + 4);
+         align256(rows * np * 4 + 4) + align256(rows * np * D * 2 + 4) + align256(rows * np * 4 + 4) +
+         align256(parts + 4);
 }
 
 cudaError_t launch_moba_tc(const nsa_params& p, const void* q, const void* k, const void* v,
@@ -905,6 +931,8 @@ cudaError_t launch_moba_tc(const nsa_params& p, const void* q, const void* k, co
   a.po = reinterpret_cast<__nv_bfloat16*>(w);
   w += align256(rows * np * D * 2 + 4);
   a.plse = reinterpret_cast<float*>(w);
+  w += align256(rows * np * 4 + 4);
+  a.kparts = reinterpret_cast<__nv_bfloat16*>(w);
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.out = static_cast<__nv_bfloat16*>(out);
   a.err = err;
@@ -920,6 +948,13 @@ cudaError_t launch_moba_tc(const nsa_params& p, const void* q, const void* k, co
 
   cudaError_t e;
   if (a.NB > 0 && (e = cudaMemsetAsync(a.cnt, 0, (size_t)a.NB * 4, stream)) != cudaSuccess) return e;
+  if (a.nfull > 0) {
+    TraceScope trace("moba_split", stream);
+    const size_t n4 = (size_t)a.B * a.nfull * a.Hkv * (D / 4);
+    const int grid = (int)std::min<size_t>((n4 + 255) / 256, (size_t)device_sm_count() * 8);
+    moba_split_kernel<<<grid, 256, 0, stream>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
   {
     TraceScope trace("moba_gate", stream);
     if ((e = ensure_dyn_smem((const void*)moba_gate_kernel, (int)kGateSmem)) != cudaSuccess)

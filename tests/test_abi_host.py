@@ -70,9 +70,10 @@ def test_workspace_size_validation():
     kbar = a256(B * (T // m) * H * 128 * 4)
     rows, nb = B * T * H, B * H * (T // m)
     moba = nsa.params(B, T, H, H, 128, sel_block=m, top_n=k)
+    parts = a256(B * (T // m) * H * 3 * 128 * 2 + 4)  # the means split into three bf16 parts
     assert nsa.workspace_size(moba, nsa.OP_MOBA_PREFILL) == (
         kbar + a256(rows * k * 4) + 4 * a256((nb + 1) * 4) + a256(rows * (k - 1) * 4 + 4) +
-        a256(rows * (k - 1) * 128 * 2 + 4) + a256(rows * (k - 1) * 4 + 4))
+        a256(rows * (k - 1) * 128 * 2 + 4) + a256(rows * (k - 1) * 4 + 4) + parts)
     moba32 = nsa.params(B, T, H, H, 128, sel_block=m, top_n=k, dtype=torch.float32)
     assert nsa.workspace_size(moba32, nsa.OP_MOBA_PREFILL) == kbar  # CUDA-core path
 
