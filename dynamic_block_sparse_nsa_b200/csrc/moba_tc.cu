@@ -9,9 +9,9 @@
 // by key block instead of by query (the gather / re-index view of the pages):
 //   moba_split each fp32 block mean split once into three bf16 parts
 //              (hi + mid + lo: 24 significant bits);
-//   moba_gate  scores per row on the tensor cores at fp32 accuracy (the
-//              parts staged by cp.async, double-buffered), the picks, the
-//              selection row, and per-(head, block) pick counts;
+//   moba_gate  scores per row at fp32 accuracy as a tcgen05 product of the
+//              query tile with the parts (TMEM accumulators), the picks,
+//              the selection row, and per-(head, block) pick counts;
 //   moba_scan  offsets of each (sequence, head, block) bucket and of its
 //              128-row tiles;
 //   moba_fill  the rows of every bucket (token, slot);
@@ -46,7 +46,7 @@ constexpr uint32_t kNegInf = 0xff800000u;
 struct MobaTcArgs {
   const __nv_bfloat16* q;
   const float* kbar;      // [B, nfull, Hkv, d]
-  __nv_bfloat16* kparts;  // [B, nfull, Hkv, 3, d]: hi, mid, lo of each block mean
+  __nv_bfloat16* kparts;  // [B, Hkv, 3, gate_rows(nfull), d]: hi, mid, lo of each block mean
   __nv_bfloat16* out;
   int32_t* sel;           // [B, T, Hq, topk]
   int32_t* cnt;           // [NB] picks per bucket (b, h, j)
@@ -86,219 +86,351 @@ __device__ __forceinline__ uint64_t mnmaj(uint32_t base, int ks) {
 // gate, scan, fill
 // ============================================================================
 
-// One thread per (token, head); 128 tokens of one head per CTA. Past blocks
-// j < t / m are scored with q . kbar[j] in fp32 and the top_k - 1 best kept
-// (higher score first, ties to the lower block: blocks arrive in increasing
-// order and only a strictly higher score displaces a kept one).
 // Block scores q . kbar_j on the tensor cores without losing fp32 accuracy:
 // q is bf16, and each fp32 block mean is split into three bf16 parts
 // (hi + mid + lo, 24 significant bits), so every product q_e * part_e is exact
-// in fp32 and the three m16n8k16 passes accumulate them in fp32, like the fp32
-// dot product on CUDA cores. A CTA takes 128 tokens of one (sequence, head)
-// (8 warps x 16 rows; the tokens share one own block, m being a multiple of
-// 128); the parts of kGateBlk block means at a time are copied (cp.async, two
-// buffers: the next chunk lands while the current one is scored) into a
-// padded layout whose fragment loads hit distinct banks.
-constexpr int kGateTok = 128;
-constexpr int kGateBlk = 64;
-constexpr int kGatePitch = D + 8;  // bf16 elements per staged row
-constexpr size_t kGateBuf = 3 * (size_t)kGateBlk * kGatePitch;  // bf16 elements per buffer
-constexpr size_t kGateSmem = 2 * kGateBuf * 2;
+// in fp32 and the tensor core sums them in fp32, like the fp32 dot product on
+// CUDA cores. A work item is 128 tokens of one (sequence, head); the tokens
+// share one own block (m is a multiple of 128), so they score the same past
+// blocks 0 .. own - 1. Per chunk of 128 blocks the three parts are loaded
+// (TMA, one part per ring stage) and S = Q [hi | mid | lo]^T accumulates in a
+// 128-column TMEM buffer that the four row warps then read: thread `row`
+// keeps the best top_k - 1 of its row (higher score first, ties to the lower
+// block: blocks arrive in increasing order and only a strictly higher score
+// displaces a kept one).
+//
+// The kernel is persistent, one CTA per SM: items are taken round-robin in
+// order of decreasing own block (the longest first) with the heads of one
+// token tile next to each other, so the CTAs running at a time read whole
+// token rows of q. The TMA warp runs ahead across items (two query tiles, a
+// four-stage ring of parts), the MMA warp fills four score buffers, and the
+// row warps drain them.
+constexpr int kGateStages = 4;
+constexpr int kGateAcc = 4;   // TMEM score buffers of 128 columns
+constexpr int kGateBox = 32;  // block rows per TMA box of the parts
 
-__device__ __forceinline__ uint32_t ld_b32(const __nv_bfloat16* p) {
-  return *reinterpret_cast<const uint32_t*>(p);
+// Rows of the parts tensor per (sequence, KV head, part): the blocks padded to
+// a whole number of TMA boxes, so every box the gate loads lies in the tensor.
+__host__ __device__ inline int gate_rows(int nfull) {
+  return nfull < kGateBox ? kGateBox : (nfull + kGateBox - 1) / kGateBox * kGateBox;
 }
 
-// Keep the best `want` (score, block) of one row: higher score first, equal
-// scores to the lower block (candidates arrive in ascending block order and
-// only a strictly better one moves ahead). `worst` is the want-th kept score
-// (-inf until the list is full): most candidates fail that one comparison.
-__device__ __forceinline__ void keep_best(float (&bs)[kMaxTopk], int (&bj)[kMaxTopk], int want,
-                                          float& worst, float s, int j) {
-  if (!(s > worst)) return;
+struct GateBars {
+  uint64_t full[kGateStages], empty[kGateStages];
+  uint64_t q_full[2], q_free[2], acc_full[kGateAcc], acc_free[kGateAcc], fin;
+  uint32_t tmem;
+  int abort;
+};
+
+size_t gate_smem() { return 1024 + (size_t)(2 + kGateStages) * TILE + sizeof(GateBars); }
+
+// Work item i of the gate: token tile, sequence and head.
+struct GateItem {
+  int t0, b, h, own, nch;
+};
+
+__device__ __forceinline__ GateItem gate_item(const MobaTcArgs& a, int i, int want) {
+  const int ntq = (a.T + KT - 1) / KT, bh = i % (a.B * a.Hq);
+  GateItem it;
+  it.t0 = (ntq - 1 - i / (a.B * a.Hq)) * KT;
+  it.b = bh / a.Hq;
+  it.h = bh % a.Hq;
+  it.own = it.t0 / a.m;
+  // 128-block chunks to score: none when every past block is taken, or none is
+  it.nch = it.own > want && want > 0 ? (it.own + KT - 1) / KT : 0;
+  return it;
+}
+
+// The selection row of token t when no block is scored: every block 0 .. own
+// when there are at most top_k of them, else (top_k = 1) the own block alone;
+// -1 after. Each past block taken counts a row into its bucket.
+__device__ void gate_emit_unscored(const MobaTcArgs& a, int b, int h, int t, int own) {
+  int32_t* dst = a.sel + ((size_t)(b * a.T + t) * a.Hq + h) * a.topk;
+  if (own < a.topk) {
+    for (int i = 0; i < a.topk; ++i) dst[i] = i <= own ? i : -1;
+    for (int j = 0; j < own; ++j) atomicAdd(a.cnt + ((size_t)b * a.Hq + h) * a.nfull + j, 1);
+  } else {
+    dst[0] = own;
+  }
+}
+
+// The best W (score, block) of one row, in registers (W = top_k - 1 is a
+// compile-time constant, so no index is dynamic), sorted by decreasing score.
+// Insertion is branch-free, so the lanes of a warp never diverge: entry i
+// takes the candidate if it beats entry i but not entry i - 1, entry i - 1 if
+// the candidate beats that too. Strict comparisons keep the lower block first
+// among equal scores (candidates arrive in increasing block order).
+template <int W>
+struct KeepBest {
+  float s[W];
+  int j[W];
+  __device__ __forceinline__ KeepBest() {
 #pragma unroll
-  for (int i = 0; i < kMaxTopk; ++i) {
-    if (i < want && s > bs[i]) {
-      const float ts = bs[i];
-      const int tj = bj[i];
-      bs[i] = s;
-      bj[i] = j;
-      s = ts;
-      j = tj;
+    for (int i = 0; i < W; ++i) {
+      s[i] = -INFINITY;
+      j[i] = -1;
     }
   }
+  __device__ __forceinline__ void offer(float x, int k) {
+    bool gt[W];
 #pragma unroll
-  for (int i = 0; i < kMaxTopk; ++i)
-    if (i == want - 1) worst = bs[i];
-}
-
-// Merge the four lane lists of a quad (disjoint blocks) into the best `want`,
-// in order: repeatedly the quad-wide best head (score desc, block asc).
-__device__ __forceinline__ void quad_merge(const float (&bs)[kMaxTopk], const int (&bj)[kMaxTopk],
-                                           int want, int (&out)[kMaxTopk]) {
-  int head = 0;
+    for (int i = 0; i < W; ++i) gt[i] = x > s[i];
 #pragma unroll
-  for (int i = 0; i < kMaxTopk; ++i) {
-    if (i >= want) break;
-    float s = -INFINITY;
-    int j = 0x7fffffff;
+    for (int i = W - 1; i > 0; --i) {
+      s[i] = gt[i] ? (gt[i - 1] ? s[i - 1] : x) : s[i];
+      j[i] = gt[i] ? (gt[i - 1] ? j[i - 1] : k) : j[i];
+    }
+    s[0] = gt[0] ? x : s[0];
+    j[0] = gt[0] ? k : j[0];
+  }
+  // The row: the picks in increasing block order, then the own block, -1
+  // after; each pick counts a row into its bucket.
+  __device__ __forceinline__ void emit(const MobaTcArgs& a, int b, int h, int t, int own) {
+    int v[W];
 #pragma unroll
-    for (int x = 0; x < kMaxTopk; ++x)
-      if (x == head && bj[x] >= 0) {
-        s = bs[x];
-        j = bj[x];
+    for (int i = 0; i < W; ++i) v[i] = j[i] < 0 ? 0x7fffffff : j[i];
+#pragma unroll
+    for (int p = 0; p < W; ++p)
+#pragma unroll
+      for (int i = 0; i + 1 < W - p; ++i)
+        if (v[i] > v[i + 1]) {
+          const int x = v[i];
+          v[i] = v[i + 1];
+          v[i + 1] = x;
+        }
+    int n = 0;
+#pragma unroll
+    for (int i = 0; i < W; ++i) n += v[i] != 0x7fffffff;
+    int32_t* dst = a.sel + ((size_t)(b * a.T + t) * a.Hq + h) * a.topk;
+    int32_t* cnt = a.cnt + ((size_t)b * a.Hq + h) * a.nfull;
+#pragma unroll
+    for (int i = 0; i < W; ++i)
+      if (i < n) {
+        dst[i] = v[i];
+        atomicAdd(cnt + v[i], 1);
       }
-    const int mine = j;
-#pragma unroll
-    for (int o = 1; o <= 2; o <<= 1) {
-      const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
-      const int j2 = __shfl_xor_sync(0xffffffffu, j, o);
-      if (s2 > s || (s2 == s && j2 < j)) {
-        s = s2;
-        j = j2;
-      }
-    }
-    out[i] = j == 0x7fffffff ? -1 : j;
-    if (mine == j && j != 0x7fffffff) ++head;
+    for (int i = n; i < a.topk; ++i) dst[i] = i == n ? own : -1;
   }
-}
+};
 
-__global__ void __launch_bounds__(256) moba_gate_kernel(MobaTcArgs a) {
-  extern __shared__ __align__(16) unsigned char gate_raw[];
-  __nv_bfloat16* kbs = reinterpret_cast<__nv_bfloat16*>(gate_raw);  // [3][kGateBlk][kGatePitch]
-  const int t0 = blockIdx.x * kGateTok, h = blockIdx.y, b = blockIdx.z;
-  const int g = h / (a.Hq / a.Hkv);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int r0 = lane >> 2, q2 = (lane & 3) * 2;
-  const int own = t0 / a.m;  // the own block of every token of the tile
-  const int want = a.topk - 1;
-  const int ta = t0 + warp * 16 + r0, tb = ta + 8;  // this lane's rows
-  uint32_t qa[D / 16][4];
-  {
-    const __nv_bfloat16* qr0 = a.q + ((size_t)(b * a.T + ta) * a.Hq + h) * D;
-    const __nv_bfloat16* qr1 = a.q + ((size_t)(b * a.T + tb) * a.Hq + h) * D;
+// Row warps 0-3 over the CTA's items: thread = row = TMEM lane. Per chunk the
+// scores of its nb blocks are read 32 columns at a time and offered in block
+// order.
+template <int W>
+__device__ __forceinline__ void gate_rows(const MobaTcArgs& a, GateBars* bars, volatile int* abort,
+                                          uint32_t tl, int row, int want) {
+  const int NI = a.B * a.Hq * ((a.T + KT - 1) / KT);
+  int ac = 0;
+  for (int i = blockIdx.x; i < NI; i += gridDim.x) {
+    const GateItem it = gate_item(a, i, want);
+    const int t = it.t0 + row;
+    if (it.nch == 0) {
+      if (t < a.T) gate_emit_unscored(a, it.b, it.h, t, it.own);
+      continue;
+    }
+    KeepBest<W> kb;
+    for (int c = 0; c < it.nch; ++c, ++ac) {
+      const int buf = ac % kGateAcc, c0 = c * KT, nb = min(KT, it.own - c0);
+      if (!wait_or_abort(&bars->acc_full[buf], (uint32_t)((ac / kGateAcc) & 1), abort, a.err))
+        return;
+      tc::fence_after_sync();
+      for (int x = 0; x < nb; x += 32) {
+        uint32_t r[32];
+        tc::ld32_sync(tl + buf * KT + x, r);
+        if (x + 32 <= nb) {
 #pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-      qa[ks][0] = ta < a.T ? __ldg(reinterpret_cast<const unsigned*>(qr0 + ks * 16 + q2)) : 0u;
-      qa[ks][1] = tb < a.T ? __ldg(reinterpret_cast<const unsigned*>(qr1 + ks * 16 + q2)) : 0u;
-      qa[ks][2] = ta < a.T ? __ldg(reinterpret_cast<const unsigned*>(qr0 + ks * 16 + 8 + q2)) : 0u;
-      qa[ks][3] = tb < a.T ? __ldg(reinterpret_cast<const unsigned*>(qr1 + ks * 16 + 8 + q2)) : 0u;
-    }
-  }
-  float bs0[kMaxTopk], bs1[kMaxTopk];
-  int bj0[kMaxTopk], bj1[kMaxTopk];
-  float worst0 = -INFINITY, worst1 = -INFINITY;
+          for (int k = 0; k < 32; ++k) kb.offer(__uint_as_float(r[k]), c0 + x + k);
+        } else {
 #pragma unroll
-  for (int i = 0; i < kMaxTopk; ++i) {
-    bs0[i] = bs1[i] = -INFINITY;
-    bj0[i] = bj1[i] = -1;
-  }
-  // the scores of 8-block tile nt (c[0], c[1]: row r0; c[2], c[3]: row r0 + 8)
-  auto take = [&](const float (&c)[4], int j0) {
-    if (j0 < own) {
-      keep_best(bs0, bj0, want, worst0, c[0], j0);
-      keep_best(bs1, bj1, want, worst1, c[2], j0);
-    }
-    if (j0 + 1 < own) {
-      keep_best(bs0, bj0, want, worst0, c[1], j0 + 1);
-      keep_best(bs1, bj1, want, worst1, c[3], j0 + 1);
-    }
-  };
-  // chunk c0 .. c0 + 63 of the parts into buffer `buf`: 16-byte granules, a
-  // block's three part rows (768 B) are contiguous in kparts
-  auto stage = [&](int c0, int buf) {
-    const int nb = min(kGateBlk, own - c0);
-    __nv_bfloat16* dstb = kbs + (size_t)buf * kGateBuf;
-    constexpr int kGran = kGateBlk * 3 * (D / 8);  // granules per chunk
-#pragma unroll 1
-    for (int r = 0; r < kGran / 256; ++r) {
-      const int idx = threadIdx.x + r * 256, j = idx / (3 * D / 8), rem = idx - j * (3 * D / 8);
-      const int pp = rem / (D / 8), gr = rem - pp * (D / 8);
-      if (j < nb)
-        ptx::cp_async16(dstb + ((size_t)pp * kGateBlk + j) * kGatePitch + gr * 8,
-                        a.kparts + (((size_t)b * a.nfull + c0 + j) * a.Hkv + g) * 3 * D + pp * D +
-                            gr * 8);
-    }
-    ptx::cp_async_commit();
-  };
-  if (own > 0) stage(0, 0);
-  for (int c0 = 0, it = 0; c0 < own; c0 += kGateBlk, ++it) {
-    const int nb = min(kGateBlk, own - c0);
-    const __nv_bfloat16* kbuf = kbs + (size_t)(it & 1) * kGateBuf;
-    if (c0 + kGateBlk < own) {
-      stage(c0 + kGateBlk, (it + 1) & 1);  // its buffer was last read before the previous barrier
-      ptx::cp_async_wait<1>();
-    } else {
-      ptx::cp_async_wait<0>();
-    }
-    __syncthreads();
-    // two 8-block tiles at a time: two independent accumulator chains. B
-    // fragment column n = r0 is block c0 + 8 nt + r0; rows past nb are stale
-    // and their columns are discarded by take().
-    const int ntl = (nb + 7) / 8;
-    for (int nt = 0; nt < ntl; nt += 2) {
-      const bool two = nt + 1 < ntl;
-      float ca[4] = {0.f, 0.f, 0.f, 0.f}, cb[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int pp = 0; pp < 3; ++pp) {
-        const __nv_bfloat16* ka = kbuf + ((size_t)pp * kGateBlk + nt * 8 + r0) * kGatePitch;
-        const __nv_bfloat16* kb2 = ka + 8 * kGatePitch;
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          ptx::mma_16816(ca, qa[ks], ld_b32(ka + ks * 16 + q2), ld_b32(ka + ks * 16 + 8 + q2));
-          if (two)
-            ptx::mma_16816(cb, qa[ks], ld_b32(kb2 + ks * 16 + q2),
-                           ld_b32(kb2 + ks * 16 + 8 + q2));
+          for (int k = 0; k < 32; ++k)
+            if (x + k < nb) kb.offer(__uint_as_float(r[k]), c0 + x + k);
         }
       }
-      take(ca, c0 + nt * 8 + q2);  // blocks of c[0], c[2] and, + 1, of c[1], c[3]
-      if (two) take(cb, c0 + nt * 8 + 8 + q2);
+      tc::fence_before_sync();
+      ptx::mbar_arrive(&bars->acc_free[buf]);
     }
-    __syncthreads();  // this buffer is refilled two chunks on
+    if (t < a.T) kb.emit(a, it.b, it.h, t, it.own);
   }
-  int pick0[kMaxTopk], pick1[kMaxTopk];
-  quad_merge(bs0, bj0, want, pick0);
-  quad_merge(bs1, bj1, want, pick1);
-  // lane q = 0 writes row r0, q = 1 row r0 + 8
-  if ((lane & 3) > 1) return;
-  const int t = (lane & 3) == 0 ? ta : tb;
-  if (t >= a.T) return;
-  int row[kMaxTopk];
-  int n = 0;
-  if (own <= want) {
-    for (int j = 0; j <= own; ++j) row[n++] = j;
-  } else {
-#pragma unroll
-    for (int i = 0; i < kMaxTopk; ++i)
-      if (i < want) row[n++] = (lane & 3) == 0 ? pick0[i] : pick1[i];
-    for (int i = 1; i < n; ++i) {  // insertion sort, n <= 7
-      const int x = row[i];
-      int p = i - 1;
-      while (p >= 0 && row[p] > x) {
-        row[p + 1] = row[p];
-        --p;
+}
+
+// Warps 0-3: the rows (TMEM lane = row); warp 4 lane 0: TMA; warp 5 lane 0:
+// MMAs. One CTA per SM (grid = min(items, SMs)).
+__global__ void __launch_bounds__(kThreads, 1)
+    moba_gate_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tp,
+                     const MobaTcArgs a) {
+  extern __shared__ unsigned char smraw[];
+  unsigned char* base = align1024(smraw);
+  unsigned char* sQ = base;  // two query tiles
+  unsigned char* ring = base + 2 * TILE;
+  GateBars* bars = reinterpret_cast<GateBars*>(ring + kGateStages * TILE);
+  volatile int* abort = &bars->abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int want = a.topk - 1;
+  const int NI = a.B * a.Hq * ((a.T + KT - 1) / KT);
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kGateStages; ++i) {
+      ptx::mbar_init(&bars->full[i], 1);
+      ptx::mbar_init(&bars->empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&bars->q_full[i], 1);
+      ptx::mbar_init(&bars->q_free[i], 1);
+    }
+    for (int i = 0; i < kGateAcc; ++i) {
+      ptx::mbar_init(&bars->acc_full[i], 1);
+      ptx::mbar_init(&bars->acc_free[i], KT);
+    }
+    ptx::mbar_init(&bars->fin, 1);
+    bars->abort = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0) {
+    tc::tmem_alloc(&bars->tmem, kGateAcc * KT);
+    tc::tmem_relinquish();
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = bars->tmem;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      ptx::prefetch_tmap(&tq);
+      ptx::prefetch_tmap(&tp);
+      const uint64_t first = ptx::policy_evict_first(), keep = ptx::policy_evict_last();
+      int lastq[2] = {-1, -1}, last[kGateStages];
+      for (int s = 0; s < kGateStages; ++s) last[s] = -1;
+      int qi = 0, st = 0;
+      bool ok = true;
+      for (int i = blockIdx.x; ok && i < NI; i += gridDim.x) {
+        const GateItem it = gate_item(a, i, want);
+        if (it.nch == 0) continue;
+        const int qb = qi & 1;
+        if (qi >= 2 &&
+            !wait_or_abort(&bars->q_free[qb], (uint32_t)(((qi - 2) >> 1) & 1), abort, a.err))
+          break;
+        unsigned char* qd = sQ + qb * TILE;
+        ptx::mbar_arrive_expect_tx(&bars->q_full[qb], TILE);
+        ptx::tma_load_3d(qd, &tq, &bars->q_full[qb], 0, it.h, it.b * a.T + it.t0, first);
+        ptx::tma_load_3d(qd + ATOM, &tq, &bars->q_full[qb], 64, it.h, it.b * a.T + it.t0, first);
+        lastq[qb] = qi++;
+        const int z = (it.b * a.Hkv + it.h / (a.Hq / a.Hkv)) * 3;
+        for (int c = 0; ok && c < it.nch; ++c) {
+          const int c0 = c * KT, nbox = (min(KT, it.own - c0) + kGateBox - 1) / kGateBox;
+          for (int pp = 0; pp < 3; ++pp, ++st) {
+            const int s = st % kGateStages;
+            if (st >= kGateStages &&
+                !wait_or_abort(&bars->empty[s], (uint32_t)(((st / kGateStages) - 1) & 1), abort,
+                               a.err)) {
+              ok = false;
+              break;
+            }
+            unsigned char* dst = ring + s * TILE;
+            ptx::mbar_arrive_expect_tx(&bars->full[s], (uint32_t)(nbox * 2 * kGateBox * 128));
+            for (int x = 0; x < nbox; ++x) {
+              ptx::tma_load_3d(dst + x * kGateBox * 128, &tp, &bars->full[s], 0,
+                               c0 + x * kGateBox, z + pp, keep);
+              ptx::tma_load_3d(dst + ATOM + x * kGateBox * 128, &tp, &bars->full[s], 64,
+                               c0 + x * kGateBox, z + pp, keep);
+            }
+            last[s] = st;
+          }
+        }
       }
-      row[p + 1] = x;
+      // every issued load lands before the CTA can exit
+      for (int s = 0; s < kGateStages; ++s)
+        if (last[s] >= 0 &&
+            !ptx::mbar_wait(&bars->full[s], (uint32_t)((last[s] / kGateStages) & 1), kWaitNs))
+          atomicOr(a.err, kErrTimeout);
+      for (int s = 0; s < 2; ++s)
+        if (lastq[s] >= 0 &&
+            !ptx::mbar_wait(&bars->q_full[s], (uint32_t)((lastq[s] >> 1) & 1), kWaitNs))
+          atomicOr(a.err, kErrTimeout);
     }
-    row[n++] = own;
+  } else if (warp == 5) {
+    if (lane == 0) {
+      const uint32_t r0 = ptx::smem_u32(ring);
+      int qi = 0, st = 0, ac = 0;
+      bool ok = true;
+      for (int i = blockIdx.x; ok && i < NI; i += gridDim.x) {
+        const GateItem it = gate_item(a, i, want);
+        if (it.nch == 0) continue;
+        const int qb = qi & 1;
+        ok = wait_or_abort(&bars->q_full[qb], (uint32_t)((qi >> 1) & 1), abort, a.err);
+        tc::fence_after_sync();
+        const uint32_t q0 = ptx::smem_u32(sQ + qb * TILE);
+        for (int c = 0; ok && c < it.nch; ++c, ++ac) {
+          const int buf = ac % kGateAcc, nb = min(KT, it.own - c * KT);
+          const uint32_t id = tc::idesc_bf16(128, (nb + 15) & ~15, false, false);
+          if (ac >= kGateAcc) {
+            ok = wait_or_abort(&bars->acc_free[buf], (uint32_t)(((ac / kGateAcc) - 1) & 1), abort,
+                               a.err);
+            tc::fence_after_sync();
+          }
+          for (int pp = 0; ok && pp < 3; ++pp, ++st) {
+            const int s = st % kGateStages;
+            ok = wait_or_abort(&bars->full[s], (uint32_t)((st / kGateStages) & 1), abort, a.err);
+            if (!ok) break;
+            tc::fence_after_sync();
+            const uint32_t kb = r0 + s * TILE;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+              tc::mma_ss(tmem + buf * KT, kmaj(q0, ks), kmaj(kb, ks), id, (pp > 0 || ks > 0));
+            tc::commit(&bars->empty[s]);
+          }
+          if (ok) tc::commit(&bars->acc_full[buf]);
+        }
+        tc::commit(&bars->q_free[qb]);
+        ++qi;
+      }
+      tc::commit(&bars->fin);
+      if (!ptx::mbar_wait(&bars->fin, 0, kWaitNs)) atomicOr(a.err, kErrTimeout);
+    }
+  } else {
+    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+    const int row = warp * 32 + lane;
+    switch (want) {
+      case 0: gate_rows<1>(a, bars, abort, tl, row, want); break;  // no item is scored
+      case 1: gate_rows<1>(a, bars, abort, tl, row, want); break;
+      case 2: gate_rows<2>(a, bars, abort, tl, row, want); break;
+      case 3: gate_rows<3>(a, bars, abort, tl, row, want); break;
+      case 4: gate_rows<4>(a, bars, abort, tl, row, want); break;
+      case 5: gate_rows<5>(a, bars, abort, tl, row, want); break;
+      case 6: gate_rows<6>(a, bars, abort, tl, row, want); break;
+      default: gate_rows<7>(a, bars, abort, tl, row, want); break;
+    }
   }
-  int32_t* dst = a.sel + ((size_t)(b * a.T + t) * a.Hq + h) * a.topk;
-  for (int i = 0; i < a.topk; ++i) dst[i] = i < n ? row[i] : -1;
-  for (int i = 0; i + 1 < n; ++i)  // every entry but the own block is a past pick
-    atomicAdd(a.cnt + ((size_t)b * a.Hq + h) * a.nfull + row[i], 1);
+
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  if (warp == 0) tc::tmem_dealloc(tmem, kGateAcc * KT);
 }
 
 // Each fp32 block mean once into three bf16 parts hi + mid + lo (hi = bf16(x),
 // mid = bf16(x - hi), lo = bf16(x - hi - mid): 24 significant bits), so every
-// product with a bf16 query element is exact in fp32.
+// product with a bf16 query element is exact in fp32. Layout
+// [B, Hkv, 3, gate_rows(nfull), d]; the padding rows are zero.
 __global__ void __launch_bounds__(256) moba_split_kernel(MobaTcArgs a) {
-  const size_t n4 = (size_t)a.B * a.nfull * a.Hkv * (D / 4);
+  const int nr = gate_rows(a.nfull);
+  const size_t n4 = (size_t)a.B * a.Hkv * nr * (D / 4);
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n4;
        i += (size_t)gridDim.x * blockDim.x) {
-    const size_t row = i / (D / 4);
-    const int e = (int)(i - row * (D / 4)) * 4;
-    const float4 x = reinterpret_cast<const float4*>(a.kbar + row * D + e)[0];
-    const float xs[4] = {x.x, x.y, x.z, x.w};
+    const size_t rest = i / (D / 4);
+    const int e = (int)(i - rest * (D / 4)) * 4;
+    const int j = (int)(rest % nr);
+    const size_t bg = rest / nr;
+    const int b = (int)(bg / a.Hkv), g = (int)(bg % a.Hkv);
+    float xs[4] = {0.f, 0.f, 0.f, 0.f};
+    if (j < a.nfull) {
+      const float4 x =
+          reinterpret_cast<const float4*>(a.kbar + (((size_t)b * a.nfull + j) * a.Hkv + g) * D + e)[0];
+      xs[0] = x.x;
+      xs[1] = x.y;
+      xs[2] = x.z;
+      xs[3] = x.w;
+    }
     __nv_bfloat16 hi[4], mid[4], lo[4];
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -307,13 +439,12 @@ __global__ void __launch_bounds__(256) moba_split_kernel(MobaTcArgs a) {
       mid[k] = __float2bfloat16_rn(r1);
       lo[k] = __float2bfloat16_rn(r1 - __bfloat162float(mid[k]));
     }
-    __nv_bfloat16* dst = a.kparts + row * 3 * D + e;
+    __nv_bfloat16* dst = a.kparts + (bg * 3 * nr + j) * D + e;
     *reinterpret_cast<uint2*>(dst) = *reinterpret_cast<const uint2*>(hi);
-    *reinterpret_cast<uint2*>(dst + D) = *reinterpret_cast<const uint2*>(mid);
-    *reinterpret_cast<uint2*>(dst + 2 * D) = *reinterpret_cast<const uint2*>(lo);
+    *reinterpret_cast<uint2*>(dst + (size_t)nr * D) = *reinterpret_cast<const uint2*>(mid);
+    *reinterpret_cast<uint2*>(dst + 2 * (size_t)nr * D) = *reinterpret_cast<const uint2*>(lo);
   }
 }
-
 // Exclusive prefix sums of the bucket counts (rows) and of their 128-row
 // tiles, in one CTA.
 __global__ void __launch_bounds__(1024) moba_scan_kernel(MobaTcArgs a) {
@@ -892,7 +1023,7 @@ size_t moba_tc_ws_bytes(const nsa_params& p, size_t kbar_bytes) {
   const size_t rows = (size_t)p.B * p.T * p.Hq;
   const size_t NB = (size_t)p.B * p.Hq * (p.T / p.sel_block);
   const size_t np = (size_t)(p.top_n - 1);
-  const size_t parts = (size_t)p.B * (p.T / p.sel_block) * p.Hkv * 3 * D * 2;
+  const size_t parts = (size_t)p.B * p.Hkv * 3 * gate_rows(p.T / p.sel_block) * D * 2;
   return align256(kbar_bytes) + align256(rows * p.top_n * 4) + 4 * align256((NB + 1) * 4) +
          align256(rows * np * 4 + 4) + align256(rows * np * D * 2 + 4) + align256(rows * np * 4 + 4) +
          align256(parts + 4);
@@ -940,8 +1071,10 @@ cudaError_t launch_moba_tc(const nsa_params& p, const void* q, const void* k, co
   a.c = scale * 1.4426950408889634f;
 
   const uint64_t BT = (uint64_t)p.B * p.T;
-  CUtensorMap tq, tk, tv;
+  CUtensorMap tq, tk, tv, tp;
   if (!make_tmap_bf16_3d(&tq, q, D, p.Hq, BT, 64, 1, KT, true) ||
+      !make_tmap_bf16_3d(&tp, a.kparts, D, gate_rows(a.nfull), (uint64_t)p.B * p.Hkv * 3, 64,
+                         kGateBox, 1, true) ||
       !make_tmap_bf16_3d(&tk, k, D, p.Hkv, BT, 64, 1, KT, true) ||
       !make_tmap_bf16_3d(&tv, v, D, p.Hkv, BT, 64, 1, KT, true))
     return cudaErrorInvalidValue;
@@ -950,17 +1083,18 @@ cudaError_t launch_moba_tc(const nsa_params& p, const void* q, const void* k, co
   if (a.NB > 0 && (e = cudaMemsetAsync(a.cnt, 0, (size_t)a.NB * 4, stream)) != cudaSuccess) return e;
   if (a.nfull > 0) {
     TraceScope trace("moba_split", stream);
-    const size_t n4 = (size_t)a.B * a.nfull * a.Hkv * (D / 4);
+    const size_t n4 = (size_t)a.B * a.Hkv * gate_rows(a.nfull) * (D / 4);
     const int grid = (int)std::min<size_t>((n4 + 255) / 256, (size_t)device_sm_count() * 8);
     moba_split_kernel<<<grid, 256, 0, stream>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   {
     TraceScope trace("moba_gate", stream);
-    if ((e = ensure_dyn_smem((const void*)moba_gate_kernel, (int)kGateSmem)) != cudaSuccess)
+    if ((e = ensure_dyn_smem((const void*)moba_gate_kernel, (int)gate_smem())) != cudaSuccess)
       return e;
-    dim3 grid((p.T + kGateTok - 1) / kGateTok, p.Hq, p.B);
-    moba_gate_kernel<<<grid, 256, kGateSmem, stream>>>(a);
+    const long long items = (long long)p.B * p.Hq * ((p.T + KT - 1) / KT);
+    const int grid = (int)std::min<long long>(items, device_sm_count());
+    moba_gate_kernel<<<grid, kThreads, gate_smem(), stream>>>(tq, tp, a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if (a.NB > 0 && p.top_n > 1) {

@@ -70,7 +70,8 @@ def test_workspace_size_validation():
     kbar = a256(B * (T // m) * H * 128 * 4)
     rows, nb = B * T * H, B * H * (T // m)
     moba = nsa.params(B, T, H, H, 128, sel_block=m, top_n=k)
-    parts = a256(B * (T // m) * H * 3 * 128 * 2 + 4)  # the means split into three bf16 parts
+    rows_g = max(32, -(-(T // m) // 32) * 32)  # block rows per part, padded to 32-row boxes
+    parts = a256(B * H * 3 * rows_g * 128 * 2 + 4)  # the means split into three bf16 parts
     assert nsa.workspace_size(moba, nsa.OP_MOBA_PREFILL) == (
         kbar + a256(rows * k * 4) + 4 * a256((nb + 1) * 4) + a256(rows * (k - 1) * 4 + 4) +
         a256(rows * (k - 1) * 128 * 2 + 4) + a256(rows * (k - 1) * 4 + 4) + parts)

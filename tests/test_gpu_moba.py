@@ -50,6 +50,14 @@ def test_moba_bf16_tensor_core_edges(over):
     gc.run_moba(w, seed=9)
 
 
+def test_moba_bf16_more_than_two_gate_chunks():
+    # 320 blocks of 128: the gate scores up to 319 past blocks in three
+    # 128-block chunks, reusing its two score buffers; ragged last tile
+    w = inputs.workload("moba_prefill_bf16_t131072", T=41000, Hq=2, Hkv=1, block=128, top_k=4)
+    rows = gc.sample_rows(41000, 160) + [(0, 40999), (0, 32768), (0, 32767), (0, 16384)]
+    gc.run_moba(w, rows=rows, seed=5)
+
+
 def test_moba_bf16_runs_the_tensor_core_kernels():
     from dynamic_block_sparse_nsa_b200 import nsa
     w = inputs.workload("moba_prefill_bf16_t131072", T=2048, Hq=2, Hkv=2, block=256, top_k=3)
