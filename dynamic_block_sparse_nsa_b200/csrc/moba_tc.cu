@@ -873,25 +873,147 @@ __global__ void __launch_bounds__(kThreads, 1)
 // moba_own: own block, causal, merged with the partials
 // ============================================================================
 
+// Work item i: 128 consecutive tokens of one (sequence, head), the heads of a
+// token tile adjacent (the tiles of one block and head, which share its keys,
+// run at about the same time on different SMs).
+struct OwnItem {
+  int b, h, t0, c0, nk;
+};
+
+__device__ __forceinline__ OwnItem own_item(const MobaTcArgs& a, int i) {
+  OwnItem it;
+  const int bh = i % (a.B * a.Hq);
+  it.b = bh / a.Hq;
+  it.h = bh % a.Hq;
+  it.t0 = (i / (a.B * a.Hq)) * KT;
+  const int tlast = min(it.t0 + KT - 1, a.T - 1);
+  it.c0 = (it.t0 / a.m) * a.m;  // own block start (a 128-token tile never straddles blocks)
+  it.nk = (tlast - it.c0) / KT + 1;
+  return it;
+}
+
+// Merge of a row: its own-block output (o / l, log2-sum-exp m + log2 l, o in
+// TMEM once the last PV MMA is done) with its np partials (normalised, bf16)
+// and their log2-sum-exps: out = sum_i 2^(lse_i - M) o_i / sum_i 2^(lse_i - M).
+__device__ __forceinline__ void merge_weights(const float* plse, int np, float m, float l,
+                                              float& wown, float (&wp)[kMaxTopk], float& inv) {
+  float lse[kMaxTopk];
+  float M = m + __log2f(l);  // key t itself is always visible: l > 0
+  const float lown = M;
+#pragma unroll
+  for (int s = 0; s < kMaxTopk - 1; ++s) {
+    lse[s] = s < np ? plse[s] : -INFINITY;
+    M = fmaxf(M, lse[s]);
+  }
+  wown = exp2f(lown - M) / l;
+  float wsum = exp2f(lown - M);
+#pragma unroll
+  for (int s = 0; s < kMaxTopk - 1; ++s) {
+    wp[s] = s < np ? exp2f(lse[s] - M) : 0.f;
+    wsum += wp[s];
+  }
+  inv = 1.f / wsum;
+}
+
+__device__ __forceinline__ void store_row16(__nv_bfloat16* dst, const float (&acc)[16], float inv) {
+  uint4 pk[2];
+  uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) pw[e] = ptx::pack_bf16(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+  reinterpret_cast<uint4*>(dst)[0] = pk[0];
+  reinterpret_cast<uint4*>(dst)[1] = pk[1];
+}
+
+__device__ __forceinline__ void add_partial(float (&acc)[16], float w, uint4 a0, uint4 a1) {
+  const __nv_bfloat162* e0 = reinterpret_cast<const __nv_bfloat162*>(&a0);
+  const __nv_bfloat162* e1 = reinterpret_cast<const __nv_bfloat162*>(&a1);
+#pragma unroll
+  for (int y = 0; y < 4; ++y) {
+    const float2 f = __bfloat1622float2(e0[y]), g = __bfloat1622float2(e1[y]);
+    acc[2 * y] = fmaf(w, f.x, acc[2 * y]);
+    acc[2 * y + 1] = fmaf(w, f.y, acc[2 * y + 1]);
+    acc[8 + 2 * y] = fmaf(w, g.x, acc[8 + 2 * y]);
+    acc[8 + 2 * y + 1] = fmaf(w, g.y, acc[8 + 2 * y + 1]);
+  }
+}
+
+// Up to two partials (top_k <= 3): both rows (2 x 256 B) and their
+// log2-sum-exps are loaded together, while the last PV MMA finishes, so the
+// merge waits for memory once.
+__device__ __forceinline__ void own_merge_preloaded(const MobaTcArgs& a, Softmax& sm, size_t prow,
+                                                    int np, float m, float l, bool live,
+                                                    __nv_bfloat16* dst) {
+  uint4 p0[16], p1[16];
+  float pl[kMaxTopk];
+  const uint4* s0 = reinterpret_cast<const uint4*>(a.po + prow * D);
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    p0[c] = np > 0 ? __ldg(s0 + c) : make_uint4(0, 0, 0, 0);
+    p1[c] = np > 1 ? __ldg(s0 + 16 + c) : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int s = 0; s < kMaxTopk; ++s) pl[s] = s < np ? a.plse[prow + s] : -INFINITY;
+  wait_or_abort(&sm.bars->o_done[(sm.j - 1) & 1], (uint32_t)(((sm.j - 1) >> 1) & 1), sm.abort,
+                sm.err);
+  tc::fence_after_sync();
+  float wown, wp[kMaxTopk], inv;
+  merge_weights(pl, np, m, l, wown, wp, inv);
+#pragma unroll
+  for (int c16 = 0; c16 < 8; ++c16) {
+    uint32_t o[16];
+    tc::ld16_sync(sm.tl + kO + c16 * 16, o);
+    float acc[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) acc[e] = __uint_as_float(o[e]) * wown;
+    add_partial(acc, wp[0], p0[2 * c16], p0[2 * c16 + 1]);
+    add_partial(acc, wp[1], p1[2 * c16], p1[2 * c16 + 1]);
+    if (live) store_row16(dst + c16 * 16, acc, inv);
+  }
+}
+
+// Any number of partials: 16 columns at a time (two chunks' loads in flight).
+__device__ __forceinline__ void own_merge_chunked(const MobaTcArgs& a, Softmax& sm, size_t prow,
+                                                  int np, float m, float l, bool live,
+                                                  __nv_bfloat16* dst) {
+  if (np > 0) ptx::bulk_prefetch_l2(a.po + prow * D, (uint32_t)(np * D * 2));
+  wait_or_abort(&sm.bars->o_done[(sm.j - 1) & 1], (uint32_t)(((sm.j - 1) >> 1) & 1), sm.abort,
+                sm.err);
+  tc::fence_after_sync();
+  float wown, wp[kMaxTopk], inv;
+  merge_weights(a.plse + prow, np, m, l, wown, wp, inv);
+#pragma unroll 2
+  for (int c16 = 0; c16 < 8; ++c16) {
+    uint32_t o[16];
+    tc::ld16_sync(sm.tl + kO + c16 * 16, o);
+    float acc[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) acc[e] = __uint_as_float(o[e]) * wown;
+#pragma unroll
+    for (int s = 0; s < kMaxTopk - 1; ++s) {
+      if (s >= np) break;
+      const uint4* ps = reinterpret_cast<const uint4*>(a.po + (prow + s) * D + c16 * 16);
+      add_partial(acc, wp[s], __ldg(ps), __ldg(ps + 1));
+    }
+    if (live) store_row16(dst + c16 * 16, acc, inv);
+  }
+}
+
+// Persistent, one CTA per SM: lanes 0-3 of warp 0 load the query tiles (two
+// buffers, lane 0) and the K / V tiles (a four-stage ring), warp 1 lane 0
+// issues the MMAs, warps 2-5 run the softmax and the merge, so one item's
+// merge overlaps the next item's first MMAs and loads.
 __global__ void __launch_bounds__(kThreads, 1)
     moba_own_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                     const __grid_constant__ CUtensorMap tv, const MobaTcArgs a) {
   extern __shared__ unsigned char smraw[];
   unsigned char* base = align1024(smraw);
-  unsigned char* sQ = base;
-  unsigned char* ring = base + TILE;
+  unsigned char* sQ = base;  // 2 x 32 KB
+  unsigned char* ring = base + 2 * TILE;
   Bars* bars = reinterpret_cast<Bars*>(ring + kStages * TILE);
   volatile int* abort = &bars->abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int ntq = (a.T + KT - 1) / KT;
-  const int bh = blockIdx.x % (a.B * a.Hq);
-  const int r = blockIdx.x / (a.B * a.Hq);
-  const int b = bh / a.Hq, h = bh % a.Hq, g = h / (a.Hq / a.Hkv);
-  const int t0 = r * KT;
-  const int tlast = min(t0 + KT - 1, a.T - 1);
-  const int c0 = (t0 / a.m) * a.m;  // own block start (a 128-token tile never straddles blocks)
-  const int nk = (tlast - c0) / KT + 1;
-  (void)ntq;
+  const int NI = a.B * a.Hq * ((a.T + KT - 1) / KT);
+  const int G = a.Hq / a.Hkv;
 
   if (threadIdx.x == 0) init_bars(bars, 1);
   if (warp == 1) {
@@ -909,90 +1031,73 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::prefetch_tmap(&tq);
         ptx::prefetch_tmap(&tk);
         ptx::prefetch_tmap(&tv);
-        ptx::mbar_arrive_expect_tx(&bars->q_full[0], TILE);
-        ptx::tma_load_3d(sQ, &tq, &bars->q_full[0], 0, h, b * a.T + t0, ptx::policy_evict_first());
-        ptx::tma_load_3d(sQ + ATOM, &tq, &bars->q_full[0], 64, h, b * a.T + t0,
-                         ptx::policy_evict_first());
       }
       Producer pr{ring, bars, abort, a.err, lane};
-      const uint64_t keep = ptx::policy_evict_last();
-      const int z0 = b * a.T + c0;
-      for (int u = 0; u < nk; ++u) {
-        pr.load(&tk, g, z0 + u * KT, keep);
-        if (u >= 1) pr.load(&tv, g, z0 + (u - 1) * KT, keep);
+      const uint64_t first = ptx::policy_evict_first(), keep = ptx::policy_evict_last();
+      int kq = 0, lastq[2] = {-1, -1};
+      for (int i = blockIdx.x; pr.ok && i < NI; i += gridDim.x, ++kq) {
+        const OwnItem it = own_item(a, i);
+        if (lane == 0) {
+          const int qb = kq & 1;
+          if (kq >= 2 &&
+              !wait_or_abort(&bars->q_free[qb], (uint32_t)(((kq >> 1) - 1) & 1), abort, a.err)) {
+            pr.ok = false;
+            break;
+          }
+          unsigned char* qd = sQ + qb * TILE;
+          ptx::mbar_arrive_expect_tx(&bars->q_full[qb], TILE);
+          ptx::tma_load_3d(qd, &tq, &bars->q_full[qb], 0, it.h, it.b * a.T + it.t0, first);
+          ptx::tma_load_3d(qd + ATOM, &tq, &bars->q_full[qb], 64, it.h, it.b * a.T + it.t0,
+                           first);
+          lastq[qb] = kq;
+        }
+        const int g = it.h / G, z0 = it.b * a.T + it.c0;
+        for (int u = 0; u < it.nk; ++u) {
+          pr.load(&tk, g, z0 + u * KT, keep);
+          if (u >= 1) pr.load(&tv, g, z0 + (u - 1) * KT, keep);
+        }
+        pr.load(&tv, g, z0 + (it.nk - 1) * KT, keep);
       }
-      pr.load(&tv, g, z0 + (nk - 1) * KT, keep);
       pr.drain();
+      if (lane == 0)  // every issued query load lands before the CTA can exit
+        for (int s = 0; s < 2; ++s)
+          if (lastq[s] >= 0 &&
+              !ptx::mbar_wait(&bars->q_full[s], (uint32_t)((lastq[s] >> 1) & 1), kWaitNs))
+            atomicOr(a.err, kErrTimeout);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       Mma mm{bars, abort, a.err, tmem, ptx::smem_u32(ring)};
-      mm.ok = wait_or_abort(&bars->q_full[0], 0, abort, a.err);
-      tc::fence_after_sync();
-      mm.tile(ptx::smem_u32(sQ), nk, 0);
+      int kq = 0;
+      for (int i = blockIdx.x; mm.ok && i < NI; i += gridDim.x, ++kq) {
+        const OwnItem it = own_item(a, i);
+        const int qb = kq & 1;
+        mm.ok = wait_or_abort(&bars->q_full[qb], (uint32_t)((kq >> 1) & 1), abort, a.err);
+        tc::fence_after_sync();
+        mm.tile(ptx::smem_u32(sQ + qb * TILE), it.nk, qb);
+      }
       tc::commit(&bars->fin);
       if (!ptx::mbar_wait(&bars->fin, 0, kWaitNs)) atomicOr(a.err, kErrTimeout);
     }
   } else {
     const int qd = warp & 3;
     const int row = qd * 32 + lane;
-    const int t = min(t0 + row, a.T - 1);
-    const bool live = t0 + row < a.T;
     Softmax sm{bars, abort, a.err, tmem + ((uint32_t)(qd * 32) << 16), a.c};
-    float m = -INFINITY, l = 0.f;
-    for (int u = 0; u < nk; ++u) sm.tile(c0 + u * KT, t + 1, m, l);
-    wait_or_abort(&bars->o_done[(nk - 1) & 1], (uint32_t)(((nk - 1) >> 1) & 1), abort, a.err);
-    tc::fence_after_sync();
-    // merge: own (o / l, lse = m + log2 l) with the row's partials
-    const int npast = min(a.topk - 1, t / a.m);
-    const size_t prow = ((size_t)(b * a.T + t) * a.Hq + h) * (a.topk - 1);
-    float lse[kMaxTopk];
-    float M = m + __log2f(l);  // key t itself is always visible: l > 0
-    const float lown = M;
-#pragma unroll
-    for (int s = 0; s < kMaxTopk - 1; ++s) {
-      lse[s] = (live && s < npast) ? a.plse[prow + s] : -INFINITY;
-      M = fmaxf(M, lse[s]);
-    }
-    const float wown = exp2f(lown - M) / l;
-    float wsum = exp2f(lown - M);
-    float wp[kMaxTopk];
-#pragma unroll
-    for (int s = 0; s < kMaxTopk - 1; ++s) {
-      wp[s] = s < npast ? exp2f(lse[s] - M) : 0.f;
-      wsum += wp[s];
-    }
-    const float inv = 1.f / wsum;
-    __nv_bfloat16* dst = a.out + ((size_t)(b * a.T + t) * a.Hq + h) * D;
-#pragma unroll 1
-    for (int c16 = 0; c16 < 8; ++c16) {
-      uint32_t o[16];
-      tc::ld16_sync(sm.tl + kO + c16 * 16, o);
-      float acc[16];
-#pragma unroll
-      for (int e = 0; e < 16; ++e) acc[e] = __uint_as_float(o[e]) * wown;
-      for (int s = 0; s < npast; ++s) {
-        const uint4* ps = reinterpret_cast<const uint4*>(a.po + (prow + s) * D + c16 * 16);
-#pragma unroll
-        for (int x = 0; x < 2; ++x) {
-          const uint4 pv = __ldg(ps + x);
-          const __nv_bfloat162* e2 = reinterpret_cast<const __nv_bfloat162*>(&pv);
-#pragma unroll
-          for (int y = 0; y < 4; ++y) {
-            const float2 f = __bfloat1622float2(e2[y]);
-            acc[8 * x + 2 * y] = fmaf(wp[s], f.x, acc[8 * x + 2 * y]);
-            acc[8 * x + 2 * y + 1] = fmaf(wp[s], f.y, acc[8 * x + 2 * y + 1]);
-          }
-        }
-      }
-      if (live) {
-        uint4 pk[2];
-        uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) pw[e] = ptx::pack_bf16(acc[2 * e] * inv, acc[2 * e + 1] * inv);
-        reinterpret_cast<uint4*>(dst + c16 * 16)[0] = pk[0];
-        reinterpret_cast<uint4*>(dst + c16 * 16)[1] = pk[1];
-      }
+    for (int i = blockIdx.x; i < NI && !*abort; i += gridDim.x) {
+      const OwnItem it = own_item(a, i);
+      const int t = min(it.t0 + row, a.T - 1);
+      const bool live = it.t0 + row < a.T;
+      const int npast = min(a.topk - 1, t / a.m);
+      const size_t prow = ((size_t)(it.b * a.T + t) * a.Hq + it.h) * (a.topk - 1);
+      float m = -INFINITY, l = 0.f;
+      for (int u = 0; u < it.nk; ++u) sm.tile(it.c0 + u * KT, t + 1, m, l);
+      __nv_bfloat16* dst = a.out + ((size_t)(it.b * a.T + t) * a.Hq + it.h) * D;
+      const int np = live ? npast : 0;
+      if (a.topk <= 3)
+        own_merge_preloaded(a, sm, prow, np, m, l, live, dst);
+      else
+        own_merge_chunked(a, sm, prow, np, m, l, live, dst);
+      tc::fence_before_sync();
     }
   }
 
@@ -1119,11 +1224,12 @@ cudaError_t launch_moba_tc(const nsa_params& p, const void* q, const void* k, co
     }
   }
   {
-    const size_t sm = attn_smem(1);
+    const size_t sm = attn_smem(2);
     if ((e = ensure_dyn_smem((const void*)moba_own_kernel, (int)sm)) != cudaSuccess) return e;
     TraceScope trace("moba_own", stream);
-    const long long grid = (long long)p.B * p.Hq * ((p.T + KT - 1) / KT);
-    moba_own_kernel<<<(unsigned)grid, kThreads, sm, stream>>>(tq, tk, tv, a);
+    const long long items = (long long)p.B * p.Hq * ((p.T + KT - 1) / KT);
+    const int grid = (int)std::min<long long>(items, device_sm_count());
+    moba_own_kernel<<<grid, kThreads, sm, stream>>>(tq, tk, tv, a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;
