@@ -54,6 +54,7 @@ struct MobaTcArgs {
   int32_t* toff;          // [NB + 1] first tile of each bucket
   int32_t* cur;           // [NB] fill cursors
   int32_t* list;          // rows: t * 8 + slot
+  int32_t* tbkt;          // [tiles] the bucket of each 128-row bucket tile
   __nv_bfloat16* po;      // [B, T, Hq, topk - 1, d] partial outputs (normalised, bf16)
   float* plse;            // [B, T, Hq, topk - 1] their log2-sum-exp
   unsigned* err;
@@ -502,8 +503,11 @@ __global__ void __launch_bounds__(1024) moba_scan_kernel(MobaTcArgs a) {
   if (threadIdx.x == 0) a.toff[a.NB] = carry[1];
 }
 
-// Rows into buckets: list[off[bucket] + k] = t * 8 + slot.
+// Rows into buckets: list[off[bucket] + k] = t * 8 + slot; and the bucket of
+// every bucket tile: tbkt[toff[bucket] + k] = bucket.
 __global__ void moba_fill_kernel(MobaTcArgs a) {
+  for (int bk = blockIdx.x * blockDim.x + threadIdx.x; bk < a.NB; bk += gridDim.x * blockDim.x)
+    for (int k = a.toff[bk]; k < a.toff[bk + 1]; ++k) a.tbkt[k] = bk;
   const long long n = (long long)a.B * a.T * a.Hq;
   for (long long r = blockIdx.x * (long long)blockDim.x + threadIdx.x; r < n;
        r += (long long)gridDim.x * blockDim.x) {
@@ -717,23 +721,13 @@ struct Softmax {
 // moba_blk: bucket tiles (gathered rows x one earlier block)
 // ============================================================================
 
-__device__ __forceinline__ int tile_bucket(const MobaTcArgs& a, int i) {
-  int lo = 0, hi = a.NB - 1;  // largest bucket with toff <= i
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (a.toff[mid] <= i) lo = mid;
-    else hi = mid - 1;
-  }
-  return lo;
-}
-
 struct BlkTile {
   int b, h, j, first, nrow;  // rows list[first .. first + nrow)
 };
 
 __device__ __forceinline__ BlkTile blk_tile(const MobaTcArgs& a, int i) {
   BlkTile w;
-  const int bk = tile_bucket(a, i);
+  const int bk = a.tbkt[i];
   w.j = bk % a.nfull;
   const int bh = bk / a.nfull;
   w.h = bh % a.Hq;
@@ -776,8 +770,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       Producer pr{ring, bars, abort, a.err, lane};
       const uint64_t keep = ptx::policy_evict_last();
+      BlkTile wn = blockIdx.x < (unsigned)ntile ? blk_tile(a, blockIdx.x) : BlkTile{};
       for (int i = blockIdx.x; pr.ok && i < ntile; i += gridDim.x) {
-        const BlkTile w = blk_tile(a, i);
+        const BlkTile w = wn;
+        if (i + (int)gridDim.x < ntile) wn = blk_tile(a, i + gridDim.x);  // in flight meanwhile
         const int g = w.h / G;
         const int z0 = w.b * a.T + w.j * a.m;
         for (int u = 0; u < nk; ++u) {
@@ -805,61 +801,83 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int qd = warp & 3;
     const int row = qd * 32 + lane;
     Softmax sm{bars, abort, a.err, tmem + ((uint32_t)(qd * 32) << 16), a.c};
-    // gather 128 query rows of tile i into Q buffer qb (zeros past the bucket)
-    auto gather = [&](int i, int kq) {
+    // The query rows of tile k + 1 are copied (cp.async, this thread's row,
+    // zeros past the bucket) while tile k's softmax runs, and handed to the
+    // MMA thread after it; the tile descriptors and list entries they need
+    // are loaded one tile further ahead still.
+    auto gather = [&](const BlkTile& w, int e, int kq) {
       const int qb = kq & 1;
       if (kq >= 2) wait_or_abort(&bars->q_free[qb], (uint32_t)(((kq >> 1) - 1) & 1), abort, a.err);
-      const BlkTile w = blk_tile(a, i);
       unsigned char* dq = sQ + qb * TILE;
-      uint4 v[16];
-      if (row < w.nrow) {
-        const int e = a.list[w.first + row];
-        const uint4* src = reinterpret_cast<const uint4*>(
-            a.q + ((size_t)(w.b * a.T + (e >> 3)) * a.Hq + w.h) * D);
-#pragma unroll
-        for (int c = 0; c < 16; ++c) v[c] = __ldg(src + c);
-      } else {
-#pragma unroll
-        for (int c = 0; c < 16; ++c) v[c] = make_uint4(0, 0, 0, 0);
-      }
+      const bool live = e >= 0;
+      const __nv_bfloat16* src =
+          a.q + ((size_t)(w.b * a.T + (live ? e >> 3 : 0)) * a.Hq + w.h) * D;
 #pragma unroll
       for (int c = 0; c < 16; ++c)
-        *reinterpret_cast<uint4*>(dq + (c >> 3) * ATOM + row * 128 + (((c & 7) ^ (row & 7)) << 4)) =
-            v[c];
-      ptx::fence_proxy_async();
-      ptx::mbar_arrive(&bars->q_full[qb]);
+        ptx::cp_async16_zfill(dq + (c >> 3) * ATOM + row * 128 + (((c & 7) ^ (row & 7)) << 4),
+                              src + c * 8, live ? 16u : 0u);
+      ptx::cp_async_commit();
     };
-    int k = 0;
-    if (blockIdx.x < (unsigned)ntile) gather(blockIdx.x, 0);
-    for (int i = blockIdx.x; i < ntile; i += gridDim.x, ++k) {
-      if (i + (int)gridDim.x < ntile) gather(i + gridDim.x, k + 1);
-      const BlkTile w = blk_tile(a, i);
-      float m = -INFINITY, l = 0.f;
-      for (int u = 0; u < nk; ++u) sm.tile(u * KT, 1 << 30, m, l);
-      wait_or_abort(&bars->o_done[(sm.j - 1) & 1], (uint32_t)(((sm.j - 1) >> 1) & 1), abort,
-                    a.err);
-      tc::fence_after_sync();
-      const bool live = row < w.nrow;
-      const int e = live ? a.list[w.first + row] : 0;
-      const size_t pr = ((size_t)(w.b * a.T + (e >> 3)) * a.Hq + w.h) * (a.topk - 1) + (e & 7);
-      const float il = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll 1
-      for (int c16 = 0; c16 < 8; ++c16) {
-        uint32_t o[16];
-        tc::ld16_sync(sm.tl + kO + c16 * 16, o);
-        if (live) {
-          uint4 pk[2];
-          uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
-#pragma unroll
-          for (int x = 0; x < 8; ++x)
-            pw[x] = ptx::pack_bf16(__uint_as_float(o[2 * x]) * il, __uint_as_float(o[2 * x + 1]) * il);
-          uint4* dst = reinterpret_cast<uint4*>(a.po + pr * D + c16 * 16);
-          dst[0] = pk[0];
-          dst[1] = pk[1];
-        }
+    auto hand_over = [&](int kq) {
+      ptx::cp_async_wait<0>();
+      ptx::fence_proxy_async();
+      ptx::mbar_arrive(&bars->q_full[kq & 1]);
+    };
+    auto entry = [&](const BlkTile& w) { return row < w.nrow ? a.list[w.first + row] : -1; };
+    if (blockIdx.x < (unsigned)ntile) {
+      const int G1 = gridDim.x;
+      BlkTile cur = blk_tile(a, blockIdx.x);
+      int ecur = entry(cur);
+      gather(cur, ecur, 0);
+      hand_over(0);
+      BlkTile nxt{};
+      int enxt = -1;
+      if ((int)blockIdx.x + G1 < ntile) {
+        nxt = blk_tile(a, blockIdx.x + G1);
+        enxt = entry(nxt);
       }
-      if (live) a.plse[pr] = m + __log2f(l);
-      tc::fence_before_sync();
+      int k = 0;
+      for (int i = blockIdx.x; i < ntile && !*abort; i += G1, ++k) {
+        const bool more = i + G1 < ntile, more2 = i + 2 * G1 < ntile;
+        if (more) gather(nxt, enxt, k + 1);
+        BlkTile nn{};
+        if (more2) nn = blk_tile(a, i + 2 * G1);  // in flight during the softmax
+        float m = -INFINITY, l = 0.f;
+        for (int u = 0; u < nk; ++u) sm.tile(u * KT, 1 << 30, m, l);
+        const int enn = more2 ? entry(nn) : -1;  // in flight during the epilogue
+        if (more) hand_over(k + 1);
+        wait_or_abort(&bars->o_done[(sm.j - 1) & 1], (uint32_t)(((sm.j - 1) >> 1) & 1), abort,
+                      a.err);
+        tc::fence_after_sync();
+        const bool live = ecur >= 0;
+        const int e = live ? ecur : 0;
+        const size_t pr =
+            ((size_t)(cur.b * a.T + (e >> 3)) * a.Hq + cur.h) * (a.topk - 1) + (e & 7);
+        const float il = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll 1
+        for (int c16 = 0; c16 < 8; ++c16) {
+          uint32_t o[16];
+          tc::ld16_sync(sm.tl + kO + c16 * 16, o);
+          if (live) {
+            uint4 pk[2];
+            uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
+#pragma unroll
+            for (int x = 0; x < 8; ++x)
+              pw[x] = ptx::pack_bf16(__uint_as_float(o[2 * x]) * il,
+                                     __uint_as_float(o[2 * x + 1]) * il);
+            uint4* dst = reinterpret_cast<uint4*>(a.po + pr * D + c16 * 16);
+            dst[0] = pk[0];
+            dst[1] = pk[1];
+          }
+        }
+        if (live) a.plse[pr] = m + __log2f(l);
+        tc::fence_before_sync();
+        cur = nxt;
+        ecur = enxt;
+        nxt = nn;
+        enxt = enn;
+      }
+      ptx::cp_async_wait<0>();  // no copy in flight past an abort
     }
   }
 
@@ -1123,7 +1141,9 @@ bool moba_tc_eligible(const nsa_params& p) {
 
 // Workspace after the block means: selection (when the caller passes none),
 // bucket counts / offsets / tile offsets / cursors, the bucket rows, the
-// partial outputs and their log-sum-exp.
+// partial outputs and their log-sum-exp, the split block means, and the
+// bucket of each bucket tile (at most one partial tile per bucket beyond
+// rows / 128 full ones).
 size_t moba_tc_ws_bytes(const nsa_params& p, size_t kbar_bytes) {
   const size_t rows = (size_t)p.B * p.T * p.Hq;
   const size_t NB = (size_t)p.B * p.Hq * (p.T / p.sel_block);
@@ -1131,7 +1151,7 @@ size_t moba_tc_ws_bytes(const nsa_params& p, size_t kbar_bytes) {
   const size_t parts = (size_t)p.B * p.Hkv * 3 * gate_rows(p.T / p.sel_block) * D * 2;
   return align256(kbar_bytes) + align256(rows * p.top_n * 4) + 4 * align256((NB + 1) * 4) +
          align256(rows * np * 4 + 4) + align256(rows * np * D * 2 + 4) + align256(rows * np * 4 + 4) +
-         align256(parts + 4);
+         align256(parts + 4) + align256((NB + rows * np / KT + 2) * 4);
 }
 
 cudaError_t launch_moba_tc(const nsa_params& p, const void* q, const void* k, const void* v,
@@ -1169,6 +1189,8 @@ cudaError_t launch_moba_tc(const nsa_params& p, const void* q, const void* k, co
   a.plse = reinterpret_cast<float*>(w);
   w += align256(rows * np * 4 + 4);
   a.kparts = reinterpret_cast<__nv_bfloat16*>(w);
+  w += align256((size_t)p.B * p.Hkv * 3 * gate_rows(a.nfull) * D * 2 + 4);
+  a.tbkt = reinterpret_cast<int32_t*>(w);
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.out = static_cast<__nv_bfloat16*>(out);
   a.err = err;
