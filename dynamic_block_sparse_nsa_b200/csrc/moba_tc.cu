@@ -54,7 +54,7 @@ struct MobaTcArgs {
   int32_t* toff;          // [NB + 1] first tile of each bucket
   int32_t* cur;           // [NB] fill cursors
   int32_t* list;          // rows: t * 8 + slot
-  int32_t* tbkt;          // [tiles] the bucket of each 128-row bucket tile
+  int4* tdesc;            // [tiles] each 128-row bucket tile: {bucket, first row, rows, 0}
   __nv_bfloat16* po;      // [B, T, Hq, topk - 1, d] partial outputs (normalised, bf16)
   float* plse;            // [B, T, Hq, topk - 1] their log2-sum-exp
   unsigned* err;
@@ -503,11 +503,12 @@ __global__ void __launch_bounds__(1024) moba_scan_kernel(MobaTcArgs a) {
   if (threadIdx.x == 0) a.toff[a.NB] = carry[1];
 }
 
-// Rows into buckets: list[off[bucket] + k] = t * 8 + slot; and the bucket of
-// every bucket tile: tbkt[toff[bucket] + k] = bucket.
+// Rows into buckets: list[off[bucket] + k] = t * 8 + slot; and the
+// descriptor of every bucket tile (one 16-byte load for moba_blk).
 __global__ void moba_fill_kernel(MobaTcArgs a) {
   for (int bk = blockIdx.x * blockDim.x + threadIdx.x; bk < a.NB; bk += gridDim.x * blockDim.x)
-    for (int k = a.toff[bk]; k < a.toff[bk + 1]; ++k) a.tbkt[k] = bk;
+    for (int k = a.toff[bk], r = 0; k < a.toff[bk + 1]; ++k, r += KT)
+      a.tdesc[k] = make_int4(bk, a.off[bk] + r, min(KT, a.cnt[bk] - r), 0);
   const long long n = (long long)a.B * a.T * a.Hq;
   for (long long r = blockIdx.x * (long long)blockDim.x + threadIdx.x; r < n;
        r += (long long)gridDim.x * blockDim.x) {
@@ -727,14 +728,13 @@ struct BlkTile {
 
 __device__ __forceinline__ BlkTile blk_tile(const MobaTcArgs& a, int i) {
   BlkTile w;
-  const int bk = a.tbkt[i];
+  const int4 d = a.tdesc[i];
+  const int bk = d.x, bh = bk / a.nfull;
   w.j = bk % a.nfull;
-  const int bh = bk / a.nfull;
   w.h = bh % a.Hq;
   w.b = bh / a.Hq;
-  const int k = i - a.toff[bk];
-  w.first = a.off[bk] + k * KT;
-  w.nrow = min(KT, a.cnt[bk] - k * KT);
+  w.first = d.y;
+  w.nrow = d.z;
   return w;
 }
 
@@ -855,19 +855,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             ((size_t)(cur.b * a.T + (e >> 3)) * a.Hq + cur.h) * (a.topk - 1) + (e & 7);
         const float il = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll 1
-        for (int c16 = 0; c16 < 8; ++c16) {
-          uint32_t o[16];
-          tc::ld16_sync(sm.tl + kO + c16 * 16, o);
+        for (int c32 = 0; c32 < 4; ++c32) {
+          uint32_t o[32];
+          tc::ld32_sync(sm.tl + kO + c32 * 32, o);
           if (live) {
-            uint4 pk[2];
+            uint4 pk[4];
             uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
 #pragma unroll
-            for (int x = 0; x < 8; ++x)
+            for (int x = 0; x < 16; ++x)
               pw[x] = ptx::pack_bf16(__uint_as_float(o[2 * x]) * il,
                                      __uint_as_float(o[2 * x + 1]) * il);
-            uint4* dst = reinterpret_cast<uint4*>(a.po + pr * D + c16 * 16);
-            dst[0] = pk[0];
-            dst[1] = pk[1];
+            uint4* dst = reinterpret_cast<uint4*>(a.po + pr * D + c32 * 32);
+#pragma unroll
+            for (int x = 0; x < 4; ++x) dst[x] = pk[x];
           }
         }
         if (live) a.plse[pr] = m + __log2f(l);
@@ -977,15 +977,19 @@ __device__ __forceinline__ void own_merge_preloaded(const MobaTcArgs& a, Softmax
   float wown, wp[kMaxTopk], inv;
   merge_weights(pl, np, m, l, wown, wp, inv);
 #pragma unroll
-  for (int c16 = 0; c16 < 8; ++c16) {
-    uint32_t o[16];
-    tc::ld16_sync(sm.tl + kO + c16 * 16, o);
-    float acc[16];
+  for (int c32 = 0; c32 < 4; ++c32) {
+    uint32_t o[32];
+    tc::ld32_sync(sm.tl + kO + c32 * 32, o);
 #pragma unroll
-    for (int e = 0; e < 16; ++e) acc[e] = __uint_as_float(o[e]) * wown;
-    add_partial(acc, wp[0], p0[2 * c16], p0[2 * c16 + 1]);
-    add_partial(acc, wp[1], p1[2 * c16], p1[2 * c16 + 1]);
-    if (live) store_row16(dst + c16 * 16, acc, inv);
+    for (int hf = 0; hf < 2; ++hf) {
+      const int c16 = 2 * c32 + hf;
+      float acc[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e) acc[e] = __uint_as_float(o[16 * hf + e]) * wown;
+      add_partial(acc, wp[0], p0[2 * c16], p0[2 * c16 + 1]);
+      add_partial(acc, wp[1], p1[2 * c16], p1[2 * c16 + 1]);
+      if (live) store_row16(dst + c16 * 16, acc, inv);
+    }
   }
 }
 
@@ -1151,7 +1155,7 @@ size_t moba_tc_ws_bytes(const nsa_params& p, size_t kbar_bytes) {
   const size_t parts = (size_t)p.B * p.Hkv * 3 * gate_rows(p.T / p.sel_block) * D * 2;
   return align256(kbar_bytes) + align256(rows * p.top_n * 4) + 4 * align256((NB + 1) * 4) +
          align256(rows * np * 4 + 4) + align256(rows * np * D * 2 + 4) + align256(rows * np * 4 + 4) +
-         align256(parts + 4) + align256((NB + rows * np / KT + 2) * 4);
+         align256(parts + 4) + align256((NB + rows * np / KT + 2) * 16);
 }
 
 cudaError_t launch_moba_tc(const nsa_params& p, const void* q, const void* k, const void* v,
@@ -1190,7 +1194,7 @@ cudaError_t launch_moba_tc(const nsa_params& p, const void* q, const void* k, co
   w += align256(rows * np * 4 + 4);
   a.kparts = reinterpret_cast<__nv_bfloat16*>(w);
   w += align256((size_t)p.B * p.Hkv * 3 * gate_rows(a.nfull) * D * 2 + 4);
-  a.tbkt = reinterpret_cast<int32_t*>(w);
+  a.tdesc = reinterpret_cast<int4*>(w);
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.out = static_cast<__nv_bfloat16*>(out);
   a.err = err;

@@ -75,7 +75,7 @@ def test_workspace_size_validation():
     assert nsa.workspace_size(moba, nsa.OP_MOBA_PREFILL) == (
         kbar + a256(rows * k * 4) + 4 * a256((nb + 1) * 4) + a256(rows * (k - 1) * 4 + 4) +
         a256(rows * (k - 1) * 128 * 2 + 4) + a256(rows * (k - 1) * 4 + 4) + parts +
-        a256((nb + rows * (k - 1) // 128 + 2) * 4))  # the bucket of each 128-row bucket tile
+        a256((nb + rows * (k - 1) // 128 + 2) * 16))  # a descriptor per 128-row bucket tile
     moba32 = nsa.params(B, T, H, H, 128, sel_block=m, top_n=k, dtype=torch.float32)
     assert nsa.workspace_size(moba32, nsa.OP_MOBA_PREFILL) == kbar  # CUDA-core path
 
