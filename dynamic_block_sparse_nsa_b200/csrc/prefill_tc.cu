@@ -155,6 +155,55 @@ struct MainBars {
 // TMEM columns of pf_main.
 constexpr uint32_t kO1 = 0, kO2 = 128, kS0 = 256;  // S buffers at 256 and 384
 
+// Exact top-k of the candidate blocks 1 .. ncand - 1 of one token (k < ncand
+// - 1), by one warp: higher score first, the lower index among equal scores.
+// Each candidate has the unique key (score bits + 1) << 32 | ~index (scores are
+// sums of probabilities, >= 0; a larger key is a better block). Every lane
+// keeps the four largest keys of its candidates (index = 1 + lane mod 32) in
+// registers; each pick is the warp maximum of the lanes' best keys, popped
+// from its lane, which rescans its candidates below the last popped key only
+// once it has given up all four. dst gets block 0, then the picks in
+// increasing order.
+__device__ void warp_topk_lists(const float* scx, int ncand, int k, int32_t* dst, int lane) {
+  auto key = [&](int jb) -> unsigned long long {
+    const float v = scx[jb];
+    const uint32_t kh = v < 0.f ? 0u : __float_as_uint(v) + 1u;
+    return ((unsigned long long)kh << 32) | (uint32_t)~(uint32_t)jb;
+  };
+  unsigned long long t0 = 0, t1 = 0, t2 = 0, t3 = 0;  // 0: empty (no key is 0)
+  auto fill = [&](unsigned long long below) {
+    t0 = t1 = t2 = t3 = 0;
+    for (int jb = 1 + lane; jb < ncand; jb += 32) {
+      const unsigned long long x = key(jb);
+      if (x >= below || x <= t3) continue;
+      const bool g0 = x > t0, g1 = x > t1, g2 = x > t2;
+      t3 = g2 ? t2 : x;
+      t2 = g2 ? (g1 ? t1 : x) : t2;
+      t1 = g1 ? (g0 ? t0 : x) : t1;
+      t0 = g0 ? x : t0;
+    }
+  };
+  fill(~0ull);
+  int mine = lane == 0 ? 0 : 0x7fffffff;
+  for (int i = 0; i < k; ++i) {
+    const uint32_t hi = (uint32_t)(t0 >> 32), lo = (uint32_t)t0;
+    const uint32_t mh = __reduce_max_sync(0xffffffffu, hi);
+    const uint32_t ml = __reduce_max_sync(0xffffffffu, hi == mh ? lo : 0u);
+    if (lane == i + 1) mine = (int)~ml;
+    if (hi == mh && lo == ml) {  // this lane's best was taken
+      const unsigned long long last = t0;
+      t0 = t1;
+      t1 = t2;
+      t2 = t3;
+      t3 = 0;
+      if (t0 == 0) fill(last);
+    }
+  }
+  int rank = 0;
+  for (int o = 0; o < 32; ++o) rank += (__shfl_sync(0xffffffffu, mine, o) < mine) ? 1 : 0;
+  if (lane <= k) dst[rank] = mine;
+}
+
 __global__ void __launch_bounds__(kMainThreads, 1)
     pf_main_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tkc,
                    const __grid_constant__ CUtensorMap tvc, const __grid_constant__ CUtensorMap tk,
@@ -543,37 +592,7 @@ __global__ void __launch_bounds__(kMainThreads, 1)
         } else if (ncand <= a.n) {
           for (int i = lane; i < a.n; i += 32) dst[i] = i < ncand ? i : -1;
         } else {
-          float* scx = sc + x * a.nblk;
-          uint32_t bh = 0, bl = 0;
-          auto rescan = [&]() {
-            uint32_t hh = 0, ll = 0;
-            for (int jb = 1 + lane; jb < ncand; jb += 32) {
-              const float vv = scx[jb];
-              const uint32_t kh = vv < 0.f ? 0u : __float_as_uint(vv) + 1u;
-              const uint32_t kl = ~(uint32_t)jb;
-              if (kh > hh || (kh == hh && kl > ll)) {
-                hh = kh;
-                ll = kl;
-              }
-            }
-            bh = hh;
-            bl = ll;
-          };
-          rescan();
-          int mine = lane == 0 ? 0 : 0x7fffffff;
-          for (int k = 0; k < a.n - 1; ++k) {
-            const uint32_t mh = __reduce_max_sync(0xffffffffu, bh);
-            const uint32_t ml = __reduce_max_sync(0xffffffffu, bh == mh ? bl : 0u);
-            const int pick = (int)~ml;
-            if (lane == k + 1) mine = pick;
-            if (((pick - 1) & 31) == lane) {
-              scx[pick] = -1.f;
-              rescan();
-            }
-          }
-          int rank = 0;
-          for (int o = 0; o < 32; ++o) rank += (__shfl_sync(0xffffffffu, mine, o) < mine) ? 1 : 0;
-          if (lane < a.n) dst[rank] = mine;
+          warp_topk_lists(sc + x * a.nblk, ncand, a.n - 1, dst, lane);
         }
       }
     }

@@ -31,9 +31,14 @@ def oracle_params_for(w):
                 top_p=w.get("top_p", 0.0))
 
 
-def compare_nsa_rows(w, op, rows_b, rows_t, q_rows, k64, v64, kc64, vc64, wg64, gpu_out, gpu_sel):
-    """Oracle on the listed rows, selection rule, forced re-run, output check."""
+def compare_nsa_rows(w, op, rows_b, rows_t, q_rows, k64, v64, kc64, vc64, wg64, gpu_out, gpu_sel,
+                     exact_sel=False):
+    """Oracle on the listed rows, selection rule, forced re-run, output check.
+    exact_sel: the selections must be equal element by element (inputs whose
+    block scores tie exactly on both sides, where only the tie rule decides)."""
     res = oracle.nsa_rows(op, rows_b, rows_t, q_rows, k64, v64, kc64, vc64, wg64)
+    if exact_sel:
+        np.testing.assert_array_equal(gpu_sel, res["sel"])
     n, bs = w["top_n"], w["sel_block"]
     differ = np.zeros(len(rows_b), dtype=bool)
     for r, t in enumerate(rows_t):
@@ -60,9 +65,10 @@ def compare_nsa_rows(w, op, rows_b, rows_t, q_rows, k64, v64, kc64, vc64, wg64, 
     return dict(max_err=stats[0], mean_err=stats[1], sel_near_ties=int(differ.sum()))
 
 
-def run_nsa_prefill(w, rows=None, seed=None):
+def run_nsa_prefill(w, rows=None, seed=None, inp=None, exact_sel=False):
     """GPU compress + prefill on workload w; oracle on `rows` (list of (b, t))."""
-    inp = inputs.make_prefill(w, seed)
+    if inp is None:
+        inp = inputs.make_prefill(w, seed)
     p = nsa_params_for(w)
     dev = {k_: v_.cuda() for k_, v_ in inp.items()}
     kc, vc = nsa.nsa_compress_kv(p, dev["k"], dev["v"], dev["w_cmp"])
@@ -83,7 +89,7 @@ def run_nsa_prefill(w, rows=None, seed=None):
     out_h = f64(out)[rb, rt]
     sel_h = sel.cpu().numpy()[rb, rt]
     return compare_nsa_rows(w, op, rb, rt, q64[rb, rt], k64, v64, kc64, vc64,
-                            f64(inp["w_gate"]), out_h, sel_h)
+                            f64(inp["w_gate"]), out_h, sel_h, exact_sel=exact_sel)
 
 
 def run_nsa_decode(w, seq_lens, check_b=None, seed=None, inp=None, quest_table=False):

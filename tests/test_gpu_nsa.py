@@ -90,6 +90,19 @@ def test_decode_bf16_fast_path_branch_alone(gates):
     gc.run_nsa_decode(w, [6000, 4033, 999, 70], seed=18)
 
 
+@pytest.mark.parametrize("top_n", [16, 5])
+def test_prefill_bf16_tensor_core_exact_ties(top_n):
+    # q = 0: every compressed score is 0, so all visible compressed blocks get
+    # the same probability and every selection block fully covered by visible
+    # ones gets bit-identical scores here and in the oracle. Only the rule
+    # "ties go to the lower index" decides, so the selections must be equal.
+    w = inputs.workload("nsa_prefill_bf16_t8192", T=3000, Hq=16, Hkv=1, top_n=top_n)
+    inp = inputs.make_prefill(w, seed=23)
+    inp["q"].zero_()
+    rows = [(0, t) for t in [0, 63, 64, 600, 1023, 1024, 1500, 2047, 2048, 2999]]
+    gc.run_nsa_prefill(w, rows=rows, inp=inp, exact_sel=True)
+
+
 def test_prefill_bf16_runs_the_tensor_core_kernels():
     from dynamic_block_sparse_nsa_b200 import nsa
     w = inputs.workload("nsa_prefill_bf16_t8192", T=600, Hq=16, Hkv=1)
