@@ -41,6 +41,7 @@ constexpr uint64_t kWaitNs = 2000000000ull;
 constexpr int kMaxTopk = 8;
 constexpr int kStages = 4;
 constexpr int kThreads = 192;     // TMA lanes, MMA thread, 4 softmax warps
+constexpr int kBlkThreads = 320;  // moba_blk: + 4 epilogue warps
 constexpr uint32_t kNegInf = 0xff800000u;
 
 struct MobaTcArgs {
@@ -536,11 +537,13 @@ __global__ void moba_fill_kernel(MobaTcArgs a) {
 struct Bars {
   uint64_t full[kStages], empty[kStages];
   uint64_t q_full[2], q_free[2], s_full[2], p_full[2], o_done[2], fin;
+  uint64_t o_full[2], o_free[2], ml_full, ml_free;  // moba_blk: O per tile parity, (m, l) hand-off
   uint32_t tmem;
   int abort;
 };
 
-constexpr uint32_t kO = 0, kS0 = 128;  // TMEM: O at 0, S buffers at 128 and 256
+// TMEM: O at 0, S buffers at 128 and 256; moba_blk's second O (odd tiles) at 384
+constexpr uint32_t kO = 0, kS0 = 128, kO2 = 384;
 
 __device__ void init_bars(Bars* bars, int q_full_count) {
   for (int i = 0; i < kStages; ++i) {
@@ -554,6 +557,12 @@ __device__ void init_bars(Bars* bars, int q_full_count) {
     ptx::mbar_init(&bars->p_full[i], 128);
     ptx::mbar_init(&bars->o_done[i], 1);
   }
+  for (int i = 0; i < 2; ++i) {
+    ptx::mbar_init(&bars->o_full[i], 1);
+    ptx::mbar_init(&bars->o_free[i], 128);
+  }
+  ptx::mbar_init(&bars->ml_full, 128);
+  ptx::mbar_init(&bars->ml_free, 128);
   ptx::mbar_init(&bars->fin, 1);
   bars->abort = 0;
   ptx::fence_mbar_init();
@@ -593,8 +602,11 @@ struct Producer {
 
 // MMA side of one query tile with `nk` key tiles: S_u = Q K_u^T into S buffer
 // (j & 1), O += P_u V_u with P from TMEM; j and c are the running tile and
-// load counters of the CTA.
-struct Mma {
+// load counters of the CTA. DBL (moba_blk): O of tile kt in O[kt & 1]; the
+// tile's first PV waits until the epilogue of tile kt - 2 has released that
+// buffer, and its last PV commits o_full[kt & 1].
+template <bool DBL>
+struct MmaT {
   Bars* bars;
   volatile int* abort;
   unsigned* err;
@@ -607,7 +619,8 @@ struct Mma {
     tc::fence_after_sync();
     return st;
   }
-  __device__ void tile(uint32_t q0, int nk, int qbuf) {
+  __device__ void tile(uint32_t q0, int nk, int qbuf, int kt = 0) {
+    const uint32_t ob = DBL && (kt & 1) ? kO2 : kO;
     const uint32_t iss = tc::idesc_bf16(128, 128, false, false);
     const uint32_t its = tc::idesc_bf16(128, 128, false, true);
     const int j0 = j;
@@ -630,16 +643,20 @@ struct Mma {
       if (u >= 1) {
         const int pj = j0 + u - 1, pb = pj & 1;
         ok = ok && wait_or_abort(&bars->p_full[pb], (uint32_t)((pj >> 1) & 1), abort, err);
+        if (DBL && u == 1 && kt >= 2)
+          ok = ok && wait_or_abort(&bars->o_free[kt & 1], (uint32_t)(((kt >> 1) - 1) & 1), abort,
+                                   err);
         tc::fence_after_sync();
         const int st = take();
         if (!ok) break;
         const uint32_t vb = r0 + st * TILE;
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          tc::mma_ts(tmem + kO, tmem + kS0 + pb * 128 + ks * 8, mnmaj(vb, ks), its,
+          tc::mma_ts(tmem + ob, tmem + kS0 + pb * 128 + ks * 8, mnmaj(vb, ks), its,
                      (u > 1 || ks > 0));
         tc::commit(&bars->empty[st]);
         tc::commit(&bars->o_done[pj & 1]);
+        if (DBL && u == nk) tc::commit(&bars->o_full[kt & 1]);
         ++c;
       }
     }
@@ -649,13 +666,15 @@ struct Mma {
 
 // Softmax side: thread `row` of the query tile, one S tile at a time; keys at
 // index >= klim are masked (the causal edge). m is kept in the log2 domain.
-struct Softmax {
+template <bool DBL>
+struct SoftmaxT {
   Bars* bars;
   volatile int* abort;
   unsigned* err;
   uint32_t tl;
   float cs;
   int j = 0;
+  uint32_t obuf = kO;  // DBL: O's TMEM column of the current tile
   __device__ void tile(int kb, int klim, float& m, float& l) {
     const int bs = j & 1;
     wait_or_abort(&bars->s_full[bs], (uint32_t)((j >> 1) & 1), abort, err);
@@ -686,10 +705,11 @@ struct Softmax {
 #pragma unroll 1
         for (int q4 = 0; q4 < 8; ++q4) {
           uint32_t w[16];
-          tc::ld16_sync(tl + kO + q4 * 16, w);
+          const uint32_t oc = tl + (DBL ? obuf : kO) + q4 * 16;
+          tc::ld16_sync(oc, w);
 #pragma unroll
           for (int e = 0; e < 16; ++e) w[e] = __float_as_uint(__uint_as_float(w[e]) * f);
-          tc::st16(tl + kO + q4 * 16, w);
+          tc::st16(oc, w);
         }
         tc::st_wait();
       }
@@ -718,6 +738,9 @@ struct Softmax {
   }
 };
 
+using Mma = MmaT<false>;
+using Softmax = SoftmaxT<false>;
+
 // ============================================================================
 // moba_blk: bucket tiles (gathered rows x one earlier block)
 // ============================================================================
@@ -738,7 +761,7 @@ __device__ __forceinline__ BlkTile blk_tile(const MobaTcArgs& a, int i) {
   return w;
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kBlkThreads, 1)
     moba_blk_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                     const MobaTcArgs a) {
   extern __shared__ unsigned char smraw[];
@@ -746,6 +769,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned char* sQ = base;              // 2 x 32 KB
   unsigned char* ring = base + 2 * TILE;
   Bars* bars = reinterpret_cast<Bars*>(ring + kStages * TILE);
+  float2* ml_s = reinterpret_cast<float2*>(bars + 1);  // [row]
   volatile int* abort = &bars->abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ntile = a.toff[a.NB];
@@ -786,25 +810,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      Mma mm{bars, abort, a.err, tmem, ptx::smem_u32(ring)};
+      MmaT<true> mm{bars, abort, a.err, tmem, ptx::smem_u32(ring)};
       int k = 0;
       for (int i = blockIdx.x; mm.ok && i < ntile; i += gridDim.x, ++k) {
         const int qb = k & 1;
         mm.ok = wait_or_abort(&bars->q_full[qb], (uint32_t)((k >> 1) & 1), abort, a.err);
         tc::fence_after_sync();
-        mm.tile(ptx::smem_u32(sQ + qb * TILE), nk, qb);
+        mm.tile(ptx::smem_u32(sQ + qb * TILE), nk, qb, k);
       }
       tc::commit(&bars->fin);
       if (!ptx::mbar_wait(&bars->fin, 0, kWaitNs)) atomicOr(a.err, kErrTimeout);
     }
-  } else {
+  } else if (warp < 6) {
+    // softmax warps: tile after tile, O of tile k in O[k & 1]; each row's
+    // (m, l) goes to the epilogue warps through shared memory
     const int qd = warp & 3;
     const int row = qd * 32 + lane;
-    Softmax sm{bars, abort, a.err, tmem + ((uint32_t)(qd * 32) << 16), a.c};
-    // The query rows of tile k + 1 are copied (cp.async, this thread's row,
-    // zeros past the bucket) while tile k's softmax runs, and handed to the
-    // MMA thread after it; the tile descriptors and list entries they need
-    // are loaded one tile further ahead still.
+    SoftmaxT<true> sm{bars, abort, a.err, tmem + ((uint32_t)(qd * 32) << 16), a.c};
+    int k = 0;
+    for (int i = blockIdx.x; i < ntile; i += gridDim.x, ++k) {
+      sm.obuf = (k & 1) ? kO2 : kO;
+      float m = -INFINITY, l = 0.f;
+      for (int u = 0; u < nk; ++u) sm.tile(u * KT, 1 << 30, m, l);
+      if (k >= 1)  // the epilogue warps have read tile k - 1's
+        wait_or_abort(&bars->ml_free, (uint32_t)((k - 1) & 1), abort, a.err);
+      ml_s[row] = make_float2(m, l);
+      ptx::mbar_arrive(&bars->ml_full);
+    }
+  } else {
+    // epilogue warps: the query rows of tile k + 2 are copied (cp.async, this
+    // thread's row, zeros past the bucket) while tile k's normalised partial
+    // outputs and log-sum-exps are written from O[k & 1], which is then
+    // released to the MMA thread; the rows are handed over at the end.
+    const int qd = warp & 3;
+    const int row = qd * 32 + lane;
+    const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
     auto gather = [&](const BlkTile& w, int e, int kq) {
       const int qb = kq & 1;
       if (kq >= 2) wait_or_abort(&bars->q_free[qb], (uint32_t)(((kq >> 1) - 1) & 1), abort, a.err);
@@ -835,29 +875,35 @@ __global__ void __launch_bounds__(kThreads, 1)
       if ((int)blockIdx.x + G1 < ntile) {
         nxt = blk_tile(a, blockIdx.x + G1);
         enxt = entry(nxt);
+        gather(nxt, enxt, 1);
+        hand_over(1);
       }
       int k = 0;
       for (int i = blockIdx.x; i < ntile && !*abort; i += G1, ++k) {
-        const bool more = i + G1 < ntile, more2 = i + 2 * G1 < ntile;
-        if (more) gather(nxt, enxt, k + 1);
-        BlkTile nn{};
-        if (more2) nn = blk_tile(a, i + 2 * G1);  // in flight during the softmax
-        float m = -INFINITY, l = 0.f;
-        for (int u = 0; u < nk; ++u) sm.tile(u * KT, 1 << 30, m, l);
-        const int enn = more2 ? entry(nn) : -1;  // in flight during the epilogue
-        if (more) hand_over(k + 1);
-        wait_or_abort(&bars->o_done[(sm.j - 1) & 1], (uint32_t)(((sm.j - 1) >> 1) & 1), abort,
-                      a.err);
+        const bool more2 = i + 2 * G1 < ntile;
+        BlkTile n2{};
+        int en2 = -1;
+        if (more2) {
+          n2 = blk_tile(a, i + 2 * G1);
+          en2 = entry(n2);
+          gather(n2, en2, k + 2);
+        }
+        wait_or_abort(&bars->ml_full, (uint32_t)(k & 1), abort, a.err);
+        const float2 ml = ml_s[row];
+        ptx::mbar_arrive(&bars->ml_free);
+        wait_or_abort(&bars->o_full[k & 1], (uint32_t)((k >> 1) & 1), abort, a.err);
         tc::fence_after_sync();
+        const float m = ml.x, l = ml.y;
         const bool live = ecur >= 0;
         const int e = live ? ecur : 0;
         const size_t pr =
             ((size_t)(cur.b * a.T + (e >> 3)) * a.Hq + cur.h) * (a.topk - 1) + (e & 7);
         const float il = l > 0.f ? 1.f / l : 0.f;
+        const uint32_t ob = (k & 1) ? kO2 : kO;
 #pragma unroll 1
         for (int c32 = 0; c32 < 4; ++c32) {
           uint32_t o[32];
-          tc::ld32_sync(sm.tl + kO + c32 * 32, o);
+          tc::ld32_sync(tl + ob + c32 * 32, o);
           if (live) {
             uint4 pk[4];
             uint32_t* pw = reinterpret_cast<uint32_t*>(pk);
@@ -872,10 +918,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (live) a.plse[pr] = m + __log2f(l);
         tc::fence_before_sync();
+        ptx::mbar_arrive(&bars->o_free[k & 1]);
+        if (more2) hand_over(k + 2);
         cur = nxt;
         ecur = enxt;
-        nxt = nn;
-        enxt = enn;
+        nxt = n2;
+        enxt = en2;
       }
       ptx::cp_async_wait<0>();  // no copy in flight past an abort
     }
@@ -1130,6 +1178,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 size_t attn_smem(int qbufs) { return 1024 + (size_t)(qbufs + kStages) * TILE + sizeof(Bars); }
+// moba_blk: + the (m, l) hand-off of each row (one buffer: the kernel then stays
+// within the 196 KB shared-memory configuration, which leaves the SM more L1)
+size_t blk_smem() { return attn_smem(2) + KT * sizeof(float2); }
 
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -1242,10 +1293,10 @@ cudaError_t launch_moba_tc(const nsa_params& p, const void* q, const void* k, co
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     {
-      const size_t sm = attn_smem(2);
+      const size_t sm = blk_smem();
       if ((e = ensure_dyn_smem((const void*)moba_blk_kernel, (int)sm)) != cudaSuccess) return e;
       TraceScope trace("moba_blk", stream);
-      moba_blk_kernel<<<device_sm_count(), kThreads, sm, stream>>>(tk, tv, a);
+      moba_blk_kernel<<<device_sm_count(), kBlkThreads, sm, stream>>>(tk, tv, a);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
   }
