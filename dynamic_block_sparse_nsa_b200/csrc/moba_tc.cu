@@ -1003,58 +1003,88 @@ __device__ __forceinline__ void add_partial(float (&acc)[16], float w, uint4 a0,
   }
 }
 
-// Up to two partials (top_k <= 3): both rows (2 x 256 B) and their
-// log2-sum-exps are loaded together, while the last PV MMA finishes, so the
-// merge waits for memory once.
-__device__ __forceinline__ void own_merge_preloaded(const MobaTcArgs& a, Softmax& sm, size_t prow,
-                                                    int np, float m, float l, bool live,
-                                                    __nv_bfloat16* dst) {
-  uint4 p0[16], p1[16];
-  float pl[kMaxTopk];
-  const uint4* s0 = reinterpret_cast<const uint4*>(a.po + prow * D);
-#pragma unroll
-  for (int c = 0; c < 16; ++c) {
-    p0[c] = np > 0 ? __ldg(s0 + c) : make_uint4(0, 0, 0, 0);
-    p1[c] = np > 1 ? __ldg(s0 + 16 + c) : make_uint4(0, 0, 0, 0);
+// The hand-offs of item k to a merge warp: the row's (m, l) from the softmax
+// warps (then released), and O[k & 1] once the item's last PV MMA is done.
+struct OwnHandoff {
+  Bars* bars;
+  volatile int* abort;
+  unsigned* err;
+  const float2* ml_s;
+  __device__ __forceinline__ float2 take_ml(int k, int row) const {
+    wait_or_abort(&bars->ml_full, (uint32_t)(k & 1), abort, err);
+    const float2 ml = ml_s[row];
+    ptx::mbar_arrive(&bars->ml_free);
+    return ml;
   }
+  __device__ __forceinline__ void wait_o(int k) const {
+    wait_or_abort(&bars->o_full[k & 1], (uint32_t)((k >> 1) & 1), abort, err);
+    tc::fence_after_sync();
+  }
+  __device__ __forceinline__ void release_o(int k) const {
+    tc::fence_before_sync();
+    ptx::mbar_arrive(&bars->o_free[k & 1]);
+  }
+};
+
+// Up to two partials (top_k <= 3): the rows' log2-sum-exps and the first
+// 64 columns of both rows are loaded before the item's O is waited for, the
+// second 64 columns while the first are merged (two waits for memory, off the
+// softmax warps' path).
+__device__ __forceinline__ void own_merge_preloaded(const MobaTcArgs& a, const OwnHandoff& hf,
+                                                    uint32_t to, int k, int row, size_t prow,
+                                                    int np, bool live, __nv_bfloat16* dst) {
+  const uint4* s0 = reinterpret_cast<const uint4*>(a.po + prow * D);
+  uint4 p0[8], p1[8];
+  auto load_half = [&](int hv) {
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      p0[c] = np > 0 ? __ldg(s0 + 8 * hv + c) : make_uint4(0, 0, 0, 0);
+      p1[c] = np > 1 ? __ldg(s0 + 16 + 8 * hv + c) : make_uint4(0, 0, 0, 0);
+    }
+  };
+  float pl[kMaxTopk];
 #pragma unroll
   for (int s = 0; s < kMaxTopk; ++s) pl[s] = s < np ? a.plse[prow + s] : -INFINITY;
-  wait_or_abort(&sm.bars->o_done[(sm.j - 1) & 1], (uint32_t)(((sm.j - 1) >> 1) & 1), sm.abort,
-                sm.err);
-  tc::fence_after_sync();
+  load_half(0);
+  const float2 ml = hf.take_ml(k, row);
   float wown, wp[kMaxTopk], inv;
-  merge_weights(pl, np, m, l, wown, wp, inv);
+  merge_weights(pl, np, ml.x, ml.y, wown, wp, inv);
+  hf.wait_o(k);
+#pragma unroll 1
+  for (int hv = 0; hv < 2; ++hv) {
+    if (hv == 1) load_half(1);
 #pragma unroll
-  for (int c32 = 0; c32 < 4; ++c32) {
-    uint32_t o[32];
-    tc::ld32_sync(sm.tl + kO + c32 * 32, o);
+    for (int c32 = 0; c32 < 2; ++c32) {
+      uint32_t o[32];
+      tc::ld32_sync(to + hv * 64 + c32 * 32, o);
 #pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-      const int c16 = 2 * c32 + hf;
-      float acc[16];
+      for (int h2 = 0; h2 < 2; ++h2) {
+        const int c = 2 * c32 + h2;  // 16-column chunk within the half
+        float acc[16];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) acc[e] = __uint_as_float(o[16 * hf + e]) * wown;
-      add_partial(acc, wp[0], p0[2 * c16], p0[2 * c16 + 1]);
-      add_partial(acc, wp[1], p1[2 * c16], p1[2 * c16 + 1]);
-      if (live) store_row16(dst + c16 * 16, acc, inv);
+        for (int e = 0; e < 16; ++e) acc[e] = __uint_as_float(o[16 * h2 + e]) * wown;
+        add_partial(acc, wp[0], p0[2 * c], p0[2 * c + 1]);
+        add_partial(acc, wp[1], p1[2 * c], p1[2 * c + 1]);
+        if (live) store_row16(dst + hv * 64 + c * 16, acc, inv);
+      }
     }
   }
+  hf.release_o(k);
 }
 
 // Any number of partials: 16 columns at a time (two chunks' loads in flight).
-__device__ __forceinline__ void own_merge_chunked(const MobaTcArgs& a, Softmax& sm, size_t prow,
-                                                  int np, float m, float l, bool live,
-                                                  __nv_bfloat16* dst) {
+__device__ __forceinline__ void own_merge_chunked(const MobaTcArgs& a, const OwnHandoff& hf,
+                                                  uint32_t to, int k, int row, size_t prow,
+                                                  int np, bool live, __nv_bfloat16* dst) {
   if (np > 0) ptx::bulk_prefetch_l2(a.po + prow * D, (uint32_t)(np * D * 2));
-  wait_or_abort(&sm.bars->o_done[(sm.j - 1) & 1], (uint32_t)(((sm.j - 1) >> 1) & 1), sm.abort,
-                sm.err);
-  tc::fence_after_sync();
+  const float2 ml = hf.take_ml(k, row);
   float wown, wp[kMaxTopk], inv;
-  merge_weights(a.plse + prow, np, m, l, wown, wp, inv);
+  merge_weights(a.plse + prow, np, ml.x, ml.y, wown, wp, inv);
+  hf.wait_o(k);
 #pragma unroll 2
   for (int c16 = 0; c16 < 8; ++c16) {
     uint32_t o[16];
-    tc::ld16_sync(sm.tl + kO + c16 * 16, o);
+    tc::ld16_sync(to + c16 * 16, o);
     float acc[16];
 #pragma unroll
     for (int e = 0; e < 16; ++e) acc[e] = __uint_as_float(o[e]) * wown;
@@ -1066,13 +1096,14 @@ __device__ __forceinline__ void own_merge_chunked(const MobaTcArgs& a, Softmax& 
     }
     if (live) store_row16(dst + c16 * 16, acc, inv);
   }
+  hf.release_o(k);
 }
 
 // Persistent, one CTA per SM: lanes 0-3 of warp 0 load the query tiles (two
 // buffers, lane 0) and the K / V tiles (a four-stage ring), warp 1 lane 0
-// issues the MMAs, warps 2-5 run the softmax and the merge, so one item's
-// merge overlaps the next item's first MMAs and loads.
-__global__ void __launch_bounds__(kThreads, 1)
+// issues the MMAs, warps 2-5 run the softmax, warps 6-9 the merge with the
+// partials, so one item's merge overlaps the next item's softmax.
+__global__ void __launch_bounds__(kBlkThreads, 1)
     moba_own_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                     const __grid_constant__ CUtensorMap tv, const MobaTcArgs a) {
   extern __shared__ unsigned char smraw[];
@@ -1080,6 +1111,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   unsigned char* sQ = base;  // 2 x 32 KB
   unsigned char* ring = base + 2 * TILE;
   Bars* bars = reinterpret_cast<Bars*>(ring + kStages * TILE);
+  float2* ml_s = reinterpret_cast<float2*>(bars + 1);  // [row]
   volatile int* abort = &bars->abort;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int NI = a.B * a.Hq * ((a.T + KT - 1) / KT);
@@ -1137,37 +1169,55 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      Mma mm{bars, abort, a.err, tmem, ptx::smem_u32(ring)};
+      MmaT<true> mm{bars, abort, a.err, tmem, ptx::smem_u32(ring)};
       int kq = 0;
       for (int i = blockIdx.x; mm.ok && i < NI; i += gridDim.x, ++kq) {
         const OwnItem it = own_item(a, i);
         const int qb = kq & 1;
         mm.ok = wait_or_abort(&bars->q_full[qb], (uint32_t)((kq >> 1) & 1), abort, a.err);
         tc::fence_after_sync();
-        mm.tile(ptx::smem_u32(sQ + qb * TILE), it.nk, qb);
+        mm.tile(ptx::smem_u32(sQ + qb * TILE), it.nk, qb, kq);
       }
       tc::commit(&bars->fin);
       if (!ptx::mbar_wait(&bars->fin, 0, kWaitNs)) atomicOr(a.err, kErrTimeout);
     }
-  } else {
+  } else if (warp < 6) {
+    // softmax warps: item after item, O of item k in O[k & 1]; each row's
+    // (m, l) goes to the merge warps through shared memory
     const int qd = warp & 3;
     const int row = qd * 32 + lane;
-    Softmax sm{bars, abort, a.err, tmem + ((uint32_t)(qd * 32) << 16), a.c};
-    for (int i = blockIdx.x; i < NI && !*abort; i += gridDim.x) {
+    SoftmaxT<true> sm{bars, abort, a.err, tmem + ((uint32_t)(qd * 32) << 16), a.c};
+    int k = 0;
+    for (int i = blockIdx.x; i < NI; i += gridDim.x, ++k) {
+      const OwnItem it = own_item(a, i);
+      const int t = min(it.t0 + row, a.T - 1);
+      sm.obuf = (k & 1) ? kO2 : kO;
+      float m = -INFINITY, l = 0.f;
+      for (int u = 0; u < it.nk; ++u) sm.tile(it.c0 + u * KT, t + 1, m, l);
+      if (k >= 1)  // the merge warps have read item k - 1's
+        wait_or_abort(&bars->ml_free, (uint32_t)((k - 1) & 1), abort, a.err);
+      ml_s[row] = make_float2(m, l);
+      ptx::mbar_arrive(&bars->ml_full);
+    }
+  } else {
+    // merge warps: item k's row, from O[k & 1] and its partials
+    const int qd = warp & 3;
+    const int row = qd * 32 + lane;
+    const uint32_t tl = tmem + ((uint32_t)(qd * 32) << 16);
+    const OwnHandoff hf{bars, abort, a.err, ml_s};
+    int k = 0;
+    for (int i = blockIdx.x; i < NI; i += gridDim.x, ++k) {
       const OwnItem it = own_item(a, i);
       const int t = min(it.t0 + row, a.T - 1);
       const bool live = it.t0 + row < a.T;
-      const int npast = min(a.topk - 1, t / a.m);
+      const int np = live ? min(a.topk - 1, t / a.m) : 0;
       const size_t prow = ((size_t)(it.b * a.T + t) * a.Hq + it.h) * (a.topk - 1);
-      float m = -INFINITY, l = 0.f;
-      for (int u = 0; u < it.nk; ++u) sm.tile(it.c0 + u * KT, t + 1, m, l);
       __nv_bfloat16* dst = a.out + ((size_t)(it.b * a.T + t) * a.Hq + it.h) * D;
-      const int np = live ? npast : 0;
+      const uint32_t to = tl + ((k & 1) ? kO2 : kO);
       if (a.topk <= 3)
-        own_merge_preloaded(a, sm, prow, np, m, l, live, dst);
+        own_merge_preloaded(a, hf, to, k, row, prow, np, live, dst);
       else
-        own_merge_chunked(a, sm, prow, np, m, l, live, dst);
-      tc::fence_before_sync();
+        own_merge_chunked(a, hf, to, k, row, prow, np, live, dst);
     }
   }
 
@@ -1301,12 +1351,12 @@ cudaError_t launch_moba_tc(const nsa_params& p, const void* q, const void* k, co
     }
   }
   {
-    const size_t sm = attn_smem(2);
+    const size_t sm = blk_smem();
     if ((e = ensure_dyn_smem((const void*)moba_own_kernel, (int)sm)) != cudaSuccess) return e;
     TraceScope trace("moba_own", stream);
     const long long items = (long long)p.B * p.Hq * ((p.T + KT - 1) / KT);
     const int grid = (int)std::min<long long>(items, device_sm_count());
-    moba_own_kernel<<<grid, kThreads, sm, stream>>>(tq, tk, tv, a);
+    moba_own_kernel<<<grid, kBlkThreads, sm, stream>>>(tq, tk, tv, a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;
