@@ -675,66 +675,81 @@ struct SoftmaxT {
   float cs;
   int j = 0;
   uint32_t obuf = kO;  // DBL: O's TMEM column of the current tile
-  __device__ void tile(int kb, int klim, float& m, float& l) {
-    const int bs = j & 1;
-    wait_or_abort(&bars->s_full[bs], (uint32_t)((j >> 1) & 1), abort, err);
-    tc::fence_after_sync();
+  // The row's nk key tiles [kb0, kb0 + 128 nk). The next tile's scores are
+  // loaded from TMEM before this tile's P stores are waited for, so the two
+  // TMEM latencies overlap (the next S is in the other buffer, and its QK MMA
+  // never waits for this tile's P).
+  __device__ void run(int nk, int kb0, int klim, float& m, float& l) {
+    if (nk <= 0) return;
     uint32_t u[128];
-    tc::ld128_sync(tl + kS0 + bs * 128, u);
-    if (kb + KT > klim) {
+    wait_or_abort(&bars->s_full[j & 1], (uint32_t)((j >> 1) & 1), abort, err);
+    tc::fence_after_sync();
+    tc::ld128_nowait(tl + kS0 + (j & 1) * 128, u);
+    tc::ld_wait128(u);
+    for (int t = 0; t < nk; ++t) {
+      const int bs = j & 1, kb = kb0 + t * KT;
+      if (kb + KT > klim) {
 #pragma unroll
-      for (int e = 0; e < 128; ++e)
-        if (kb + e >= klim) u[e] = kNegInf;
-    }
-    float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+        for (int e = 0; e < 128; ++e)
+          if (kb + e >= klim) u[e] = kNegInf;
+      }
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-    for (int e = 0; e < 128; e += 4) {
-      mx0 = fmaxf(mx0, __uint_as_float(u[e]));
-      mx1 = fmaxf(mx1, __uint_as_float(u[e + 1]));
-      mx2 = fmaxf(mx2, __uint_as_float(u[e + 2]));
-      mx3 = fmaxf(mx3, __uint_as_float(u[e + 3]));
-    }
-    const float mt = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * cs;
-    const float mn = fmaxf(m, mt);
-    if (mn != -INFINITY && (m == -INFINITY || mn > m + 8.f)) {
-      if (m != -INFINITY) {
-        const float f = exp2f(m - mn);
-        l *= f;
-        wait_or_abort(&bars->o_done[(j - 1) & 1], (uint32_t)(((j - 1) >> 1) & 1), abort, err);
-        tc::fence_after_sync();
+      for (int e = 0; e < 128; e += 4) {
+        mx0 = fmaxf(mx0, __uint_as_float(u[e]));
+        mx1 = fmaxf(mx1, __uint_as_float(u[e + 1]));
+        mx2 = fmaxf(mx2, __uint_as_float(u[e + 2]));
+        mx3 = fmaxf(mx3, __uint_as_float(u[e + 3]));
+      }
+      const float mt = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * cs;
+      const float mn = fmaxf(m, mt);
+      if (mn != -INFINITY && (m == -INFINITY || mn > m + 8.f)) {
+        if (m != -INFINITY) {
+          const float f = exp2f(m - mn);
+          l *= f;
+          wait_or_abort(&bars->o_done[(j - 1) & 1], (uint32_t)(((j - 1) >> 1) & 1), abort, err);
+          tc::fence_after_sync();
 #pragma unroll 1
-        for (int q4 = 0; q4 < 8; ++q4) {
-          uint32_t w[16];
-          const uint32_t oc = tl + (DBL ? obuf : kO) + q4 * 16;
-          tc::ld16_sync(oc, w);
+          for (int q4 = 0; q4 < 8; ++q4) {
+            uint32_t w[16];
+            const uint32_t oc = tl + (DBL ? obuf : kO) + q4 * 16;
+            tc::ld16_sync(oc, w);
 #pragma unroll
-          for (int e = 0; e < 16; ++e) w[e] = __float_as_uint(__uint_as_float(w[e]) * f);
-          tc::st16(oc, w);
+            for (int e = 0; e < 16; ++e) w[e] = __float_as_uint(__uint_as_float(w[e]) * f);
+            tc::st16(oc, w);
+          }
+          tc::st_wait();
         }
-        tc::st_wait();
+        m = mn;
       }
-      m = mn;
-    }
-    const float nm = m == -INFINITY ? 0.f : -m;
-    float ls0 = 0.f, ls1 = 0.f;
+      const float nm = m == -INFINITY ? 0.f : -m;
+      float ls0 = 0.f, ls1 = 0.f;
 #pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) {
-      uint32_t pk[16];
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t pk[16];
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        const float p0 = ptx::ex2(fmaf(__uint_as_float(u[q4 * 32 + 2 * e]), cs, nm));
-        const float p1 = ptx::ex2(fmaf(__uint_as_float(u[q4 * 32 + 2 * e + 1]), cs, nm));
-        ls0 += p0;
-        ls1 += p1;
-        pk[e] = ptx::pack_bf16(p0, p1);
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = ptx::ex2(fmaf(__uint_as_float(u[q4 * 32 + 2 * e]), cs, nm));
+          const float p1 = ptx::ex2(fmaf(__uint_as_float(u[q4 * 32 + 2 * e + 1]), cs, nm));
+          ls0 += p0;
+          ls1 += p1;
+          pk[e] = ptx::pack_bf16(p0, p1);
+        }
+        tc::st16(tl + kS0 + bs * 128 + q4 * 16, pk);
       }
-      tc::st16(tl + kS0 + bs * 128 + q4 * 16, pk);
+      l += ls0 + ls1;
+      const bool more = t + 1 < nk;
+      if (more) {
+        wait_or_abort(&bars->s_full[(j + 1) & 1], (uint32_t)(((j + 1) >> 1) & 1), abort, err);
+        tc::fence_after_sync();
+        tc::ld128_nowait(tl + kS0 + ((j + 1) & 1) * 128, u);
+      }
+      tc::st_wait();
+      tc::fence_before_sync();
+      ptx::mbar_arrive(&bars->p_full[bs]);
+      if (more) tc::ld_wait128(u);
+      ++j;
     }
-    l += ls0 + ls1;
-    tc::st_wait();
-    tc::fence_before_sync();
-    ptx::mbar_arrive(&bars->p_full[bs]);
-    ++j;
   }
 };
 
@@ -831,7 +846,7 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
     for (int i = blockIdx.x; i < ntile; i += gridDim.x, ++k) {
       sm.obuf = (k & 1) ? kO2 : kO;
       float m = -INFINITY, l = 0.f;
-      for (int u = 0; u < nk; ++u) sm.tile(u * KT, 1 << 30, m, l);
+      sm.run(nk, 0, 1 << 30, m, l);
       if (k >= 1)  // the epilogue warps have read tile k - 1's
         wait_or_abort(&bars->ml_free, (uint32_t)((k - 1) & 1), abort, a.err);
       ml_s[row] = make_float2(m, l);
@@ -1193,7 +1208,7 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
       const int t = min(it.t0 + row, a.T - 1);
       sm.obuf = (k & 1) ? kO2 : kO;
       float m = -INFINITY, l = 0.f;
-      for (int u = 0; u < it.nk; ++u) sm.tile(it.c0 + u * KT, t + 1, m, l);
+      sm.run(it.nk, it.c0, t + 1, m, l);
       if (k >= 1)  // the merge warps have read item k - 1's
         wait_or_abort(&bars->ml_free, (uint32_t)((k - 1) & 1), abort, a.err);
       ml_s[row] = make_float2(m, l);
