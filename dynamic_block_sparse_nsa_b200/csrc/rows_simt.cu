@@ -531,6 +531,51 @@ __global__ void __launch_bounds__(256) moba_block_mean_kernel(const T* __restric
   }
 }
 
+// The same for bf16 keys with d a multiple of 8: each thread sums 8 adjacent
+// dimensions (16-byte loads, eight fp64 accumulators, eight rows' loads in
+// flight), so the kernel streams the keys at HBM rate.
+__global__ void __launch_bounds__(256) moba_block_mean8_kernel(const __nv_bfloat16* __restrict__ k,
+                                                               float* __restrict__ kbar, int B,
+                                                               int T_, int Hkv, int d, int m) {
+  const int nfull = T_ / m;
+  const long row = (long)Hkv * d;
+  const long total8 = (long)B * nfull * row / 8;
+  for (long o8 = blockIdx.x * (long)blockDim.x + threadIdx.x; o8 < total8;
+       o8 += (long)gridDim.x * blockDim.x) {
+    const long o = o8 * 8;
+    const int b = (int)(o / ((long)nfull * row));
+    const long r = o - (long)b * nfull * row;
+    const int j = (int)(r / row);
+    const long ge = r - (long)j * row;
+    const __nv_bfloat16* src = k + ((long)b * T_ + (long)j * m) * row + ge;
+    double acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.0;
+#pragma unroll 8
+    for (int u = 0; u < m; ++u) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(src + (long)u * row));
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(h2[e]);
+        acc[2 * e] += (double)f.x;
+        acc[2 * e + 1] += (double)f.y;
+      }
+    }
+    float4 lo, hi;
+    lo.x = (float)(acc[0] / m);
+    lo.y = (float)(acc[1] / m);
+    lo.z = (float)(acc[2] / m);
+    lo.w = (float)(acc[3] / m);
+    hi.x = (float)(acc[4] / m);
+    hi.y = (float)(acc[5] / m);
+    hi.z = (float)(acc[6] / m);
+    hi.w = (float)(acc[7] / m);
+    reinterpret_cast<float4*>(kbar + o)[0] = lo;
+    reinterpret_cast<float4*>(kbar + o)[1] = hi;
+  }
+}
+
 template <typename T>
 __global__ void __launch_bounds__(kThreads) moba_rows_kernel(MobaArgs a) {
   extern __shared__ float sm[];
@@ -620,7 +665,14 @@ cudaError_t launch_moba_block_mean(const MobaArgs& a, cudaStream_t stream) {
     const long cap = (long)device_sms() * 16;
     if (blocks > cap) blocks = cap;
     TraceScope trace("moba_block_mean", stream);
-    if (a.dtype == NSA_DTYPE_BF16)
+    const bool vec = a.dtype == NSA_DTYPE_BF16 && a.d % 8 == 0 &&
+                     reinterpret_cast<uintptr_t>(a.k) % 16 == 0 &&
+                     reinterpret_cast<uintptr_t>(a.kbar) % 16 == 0;
+    if (vec) {
+      const long b8 = (total / 8 + 255) / 256;
+      moba_block_mean8_kernel<<<(unsigned)(b8 < cap ? b8 : cap), 256, 0, stream>>>(
+          (const __nv_bfloat16*)a.k, a.kbar, a.B, a.T, a.Hkv, a.d, a.m);
+    } else if (a.dtype == NSA_DTYPE_BF16)
       moba_block_mean_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, stream>>>(
           (const __nv_bfloat16*)a.k, a.kbar, a.B, a.T, a.Hkv, a.d, a.m);
     else
