@@ -14,12 +14,17 @@
 //              the selection row, and per-(head, block) pick counts;
 //   moba_scan  offsets of each (sequence, head, block) bucket and of its
 //              128-row tiles;
-//   moba_fill  the rows of every bucket (token, slot);
+//   moba_fill  the rows of every bucket (token, slot) and each bucket tile's
+//              descriptor;
 //   moba_blk   per bucket tile: 128 gathered query rows against the block's m
 //              keys (tcgen05, TMEM accumulators), written as a normalised
 //              partial output and its log-sum-exp;
 //   moba_own   per 128 consecutive tokens of one head: causal attention over
 //              the own block, merged with the row's partials into the output.
+// The gate and both attention kernels are persistent (one CTA per SM) and
+// warp-specialised: a TMA warp, one MMA-issuing thread, and row warps; in the
+// attention kernels four softmax warps hand each tile's O (double-buffered in
+// TMEM) and its rows' (m, l) to four epilogue / merge warps.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -600,13 +605,12 @@ struct Producer {
   }
 };
 
-// MMA side of one query tile with `nk` key tiles: S_u = Q K_u^T into S buffer
+// MMA side of query tile kt with `nk` key tiles: S_u = Q K_u^T into S buffer
 // (j & 1), O += P_u V_u with P from TMEM; j and c are the running tile and
-// load counters of the CTA. DBL (moba_blk): O of tile kt in O[kt & 1]; the
-// tile's first PV waits until the epilogue of tile kt - 2 has released that
-// buffer, and its last PV commits o_full[kt & 1].
-template <bool DBL>
-struct MmaT {
+// load counters of the CTA. O of tile kt is O[kt & 1]: the tile's first PV
+// waits until the epilogue of tile kt - 2 has released that buffer, and its
+// last PV commits o_full[kt & 1].
+struct Mma {
   Bars* bars;
   volatile int* abort;
   unsigned* err;
@@ -620,7 +624,7 @@ struct MmaT {
     return st;
   }
   __device__ void tile(uint32_t q0, int nk, int qbuf, int kt = 0) {
-    const uint32_t ob = DBL && (kt & 1) ? kO2 : kO;
+    const uint32_t ob = (kt & 1) ? kO2 : kO;
     const uint32_t iss = tc::idesc_bf16(128, 128, false, false);
     const uint32_t its = tc::idesc_bf16(128, 128, false, true);
     const int j0 = j;
@@ -643,7 +647,7 @@ struct MmaT {
       if (u >= 1) {
         const int pj = j0 + u - 1, pb = pj & 1;
         ok = ok && wait_or_abort(&bars->p_full[pb], (uint32_t)((pj >> 1) & 1), abort, err);
-        if (DBL && u == 1 && kt >= 2)
+        if (u == 1 && kt >= 2)
           ok = ok && wait_or_abort(&bars->o_free[kt & 1], (uint32_t)(((kt >> 1) - 1) & 1), abort,
                                    err);
         tc::fence_after_sync();
@@ -656,7 +660,7 @@ struct MmaT {
                      (u > 1 || ks > 0));
         tc::commit(&bars->empty[st]);
         tc::commit(&bars->o_done[pj & 1]);
-        if (DBL && u == nk) tc::commit(&bars->o_full[kt & 1]);
+        if (u == nk) tc::commit(&bars->o_full[kt & 1]);
         ++c;
       }
     }
@@ -666,15 +670,14 @@ struct MmaT {
 
 // Softmax side: thread `row` of the query tile, one S tile at a time; keys at
 // index >= klim are masked (the causal edge). m is kept in the log2 domain.
-template <bool DBL>
-struct SoftmaxT {
+struct Softmax {
   Bars* bars;
   volatile int* abort;
   unsigned* err;
   uint32_t tl;
   float cs;
   int j = 0;
-  uint32_t obuf = kO;  // DBL: O's TMEM column of the current tile
+  uint32_t obuf = kO;  // O's TMEM column of the current tile
   // The row's nk key tiles [kb0, kb0 + 128 nk). The next tile's scores are
   // loaded from TMEM before this tile's P stores are waited for, so the two
   // TMEM latencies overlap (the next S is in the other buffer, and its QK MMA
@@ -712,7 +715,7 @@ struct SoftmaxT {
 #pragma unroll 1
           for (int q4 = 0; q4 < 8; ++q4) {
             uint32_t w[16];
-            const uint32_t oc = tl + (DBL ? obuf : kO) + q4 * 16;
+            const uint32_t oc = tl + obuf + q4 * 16;
             tc::ld16_sync(oc, w);
 #pragma unroll
             for (int e = 0; e < 16; ++e) w[e] = __float_as_uint(__uint_as_float(w[e]) * f);
@@ -753,8 +756,6 @@ struct SoftmaxT {
   }
 };
 
-using Mma = MmaT<false>;
-using Softmax = SoftmaxT<false>;
 
 // ============================================================================
 // moba_blk: bucket tiles (gathered rows x one earlier block)
@@ -825,7 +826,7 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      MmaT<true> mm{bars, abort, a.err, tmem, ptx::smem_u32(ring)};
+      Mma mm{bars, abort, a.err, tmem, ptx::smem_u32(ring)};
       int k = 0;
       for (int i = blockIdx.x; mm.ok && i < ntile; i += gridDim.x, ++k) {
         const int qb = k & 1;
@@ -841,7 +842,7 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
     // (m, l) goes to the epilogue warps through shared memory
     const int qd = warp & 3;
     const int row = qd * 32 + lane;
-    SoftmaxT<true> sm{bars, abort, a.err, tmem + ((uint32_t)(qd * 32) << 16), a.c};
+    Softmax sm{bars, abort, a.err, tmem + ((uint32_t)(qd * 32) << 16), a.c};
     int k = 0;
     for (int i = blockIdx.x; i < ntile; i += gridDim.x, ++k) {
       sm.obuf = (k & 1) ? kO2 : kO;
@@ -1184,7 +1185,7 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      MmaT<true> mm{bars, abort, a.err, tmem, ptx::smem_u32(ring)};
+      Mma mm{bars, abort, a.err, tmem, ptx::smem_u32(ring)};
       int kq = 0;
       for (int i = blockIdx.x; mm.ok && i < NI; i += gridDim.x, ++kq) {
         const OwnItem it = own_item(a, i);
@@ -1201,7 +1202,7 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
     // (m, l) goes to the merge warps through shared memory
     const int qd = warp & 3;
     const int row = qd * 32 + lane;
-    SoftmaxT<true> sm{bars, abort, a.err, tmem + ((uint32_t)(qd * 32) << 16), a.c};
+    Softmax sm{bars, abort, a.err, tmem + ((uint32_t)(qd * 32) << 16), a.c};
     int k = 0;
     for (int i = blockIdx.x; i < NI; i += gridDim.x, ++k) {
       const OwnItem it = own_item(a, i);
