@@ -119,13 +119,8 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       : "memory");
 }
 
-// 16-byte global -> shared copy through L2 only (cp.async, completes by group).
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)),
-               "l"(reinterpret_cast<uint64_t>(src))
-               : "memory");
-}
-// The same with the bytes past `src_bytes` (0 or 16) filled with zeros.
+// 16-byte global -> shared copy through L2 only (cp.async, completes by group),
+// the bytes past `src_bytes` (0 or 16) filled with zeros.
 __device__ __forceinline__ void cp_async16_zfill(void* dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)),
                "l"(reinterpret_cast<uint64_t>(src)), "r"(src_bytes)
