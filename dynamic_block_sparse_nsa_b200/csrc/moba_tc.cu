@@ -547,7 +547,7 @@ struct Bars {
   int abort;
 };
 
-// TMEM: O at 0, S buffers at 128 and 256; moba_blk's second O (odd tiles) at 384
+// TMEM: O at 0, S buffers at 128 and 256, the second O (odd tiles or items) at 384
 constexpr uint32_t kO = 0, kS0 = 128, kO2 = 384;
 
 __device__ void init_bars(Bars* bars, int q_full_count) {
@@ -1244,8 +1244,9 @@ __global__ void __launch_bounds__(kBlkThreads, 1)
 }
 
 size_t attn_smem(int qbufs) { return 1024 + (size_t)(qbufs + kStages) * TILE + sizeof(Bars); }
-// moba_blk: + the (m, l) hand-off of each row (one buffer: the kernel then stays
-// within the 196 KB shared-memory configuration, which leaves the SM more L1)
+// Both attention kernels: + the (m, l) hand-off of each row (one buffer: the
+// kernels then stay within the 196 KB shared-memory configuration, which
+// leaves the SM more L1)
 size_t blk_smem() { return attn_smem(2) + KT * sizeof(float2); }
 
 
@@ -1263,7 +1264,7 @@ bool moba_tc_eligible(const nsa_params& p) {
 // Workspace after the block means: selection (when the caller passes none),
 // bucket counts / offsets / tile offsets / cursors, the bucket rows, the
 // partial outputs and their log-sum-exp, the split block means, and the
-// bucket of each bucket tile (at most one partial tile per bucket beyond
+// descriptor of each bucket tile (at most one partial tile per bucket beyond
 // rows / 128 full ones).
 size_t moba_tc_ws_bytes(const nsa_params& p, size_t kbar_bytes) {
   const size_t rows = (size_t)p.B * p.T * p.Hq;
